@@ -1,0 +1,287 @@
+"""The synthetic verify-step workloads and their seeded raw inputs.
+
+Shapes follow the five benchmark configurations (tiny one-layer step; batch 1
+at 8k context with a sliding-window and a key-equals-value global layer;
+batch 8 ragged 4k-32k global-only; batch 64 six-layer throughput case; the
+4-layer 131k-prompt speculative loop), plus scaled-down variants of the same
+structure for parity tests that the CPU oracle finishes in seconds.
+
+Everything here is a draw or a layout decision: weights N(0, 0.02) bf16,
+context pre-RoPE keys/values N(0, 1) bf16, token ids uniform, the per-token
+accept coin flips that decide where a draft first goes wrong, and a seeded
+random permutation of the page pool.  No model arithmetic happens here.
+"""
+from __future__ import annotations
+
+import dataclasses
+from dataclasses import dataclass, field
+
+import numpy as np
+
+from . import gen
+
+PAGE = 64
+
+
+@dataclass(frozen=True)
+class LayerSpec:
+    window: int = 0            # 0 = global attention; else sliding window (keys incl. self)
+    kv_equal: bool = False     # key-equals-value global layer (V = pre-RoPE K)
+    rope_fraction: float = 1.0 # fraction of rotary pairs rotated (highest frequencies first)
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    batch: int
+    k: int
+    d_model: int
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    vocab: int
+    layers: tuple
+    ctx_lo: int                 # context lengths uniform in [ctx_lo, ctx_hi] (inclusive)
+    ctx_hi: int
+    accept: tuple               # draft recipe, see make_drafts
+    split_tokens: int = 256     # absolute split-KV chunk of the attention reduction
+    page_size: int = PAGE
+    rope_theta: float = 10000.0
+    rms_eps: float = 1e-6
+    weight_std: float = 0.02
+    seed: int = 0
+    steps: int = 1              # verify steps (the loop workload runs many)
+    prompt_tokens: int = 0      # >0: context is a prefilled random prompt, not drawn K/V
+
+    @property
+    def q_rows(self) -> int:
+        return self.k + 1
+
+    @property
+    def group(self) -> int:
+        return self.n_q_heads // self.n_kv_heads
+
+    def qkv_out(self, layer: LayerSpec) -> int:
+        nv = 0 if layer.kv_equal else self.n_kv_heads
+        return (self.n_q_heads + self.n_kv_heads + nv) * self.head_dim
+
+    def with_(self, **kw) -> "Workload":
+        return dataclasses.replace(self, **kw)
+
+
+LOCAL1024 = LayerSpec(window=1024, kv_equal=False, rope_fraction=1.0)
+GLOBAL_KV = LayerSpec(window=0, kv_equal=True, rope_fraction=0.25)
+GLOBAL_FULL = LayerSpec(window=0, kv_equal=False, rope_fraction=1.0)
+
+WORKLOADS = {
+    # Tiny verify step: 1 layer, 8 q heads / 1 kv head, D 128, d 512, V 4096, ctx 256.
+    "tiny": Workload("tiny", batch=1, k=4, d_model=512, n_q_heads=8, n_kv_heads=1, head_dim=128,
+                     vocab=4096, layers=(GLOBAL_FULL,), ctx_lo=256, ctx_hi=256,
+                     accept=("one_wrong", 0.5)),
+    # Batch 1, 8k context, k=4: sliding-window layer + key-equals-value global layer.
+    "b1_ctx8k": Workload("b1_ctx8k", batch=1, k=4, d_model=2560, n_q_heads=16, n_kv_heads=8,
+                         head_dim=256, vocab=262144, layers=(LOCAL1024, GLOBAL_KV),
+                         ctx_lo=8192, ctx_hi=8192, accept=("geometric", 0.8)),
+    # Batch 8 ragged 4k-32k, global key-equals-value layer only.
+    "b8_ragged": Workload("b8_ragged", batch=8, k=4, d_model=5376, n_q_heads=32, n_kv_heads=4,
+                          head_dim=256, vocab=262144, layers=(GLOBAL_KV,), ctx_lo=4096,
+                          ctx_hi=32768, accept=("geometric", 0.8)),
+    # Batch 64, k=3, 5 sliding-window layers + 1 key-equals-value global layer.
+    "b64_6layer": Workload("b64_6layer", batch=64, k=3, d_model=3840, n_q_heads=16, n_kv_heads=8,
+                           head_dim=256, vocab=262144,
+                           layers=(LOCAL1024,) * 5 + (GLOBAL_KV,), ctx_lo=1024, ctx_hi=16384,
+                           accept=("geometric_per_seq", 0.5, 0.9)),
+    # Speculative loop: 4 layers (3 sliding + 1 global K=V), 131072-token prompt, k=8, 512 steps.
+    "loop_131k": Workload("loop_131k", batch=1, k=8, d_model=2048, n_q_heads=8, n_kv_heads=2,
+                          head_dim=256, vocab=262144, layers=(LOCAL1024,) * 3 + (GLOBAL_KV,),
+                          ctx_lo=131072, ctx_hi=131072, accept=("corrupted_greedy", 0.8),
+                          split_tokens=1024, steps=512, prompt_tokens=131072),
+}
+
+# Scaled-down variants with the same structure, sized for the CPU oracle to
+# finish in seconds while still spanning several tiles, pages and splits and
+# leaving ragged tails (vocab not a multiple of the 128-row tile, contexts
+# not a multiple of the 64-token page or the split).
+WORKLOADS.update({
+    "small_b1": WORKLOADS["b1_ctx8k"].with_(name="small_b1", vocab=9000, ctx_lo=1500, ctx_hi=1500,
+                                              layers=(LayerSpec(window=300), GLOBAL_KV)),
+    "small_ragged": WORKLOADS["b8_ragged"].with_(name="small_ragged", batch=4, d_model=1024,
+                                                  vocab=5000, ctx_lo=100, ctx_hi=1400),
+    "small_b16": WORKLOADS["b64_6layer"].with_(name="small_b16", batch=16, d_model=768,
+                                                vocab=4100, ctx_lo=60, ctx_hi=900,
+                                                layers=(LayerSpec(window=200),) * 2 + (GLOBAL_KV,)),
+    "small_loop": WORKLOADS["loop_131k"].with_(name="small_loop", vocab=6000, d_model=512,
+                                                ctx_lo=700, ctx_hi=700, prompt_tokens=700,
+                                                layers=(LayerSpec(window=128),) * 3 + (GLOBAL_KV,),
+                                                split_tokens=256, steps=24),
+})
+
+
+def get_workload(name: str) -> Workload:
+    return WORKLOADS[name]
+
+
+# --------------------------------------------------------------------------
+# Weights
+# --------------------------------------------------------------------------
+
+def _w(wl: Workload, name: str, rows: int, cols: int) -> np.ndarray:
+    out = gen.normal_bf16(wl.seed, f"{wl.name}/{name}", 0, rows * cols, wl.weight_std)
+    return out.reshape(rows, cols)
+
+
+def lm_head_weight(wl: Workload) -> np.ndarray:
+    """Tied embedding / LM-head matrix, bf16 bits, [vocab][d_model]."""
+    return _w(wl, "w_lm", wl.vocab, wl.d_model)
+
+
+def layer_weights(wl: Workload, l: int):
+    """(W_qkv [Nqkv][d], W_o [d][Hq*D]) bf16 bits, rows = output features.
+
+    W_qkv rows are ordered [q heads | k heads | v heads (absent on K=V layers)],
+    each head's head_dim rows contiguous."""
+    spec = wl.layers[l]
+    wqkv = _w(wl, f"l{l}/w_qkv", wl.qkv_out(spec), wl.d_model)
+    wo = _w(wl, f"l{l}/w_o", wl.d_model, wl.n_q_heads * wl.head_dim)
+    return wqkv, wo
+
+
+# --------------------------------------------------------------------------
+# Per-sequence inputs
+# --------------------------------------------------------------------------
+
+def context_lengths(wl: Workload) -> np.ndarray:
+    if wl.ctx_lo == wl.ctx_hi:
+        return np.full(wl.batch, wl.ctx_lo, dtype=np.int64)
+    return gen.randint(wl.seed, f"{wl.name}/ctx_len", 0, wl.batch, wl.ctx_lo, wl.ctx_hi + 1)
+
+
+def visible_start(wl: Workload, spec: LayerSpec, L: int) -> int:
+    """First context position any of the q rows (positions L..L+k) can see.
+
+    Row at position t sees keys j with t - W < j <= t on a window-W layer, so
+    over the rows the earliest visible key is L - W + 1."""
+    if spec.window == 0:
+        return 0
+    return max(0, L - spec.window + 1)
+
+
+def context_kv(wl: Workload, b: int, attempt: int, l: int, L: int):
+    """Raw (pre-RoPE) context keys and values for positions [lo, L) of layer l.
+
+    Returns (lo, k_raw [n][Hkv][D] bf16 bits, v_raw or None).  Element
+    (pos j, head h, dim e) is counter (j*Hkv + h)*D + e of its stream, so a
+    position's values do not depend on which slice is generated.  K=V layers
+    have no separate V."""
+    spec = wl.layers[l]
+    lo = visible_start(wl, spec, L)
+    n = L - lo
+    hd = wl.n_kv_heads * wl.head_dim
+    base = f"{wl.name}/b{b}/t{attempt}/l{l}"
+    k = gen.normal_bf16(wl.seed, base + "/ctx_k", lo * hd, n * hd, 1.0).reshape(n, wl.n_kv_heads,
+                                                                                 wl.head_dim)
+    v = None
+    if not spec.kv_equal:
+        v = gen.normal_bf16(wl.seed, base + "/ctx_v", lo * hd, n * hd, 1.0).reshape(
+            n, wl.n_kv_heads, wl.head_dim)
+    return lo, k, v
+
+
+def last_token(wl: Workload, b: int, attempt: int) -> int:
+    return int(gen.randint(wl.seed, f"{wl.name}/b{b}/t{attempt}/last_token", 0, 1, 0, wl.vocab)[0])
+
+
+def prompt_tokens(wl: Workload, b: int = 0) -> np.ndarray:
+    """Random prompt token ids for the prefilled-loop workload."""
+    return gen.randint(wl.seed, f"{wl.name}/b{b}/prompt", 0, wl.prompt_tokens, 0, wl.vocab)
+
+
+def rejection_point(wl: Workload, b: int, attempt: int) -> int:
+    """Index r of the first wrong draft (r == k: all drafts correct).
+
+    geometric(p): r = number of leading successes of per-token Bernoulli(p)
+    coin flips, capped at k.  geometric_per_seq(lo, hi): the same with
+    p_b ~ U[lo, hi] drawn once per sequence.  one_wrong(q): with probability
+    q one position j ~ U[0, k) is wrong, else none."""
+    kind = wl.accept[0]
+    base = f"{wl.name}/b{b}/t{attempt}"
+    if kind == "one_wrong":
+        coin = gen.uniform(wl.seed, base + "/wrong_coin", 0, 1)[0]
+        if coin < wl.accept[1]:
+            return int(gen.randint(wl.seed, base + "/wrong_pos", 0, 1, 0, wl.k)[0])
+        return wl.k
+    if kind == "geometric":
+        p = wl.accept[1]
+    elif kind == "geometric_per_seq":
+        p = wl.accept[1] + (wl.accept[2] - wl.accept[1]) * gen.uniform(
+            wl.seed, f"{wl.name}/b{b}/accept_p", 0, 1)[0]
+    else:
+        raise ValueError(f"no fixed rejection point for draft recipe {kind}")
+    flips = gen.uniform(wl.seed, base + "/accept_flips", 0, wl.k)
+    r = 0
+    while r < wl.k and flips[r] < p:
+        r += 1
+    return r
+
+
+def make_drafts(wl: Workload, b: int, attempt: int, greedy: np.ndarray) -> tuple[np.ndarray, int]:
+    """Drafts from the greedy continuation `greedy` (at least r+1 tokens).
+
+    drafts[i] = greedy[i] for i < r; drafts[r] = a random id != greedy[r];
+    later drafts are random ids.  one_wrong keeps greedy tokens after the
+    replaced position.  Returns (drafts[k] int32, r)."""
+    r = rejection_point(wl, b, attempt)
+    stream = f"{wl.name}/b{b}/t{attempt}/draft_rand"
+    ids = gen.randint(wl.seed, stream, 0, 4 * wl.k + 64, 0, wl.vocab)
+    drafts = np.empty(wl.k, dtype=np.int32)
+    ctr = 0
+    for i in range(wl.k):
+        if i < r:
+            drafts[i] = greedy[i]
+        elif i == r:
+            while ids[ctr] == greedy[r]:
+                ctr += 1
+            drafts[i] = ids[ctr]
+            ctr += 1
+        elif wl.accept[0] == "one_wrong":
+            drafts[i] = greedy[i]
+        else:
+            drafts[i] = ids[ctr]
+            ctr += 1
+    return drafts, r
+
+
+def loop_draft_flips(wl: Workload, step: int) -> tuple[np.ndarray, np.ndarray]:
+    """Coin flips and random ids of the corrupted-greedy drafter at one loop step:
+    draft i is the true greedy token if flip[i] < p else ids[i]."""
+    flips = gen.uniform(wl.seed, f"{wl.name}/loop_flips", step * wl.k, wl.k)
+    ids = gen.randint(wl.seed, f"{wl.name}/loop_ids", step * wl.k, wl.k, 0, wl.vocab)
+    return flips, ids
+
+
+# --------------------------------------------------------------------------
+# Paged layout
+# --------------------------------------------------------------------------
+
+def pages_needed(L: int, k: int, page: int = PAGE, extra_tokens: int = 0) -> int:
+    return -(-(L + k + 1 + extra_tokens) // page)
+
+
+def page_assignment(wl: Workload, lens, extra_tokens: int = 0):
+    """Seeded random permutation of the pool, handed out sequence by sequence.
+
+    Returns (num_pages, block_table [B][max_pages] int32, -1 padded)."""
+    need = [pages_needed(int(L), wl.k, wl.page_size, extra_tokens) for L in lens]
+    total = int(sum(need))
+    u = gen.uniform(wl.seed, f"{wl.name}/page_perm", 0, total)
+    perm = np.arange(total, dtype=np.int64)
+    for i in range(total - 1, 0, -1):       # Fisher-Yates, driven by the counter stream
+        j = int(u[i] * (i + 1))
+        perm[i], perm[j] = perm[j], perm[i]
+    maxp = max(need)
+    table = np.full((len(lens), maxp), -1, dtype=np.int32)
+    pos = 0
+    for b, n in enumerate(need):
+        table[b, :n] = perm[pos:pos + n]
+        pos += n
+    return total, table

@@ -1,0 +1,93 @@
+"""Test-side glue: turn a workload's seeded raw inputs into oracle objects and
+into the drafts/expected outcomes the parity tests compare against.
+
+Only tests (and the golden-fixture script) use this module; it imports the
+oracle and the input generator, never the CUDA binding.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+
+import oracle
+from speculative_decoding_verification_91_b200.inputs import workloads as W
+
+MARGIN_ABS = 2e-2      # float tolerance of logits: 2e-2 absolute ...
+MARGIN_REL = 1e-2      # ... plus 1e-2 relative
+
+
+def margin_ok(top1: float, top2: float) -> bool:
+    """Top-2 logit gap wider than the logits' float tolerance, so that any
+    implementation within tolerance takes the same argmax."""
+    return (top1 - top2) >= MARGIN_ABS + MARGIN_REL * abs(top1)
+
+
+def oracle_model(wl: W.Workload) -> oracle.Model:
+    layers = []
+    for l, spec in enumerate(wl.layers):
+        wqkv, wo = W.layer_weights(wl, l)
+        layers.append(oracle.LayerDef(spec.window, spec.kv_equal, spec.rope_fraction,
+                                      oracle.bf16_from_bits(wqkv), oracle.bf16_from_bits(wo)))
+    return oracle.Model(wl.d_model, wl.n_q_heads, wl.n_kv_heads, wl.head_dim,
+                        W.lm_head_weight(wl), layers, wl.rope_theta, wl.rms_eps)
+
+
+def context_caches(wl: W.Workload, model: oracle.Model, b: int, attempt: int, L: int):
+    caches = []
+    for l in range(len(wl.layers)):
+        lo, k, v = W.context_kv(wl, b, attempt, l, L)
+        caches.append(oracle.cache_from_raw(model, l, lo, oracle.bf16_from_bits(k),
+                                            None if v is None else oracle.bf16_from_bits(v)))
+    return caches
+
+
+def greedy_continuation(model, caches, L, last, n):
+    """First n greedy tokens after `last` (one oracle forward per token)."""
+    toks = [int(last)]
+    out = []
+    for _ in range(n):
+        fw = model_forward_last(model, caches, L, toks)
+        out.append(int(fw.g[0]))
+        toks.append(out[-1])
+    return np.array(out, dtype=np.int64)
+
+
+def model_forward_last(model, caches, L, toks):
+    return oracle.verify_forward(model, caches, L, toks, lm_rows=[len(toks) - 1])
+
+
+@dataclass
+class SeqCase:
+    b: int
+    attempt: int
+    L: int
+    last: int
+    drafts: np.ndarray
+    r: int
+    result: object          # oracle.StepResult
+    guarded: bool           # rows 0..a all have a safe top-2 margin
+
+
+def build_sequence(wl, model, b, L, attempt, guard=True) -> SeqCase:
+    caches = context_caches(wl, model, b, attempt, L)
+    last = W.last_token(wl, b, attempt)
+    r = W.rejection_point(wl, b, attempt)
+    n_greedy = wl.k if (r == wl.k or wl.accept[0] == "one_wrong") else r + 1
+    greedy = greedy_continuation(model, caches, L, last, n_greedy)
+    drafts, r2 = W.make_drafts(wl, b, attempt, np.concatenate([greedy, np.zeros(1, np.int64)]))
+    assert r2 == r
+    res = oracle.verify_step(model, caches, L, last, drafts)
+    ok = res.accept_len == r and all(margin_ok(res.top1[i], res.top2[i])
+                                     for i in range(res.accept_len + 1))
+    return SeqCase(b, attempt, L, last, drafts, r, res, ok)
+
+
+def guarded_sequence(wl, model, b, L, max_attempts=40, start=0) -> SeqCase:
+    """Redraw the sequence's sub-seed (context, last token, drafts) until every
+    argmax the acceptance depends on has a safe margin."""
+    for t in range(start, start + max_attempts):
+        case = build_sequence(wl, model, b, L, t)
+        if case.guarded:
+            return case
+    raise RuntimeError(f"no margin-safe draw for sequence {b} in {max_attempts} attempts")
