@@ -1,0 +1,382 @@
+"""Benchmark of the fused verify step (spec_verify_step) on synthetic inputs.
+
+Default workload: batch 1, 8192-token context, k = 4 drafts, two layers (a
+1024-token sliding-window layer with separate K/V and a key-equals-value
+global layer with p-RoPE p = 0.25), 16 query / 8 KV heads, head_dim 256,
+d_model 2560, 262,144-token vocabulary, 64-token pages scattered in the pool.
+
+Prints one JSON line.  `value` is verified tokens per second (tokens the
+step emits: accepted drafts plus the target's own token), whole job over
+all ranks, timed on the device with CUDA events around each step while the
+inputs are resident; `e2e` is the same metric through the C ABI with the
+step's inputs copied from pinned host memory and its results copied back
+inside the timed region.  `roofline` reports the LM-head kernel (the step's
+largest byte mover) against the measured HBM copy bandwidth.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cuda|reference]
+
+Under torchrun each rank runs its own replica of the workload (independent
+sequences; no collective on the data path) and rank 0 prints the line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "verified tokens/s (k=4) & us per verify step; HBM GB/s as % of B200 peak"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
+    ap.add_argument("--workload", default="b1_ctx8k")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------
+# Inputs: drafts from the workload's recipe; the greedy continuation they
+# need comes from the CUDA path itself (k = 0 steps), which only chooses
+# inputs and is not a parity claim.
+# --------------------------------------------------------------------------
+
+def gpu_greedy_drafts(sess, wl, W):
+    import torch
+    greedy = np.zeros((wl.batch, wl.k + 1), dtype=np.int64)
+    last = np.array([W.last_token(wl, b, sess.attempts[b]) for b in range(wl.batch)], np.int32)
+    from speculative_decoding_verification_91_b200.session import WorkloadSession
+    g = WorkloadSession(wl.with_(k=0), attempts=sess.attempts, device=sess.device, poison=False)
+    cur = last.copy()
+    for i in range(wl.k + 1):
+        g.set_inputs(cur, [])
+        g.step()
+        o = g.outputs()
+        greedy[:, i] = o["target_ids"][:, 0]
+        cur = o["new_last"].astype(np.int32)
+    del g
+    torch.cuda.empty_cache()
+    drafts = np.stack([W.make_drafts(wl, b, sess.attempts[b], greedy[b])[0] for b in range(wl.batch)])
+    return last, drafts
+
+
+def algorithmic_bytes(wl, lens):
+    """North-star bytes of one step: visible KV pages read (union of the rows'
+    keys; key-equals-value layers at (1+p)*D per token-head) + LM-head weights."""
+    kv = 0
+    for spec in wl.layers:
+        for L in lens:
+            hi = L + wl.k + 1
+            lo = 0 if spec.window == 0 else max(0, L - spec.window + 1)
+            per = (wl.head_dim * (1 + spec.rope_fraction) if spec.kv_equal else 2 * wl.head_dim) * 2
+            kv += (hi - lo) * wl.n_kv_heads * per
+    lm = wl.vocab * wl.d_model * 2
+    proj = sum((wl.qkv_out(s) * wl.d_model + wl.d_model * wl.n_q_heads * wl.head_dim) * 2
+               for s in wl.layers)
+    return int(kv), int(lm), int(proj)
+
+
+def run_cuda(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from speculative_decoding_verification_91_b200 import binding as B
+    from speculative_decoding_verification_91_b200.inputs import workloads as W
+    from speculative_decoding_verification_91_b200.session import WorkloadSession
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = W.get_workload(args.workload)
+    B.lib()
+    sess = WorkloadSession(wl, device=dev, poison=False)
+    last, drafts = gpu_greedy_drafts(sess, wl, W)
+    sess.set_inputs(last, drafts)
+    stream = torch.cuda.current_stream(dev)
+
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    # ---- warm-up (untimed), also fixes the emitted-token count of the step
+    for _ in range(args.warmup):
+        sess.reset_lengths()
+        sess.step(stream=stream)
+    torch.cuda.synchronize(dev)
+    out = sess.outputs()
+    if sess.ws.device_status(stream) != 0:
+        raise RuntimeError("device status flagged during warm-up")
+    tokens_per_step = int(np.sum(out["accept_len"] + 1))
+
+    # ---- timed: device-resident inputs, L2 flushed before every step
+    starts = [ev() for _ in range(args.steps)]
+    stops = [ev() for _ in range(args.steps)]
+    lm0 = [ev() for _ in range(args.steps)]
+    lm1 = [ev() for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local_rank) as clocks:
+        for i in range(args.steps):
+            flush.zero_()
+            sess.reset_lengths()
+            B.spec_set_profile_events(B.SPEC_PROF_STEP, starts[i], stops[i])
+            B.spec_set_profile_events(B.SPEC_PROF_LMHEAD, lm0[i], lm1[i])
+            sess.step(stream=stream, with_targets=False)
+        B.spec_set_profile_events(B.SPEC_PROF_STEP, None, None)
+        B.spec_set_profile_events(B.SPEC_PROF_LMHEAD, None, None)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, stops)]
+    lm_ms = [s.elapsed_time(e) for s, e in zip(lm0, lm1)]
+    if sess.ws.device_status(stream) != 0:
+        raise RuntimeError("device status flagged during the timed steps")
+
+    # ---- e2e: the public C-ABI call fed from pinned host buffers
+    Bn, k = wl.batch, wl.k
+    h_in = torch.empty(Bn * (2 + k), dtype=torch.int32).pin_memory()
+    h_in[:Bn] = torch.from_numpy(last)
+    h_in[Bn:Bn + Bn * k] = torch.from_numpy(drafts.reshape(-1).astype(np.int32))
+    h_in[Bn + Bn * k:] = torch.from_numpy(sess.lens.astype(np.int32))
+    h_out = torch.empty(Bn * (k + 1) + 3 * Bn, dtype=torch.int32).pin_memory()
+    e0 = [ev() for _ in range(args.steps)]
+    e1 = [ev() for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.zero_()
+        e0[i].record(stream)
+        sess.last_token.copy_(h_in[:Bn], non_blocking=True)
+        sess.drafts[:Bn * k].copy_(h_in[Bn:Bn + Bn * k], non_blocking=True)
+        sess.seq_lens.copy_(h_in[Bn + Bn * k:], non_blocking=True)
+        sess.step(stream=stream, with_targets=False)
+        h_out[:Bn * (k + 1)].copy_(sess.emitted, non_blocking=True)
+        h_out[Bn * (k + 1):Bn * (k + 2)].copy_(sess.accept_len, non_blocking=True)
+        h_out[Bn * (k + 2):Bn * (k + 3)].copy_(sess.new_last, non_blocking=True)
+        h_out[Bn * (k + 3):].copy_(sess.seq_lens, non_blocking=True)
+        e1[i].record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = [s.elapsed_time(e) for s, e in zip(e0, e1)]
+    got_acc = h_out[Bn * (k + 1):Bn * (k + 2)].numpy()
+    assert np.array_equal(got_acc, out["accept_len"]), "e2e step disagrees with the device-timed step"
+
+    mean_step = float(np.mean(step_ms))
+    mean_lm = float(np.mean(lm_ms))
+    mean_e2e = float(np.mean(e2e_ms))
+    if world > 1:
+        t = torch.tensor([mean_step, mean_e2e, mean_lm], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        mean_step, mean_e2e, mean_lm = [float(v) for v in t.tolist()]
+    kv_b, lm_b, proj_b = algorithmic_bytes(wl, sess.lens)
+    launches_per_step = 4 + 6 * len(wl.layers)
+    return dict(wl=wl, lens=sess.lens, tokens_per_step=tokens_per_step, mean_step=mean_step,
+                mean_lm=mean_lm, mean_e2e=mean_e2e, kv_b=kv_b, lm_b=lm_b, proj_b=proj_b,
+                launches=launches_per_step * args.steps, clocks=clocks.summary(),
+                h2d=int(h_in.numel() * 4), d2h=int(h_out.numel() * 4), step_ms=step_ms,
+                M=wl.batch * wl.q_rows)
+
+
+# --------------------------------------------------------------------------
+# CPU oracle leg (baseline only; bounded sample)
+# --------------------------------------------------------------------------
+
+def oracle_sample(wl_name: str, budget_s: float = 25.0):
+    """Times the CPU oracle on one sequence of the workload: a full verify
+    step (all layers, all k+1 rows, full-vocabulary LM head).  Returns
+    (tokens/s, seconds, threads, description)."""
+    import oracle
+    from speculative_decoding_verification_91_b200.inputs import workloads as W
+    from speculative_decoding_verification_91_b200.inputs import gen
+    wl = W.get_workload(wl_name)
+    L = int(W.context_lengths(wl)[0])
+    layers = []
+    for l, spec in enumerate(wl.layers):
+        wqkv, wo = W.layer_weights(wl, l)
+        layers.append(oracle.LayerDef(spec.window, spec.kv_equal, spec.rope_fraction,
+                                      oracle.bf16_from_bits(wqkv), oracle.bf16_from_bits(wo)))
+    model = oracle.Model(wl.d_model, wl.n_q_heads, wl.n_kv_heads, wl.head_dim,
+                         W.lm_head_weight(wl), layers, wl.rope_theta, wl.rms_eps)
+    caches = []
+    for l in range(len(wl.layers)):
+        lo, k, v = W.context_kv(wl, 0, 0, l, L)
+        caches.append(oracle.cache_from_raw(model, l, lo, oracle.bf16_from_bits(k),
+                                            None if v is None else oracle.bf16_from_bits(v)))
+    last = W.last_token(wl, 0, 0)
+    drafts = gen.randint(wl.seed, f"{wl.name}/bench_drafts", 0, wl.k, 0, wl.vocab)
+    t0 = time.perf_counter()
+    n = 0
+    tokens = 0
+    while True:
+        res = oracle.verify_step(model, caches, L, last, drafts)
+        tokens += res.accept_len + 1
+        n += 1
+        if time.perf_counter() - t0 > budget_s * 0.5 or n >= 3:
+            break
+    dt = time.perf_counter() - t0
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    desc = (f"{n} full oracle verify step(s) of sequence 0 ({wl.name}: {len(wl.layers)} layers, "
+            f"k={wl.k}, ctx {L}, vocab {wl.vocab}); numpy float64, BLAS threads={threads}")
+    return tokens / dt, dt / n, threads, desc
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        steps_tok, steps_s = [], []
+        for _ in range(args.warmup + args.steps):
+            tps, sec, threads, desc = oracle_sample(args.workload, budget_s=4.0)
+            steps_tok.append(tps)
+            steps_s.append(sec)
+        tps = float(np.mean(steps_tok[args.warmup:]))
+        sec = float(np.mean(steps_s[args.warmup:]))
+        line = {"metric": METRIC, "value": tps, "unit": "tokens/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "impl": "reference",
+                "config": {"workload": args.workload},
+                "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": threads,
+                                 "kind": "oracle", "sample": desc},
+                "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        dist.init_process_group("nccl", init_method="env://",
+                                timeout=__import__("datetime").timedelta(seconds=300))
+    try:
+        r = run_cuda(args, rank, world, local_rank)
+    finally:
+        pass
+    if rank == 0:
+        wl = r["wl"]
+        peak, peak_kind = measured_peaks()
+        step_s = r["mean_step"] / 1e3
+        lm_s = r["mean_lm"] / 1e3
+        value = r["tokens_per_step"] * world / step_s
+        lm_bytes = r["lm_b"] + r["M"] * wl.d_model * 2
+        achieved = lm_bytes / lm_s / 1e9
+        step_bytes = r["kv_b"] + r["lm_b"]
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["mean_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": wl.name, "batch": wl.batch, "k": wl.k,
+                       "context": [int(x) for x in r["lens"]], "layers": len(wl.layers),
+                       "d_model": wl.d_model, "vocab": wl.vocab,
+                       "l2": f"flushed ({L2_FLUSH_BYTES >> 20} MiB write) before every timed step",
+                       "tokens_per_step": r["tokens_per_step"]},
+            "us_per_step": r["mean_step"] * 1e3,
+            "step_hbm": {"bytes": step_bytes, "bytes_with_projections": step_bytes + r["proj_b"],
+                         "gbs": step_bytes / step_s / 1e9,
+                         "frac_of_8tbs": step_bytes / step_s / 1e9 / NOMINAL_HBM_GBS,
+                         "frac_of_measured": step_bytes / step_s / 1e9 / peak},
+            "roofline": {"kernel": "stream_gemm_kernel<argmax> (LM head + argmax)", "bound": "hbm",
+                         "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "peak_kind": peak_kind, "traffic": None,
+                         "bytes_per_launch": lm_bytes, "us_per_launch": r["mean_lm"] * 1e3},
+            "e2e": {"value": r["tokens_per_step"] * world / (r["mean_e2e"] / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
+            "gpu_launches": r["launches"],
+            "clocks": r["clocks"],
+        }
+        if not args.no_cpu_baseline and world == 1:
+            tps, sec, threads, desc = oracle_sample(wl.name)
+            line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": threads,
+                                    "kind": "oracle", "sample": desc}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

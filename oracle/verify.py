@@ -372,6 +372,9 @@ def verify_forward(model: Model, caches: list, L: int, tokens, lm_rows=None) -> 
         x = f32(x.astype(np.float64) + y.astype(np.float64))
     rows = np.arange(nq) if lm_rows is None else np.asarray(lm_rows, dtype=np.int64)
     h = bf16(rmsnorm(x[rows], model.rms_eps))
+    if rows.size == 0:                      # caller forms the logits itself (batched)
+        empty = np.zeros(0)
+        return Forward(empty.astype(np.int64), empty, empty, h, new_entries, attn_out, x)
     g, t1, t2 = lm_head_top2(h, model.w_lm_bits)
     return Forward(g, t1, t2, h, new_entries, attn_out, x)
 

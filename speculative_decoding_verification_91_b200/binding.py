@@ -1,0 +1,200 @@
+"""ctypes binding of libspecverify.so: argument marshalling only.
+
+Every function here has the name and argument order of the C entry point in
+include/specverify.h.  Tensor arguments may be ints (device addresses),
+objects with ``data_ptr()`` (torch tensors) or None (NULL).  A non-zero
+status raises SpecError.  There is no fallback: if the library is missing
+the import of the first entry point raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import POINTER, c_float, c_int, c_size_t, c_uint, c_void_p
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libspecverify.so")
+
+SPEC_OK = 0
+SPEC_EINVAL = -1
+SPEC_EUNSUPPORTED = -2
+SPEC_ECUDA = -3
+SPEC_EDEVICE = -4
+SPEC_ETIMEOUT = -5
+SPEC_DEV_BAD_PAGE = 0x1
+SPEC_DEV_BAD_LENGTH = 0x2
+SPEC_DEV_TIMEOUT = 0x4
+SPEC_DEV_BAD_TOKEN = 0x8
+SPEC_MAX_K = 16
+SPEC_PAGE_SIZE = 64
+
+EXPORTED = [
+    "spec_status_string", "spec_layer_pool_bytes", "spec_workspace_bytes",
+    "spec_lmhead_workspace_bytes", "spec_workspace_init", "spec_read_device_status",
+    "spec_cache_write", "spec_verify_attn", "spec_lmhead_argmax", "spec_accept_commit",
+    "spec_verify_step", "spec_set_profile_events",
+]
+SPEC_PROF_LMHEAD = 0
+SPEC_PROF_STEP = 1
+
+
+class SpecError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status} ({status_string(status)})")
+
+
+class SpecLayer(ctypes.Structure):
+    _fields_ = [
+        ("w_qkv", c_void_p), ("w_o", c_void_p),
+        ("k_pool", c_void_p), ("v_pool", c_void_p), ("ksb_pool", c_void_p),
+        ("window", c_int), ("kv_equal", c_int), ("rope_fraction", c_float),
+    ]
+
+
+class SpecModel(ctypes.Structure):
+    _fields_ = [
+        ("n_layers", c_int), ("d_model", c_int), ("n_q_heads", c_int), ("n_kv_heads", c_int),
+        ("head_dim", c_int), ("vocab", c_int), ("page_size", c_int), ("num_pages", c_int),
+        ("split_tokens", c_int), ("rope_theta", c_float), ("rms_eps", c_float),
+        ("w_lm", c_void_p), ("layers", POINTER(SpecLayer)),
+    ]
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def lib():
+    """The loaded library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(
+                f"{_LIB_PATH} is missing: build it with "
+                "`python -m speculative_decoding_verification_91_b200.build`")
+        L = ctypes.CDLL(_LIB_PATH)
+        pm = POINTER(SpecModel)
+        L.spec_status_string.restype = ctypes.c_char_p
+        L.spec_status_string.argtypes = [c_int]
+        L.spec_layer_pool_bytes.restype = c_size_t
+        L.spec_layer_pool_bytes.argtypes = [pm, c_int, c_int]
+        L.spec_workspace_bytes.restype = c_size_t
+        L.spec_workspace_bytes.argtypes = [pm, c_int, c_int, c_int]
+        L.spec_lmhead_workspace_bytes.restype = c_size_t
+        L.spec_lmhead_workspace_bytes.argtypes = [c_int, c_int]
+        L.spec_workspace_init.argtypes = [c_void_p, c_size_t, c_void_p]
+        L.spec_read_device_status.argtypes = [c_void_p, c_size_t, c_void_p, POINTER(c_uint)]
+        L.spec_cache_write.argtypes = [pm, c_int, c_void_p, c_int, c_int, c_int, c_void_p, c_void_p,
+                                       c_void_p]
+        L.spec_verify_attn.argtypes = [pm, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_int,
+                                       c_void_p, c_int, c_int, c_void_p, c_void_p, c_size_t,
+                                       c_void_p]
+        L.spec_lmhead_argmax.argtypes = [c_void_p, c_void_p, c_int, c_int, c_int, c_void_p,
+                                         c_void_p, c_void_p, c_size_t, c_void_p]
+        L.spec_accept_commit.argtypes = [c_void_p, c_void_p, c_int, c_int, c_void_p, c_void_p,
+                                         c_void_p, c_void_p, c_void_p]
+        L.spec_verify_step.argtypes = [pm, c_void_p, c_int, c_void_p, c_void_p, c_int, c_int,
+                                       c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                       c_void_p, c_size_t, c_void_p]
+        L.spec_set_profile_events.argtypes = [c_int, c_void_p, c_void_p]
+        for name in EXPORTED[4:]:
+            getattr(L, name).restype = c_int
+        _lib = L
+    return _lib
+
+
+def _p(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _s(stream):
+    if stream is None:
+        return None
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(rc: int, where: str) -> int:
+    if rc != SPEC_OK:
+        raise SpecError(rc, where)
+    return rc
+
+
+def status_string(status: int) -> str:
+    return lib().spec_status_string(status).decode()
+
+
+def spec_layer_pool_bytes(model: SpecModel, layer: int, which: int) -> int:
+    return int(lib().spec_layer_pool_bytes(ctypes.byref(model), layer, which))
+
+
+def spec_workspace_bytes(model: SpecModel, max_batch: int, max_k: int, max_pages: int) -> int:
+    return int(lib().spec_workspace_bytes(ctypes.byref(model), max_batch, max_k, max_pages))
+
+
+def spec_lmhead_workspace_bytes(M: int, V: int) -> int:
+    return int(lib().spec_lmhead_workspace_bytes(M, V))
+
+
+def spec_workspace_init(ws, ws_bytes: int, stream=None) -> int:
+    return _check(lib().spec_workspace_init(_p(ws), ws_bytes, _s(stream)), "spec_workspace_init")
+
+
+def spec_read_device_status(ws, ws_bytes: int, stream=None) -> int:
+    """Returns the SPEC_DEV_* bits (and clears them); never raises on bits."""
+    v = c_uint(0)
+    rc = lib().spec_read_device_status(_p(ws), ws_bytes, _s(stream), ctypes.byref(v))
+    if rc not in (SPEC_OK, SPEC_EDEVICE, SPEC_ETIMEOUT):
+        raise SpecError(rc, "spec_read_device_status")
+    return int(v.value)
+
+
+def spec_cache_write(model, layer, block_table_row, max_pages, pos0, n_tok, k_raw, v_raw,
+                     stream=None) -> int:
+    return _check(lib().spec_cache_write(ctypes.byref(model), layer, _p(block_table_row), max_pages,
+                                         pos0, n_tok, _p(k_raw), _p(v_raw), _s(stream)),
+                  "spec_cache_write")
+
+
+def spec_verify_attn(model, layer, q, k_new, v_new, block_table, max_pages, seq_lens, B, k, out,
+                     ws, ws_bytes, stream=None) -> int:
+    return _check(lib().spec_verify_attn(ctypes.byref(model), layer, _p(q), _p(k_new), _p(v_new),
+                                         _p(block_table), max_pages, _p(seq_lens), B, k, _p(out),
+                                         _p(ws), ws_bytes, _s(stream)), "spec_verify_attn")
+
+
+def spec_lmhead_argmax(h, w, M, d, V, ids, maxlogit, ws, ws_bytes, stream=None) -> int:
+    return _check(lib().spec_lmhead_argmax(_p(h), _p(w), M, d, V, _p(ids), _p(maxlogit), _p(ws),
+                                           ws_bytes, _s(stream)), "spec_lmhead_argmax")
+
+
+def spec_accept_commit(drafts, target, B, k, seq_lens, accept_len, emitted, last_token,
+                       stream=None) -> int:
+    return _check(lib().spec_accept_commit(_p(drafts), _p(target), B, k, _p(seq_lens),
+                                           _p(accept_len), _p(emitted), _p(last_token), _s(stream)),
+                  "spec_accept_commit")
+
+
+def spec_verify_step(model, block_table, max_pages, last_token, drafts, B, k, seq_lens, accept_len,
+                     emitted, new_last_token, target_ids, target_maxlogit, ws, ws_bytes,
+                     stream=None) -> int:
+    return _check(lib().spec_verify_step(ctypes.byref(model), _p(block_table), max_pages,
+                                         _p(last_token), _p(drafts), B, k, _p(seq_lens),
+                                         _p(accept_len), _p(emitted), _p(new_last_token),
+                                         _p(target_ids), _p(target_maxlogit), _p(ws), ws_bytes,
+                                         _s(stream)), "spec_verify_step")
+
+
+def spec_set_profile_events(stage: int, ev_start, ev_stop) -> int:
+    """ev_start / ev_stop: torch.cuda.Event (recorded by the library) or None."""
+    h = lambda e: None if e is None else e.cuda_event
+    return _check(lib().spec_set_profile_events(stage, h(ev_start), h(ev_stop)),
+                  "spec_set_profile_events")

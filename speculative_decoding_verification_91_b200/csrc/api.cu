@@ -1,0 +1,433 @@
+// C ABI of the verify step: argument validation, workspace layout, launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "../../include/specverify.h"
+#include "common.cuh"
+#include "internal.h"
+
+namespace sv {
+
+// ------------------------------------------------------------------ TMA maps
+namespace {
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                              const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                              CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                              CUtensorMapFloatOOBfill);
+EncodeFn g_encode = nullptr;
+std::once_flag g_encode_once;
+
+void resolve_encode() {
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    g_encode = reinterpret_cast<EncodeFn>(fn);
+}
+}  // namespace
+
+bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                       uint32_t box_rows, uint32_t box_cols) {
+  std::call_once(g_encode_once, resolve_encode);
+  if (!g_encode || !base) return false;
+  if ((reinterpret_cast<uintptr_t>(base) & 15) || (cols * 2) % 16 || box_cols * 2 > 128) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+int n_rot_of(const spec_model* m, const spec_layer& L) {
+  return (int)lrintf(L.rope_fraction * (float)m->head_dim / 2.0f);
+}
+
+int qkv_out(const spec_model* m, const spec_layer& L) {
+  return (m->n_q_heads + m->n_kv_heads + (L.kv_equal ? 0 : m->n_kv_heads)) * m->head_dim;
+}
+
+int check_model(const spec_model* m) {
+  if (!m || !m->layers || !m->w_lm) return SPEC_EINVAL;
+  if (m->n_layers < 1 || m->d_model < 8 || m->d_model % 8 || m->n_q_heads < 1 || m->n_kv_heads < 1 ||
+      m->n_q_heads % m->n_kv_heads || m->vocab < 1 || m->num_pages < 1)
+    return SPEC_EINVAL;
+  if (m->page_size != SPEC_PAGE_SIZE) return SPEC_EUNSUPPORTED;
+  if (m->head_dim != 128 && m->head_dim != 256) return SPEC_EUNSUPPORTED;
+  if (m->split_tokens < m->page_size || m->split_tokens % m->page_size) return SPEC_EINVAL;
+  if (!(m->rope_theta > 0.f) || !(m->rms_eps >= 0.f)) return SPEC_EINVAL;
+  if ((uint64_t)m->num_pages * m->n_kv_heads * m->page_size > 0x7fffffffull) return SPEC_EUNSUPPORTED;
+  if (reinterpret_cast<uintptr_t>(m->w_lm) & 15) return SPEC_EINVAL;
+  for (int l = 0; l < m->n_layers; ++l) {
+    const spec_layer& L = m->layers[l];
+    if (!L.w_qkv || !L.w_o || !L.k_pool) return SPEC_EINVAL;
+    if (L.window < 0) return SPEC_EINVAL;
+    if (!(L.rope_fraction >= 0.f && L.rope_fraction <= 1.f)) return SPEC_EINVAL;
+    const int nr = n_rot_of(m, L);
+    if (L.kv_equal) {
+      if (!L.ksb_pool || L.v_pool) return SPEC_EINVAL;
+      if (2 * nr != 64) return SPEC_EUNSUPPORTED;   // side-band tile is 64 wide
+    } else if (!L.v_pool) {
+      return SPEC_EINVAL;
+    }
+    const void* ptrs[5] = {L.w_qkv, L.w_o, L.k_pool, L.v_pool, L.ksb_pool};
+    for (const void* p : ptrs)
+      if (reinterpret_cast<uintptr_t>(p) & 15) return SPEC_EINVAL;
+  }
+  return SPEC_OK;
+}
+
+// Workspace layout of one verify step for (B, k, max_pages).
+struct StepLayout {
+  size_t x, hn, qkv, qrot, attn_out, attn_part, gemm_part, arg_val, arg_idx, ids, maxv, total;
+  int tickets;
+};
+
+StepLayout step_layout(const spec_model* m, int B, int k, int max_pages) {
+  StepLayout s{};
+  const int q = k + 1, M = B * q, d = m->d_model, D = m->head_dim;
+  int nqkv = 0;
+  size_t attn_floats = 0, gemm_floats = 0;
+  int tickets = 0;
+  for (int l = 0; l < m->n_layers; ++l) {
+    const spec_layer& L = m->layers[l];
+    nqkv = std::max(nqkv, qkv_out(m, L));
+    AttnGeom g = plan_attn(B, q, m->n_q_heads, m->n_kv_heads, D, m->page_size, m->num_pages,
+                           max_pages, L.window, L.kv_equal, 2 * n_rot_of(m, L), m->split_tokens);
+    attn_floats = std::max(attn_floats, attn_partial_floats(g));
+    GemmPlan pq = plan_gemm(M, qkv_out(m, L), d, kGemmStore);
+    GemmPlan po = plan_gemm(M, d, m->n_q_heads * D, kGemmResidual);
+    gemm_floats = std::max({gemm_floats, gemm_partial_floats(pq), gemm_partial_floats(po)});
+    tickets = std::max({tickets, gemm_tickets(pq), gemm_tickets(po)});
+  }
+  GemmPlan pl = plan_gemm(M, m->vocab, d, kGemmArgmax);
+  tickets = std::max(tickets, pl.mblocks);
+  size_t off = kWsHeaderBytes;
+  s.x = off;         off = up(off + (size_t)M * d * 4);
+  s.hn = off;        off = up(off + (size_t)M * d * 2);
+  s.qkv = off;       off = up(off + (size_t)M * nqkv * 4);
+  s.qrot = off;      off = up(off + (size_t)M * m->n_q_heads * D * 2);
+  s.attn_out = off;  off = up(off + (size_t)M * m->n_q_heads * D * 2);
+  s.attn_part = off; off = up(off + attn_floats * 4);
+  s.gemm_part = off; off = up(off + gemm_floats * 4);
+  s.arg_val = off;   off = up(off + gemm_argmax_entries(pl) * 4);
+  s.arg_idx = off;   off = up(off + gemm_argmax_entries(pl) * 4);
+  s.ids = off;       off = up(off + (size_t)M * 4);
+  s.maxv = off;      off = up(off + (size_t)M * 4);
+  s.total = off;
+  s.tickets = tickets;
+  return s;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? SPEC_OK : SPEC_ECUDA; }
+
+cudaEvent_t g_prof[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};
+inline void prof_mark(int stage, int which, cudaStream_t st) {
+  if (g_prof[stage][which]) cudaEventRecord(g_prof[stage][which], st);
+}
+
+}  // namespace
+}  // namespace sv
+
+using namespace sv;
+
+extern "C" {
+
+int spec_set_profile_events(int stage, void* ev_start, void* ev_stop) {
+  if (stage != SPEC_PROF_LMHEAD && stage != SPEC_PROF_STEP) return SPEC_EINVAL;
+  g_prof[stage][0] = static_cast<cudaEvent_t>(ev_start);
+  g_prof[stage][1] = static_cast<cudaEvent_t>(ev_stop);
+  return SPEC_OK;
+}
+
+const char* spec_status_string(int s) {
+  switch (s) {
+    case SPEC_OK: return "ok";
+    case SPEC_EINVAL: return "invalid argument";
+    case SPEC_EUNSUPPORTED: return "unsupported configuration";
+    case SPEC_ECUDA: return "CUDA error";
+    case SPEC_EDEVICE: return "device reported bad data";
+    case SPEC_ETIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+size_t spec_layer_pool_bytes(const spec_model* m, int layer, int which) {
+  if (!m || !m->layers || layer < 0 || layer >= m->n_layers) return 0;
+  const spec_layer& L = m->layers[layer];
+  const size_t tok_heads = (size_t)m->num_pages * m->n_kv_heads * m->page_size;
+  switch (which) {
+    case 0: return tok_heads * m->head_dim * 2;
+    case 1: return L.kv_equal ? 0 : tok_heads * m->head_dim * 2;
+    case 2: return L.kv_equal ? tok_heads * 2 * n_rot_of(m, L) * 2 : 0;
+  }
+  return 0;
+}
+
+size_t spec_workspace_bytes(const spec_model* m, int max_batch, int max_k, int max_pages) {
+  if (!m || !m->layers || max_batch < 1 || max_k < 0 || max_k > SPEC_MAX_K || max_pages < 1) return 0;
+  StepLayout s = step_layout(m, max_batch, max_k, max_pages);
+  if (s.tickets > kMaxTickets) return 0;
+  return s.total;
+}
+
+size_t spec_lmhead_workspace_bytes(int M, int V) {
+  if (M < 1 || V < 1) return 0;
+  GemmPlan p = plan_gemm(M, V, 64, kGemmArgmax);
+  return kWsHeaderBytes + up(gemm_argmax_entries(p) * 4) * 2;
+}
+
+int spec_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  if (!ws || ws_bytes < kWsHeaderBytes) return SPEC_EINVAL;
+  return cuda_status(cudaMemsetAsync(ws, 0, kWsHeaderBytes, static_cast<cudaStream_t>(stream)));
+}
+
+int spec_read_device_status(void* ws, size_t ws_bytes, void* stream, unsigned* status) {
+  if (!ws || ws_bytes < kWsHeaderBytes || !status) return SPEC_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned v = 0;
+  if (cudaMemcpyAsync(&v, ws, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess) return SPEC_ECUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return SPEC_ECUDA;
+  if (v && cudaMemsetAsync(ws, 0, 4, st) != cudaSuccess) return SPEC_ECUDA;
+  *status = v;
+  if (v & SPEC_DEV_TIMEOUT) return SPEC_ETIMEOUT;
+  return v ? SPEC_EDEVICE : SPEC_OK;
+}
+
+int spec_cache_write(const spec_model* m, int layer, const int32_t* block_table_row, int max_pages,
+                     int pos0, int n_tok, const void* k_raw, const void* v_raw, void* stream) {
+  int rc = check_model(m);
+  if (rc) return rc;
+  if (layer < 0 || layer >= m->n_layers || !block_table_row || max_pages < 1 || pos0 < 0 ||
+      n_tok < 0 || !k_raw)
+    return SPEC_EINVAL;
+  const spec_layer& L = m->layers[layer];
+  if (!L.kv_equal && !v_raw) return SPEC_EINVAL;
+  if ((int64_t)pos0 + n_tok > (int64_t)max_pages * m->page_size) return SPEC_EINVAL;
+  if (n_tok == 0) return SPEC_OK;
+  RopeAppend a{};
+  a.n_q_heads = m->n_q_heads;
+  a.n_kv_heads = m->n_kv_heads;
+  a.head_dim = m->head_dim;
+  a.n_rot = n_rot_of(m, L);
+  a.theta = m->rope_theta;
+  a.page_size = m->page_size;
+  a.num_pages = m->num_pages;
+  a.max_pages = max_pages;
+  a.n_rows = n_tok;
+  a.pos0 = pos0;
+  a.block_table = block_table_row;
+  a.src_k = k_raw;
+  a.k_row_stride = (long)m->n_kv_heads * m->head_dim;
+  a.src_v = L.kv_equal ? nullptr : v_raw;
+  a.v_row_stride = a.k_row_stride;
+  a.k_pool = static_cast<uint16_t*>(L.k_pool);
+  a.v_pool = static_cast<uint16_t*>(L.v_pool);
+  a.ksb_pool = static_cast<uint16_t*>(L.ksb_pool);
+  return cuda_status(launch_rope_append(a, 1, static_cast<cudaStream_t>(stream)));
+}
+
+int spec_verify_attn(const spec_model* m, int layer, const void* q, const void* k_new,
+                     const void* v_new, const int32_t* block_table, int max_pages,
+                     const int32_t* seq_lens, int B, int k, void* out, void* ws, size_t ws_bytes,
+                     void* stream) {
+  int rc = check_model(m);
+  if (rc) return rc;
+  if (layer < 0 || layer >= m->n_layers || !q || !k_new || !block_table || !seq_lens || !out || !ws)
+    return SPEC_EINVAL;
+  if (B < 1 || k < 0 || k > SPEC_MAX_K || max_pages < 1) return SPEC_EINVAL;
+  const spec_layer& L = m->layers[layer];
+  if (!L.kv_equal && !v_new) return SPEC_EINVAL;
+  const int qn = k + 1, D = m->head_dim;
+  StepLayout s = step_layout(m, B, k, max_pages);
+  if (ws_bytes < s.total) return SPEC_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  WsHeader hdr = ws_header(ws);
+
+  RopeAppend a{};
+  a.n_q_heads = m->n_q_heads;
+  a.n_kv_heads = m->n_kv_heads;
+  a.head_dim = D;
+  a.n_rot = n_rot_of(m, L);
+  a.theta = m->rope_theta;
+  a.page_size = m->page_size;
+  a.num_pages = m->num_pages;
+  a.max_pages = max_pages;
+  a.n_rows = qn;
+  a.seq_lens = seq_lens;
+  a.block_table = block_table;
+  a.src_q = q;
+  a.q_row_stride = (long)m->n_q_heads * D;
+  a.q_seq_stride = a.q_row_stride * qn;
+  a.src_k = k_new;
+  a.k_row_stride = (long)m->n_kv_heads * D;
+  a.k_seq_stride = a.k_row_stride * qn;
+  a.src_v = L.kv_equal ? nullptr : v_new;
+  a.v_row_stride = a.k_row_stride;
+  a.v_seq_stride = a.k_seq_stride;
+  a.q_out = at<uint16_t>(ws, s.qrot);
+  a.k_pool = static_cast<uint16_t*>(L.k_pool);
+  a.v_pool = static_cast<uint16_t*>(L.v_pool);
+  a.ksb_pool = static_cast<uint16_t*>(L.ksb_pool);
+  a.status = hdr.status;
+  rc = cuda_status(launch_rope_append(a, B, st));
+  if (rc) return rc;
+  AttnGeom g = plan_attn(B, qn, m->n_q_heads, m->n_kv_heads, D, m->page_size, m->num_pages,
+                         max_pages, L.window, L.kv_equal, 2 * a.n_rot, m->split_tokens);
+  return cuda_status(launch_attention(g, at<uint16_t>(ws, s.qrot), L.k_pool, L.v_pool, L.ksb_pool,
+                                      block_table, seq_lens, at<float>(ws, s.attn_part),
+                                      static_cast<uint16_t*>(out), hdr.status, st));
+}
+
+int spec_lmhead_argmax(const void* h, const void* w, int M, int d, int V, int32_t* ids,
+                       float* maxlogit, void* ws, size_t ws_bytes, void* stream) {
+  if (!h || !w || !ids || !ws || M < 1 || V < 1 || d < 8 || d % 8) return SPEC_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(h) & 15) || (reinterpret_cast<uintptr_t>(w) & 15)) return SPEC_EINVAL;
+  GemmPlan p = plan_gemm(M, V, d, kGemmArgmax);
+  if (p.mblocks > kMaxTickets) return SPEC_EUNSUPPORTED;
+  const size_t need = spec_lmhead_workspace_bytes(M, V);
+  if (ws_bytes < need) return SPEC_EINVAL;
+  WsHeader hdr = ws_header(ws);
+  GemmBuffers b{};
+  b.arg_val = at<float>(ws, kWsHeaderBytes);
+  b.arg_idx = at<int>(ws, kWsHeaderBytes + up(gemm_argmax_entries(p) * 4));
+  b.ids = ids;
+  b.maxv = maxlogit;
+  b.tickets = hdr.tickets;
+  b.status = hdr.status;
+  return cuda_status(launch_gemm(p, kGemmArgmax, h, w, b, static_cast<cudaStream_t>(stream)));
+}
+
+int spec_accept_commit(const int32_t* drafts, const int32_t* target, int B, int k,
+                       int32_t* seq_lens, int32_t* accept_len, int32_t* emitted,
+                       int32_t* last_token, void* stream) {
+  if (!target || !seq_lens || !accept_len || !emitted || !last_token) return SPEC_EINVAL;
+  if (B < 1 || k < 0 || k > SPEC_MAX_K || (k > 0 && !drafts)) return SPEC_EINVAL;
+  return cuda_status(launch_accept(drafts, target, B, k, seq_lens, accept_len, emitted, last_token,
+                                   nullptr, nullptr, nullptr, static_cast<cudaStream_t>(stream)));
+}
+
+int spec_verify_step(const spec_model* m, const int32_t* block_table, int max_pages,
+                     const int32_t* last_token, const int32_t* drafts, int B, int k,
+                     int32_t* seq_lens, int32_t* accept_len, int32_t* emitted,
+                     int32_t* new_last_token, int32_t* target_ids, float* target_maxlogit,
+                     void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_model(m);
+  if (rc) return rc;
+  if (!block_table || !last_token || !seq_lens || !accept_len || !emitted || !new_last_token || !ws)
+    return SPEC_EINVAL;
+  if (B < 1 || k < 0 || k > SPEC_MAX_K || max_pages < 1 || (k > 0 && !drafts)) return SPEC_EINVAL;
+  StepLayout s = step_layout(m, B, k, max_pages);
+  if (s.tickets > kMaxTickets) return SPEC_EUNSUPPORTED;
+  if (ws_bytes < s.total) return SPEC_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  WsHeader hdr = ws_header(ws);
+  const int q = k + 1, M = B * q, d = m->d_model, D = m->head_dim;
+  float* x = at<float>(ws, s.x);
+  uint16_t* hn = at<uint16_t>(ws, s.hn);
+  float* qkv = at<float>(ws, s.qkv);
+  uint16_t* qrot = at<uint16_t>(ws, s.qrot);
+  uint16_t* attn_out = at<uint16_t>(ws, s.attn_out);
+
+  prof_mark(SPEC_PROF_STEP, 0, st);
+  rc = cuda_status(launch_embed(m->w_lm, m->vocab, d, last_token, drafts, B, q, x, hdr.status, st));
+  if (rc) return rc;
+  for (int l = 0; l < m->n_layers; ++l) {
+    const spec_layer& L = m->layers[l];
+    const int nqkv = qkv_out(m, L);
+    rc = cuda_status(launch_rmsnorm(x, M, d, m->rms_eps, hn, st));
+    if (rc) return rc;
+    GemmPlan pq = plan_gemm(M, nqkv, d, kGemmStore);
+    GemmBuffers bq{};
+    bq.out = qkv;
+    bq.partial = at<float>(ws, s.gemm_part);
+    bq.tickets = hdr.tickets;
+    bq.status = hdr.status;
+    rc = cuda_status(launch_gemm(pq, kGemmStore, hn, L.w_qkv, bq, st));
+    if (rc) return rc;
+
+    RopeAppend a{};
+    a.n_q_heads = m->n_q_heads;
+    a.n_kv_heads = m->n_kv_heads;
+    a.head_dim = D;
+    a.n_rot = n_rot_of(m, L);
+    a.theta = m->rope_theta;
+    a.page_size = m->page_size;
+    a.num_pages = m->num_pages;
+    a.max_pages = max_pages;
+    a.n_rows = q;
+    a.seq_lens = seq_lens;
+    a.block_table = block_table;
+    a.src_is_f32 = 1;
+    a.src_q = qkv;
+    a.q_row_stride = nqkv;
+    a.q_seq_stride = (long)nqkv * q;
+    a.src_k = qkv + (size_t)m->n_q_heads * D;
+    a.k_row_stride = nqkv;
+    a.k_seq_stride = (long)nqkv * q;
+    a.src_v = L.kv_equal ? nullptr : qkv + (size_t)(m->n_q_heads + m->n_kv_heads) * D;
+    a.v_row_stride = nqkv;
+    a.v_seq_stride = (long)nqkv * q;
+    a.q_out = qrot;
+    a.k_pool = static_cast<uint16_t*>(L.k_pool);
+    a.v_pool = static_cast<uint16_t*>(L.v_pool);
+    a.ksb_pool = static_cast<uint16_t*>(L.ksb_pool);
+    a.status = hdr.status;
+    rc = cuda_status(launch_rope_append(a, B, st));
+    if (rc) return rc;
+
+    AttnGeom g = plan_attn(B, q, m->n_q_heads, m->n_kv_heads, D, m->page_size, m->num_pages,
+                           max_pages, L.window, L.kv_equal, 2 * a.n_rot, m->split_tokens);
+    rc = cuda_status(launch_attention(g, qrot, L.k_pool, L.v_pool, L.ksb_pool, block_table, seq_lens,
+                                      at<float>(ws, s.attn_part), attn_out, hdr.status, st));
+    if (rc) return rc;
+
+    GemmPlan po = plan_gemm(M, d, m->n_q_heads * D, kGemmResidual);
+    GemmBuffers bo{};
+    bo.out = x;
+    bo.partial = at<float>(ws, s.gemm_part);
+    bo.tickets = hdr.tickets;
+    bo.status = hdr.status;
+    rc = cuda_status(launch_gemm(po, kGemmResidual, attn_out, L.w_o, bo, st));
+    if (rc) return rc;
+  }
+  rc = cuda_status(launch_rmsnorm(x, M, d, m->rms_eps, hn, st));
+  if (rc) return rc;
+  GemmPlan pl = plan_gemm(M, m->vocab, d, kGemmArgmax);
+  GemmBuffers bl{};
+  bl.arg_val = at<float>(ws, s.arg_val);
+  bl.arg_idx = at<int>(ws, s.arg_idx);
+  bl.ids = at<int32_t>(ws, s.ids);
+  bl.maxv = at<float>(ws, s.maxv);
+  bl.tickets = hdr.tickets;
+  bl.status = hdr.status;
+  prof_mark(SPEC_PROF_LMHEAD, 0, st);
+  rc = cuda_status(launch_gemm(pl, kGemmArgmax, hn, m->w_lm, bl, st));
+  prof_mark(SPEC_PROF_LMHEAD, 1, st);
+  if (rc) return rc;
+  rc = cuda_status(launch_accept(drafts, at<int32_t>(ws, s.ids), B, k, seq_lens, accept_len,
+                                 emitted, new_last_token, target_ids, target_maxlogit,
+                                 at<float>(ws, s.maxv), st));
+  prof_mark(SPEC_PROF_STEP, 1, st);
+  return rc;
+}
+
+}  // extern "C"

@@ -1,0 +1,415 @@
+// Streaming skinny GEMM for the verify step: Y = X . W^T where X holds the
+// few verify rows (M = B*(k+1), tens of rows) and W is a large bf16 weight
+// matrix read once from HBM.  Used for the QKV projection, the output
+// projection (+ residual) and the tied LM head with a fused argmax.
+//
+// Design (sm_100a):
+//   * one producer warp issues TMA tile loads (W box 128 rows x 64 k, X box
+//     (8*NT) rows x 64 k, both 128-byte swizzled) into a ring of stages
+//     guarded by mbarriers; W uses an evict-first L2 policy (read once), X
+//     evict-last (re-read by every CTA);
+//   * four consumer warps each own 32 W rows of the 128-row tile and all
+//     M-block rows: swap-AB mma.sync m16n8k16 (W rows are the MMA's M side,
+//     the verify rows its N side), fp32 accumulators in registers;
+//   * split-K over a fixed number of K chunks per CTA (a function of N and K
+//     only, never of M, so a row's sum order does not depend on the batch);
+//     partial sums are added in split order by the last CTA to finish a tile
+//     (atomic ticket, no spin waits);
+//   * argmax epilogue: per-tile (max, index) per row, ties to the lowest
+//     index, reduced across tiles by the last CTA; logits never reach HBM.
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace sv {
+
+namespace {
+
+constexpr int kTileN = 128;
+constexpr int kTileK = 64;
+constexpr int kConsumerWarps = 4;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kMBlock = 64;
+
+template <int NT>
+struct Cfg {
+  static constexpr int kStages = NT <= 2 ? 6 : 5;
+  static constexpr int kWBytes = kTileN * 128;
+  static constexpr int kXBytes = NT * 8 * 128;
+  static constexpr int kStageBytes = kWBytes + kXBytes;
+  static constexpr int kRedBytes = 2 * kConsumerWarps * NT * 8 * 4;
+  static constexpr int kSmem = 1024 + kStages * kStageBytes + 2 * kStages * 8 + kRedBytes + 64;
+};
+
+struct Args {
+  int M, N, K, kchunks, splits, n_tiles;
+  float* out;
+  float* partial;
+  float* arg_val;
+  int* arg_idx;
+  int32_t* ids;
+  float* maxv;
+  unsigned* tickets;
+  unsigned* status;
+};
+
+template <int NT, int MODE>
+__global__ void __launch_bounds__(kThreads) stream_gemm_kernel(
+    const __grid_constant__ CUtensorMap tw, const __grid_constant__ CUtensorMap tx, Args a) {
+  using C = Cfg<NT>;
+  constexpr int MP = NT * 8;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
+  uint64_t* empty = full + C::kStages;
+  float* red_v = reinterpret_cast<float*>(empty + C::kStages);
+  int* red_i = reinterpret_cast<int*>(red_v + kConsumerWarps * MP);
+  int* flag = red_i + kConsumerWarps * MP;
+  volatile int* fail = flag + 1;  // set by any consumer warp whose wait ran out
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_tile = blockIdx.x, split = blockIdx.y, mblk = blockIdx.z;
+  const int m0 = mblk * kMBlock;
+  const int kc0 = (int)((long)split * a.kchunks / a.splits);
+  const int kc1 = (int)((long)(split + 1) * a.kchunks / a.splits);
+  const int nk = kc1 - kc0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumerWarps);
+    }
+    *fail = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  if (warp == kConsumerWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tw);
+      prefetch_tmap(&tx);
+      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_x = policy_evict_last();
+      int issued = 0;
+      for (int it = 0; it < nk; ++it) {
+        const int s = it % C::kStages;
+        if (it >= C::kStages && !mbar_wait(&empty[s], ((it / C::kStages) - 1) & 1, a.status)) break;
+        uint8_t* st = smem + s * C::kStageBytes;
+        mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+        const int kx = (kc0 + it) * kTileK;
+        tma_load_2d(st, &tw, &full[s], kx, n_tile * kTileN, pol_w);
+        tma_load_2d(st + C::kWBytes, &tx, &full[s], kx, m0, pol_x);
+        issued = it + 1;
+      }
+      // Drain: every issued stage must have landed before the CTA may exit.
+      for (int it = (issued > C::kStages ? issued - C::kStages : 0); it < issued; ++it)
+        mbar_wait(&full[it % C::kStages], (it / C::kStages) & 1, a.status);
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  float acc[2][NT][4];
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
+
+  // On a timed-out wait a warp stops consuming but still reaches every named
+  // barrier below, so the other warps never block on it; the CTA then skips
+  // its outputs as a whole.
+  for (int it = 0; it < nk; ++it) {
+    const int s = it % C::kStages;
+    if (*fail) break;
+    if (!mbar_wait(&full[s], (it / C::kStages) & 1, a.status)) {
+      *fail = 1;
+      break;
+    }
+    const uint32_t wb = smem_u32(smem + s * C::kStageBytes);
+    const uint32_t xb = wb + C::kWBytes;
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+      uint32_t af[2][4];
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+        const uint32_t row = warp * 32 + mt * 16 + (lane & 15);
+        ldsm_x4(wb + swz128(row, ks * 2 + (lane >> 4)), af[mt][0], af[mt][1], af[mt][2], af[mt][3]);
+      }
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        uint32_t b0, b1;
+        const uint32_t row = nt * 8 + (lane & 7);
+        ldsm_x2(xb + swz128(row, ks * 2 + ((lane >> 3) & 1)), b0, b1);
+        mma_bf16(acc[0][nt], af[0], b0, b1);
+        mma_bf16(acc[1][nt], af[1], b0, b1);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+  }
+  named_bar(1, kConsumerWarps * 32);
+  if (*fail) return;
+
+  const int g = lane >> 2, t = lane & 3;
+  const int ctid = threadIdx.x;  // 0..127 among consumers
+
+  if (MODE == kGemmArgmax) {
+    // ---- per-tile argmax of every verify row (column of the MMA tile)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        float bv = -INFINITY;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int n = n_tile * kTileN + warp * 32 + mt * 16 + g + h * 8;
+            const float v = acc[mt][nt][h * 2 + j];
+            if (n < a.N && better(v, n, bv, bi)) {
+              bv = v;
+              bi = n;
+            }
+          }
+        }
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+          const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+          const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+          if (better(ov, oi, bv, bi)) {
+            bv = ov;
+            bi = oi;
+          }
+        }
+        if (g == 0) {
+          const int col = nt * 8 + 2 * t + j;
+          red_v[warp * MP + col] = bv;
+          red_i[warp * MP + col] = bi;
+        }
+      }
+    }
+    named_bar(1, kConsumerWarps * 32);
+    if (ctid < MP && m0 + ctid < a.M) {
+      float bv = red_v[ctid];
+      int bi = red_i[ctid];
+      for (int w = 1; w < kConsumerWarps; ++w) {
+        const float v = red_v[w * MP + ctid];
+        const int i = red_i[w * MP + ctid];
+        if (better(v, i, bv, bi)) {
+          bv = v;
+          bi = i;
+        }
+      }
+      const size_t o = (size_t)n_tile * a.M + m0 + ctid;
+      a.arg_val[o] = bv;
+      a.arg_idx[o] = bi;
+    }
+    __threadfence();
+    named_bar(1, kConsumerWarps * 32);
+    if (ctid == 0) {
+      const unsigned prev = atomicAdd(&a.tickets[mblk], 1u);
+      *flag = (prev == (unsigned)(a.n_tiles - 1));
+    }
+    named_bar(1, kConsumerWarps * 32);
+    if (!*flag) return;
+    __threadfence();
+    // ---- last CTA of this M-block: reduce over all tiles, lowest index wins ties
+    const int mcount = min(kMBlock, a.M - m0);
+    for (int mm = 0; mm < mcount; ++mm) {
+      const int m = m0 + mm;
+      float bv = -INFINITY;
+      int bi = 0x7fffffff;
+      for (int tile = ctid; tile < a.n_tiles; tile += kConsumerWarps * 32) {
+        const float v = __ldcg(&a.arg_val[(size_t)tile * a.M + m]);
+        const int i = __ldcg(&a.arg_idx[(size_t)tile * a.M + m]);
+        if (better(v, i, bv, bi)) {
+          bv = v;
+          bi = i;
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+        if (better(ov, oi, bv, bi)) {
+          bv = ov;
+          bi = oi;
+        }
+      }
+      if (lane == 0) {
+        red_v[warp] = bv;
+        red_i[warp] = bi;
+      }
+      named_bar(1, kConsumerWarps * 32);
+      if (ctid == 0) {
+        for (int w = 1; w < kConsumerWarps; ++w)
+          if (better(red_v[w], red_i[w], bv, bi)) {
+            bv = red_v[w];
+            bi = red_i[w];
+          }
+        a.ids[m] = bi;
+        if (a.maxv) a.maxv[m] = bv;
+      }
+      named_bar(1, kConsumerWarps * 32);
+    }
+    if (ctid == 0) a.tickets[mblk] = 0u;
+    return;
+  }
+
+  // ---- store / residual epilogues
+  if (a.splits == 1) {
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int n = n_tile * kTileN + warp * 32 + mt * 16 + g + (e >> 1) * 8;
+          const int m = m0 + nt * 8 + 2 * t + (e & 1);
+          if (n < a.N && m < a.M) {
+            float* dst = a.out + (size_t)m * a.N + n;
+            if (MODE == kGemmResidual)
+              *dst = __fadd_rn(*dst, acc[mt][nt][e]);
+            else
+              *dst = acc[mt][nt][e];
+          }
+        }
+    return;
+  }
+  // split-K: publish this split's partial tile [128][MP]
+  float* mine = a.partial + (((size_t)mblk * a.splits + split) * a.n_tiles + n_tile) * kTileN * MP;
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int r = warp * 32 + mt * 16 + g + h * 8;
+        const int c = nt * 8 + 2 * t;
+        __stcg(reinterpret_cast<float2*>(mine + (size_t)r * MP + c),
+               make_float2(acc[mt][nt][h * 2], acc[mt][nt][h * 2 + 1]));
+      }
+  __threadfence();
+  named_bar(1, kConsumerWarps * 32);
+  if (ctid == 0) {
+    unsigned* tk = &a.tickets[mblk * a.n_tiles + n_tile];
+    const unsigned prev = atomicAdd(tk, 1u);
+    *flag = (prev == (unsigned)(a.splits - 1));
+  }
+  named_bar(1, kConsumerWarps * 32);
+  if (!*flag) return;
+  __threadfence();
+  // last split of this tile: sum partials in split order, then the epilogue
+  const int r = ctid;  // one W row (output feature) per consumer thread
+  const int n = n_tile * kTileN + r;
+  if (n < a.N) {
+    const int mcount = min(MP, a.M - m0);
+    for (int mm = 0; mm < mcount; ++mm) {
+      float s = 0.f;
+      for (int sp = 0; sp < a.splits; ++sp) {
+        const float* p =
+            a.partial + (((size_t)mblk * a.splits + sp) * a.n_tiles + n_tile) * kTileN * MP;
+        s = __fadd_rn(s, __ldcg(p + (size_t)r * MP + mm));
+      }
+      float* dst = a.out + (size_t)(m0 + mm) * a.N + n;
+      if (MODE == kGemmResidual)
+        *dst = __fadd_rn(*dst, s);
+      else
+        *dst = s;
+    }
+  }
+  if (ctid == 0) a.tickets[mblk * a.n_tiles + n_tile] = 0u;
+}
+
+template <int NT, int MODE>
+cudaError_t launch_nt(const GemmPlan& p, const CUtensorMap& tw, const CUtensorMap& tx,
+                      const Args& a, cudaStream_t st) {
+  auto kern = stream_gemm_kernel<NT, MODE>;
+  const int smem = Cfg<NT>::kSmem;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(p.n_tiles, p.splits, p.mblocks);
+  kern<<<grid, kThreads, smem, st>>>(tw, tx, a);
+  return cudaGetLastError();
+}
+
+template <int MODE>
+cudaError_t launch_mode(const GemmPlan& p, const CUtensorMap& tw, const CUtensorMap& tx,
+                        const Args& a, cudaStream_t st) {
+  switch (p.nt) {
+    case 1: return launch_nt<1, MODE>(p, tw, tx, a, st);
+    case 2: return launch_nt<2, MODE>(p, tw, tx, a, st);
+    case 3: return launch_nt<3, MODE>(p, tw, tx, a, st);
+    case 4: return launch_nt<4, MODE>(p, tw, tx, a, st);
+    case 5: return launch_nt<5, MODE>(p, tw, tx, a, st);
+    case 6: return launch_nt<6, MODE>(p, tw, tx, a, st);
+    case 7: return launch_nt<7, MODE>(p, tw, tx, a, st);
+    case 8: return launch_nt<8, MODE>(p, tw, tx, a, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+GemmPlan plan_gemm(int M, int N, int K, int mode) {
+  GemmPlan p{};
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.n_tiles = (N + kTileN - 1) / kTileN;
+  p.kchunks = (K + kTileK - 1) / kTileK;
+  p.mblocks = (M + kMBlock - 1) / kMBlock;
+  p.nt = (std::min(M, kMBlock) + 7) / 8;
+  if (mode == kGemmArgmax) {
+    p.splits = 1;
+  } else {
+    // about 256 CTAs per M-block, at least 4 K chunks each; depends on N, K only
+    int s = (256 + p.n_tiles - 1) / p.n_tiles;
+    s = std::min(s, std::max(1, p.kchunks / 4));
+    p.splits = std::max(1, s);
+  }
+  return p;
+}
+
+size_t gemm_partial_floats(const GemmPlan& p) {
+  if (p.splits <= 1) return 0;
+  return (size_t)p.mblocks * p.splits * p.n_tiles * kTileN * (p.nt * 8);
+}
+size_t gemm_argmax_entries(const GemmPlan& p) { return (size_t)p.n_tiles * p.M; }
+int gemm_tickets(const GemmPlan& p) { return p.mblocks * p.n_tiles; }
+
+cudaError_t launch_gemm(const GemmPlan& p, int mode, const void* x, const void* w,
+                        const GemmBuffers& b, cudaStream_t st) {
+  CUtensorMap tw, tx;
+  if (!make_tmap_bf16_2d(&tw, w, p.N, p.K, kTileN, kTileK)) return cudaErrorInvalidValue;
+  if (!make_tmap_bf16_2d(&tx, x, p.M, p.K, p.nt * 8, kTileK)) return cudaErrorInvalidValue;
+  Args a{};
+  a.M = p.M;
+  a.N = p.N;
+  a.K = p.K;
+  a.kchunks = p.kchunks;
+  a.splits = p.splits;
+  a.n_tiles = p.n_tiles;
+  a.out = b.out;
+  a.partial = b.partial;
+  a.arg_val = b.arg_val;
+  a.arg_idx = b.arg_idx;
+  a.ids = b.ids;
+  a.maxv = b.maxv;
+  a.tickets = b.tickets;
+  a.status = b.status;
+  switch (mode) {
+    case kGemmStore: return launch_mode<kGemmStore>(p, tw, tx, a, st);
+    case kGemmResidual: return launch_mode<kGemmResidual>(p, tw, tx, a, st);
+    case kGemmArgmax: return launch_mode<kGemmArgmax>(p, tw, tx, a, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace sv

@@ -1,0 +1,101 @@
+// Host-side launchers shared by the C-ABI layer (api.cu) and the kernel files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace sv {
+
+// ----------------------------------------------------------------- TMA maps
+// 2D row-major bf16 tensor [rows][cols], box {box_cols, box_rows}, 128-byte
+// swizzle, zero fill outside the tensor.  Returns false if the driver call
+// fails (the caller reports SPEC_ECUDA) or the layout is not encodable.
+bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                       uint32_t box_rows, uint32_t box_cols);
+
+// --------------------------------------------------------- streaming GEMM
+// Y = X . W^T with X [M][K] bf16 (row-major), W [N][K] bf16 (row-major),
+// fp32 accumulation, W streamed once per M-block by TMA.
+enum GemmMode { kGemmStore = 0, kGemmResidual = 1, kGemmArgmax = 2 };
+
+struct GemmPlan {
+  int M, N, K;
+  int n_tiles;   // ceil(N / 128)
+  int kchunks;   // ceil(K / 64)
+  int splits;    // split-K factor (1 for argmax)
+  int mblocks;   // ceil(M / 64)
+  int nt;        // n8 tiles per M-block: ceil(min(M, 64) / 8)
+};
+GemmPlan plan_gemm(int M, int N, int K, int mode);
+size_t gemm_partial_floats(const GemmPlan& p);   // split-K partial sums
+size_t gemm_argmax_entries(const GemmPlan& p);   // per-tile argmax partials
+int gemm_tickets(const GemmPlan& p);
+
+struct GemmBuffers {
+  float* out;          // kGemmStore: [M][N]; kGemmResidual: [M][N] updated in place
+  float* partial;      // gemm_partial_floats()
+  float* arg_val;      // gemm_argmax_entries()
+  int* arg_idx;
+  int32_t* ids;        // kGemmArgmax: [M]
+  float* maxv;         // kGemmArgmax: [M] or null
+  unsigned* tickets;   // gemm_tickets() counters, zero on entry, zero on exit
+  unsigned* status;
+};
+cudaError_t launch_gemm(const GemmPlan& p, int mode, const void* x, const void* w,
+                        const GemmBuffers& buf, cudaStream_t st);
+
+// ------------------------------------------------------------- small kernels
+cudaError_t launch_embed(const void* w_lm, int vocab, int d, const int32_t* last_token,
+                         const int32_t* drafts, int B, int q, float* x, unsigned* status,
+                         cudaStream_t st);
+cudaError_t launch_rmsnorm(const float* x, int M, int d, float eps, uint16_t* out,
+                           cudaStream_t st);
+cudaError_t launch_accept(const int32_t* drafts, const int32_t* target, int B, int k,
+                          int32_t* seq_lens, int32_t* accept_len, int32_t* emitted,
+                          int32_t* last_token, int32_t* copy_ids, float* copy_max,
+                          const float* maxv, cudaStream_t st);
+
+// ------------------------------------------------------- RoPE + cache append
+struct RopeAppend {
+  // geometry
+  int n_q_heads, n_kv_heads, head_dim, n_rot;   // n_rot rotated pairs
+  float theta;
+  int page_size, num_pages, max_pages;
+  // rows: blockIdx.x = i in [0, n_rows), blockIdx.y = sequence b
+  int n_rows;
+  const int32_t* seq_lens;   // position of row i = seq_lens[b] + i   (if non-null)
+  int pos0;                  // ... else pos0 + i
+  const int32_t* block_table;
+  // sources (pre-RoPE), element strides in elements
+  const void* src_q; long q_row_stride, q_seq_stride;   // null: no queries
+  const void* src_k; long k_row_stride, k_seq_stride;
+  const void* src_v; long v_row_stride, v_seq_stride;   // null on key-equals-value layers
+  int src_is_f32;
+  // destinations
+  uint16_t* q_out;           // [B][n_rows][Hq][D] bf16 rotated queries
+  uint16_t* k_pool;
+  uint16_t* v_pool;
+  uint16_t* ksb_pool;        // key-equals-value side-band
+  unsigned* status;
+};
+cudaError_t launch_rope_append(const RopeAppend& a, int B, cudaStream_t st);
+
+// ---------------------------------------------------------- split-KV attention
+struct AttnGeom {
+  int B, q, n_q_heads, n_kv_heads, head_dim, page_size, num_pages, max_pages;
+  int window, kv_equal, sb_width, split_tokens;
+  int n_splits_grid;   // CTAs per (sequence, kv head, row block)
+  int rows;            // G * q
+  int row_blocks;      // ceil(rows / 64)
+};
+AttnGeom plan_attn(int B, int q, int Hq, int Hkv, int D, int page, int num_pages, int max_pages,
+                   int window, int kv_equal, int sb_width, int split_tokens);
+size_t attn_partial_floats(const AttnGeom& g);
+cudaError_t launch_attention(const AttnGeom& g, const uint16_t* qrot, const void* k_pool,
+                             const void* v_pool, const void* ksb_pool, const int32_t* block_table,
+                             const int32_t* seq_lens, float* part, uint16_t* out, unsigned* status,
+                             cudaStream_t st);
+
+}  // namespace sv

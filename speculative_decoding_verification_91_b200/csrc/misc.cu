@@ -1,0 +1,108 @@
+// Small verify-step kernels: token embedding gather, RMSNorm, and the
+// acceptance / bonus-token / commit kernel.
+#include "common.cuh"
+#include "internal.h"
+
+namespace sv {
+
+namespace {
+
+// Row m = b*q + i holds token last_token[b] (i = 0) or drafts[b][i-1]; its
+// residual stream starts as the tied embedding row, widened to fp32.
+__global__ void embed_kernel(const uint16_t* __restrict__ w_lm, int vocab, int d,
+                             const int32_t* __restrict__ last_token,
+                             const int32_t* __restrict__ drafts, int q, float* __restrict__ x,
+                             unsigned* status) {
+  const int m = blockIdx.x;
+  const int b = m / q, i = m % q;
+  int tok = (i == 0) ? last_token[b] : drafts[b * (q - 1) + (i - 1)];
+  float* row = x + (size_t)m * d;
+  if (tok < 0 || tok >= vocab) {
+    if (threadIdx.x == 0) flag_status(status, SPEC_DEV_BAD_TOKEN);
+    for (int e = threadIdx.x; e < d; e += blockDim.x) row[e] = 0.f;
+    return;
+  }
+  const uint16_t* src = w_lm + (size_t)tok * d;
+  for (int e = threadIdx.x; e < d; e += blockDim.x) row[e] = bf16_to_f32(src[e]);
+}
+
+// out[m] = bf16(x[m] / sqrt(mean(x[m]^2) + eps)); fixed reduction order.
+constexpr int kNormThreads = 256;
+__global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(const float* __restrict__ x, int d,
+                                                               float eps,
+                                                               uint16_t* __restrict__ out) {
+  __shared__ float red[kNormThreads / 32];
+  const int m = blockIdx.x;
+  const float* row = x + (size_t)m * d;
+  float ss = 0.f;
+  for (int e = threadIdx.x; e < d; e += kNormThreads) ss = __fmaf_rn(row[e], row[e], ss);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  float tot = 0.f;
+#pragma unroll
+  for (int w = 0; w < kNormThreads / 32; ++w) tot += red[w];
+  const float inv = 1.0f / sqrtf(tot / (float)d + eps);
+  uint16_t* o = out + (size_t)m * d;
+  for (int e = threadIdx.x; e < d; e += kNormThreads) o[e] = f32_to_bf16(__fmul_rn(row[e], inv));
+}
+
+// One warp per sequence: a = number of leading drafts equal to the target's
+// argmax (ballot of matches, first zero bit), emit them and target[a], commit
+// a+1 positions.
+__global__ void accept_kernel(const int32_t* __restrict__ drafts, const int32_t* __restrict__ target,
+                              int B, int k, int32_t* seq_lens, int32_t* accept_len,
+                              int32_t* emitted, int32_t* last_token, int32_t* copy_ids,
+                              float* copy_max, const float* maxv) {
+  const int b = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (b >= B) return;
+  const int q = k + 1;
+  const int32_t* tg = target + (size_t)b * q;
+  const bool match = lane < k && drafts[(size_t)b * k + lane] == tg[lane];
+  const unsigned mism = ~__ballot_sync(0xffffffffu, match);   // bit i set: draft i not accepted
+  const int a = min(__ffs(mism) - 1, k);
+  if (lane < q) {
+    int v = -1;
+    if (lane < a) v = drafts[(size_t)b * k + lane];
+    else if (lane == a) v = tg[a];
+    emitted[(size_t)b * q + lane] = v;
+    if (copy_ids) copy_ids[(size_t)b * q + lane] = tg[lane];
+    if (copy_max) copy_max[(size_t)b * q + lane] = maxv[(size_t)b * q + lane];
+  }
+  __syncwarp();
+  if (lane == 0) {
+    accept_len[b] = a;
+    last_token[b] = tg[a];
+    seq_lens[b] += a + 1;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_embed(const void* w_lm, int vocab, int d, const int32_t* last_token,
+                         const int32_t* drafts, int B, int q, float* x, unsigned* status,
+                         cudaStream_t st) {
+  embed_kernel<<<B * q, 256, 0, st>>>(static_cast<const uint16_t*>(w_lm), vocab, d, last_token,
+                                      drafts, q, x, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rmsnorm(const float* x, int M, int d, float eps, uint16_t* out,
+                           cudaStream_t st) {
+  rmsnorm_kernel<<<M, kNormThreads, 0, st>>>(x, d, eps, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_accept(const int32_t* drafts, const int32_t* target, int B, int k,
+                          int32_t* seq_lens, int32_t* accept_len, int32_t* emitted,
+                          int32_t* last_token, int32_t* copy_ids, float* copy_max,
+                          const float* maxv, cudaStream_t st) {
+  const int warps = 4;
+  accept_kernel<<<(B + warps - 1) / warps, warps * 32, 0, st>>>(
+      drafts, target, B, k, seq_lens, accept_len, emitted, last_token, copy_ids, copy_max, maxv);
+  return cudaGetLastError();
+}
+
+}  // namespace sv

@@ -1,0 +1,100 @@
+"""Device-side state for the verify step: weights, paged cache pools,
+workspace and the spec_model descriptor handed to the C ABI.
+
+PyTorch provides device memory and streams here; all arithmetic of the
+verify step runs in libspecverify.so.
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+from . import binding as B
+
+BF16_NAN = 0x7FC0
+
+
+def to_device_bf16(bits: np.ndarray, device) -> torch.Tensor:
+    """Upload bf16 bit patterns (numpy uint16) as a bfloat16 tensor."""
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16))
+    return t.to(device=device, non_blocking=False).view(torch.bfloat16)
+
+
+@dataclass
+class LayerConfig:
+    window: int
+    kv_equal: bool
+    rope_fraction: float
+
+
+class DeviceModel:
+    """Weights and cache pools of one synthetic target on one GPU.
+
+    Pools are allocated for num_pages pages and filled with bf16 NaN when
+    `poison` is set, so that any read of a slot that was never written shows
+    up in the results."""
+
+    def __init__(self, *, d_model, n_q_heads, n_kv_heads, head_dim, vocab, layers, w_lm_bits,
+                 layer_weights, num_pages, split_tokens, rope_theta=10000.0, rms_eps=1e-6,
+                 device="cuda", poison=True):
+        self.device = torch.device(device)
+        self.d_model, self.n_q_heads, self.n_kv_heads = d_model, n_q_heads, n_kv_heads
+        self.head_dim, self.vocab, self.num_pages = head_dim, vocab, num_pages
+        self.layers = list(layers)
+        self.w_lm = to_device_bf16(w_lm_bits, self.device)
+        self.w_qkv, self.w_o, self.k_pool, self.v_pool, self.ksb_pool = [], [], [], [], []
+        P, H, D = num_pages, n_kv_heads, head_dim
+        for (wqkv, wo), spec in zip(layer_weights, self.layers):
+            self.w_qkv.append(to_device_bf16(wqkv, self.device))
+            self.w_o.append(to_device_bf16(wo, self.device))
+            n_rot = int(round(spec.rope_fraction * D / 2))
+            self.k_pool.append(self._pool((P, H, B.SPEC_PAGE_SIZE, D), poison))
+            if spec.kv_equal:
+                self.v_pool.append(None)
+                self.ksb_pool.append(self._pool((P, H, B.SPEC_PAGE_SIZE, 2 * n_rot), poison))
+            else:
+                self.v_pool.append(self._pool((P, H, B.SPEC_PAGE_SIZE, D), poison))
+                self.ksb_pool.append(None)
+        self._layers_c = (B.SpecLayer * len(self.layers))()
+        for l, spec in enumerate(self.layers):
+            self._layers_c[l] = B.SpecLayer(
+                self.w_qkv[l].data_ptr(), self.w_o[l].data_ptr(), self.k_pool[l].data_ptr(),
+                self.v_pool[l].data_ptr() if self.v_pool[l] is not None else None,
+                self.ksb_pool[l].data_ptr() if self.ksb_pool[l] is not None else None,
+                int(spec.window), int(spec.kv_equal), float(spec.rope_fraction))
+        self.desc = B.SpecModel(len(self.layers), d_model, n_q_heads, n_kv_heads, head_dim, vocab,
+                                B.SPEC_PAGE_SIZE, num_pages, split_tokens, float(rope_theta),
+                                float(rms_eps), self.w_lm.data_ptr(),
+                                ctypes.cast(self._layers_c, ctypes.POINTER(B.SpecLayer)))
+
+    def _pool(self, shape, poison):
+        if poison:
+            return torch.full(shape, BF16_NAN, dtype=torch.int16, device=self.device).view(torch.bfloat16)
+        return torch.empty(shape, dtype=torch.bfloat16, device=self.device)
+
+    def pool_bytes(self) -> int:
+        n = 0
+        for l in range(len(self.layers)):
+            for which in range(3):
+                n += B.spec_layer_pool_bytes(self.desc, l, which)
+        return n
+
+
+class Workspace:
+    """Caller-owned scratch for the kernels, cleared once at creation."""
+
+    def __init__(self, nbytes: int, device="cuda", stream=None):
+        if nbytes <= 0:
+            raise ValueError("workspace size must be positive (check the model / batch limits)")
+        self.nbytes = int(nbytes)
+        self.buf = torch.empty(self.nbytes, dtype=torch.uint8, device=device)
+        B.spec_workspace_init(self.buf, self.nbytes, stream)
+
+    def ptr(self) -> int:
+        return self.buf.data_ptr()
+
+    def device_status(self, stream=None) -> int:
+        return B.spec_read_device_status(self.buf, self.nbytes, stream)

@@ -1,0 +1,111 @@
+"""The C-ABI library builds, loads and exports what include/specverify.h
+declares; host-side validation and layout queries work without a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from speculative_decoding_verification_91_b200 import binding as B
+from speculative_decoding_verification_91_b200 import build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "specverify.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return B.lib()
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_ \*]*?\b(spec_[a-z_]+)\s*\(",
+                                 text, flags=re.M)))
+
+
+def test_every_declared_function_is_exported(lib):
+    names = _declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(names) == sorted(B.EXPORTED)
+
+
+def test_status_strings(lib):
+    assert B.status_string(0) == "ok"
+    assert "invalid" in B.status_string(-1)
+    assert B.status_string(12345) == "unknown status"
+
+
+FAKE = 0x10000  # 16-byte aligned dummy address; never dereferenced on the host paths tested
+
+
+def _model(kv_equal=True, D=256, frac=0.25, num_pages=100, n_layers=1):
+    layers = (B.SpecLayer * n_layers)()
+    for l in range(n_layers):
+        layers[l] = B.SpecLayer(FAKE, FAKE, FAKE, None if kv_equal else FAKE, FAKE if kv_equal else None,
+                                0, int(kv_equal), frac)
+    m = B.SpecModel(n_layers, 2560, 16, 8, D, 262144, 64, num_pages, 256, 10000.0, 1e-6, FAKE,
+                    ctypes.cast(layers, ctypes.POINTER(B.SpecLayer)))
+    m._keep = layers
+    return m
+
+
+def test_key_equals_value_pool_is_37_5_percent_smaller(lib):
+    kv = _model(True)
+    sep = _model(False, frac=1.0)
+    kv_bytes = sum(B.spec_layer_pool_bytes(kv, 0, w) for w in range(3))
+    sep_bytes = sum(B.spec_layer_pool_bytes(sep, 0, w) for w in range(3))
+    assert kv_bytes == 100 * 8 * 64 * (256 + 64) * 2
+    assert 1 - kv_bytes / sep_bytes == 0.375
+    assert B.spec_layer_pool_bytes(kv, 0, 1) == 0 and B.spec_layer_pool_bytes(sep, 0, 2) == 0
+
+
+def test_workspace_sizes(lib):
+    m = _model()
+    ws = B.spec_workspace_bytes(m, 8, 4, 520)
+    assert ws > 4096
+    assert B.spec_workspace_bytes(m, 8, 17, 520) == 0      # k above the limit
+    assert B.spec_workspace_bytes(m, 0, 4, 520) == 0
+    assert B.spec_workspace_bytes(m, 16, 4, 520) > ws
+    assert B.spec_lmhead_workspace_bytes(5, 262144) > 4096
+
+
+def test_invalid_arguments_are_rejected_before_any_launch(lib):
+    m = _model()
+    L = lib
+    pm = ctypes.byref(m)
+    # null workspace / pointers
+    assert L.spec_verify_step(pm, FAKE, 10, FAKE, FAKE, 1, 4, FAKE, FAKE, FAKE, FAKE, None, None,
+                              None, 0, None) == B.SPEC_EINVAL
+    # k out of range
+    assert L.spec_verify_step(pm, FAKE, 10, FAKE, FAKE, 1, 17, FAKE, FAKE, FAKE, FAKE, None, None,
+                              FAKE, 1 << 30, None) == B.SPEC_EINVAL
+    # drafts missing with k > 0
+    assert L.spec_verify_step(pm, FAKE, 10, FAKE, None, 1, 2, FAKE, FAKE, FAKE, FAKE, None, None,
+                              FAKE, 1 << 30, None) == B.SPEC_EINVAL
+    # workspace too small
+    assert L.spec_verify_step(pm, FAKE, 10, FAKE, FAKE, 1, 4, FAKE, FAKE, FAKE, FAKE, None, None,
+                              FAKE, 100, None) == B.SPEC_EINVAL
+    # misaligned LM head weights
+    assert L.spec_lmhead_argmax(FAKE, FAKE + 2, 4, 512, 1000, FAKE, None, FAKE, 1 << 20,
+                                None) == B.SPEC_EINVAL
+    assert L.spec_lmhead_argmax(FAKE, FAKE, 4, 511, 1000, FAKE, None, FAKE, 1 << 20,
+                                None) == B.SPEC_EINVAL
+    assert L.spec_accept_commit(None, FAKE, 1, 4, FAKE, FAKE, FAKE, FAKE, None) == B.SPEC_EINVAL
+    assert L.spec_cache_write(pm, 0, FAKE, 2, 100, 60, FAKE, None, None) == B.SPEC_EINVAL
+
+
+def test_unsupported_shapes_are_reported(lib):
+    m = _model(D=192)
+    assert lib.spec_verify_step(ctypes.byref(m), FAKE, 10, FAKE, FAKE, 1, 4, FAKE, FAKE, FAKE, FAKE,
+                                None, None, FAKE, 1 << 30, None) == B.SPEC_EUNSUPPORTED
+    m2 = _model(kv_equal=True, frac=0.5)          # side-band wider than the 64-wide tile
+    assert lib.spec_verify_step(ctypes.byref(m2), FAKE, 10, FAKE, FAKE, 1, 4, FAKE, FAKE, FAKE, FAKE,
+                                None, None, FAKE, 1 << 30, None) == B.SPEC_EUNSUPPORTED
+    m3 = _model()
+    m3.page_size = 32
+    assert lib.spec_verify_step(ctypes.byref(m3), FAKE, 10, FAKE, FAKE, 1, 4, FAKE, FAKE, FAKE, FAKE,
+                                None, None, FAKE, 1 << 30, None) == B.SPEC_EUNSUPPORTED

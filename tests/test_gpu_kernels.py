@@ -1,0 +1,268 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Integer outputs (accept lengths, emitted tokens, lengths, argmax ids at
+margin-safe rows) must be identical; cache entries written from identical
+bf16 inputs must be bit-identical; attention outputs and logits must agree
+within 2e-2 absolute + 1e-2 relative (bf16 inputs, fp32 accumulation).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from speculative_decoding_verification_91_b200 import binding as B
+from speculative_decoding_verification_91_b200.inputs import gen
+from speculative_decoding_verification_91_b200.inputs import workloads as W
+from speculative_decoding_verification_91_b200.runtime import Workspace, to_device_bf16
+from speculative_decoding_verification_91_b200.session import WorkloadSession
+
+from . import harness
+
+pytestmark = pytest.mark.gpu
+
+ATOL, RTOL = 2e-2, 1e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.fail("CUDA device required for -m gpu tests")
+    B.lib()
+    yield
+    torch.cuda.synchronize()
+
+
+def _bits(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+# ---------------------------------------------------------------- acceptance
+
+@pytest.mark.parametrize("k", [0, 1, 2, 3, 4, 8, 16])
+def test_accept_commit_matches_oracle(k):
+    rng = np.random.default_rng(100 + k)
+    Bn = 37
+    g = rng.integers(0, 50, (Bn, k + 1)).astype(np.int32)
+    drafts = g[:, :k].copy()
+    for b in range(Bn):
+        if rng.random() < 0.7 and k > 0:
+            j = rng.integers(0, k)
+            drafts[b, j] += 1 + rng.integers(0, 5)
+    lens = rng.integers(0, 10000, Bn).astype(np.int32)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    d_dr, d_g, d_len = dev(drafts), dev(g), dev(lens)
+    acc = torch.zeros(Bn, dtype=torch.int32, device="cuda")
+    emi = torch.zeros(Bn * (k + 1), dtype=torch.int32, device="cuda")
+    last = torch.zeros(Bn, dtype=torch.int32, device="cuda")
+    B.spec_accept_commit(d_dr if k else None, d_g, Bn, k, d_len, acc, emi, last)
+    torch.cuda.synchronize()
+    emi = emi.cpu().numpy().reshape(Bn, k + 1)
+    for b in range(Bn):
+        a, emitted, nxt = oracle.accept_longest_prefix(drafts[b], g[b])
+        assert acc[b].item() == a
+        assert emi[b].tolist() == emitted
+        assert last[b].item() == nxt
+        assert d_len[b].item() == lens[b] + a + 1
+
+
+# ---------------------------------------------------------------- LM head
+
+@pytest.mark.parametrize("M,d,V", [(1, 512, 4096), (5, 2560, 9000), (9, 256, 1000),
+                                   (40, 1024, 5000), (100, 512, 3000), (64, 2048, 131)])
+def test_lmhead_argmax_matches_oracle(M, d, V):
+    h = gen.normal_bf16(1, f"test/lm/h/{M}/{d}", 0, M * d, 1.0).reshape(M, d)
+    w = gen.normal_bf16(1, f"test/lm/w/{d}/{V}", 0, V * d, 0.02).reshape(V, d)
+    ids_o, t1, t2 = oracle.lm_head_top2(oracle.bf16_from_bits(h), w)
+    hd, wd = to_device_bf16(h, "cuda"), to_device_bf16(w, "cuda")
+    ws = Workspace(B.spec_lmhead_workspace_bytes(M, V))
+    ids = torch.zeros(M, dtype=torch.int32, device="cuda")
+    mx = torch.zeros(M, dtype=torch.float32, device="cuda")
+    for rep in range(2):                      # second call: counters were left at zero
+        B.spec_lmhead_argmax(hd, wd, M, d, V, ids, mx, ws.buf, ws.nbytes)
+        torch.cuda.synchronize()
+        gi, gm = ids.cpu().numpy(), mx.cpu().numpy()
+        wv = oracle.bf16_from_bits(w).astype(np.float64)
+        hv = oracle.bf16_from_bits(h).astype(np.float64)
+        for m in range(M):
+            assert abs(gm[m] - t1[m]) <= ATOL + RTOL * abs(t1[m])
+            if harness.margin_ok(t1[m], t2[m]):
+                assert gi[m] == ids_o[m], (m, gi[m], ids_o[m])
+            else:                              # a near tie: the pick must be a valid maximum
+                assert 0 <= gi[m] < V
+                assert abs(hv[m] @ wv[gi[m]] - t1[m]) <= ATOL + RTOL * abs(t1[m])
+    assert ws.device_status() == 0
+
+
+def test_lmhead_ties_go_to_lowest_id():
+    M, d, V = 3, 256, 2000
+    h = gen.normal_bf16(2, "test/tie/h", 0, M * d, 1.0).reshape(M, d)
+    w = gen.normal_bf16(2, "test/tie/w", 0, V * d, 0.02).reshape(V, d)
+    ids_o, _, _ = oracle.lm_head_top2(oracle.bf16_from_bits(h), w)
+    w2 = w.copy()
+    for m in range(M):                 # copies of each row's winner at later and earlier ids
+        best = ids_o[m]
+        w2[(best + 977 + m) % V] = w[best]
+        w2[1999 - m] = w[best]
+    ids_o2, t1, t2 = oracle.lm_head_top2(oracle.bf16_from_bits(h), w2)
+    ws = Workspace(B.spec_lmhead_workspace_bytes(M, V))
+    ids = torch.zeros(M, dtype=torch.int32, device="cuda")
+    B.spec_lmhead_argmax(to_device_bf16(h, "cuda"), to_device_bf16(w2, "cuda"), M, d, V, ids, None,
+                         ws.buf, ws.nbytes)
+    torch.cuda.synchronize()
+    assert ids.cpu().numpy().tolist() == ids_o2.tolist()
+
+
+# ---------------------------------------------------------------- cache + attention
+
+@pytest.mark.parametrize("name", ["tiny", "small_b1", "small_ragged"])
+def test_cache_write_matches_oracle_bitwise(name):
+    wl = W.get_workload(name)
+    model = harness.oracle_model(wl)
+    s = WorkloadSession(wl)
+    for b in range(min(wl.batch, 3)):
+        L = int(s.lens[b])
+        caches = harness.context_caches(wl, model, b, 0, L)
+        for l, spec in enumerate(wl.layers):
+            c = caches[l]
+            k, v, sb = s.read_cache(l, b, c.lo, L)
+            assert np.array_equal(k, oracle.bits_from_bf16(c.k)), (b, l)
+            if spec.kv_equal:
+                n = oracle.rope_rotated_pairs(wl.head_dim, spec.rope_fraction)
+                h = wl.head_dim // 2
+                want = np.concatenate([c.kpre[..., :n], c.kpre[..., h:h + n]], axis=-1)
+                assert np.array_equal(sb, oracle.bits_from_bf16(want))
+            else:
+                assert np.array_equal(v, oracle.bits_from_bf16(c.v))
+
+
+@pytest.mark.parametrize("name,layer", [("tiny", 0), ("small_b1", 0), ("small_b1", 1),
+                                        ("small_ragged", 0), ("small_b16", 0), ("small_b16", 2)])
+def test_verify_attn_matches_oracle(name, layer):
+    wl = W.get_workload(name)
+    spec = wl.layers[layer]
+    model = harness.oracle_model(wl)
+    s = WorkloadSession(wl)
+    Bn, q, Hq, Hkv, D = wl.batch, wl.q_rows, wl.n_q_heads, wl.n_kv_heads, wl.head_dim
+    qb = gen.normal_bf16(3, f"test/attn/{name}/q", 0, Bn * q * Hq * D, 1.0).reshape(Bn, q, Hq, D)
+    kb = gen.normal_bf16(3, f"test/attn/{name}/k", 0, Bn * q * Hkv * D, 1.0).reshape(Bn, q, Hkv, D)
+    vb = gen.normal_bf16(3, f"test/attn/{name}/v", 0, Bn * q * Hkv * D, 1.0).reshape(Bn, q, Hkv, D)
+    pools = [p for p in (s.dm.k_pool[layer], s.dm.v_pool[layer], s.dm.ksb_pool[layer]) if p is not None]
+    before = [_bits(p).copy() for p in pools]
+    out = torch.zeros(Bn * q * Hq * D, dtype=torch.bfloat16, device="cuda")
+    B.spec_verify_attn(s.dm.desc, layer, to_device_bf16(qb, "cuda"), to_device_bf16(kb, "cuda"),
+                       None if spec.kv_equal else to_device_bf16(vb, "cuda"), s.block_table,
+                       s.max_pages, s.seq_lens, Bn, wl.k, out, s.ws.buf, s.ws.nbytes)
+    torch.cuda.synchronize()
+    assert s.ws.device_status() == 0
+    got = oracle.bf16_from_bits(_bits(out)).reshape(Bn, q, Hq, D)
+    table = s.block_table.cpu().numpy()
+    after = [_bits(p) for p in pools]
+    touched = np.zeros(before[0].shape[:3], dtype=bool)           # [page][head][slot]
+    for b in range(Bn):
+        L = int(s.lens[b])
+        cache = harness.context_caches(wl, model, b, 0, L)[layer]
+        want, (k_new, v_new, kpre_new) = oracle.attention_layer(
+            model, layer, cache, L, oracle.bf16_from_bits(qb[b]), oracle.bf16_from_bits(kb[b]),
+            None if spec.kv_equal else oracle.bf16_from_bits(vb[b]))
+        assert np.all(np.isclose(got[b], want, atol=ATOL, rtol=RTOL)), (
+            b, np.abs(got[b] - want).max())
+        assert np.mean(np.abs(got[b] - want)) < 2e-3
+        k, v, sb = s.read_cache(layer, b, L, L + q)
+        assert np.array_equal(k, oracle.bits_from_bf16(k_new))
+        if spec.kv_equal:
+            n = oracle.rope_rotated_pairs(D, spec.rope_fraction)
+            want_sb = np.concatenate([kpre_new[..., :n], kpre_new[..., D // 2:D // 2 + n]], axis=-1)
+            assert np.array_equal(sb, oracle.bits_from_bf16(want_sb))
+        else:
+            assert np.array_equal(v, oracle.bits_from_bf16(v_new))
+        for pos in range(L, L + q):
+            touched[table[b, pos // 64], :, pos % 64] = True
+    for bef, aft in zip(before, after):       # every other cache byte is unchanged
+        assert np.array_equal(bef[~touched], aft[~touched])
+
+
+# ---------------------------------------------------------------- whole step
+
+def _run_step(wl, cases):
+    s = WorkloadSession(wl, attempts=[c.attempt for c in cases])
+    s.set_inputs([c.last for c in cases], np.stack([c.drafts for c in cases]) if wl.k else [])
+    s.step()
+    return s, s.outputs()
+
+
+@pytest.mark.parametrize("name", ["tiny", "small_b1", "small_ragged", "small_b16"])
+def test_verify_step_matches_oracle(name):
+    wl = W.get_workload(name)
+    model = harness.oracle_model(wl)
+    lens = W.context_lengths(wl)
+    cases = [harness.guarded_sequence(wl, model, b, int(lens[b])) for b in range(wl.batch)]
+    s, out = _run_step(wl, cases)
+    assert s.ws.device_status() == 0
+    flips = total = 0
+    for b, c in enumerate(cases):
+        res = c.result
+        a = res.accept_len
+        assert out["accept_len"][b] == a
+        assert out["emitted"][b].tolist() == res.emitted
+        assert out["new_last"][b] == res.next_last_token
+        assert out["seq_lens"][b] == res.new_len
+        assert np.array_equal(out["target_ids"][b][:a + 1], res.g[:a + 1])
+        for i in range(wl.q_rows):
+            assert abs(out["target_max"][b][i] - res.top1[i]) <= ATOL + RTOL * abs(res.top1[i])
+        # committed cache entries (positions L..L+a) against the oracle's
+        for l, spec in enumerate(wl.layers):
+            k_new, v_new, kpre_new = res.forward.new_entries[l]
+            k, v, sb = s.read_cache(l, b, c.L, c.L + a + 1)
+            kw = oracle.bits_from_bf16(k_new[:a + 1])
+            gk = oracle.bf16_from_bits(k)
+            assert np.all(np.isclose(gk, k_new[:a + 1], atol=ATOL, rtol=RTOL))
+            flips += int(np.sum(k != kw))
+            total += k.size
+            vv = v if not spec.kv_equal else sb
+            if not spec.kv_equal:
+                assert np.all(np.isclose(oracle.bf16_from_bits(v), v_new[:a + 1], atol=ATOL, rtol=RTOL))
+                flips += int(np.sum(v != oracle.bits_from_bf16(v_new[:a + 1])))
+                total += v.size
+    # entries computed from a differently ordered fp32 sum may differ by a bf16 ulp, rarely
+    assert flips <= max(2, total // 500), (flips, total)
+
+
+@pytest.mark.parametrize("name", ["small_b1", "small_ragged"])
+def test_step_is_invariant_to_k(name):
+    """Greedy decoding with k = 0, one token per step, and one verify step with
+    k = 8 whose drafts are those greedy tokens give bit-identical rows: the
+    same argmax logits and the same cache entries (fixed split boundaries,
+    M-independent reduction orders)."""
+    base = W.get_workload(name)
+    g0 = WorkloadSession(base.with_(k=0))
+    Bn = base.batch
+    last = np.array([W.last_token(base, b, 0) for b in range(Bn)], dtype=np.int32)
+    tokens, maxes = [], []
+    cur = last.copy()
+    for step in range(3):
+        g0.set_inputs(cur, [])
+        g0.step()
+        o = g0.outputs()
+        tokens.append(o["target_ids"][:, 0].copy())
+        maxes.append(o["target_max"][:, 0].copy())
+        cur = o["new_last"].astype(np.int32)
+    s8 = WorkloadSession(base.with_(k=8))
+    drafts = np.zeros((Bn, 8), dtype=np.int32)
+    drafts[:, :3] = np.stack(tokens, axis=1)
+    drafts[:, 3:] = 7
+    s8.set_inputs(last, drafts)
+    s8.step()
+    o8 = s8.outputs()
+    for b in range(Bn):
+        assert o8["accept_len"][b] >= 3
+        for i in range(3):
+            assert o8["target_ids"][b][i] == tokens[i][b]
+            assert np.float32(o8["target_max"][b][i]).view(np.uint32) == \
+                np.float32(maxes[i][b]).view(np.uint32)
+        L = int(g0.lens[b])
+        for l in range(len(base.layers)):
+            a = g0.read_cache(l, b, L, L + 3)
+            c = s8.read_cache(l, b, L, L + 3)
+            for x, y in zip(a, c):
+                if x is not None:
+                    assert np.array_equal(x, y)
