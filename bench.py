@@ -43,8 +43,8 @@ L2_FLUSH_BYTES = 256 << 20
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
     ap.add_argument("--workload", default="b1_ctx8k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -76,12 +76,17 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
+            t0 = time.time()                      # first sample before timing starts
+            while not self.lines and time.time() - t0 < 3.0:
+                time.sleep(0.02)
+            self.skip = len(self.lines)
         except OSError:
             self.proc = None
+            self.skip = 0
         return self
 
     def _read(self):
@@ -99,7 +104,7 @@ class ClockSampler:
     def summary(self):
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for ln in self.lines[self.skip:] or self.lines[-1:]:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 9:
                 continue
@@ -187,28 +192,22 @@ def run_cuda(args, rank, world, local_rank):
         raise RuntimeError("device status flagged during warm-up")
     tokens_per_step = int(np.sum(out["accept_len"] + 1))
 
-    # ---- timed: device-resident inputs, L2 flushed before every step
-    starts = [ev() for _ in range(args.steps)]
-    stops = [ev() for _ in range(args.steps)]
-    lm0 = [ev() for _ in range(args.steps)]
-    lm1 = [ev() for _ in range(args.steps)]
+    # ---- timed: device-resident inputs, L2 flushed before every step; the
+    #      library records its own CUDA events around each step and its
+    #      LM-head launch on the launching stream
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
+    B.spec_profile_start(args.steps)
     with ClockSampler(local_rank) as clocks:
         for i in range(args.steps):
             flush.zero_()
             sess.reset_lengths()
-            B.spec_set_profile_events(B.SPEC_PROF_STEP, starts[i], stops[i])
-            B.spec_set_profile_events(B.SPEC_PROF_LMHEAD, lm0[i], lm1[i])
             sess.step(stream=stream, with_targets=False)
-        B.spec_set_profile_events(B.SPEC_PROF_STEP, None, None)
-        B.spec_set_profile_events(B.SPEC_PROF_LMHEAD, None, None)
         torch.cuda.synchronize(dev)
+    step_ms, lm_ms = B.spec_profile_collect(args.steps)
     if world > 1:
         dist.barrier()
-    step_ms = [s.elapsed_time(e) for s, e in zip(starts, stops)]
-    lm_ms = [s.elapsed_time(e) for s, e in zip(lm0, lm1)]
     if sess.ws.device_status(stream) != 0:
         raise RuntimeError("device status flagged during the timed steps")
 
@@ -369,9 +368,11 @@ def main():
             "clocks": r["clocks"],
         }
         if not args.no_cpu_baseline and world == 1:
-            tps, sec, threads, desc = oracle_sample(wl.name)
-            line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": threads,
-                                    "kind": "oracle", "sample": desc}
+            _, sec, threads, desc = oracle_sample(wl.name)
+            line["cpu_baseline"] = {"value": r["tokens_per_step"] / sec, "unit": "tokens/s",
+                                    "cores": threads, "kind": "oracle",
+                                    "sample": desc + f"; s/step {sec:.2f}, scaled by the "
+                                    f"workload's {r['tokens_per_step']} emitted tokens per step"}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

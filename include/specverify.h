@@ -211,14 +211,16 @@ int spec_verify_step(const spec_model* m, const int32_t* block_table, int max_pa
                      int32_t* new_last_token, int32_t* target_ids, float* target_maxlogit,
                      void* ws, size_t ws_bytes, void* stream);
 
-/* Timing hook (no counterpart in the pages; measurement only).  When set,
- * spec_verify_step records ev_start / ev_stop (cudaEvent_t passed as void*)
- * on its stream immediately before and after the named stage's launches.
- * stage: SPEC_PROF_LMHEAD (the LM-head argmax kernel) or SPEC_PROF_STEP (the
- * whole step).  NULL events clear the hook.  Process-wide; not thread-safe. */
-#define SPEC_PROF_LMHEAD 0
-#define SPEC_PROF_STEP 1
-int spec_set_profile_events(int stage, void* ev_start, void* ev_stop);
+/* Timing hook (no counterpart in the pages; measurement only).
+ * spec_profile_start(n): the next n spec_verify_step calls record CUDA events
+ * (created and owned by the library) on their stream around the whole step
+ * and around the LM-head launch.  spec_profile_collect(step_ms, lmhead_ms, n)
+ * waits for those events, writes the n per-step durations in milliseconds
+ * (host arrays) and releases the events.  Process-wide; not thread-safe.
+ * n must be in [1, 65536]; collect returns SPEC_EINVAL if fewer than n steps
+ * were recorded. */
+int spec_profile_start(int n_steps);
+int spec_profile_collect(float* step_ms, float* lmhead_ms, int n_steps);
 
 #ifdef __cplusplus
 }

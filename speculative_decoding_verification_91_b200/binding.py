@@ -31,10 +31,8 @@ EXPORTED = [
     "spec_status_string", "spec_layer_pool_bytes", "spec_workspace_bytes",
     "spec_lmhead_workspace_bytes", "spec_workspace_init", "spec_read_device_status",
     "spec_cache_write", "spec_verify_attn", "spec_lmhead_argmax", "spec_accept_commit",
-    "spec_verify_step", "spec_set_profile_events",
+    "spec_verify_step", "spec_profile_start", "spec_profile_collect",
 ]
-SPEC_PROF_LMHEAD = 0
-SPEC_PROF_STEP = 1
 
 
 class SpecError(RuntimeError):
@@ -99,7 +97,8 @@ def lib():
         L.spec_verify_step.argtypes = [pm, c_void_p, c_int, c_void_p, c_void_p, c_int, c_int,
                                        c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                        c_void_p, c_size_t, c_void_p]
-        L.spec_set_profile_events.argtypes = [c_int, c_void_p, c_void_p]
+        L.spec_profile_start.argtypes = [c_int]
+        L.spec_profile_collect.argtypes = [POINTER(c_float), POINTER(c_float), c_int]
         for name in EXPORTED[4:]:
             getattr(L, name).restype = c_int
         _lib = L
@@ -193,8 +192,14 @@ def spec_verify_step(model, block_table, max_pages, last_token, drafts, B, k, se
                                          _s(stream)), "spec_verify_step")
 
 
-def spec_set_profile_events(stage: int, ev_start, ev_stop) -> int:
-    """ev_start / ev_stop: torch.cuda.Event (recorded by the library) or None."""
-    h = lambda e: None if e is None else e.cuda_event
-    return _check(lib().spec_set_profile_events(stage, h(ev_start), h(ev_stop)),
-                  "spec_set_profile_events")
+
+def spec_profile_start(n_steps: int) -> int:
+    return _check(lib().spec_profile_start(n_steps), "spec_profile_start")
+
+
+def spec_profile_collect(n_steps: int):
+    """(step_ms list, lmhead_ms list) of the last n profiled steps."""
+    a = (c_float * n_steps)()
+    b = (c_float * n_steps)()
+    _check(lib().spec_profile_collect(a, b, n_steps), "spec_profile_collect")
+    return list(a), list(b)

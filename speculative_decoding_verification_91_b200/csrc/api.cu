@@ -6,6 +6,7 @@
 
 #include <algorithm>
 #include <mutex>
+#include <vector>
 
 #include "../../include/specverify.h"
 #include "common.cuh"
@@ -139,9 +140,25 @@ T* at(void* ws, size_t off) {
 
 inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? SPEC_OK : SPEC_ECUDA; }
 
-cudaEvent_t g_prof[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};
-inline void prof_mark(int stage, int which, cudaStream_t st) {
-  if (g_prof[stage][which]) cudaEventRecord(g_prof[stage][which], st);
+// Profiling events: per recorded step {step start, LM-head start, LM-head
+// stop, step stop}.
+struct Prof {
+  std::vector<cudaEvent_t> ev;
+  int n = 0, used = 0;
+  bool on = false;
+};
+Prof g_prof;
+inline void prof_mark(int which, cudaStream_t st) {
+  if (g_prof.on && g_prof.used < g_prof.n) cudaEventRecord(g_prof.ev[4 * g_prof.used + which], st);
+}
+inline void prof_step_done() {
+  if (g_prof.on && g_prof.used < g_prof.n) ++g_prof.used;
+}
+void prof_release() {
+  for (cudaEvent_t e : g_prof.ev) cudaEventDestroy(e);
+  g_prof.ev.clear();
+  g_prof.n = g_prof.used = 0;
+  g_prof.on = false;
 }
 
 }  // namespace
@@ -151,11 +168,35 @@ using namespace sv;
 
 extern "C" {
 
-int spec_set_profile_events(int stage, void* ev_start, void* ev_stop) {
-  if (stage != SPEC_PROF_LMHEAD && stage != SPEC_PROF_STEP) return SPEC_EINVAL;
-  g_prof[stage][0] = static_cast<cudaEvent_t>(ev_start);
-  g_prof[stage][1] = static_cast<cudaEvent_t>(ev_stop);
+int spec_profile_start(int n_steps) {
+  if (n_steps < 1 || n_steps > 65536) return SPEC_EINVAL;
+  prof_release();
+  g_prof.ev.resize(4 * (size_t)n_steps, nullptr);
+  for (auto& e : g_prof.ev)
+    if (cudaEventCreate(&e) != cudaSuccess) {
+      prof_release();
+      return SPEC_ECUDA;
+    }
+  g_prof.n = n_steps;
+  g_prof.on = true;
   return SPEC_OK;
+}
+
+int spec_profile_collect(float* step_ms, float* lmhead_ms, int n_steps) {
+  if (!g_prof.on || n_steps != g_prof.n || g_prof.used < n_steps || !step_ms) {
+    prof_release();
+    return SPEC_EINVAL;
+  }
+  int rc = SPEC_OK;
+  for (int i = 0; i < n_steps && rc == SPEC_OK; ++i) {
+    cudaEvent_t* e = &g_prof.ev[4 * (size_t)i];
+    if (cudaEventSynchronize(e[3]) != cudaSuccess ||
+        cudaEventElapsedTime(&step_ms[i], e[0], e[3]) != cudaSuccess ||
+        (lmhead_ms && cudaEventElapsedTime(&lmhead_ms[i], e[1], e[2]) != cudaSuccess))
+      rc = SPEC_ECUDA;
+  }
+  prof_release();
+  return rc;
 }
 
 const char* spec_status_string(int s) {
@@ -347,7 +388,7 @@ int spec_verify_step(const spec_model* m, const int32_t* block_table, int max_pa
   uint16_t* qrot = at<uint16_t>(ws, s.qrot);
   uint16_t* attn_out = at<uint16_t>(ws, s.attn_out);
 
-  prof_mark(SPEC_PROF_STEP, 0, st);
+  prof_mark(0, st);
   rc = cuda_status(launch_embed(m->w_lm, m->vocab, d, last_token, drafts, B, q, x, hdr.status, st));
   if (rc) return rc;
   for (int l = 0; l < m->n_layers; ++l) {
@@ -419,14 +460,15 @@ int spec_verify_step(const spec_model* m, const int32_t* block_table, int max_pa
   bl.maxv = at<float>(ws, s.maxv);
   bl.tickets = hdr.tickets;
   bl.status = hdr.status;
-  prof_mark(SPEC_PROF_LMHEAD, 0, st);
+  prof_mark(1, st);
   rc = cuda_status(launch_gemm(pl, kGemmArgmax, hn, m->w_lm, bl, st));
-  prof_mark(SPEC_PROF_LMHEAD, 1, st);
+  prof_mark(2, st);
   if (rc) return rc;
   rc = cuda_status(launch_accept(drafts, at<int32_t>(ws, s.ids), B, k, seq_lens, accept_len,
                                  emitted, new_last_token, target_ids, target_maxlogit,
                                  at<float>(ws, s.maxv), st));
-  prof_mark(SPEC_PROF_STEP, 1, st);
+  prof_mark(3, st);
+  prof_step_done();
   return rc;
 }
 
