@@ -174,8 +174,19 @@ def run_cuda(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     wl = W.get_workload(args.workload)
     B.lib()
-    sess = WorkloadSession(wl, device=dev, poison=False)
-    last, drafts = gpu_greedy_drafts(sess, wl, W)
+    fixture = os.path.join(ROOT, "tests", "golden", f"verify_{wl.name}.json")
+    if os.path.exists(fixture):
+        # margin-guarded inputs shared with the parity tests
+        with open(fixture) as f:
+            seqs = json.load(f)["sequences"]
+        sess = WorkloadSession(wl, attempts=[q["attempt"] for q in seqs], device=dev, poison=False)
+        last = np.array([q["last_token"] for q in seqs], dtype=np.int32)
+        drafts = np.array([q["drafts"] for q in seqs], dtype=np.int32)
+        inputs = "margin-guarded fixture " + os.path.relpath(fixture, ROOT)
+    else:
+        sess = WorkloadSession(wl, device=dev, poison=False)
+        last, drafts = gpu_greedy_drafts(sess, wl, W)
+        inputs = "attempt-0 draws; drafts from the workload recipe on the CUDA greedy path"
     sess.set_inputs(last, drafts)
     stream = torch.cuda.current_stream(dev)
 
@@ -247,7 +258,7 @@ def run_cuda(args, rank, world, local_rank):
         mean_step, mean_e2e, mean_lm = [float(v) for v in t.tolist()]
     kv_b, lm_b, proj_b = algorithmic_bytes(wl, sess.lens)
     launches_per_step = 4 + 6 * len(wl.layers)
-    return dict(wl=wl, lens=sess.lens, tokens_per_step=tokens_per_step, mean_step=mean_step,
+    return dict(wl=wl, lens=sess.lens, tokens_per_step=tokens_per_step, mean_step=mean_step, inputs=inputs,
                 mean_lm=mean_lm, mean_e2e=mean_e2e, kv_b=kv_b, lm_b=lm_b, proj_b=proj_b,
                 launches=launches_per_step * args.steps, clocks=clocks.summary(),
                 h2d=int(h_in.numel() * 4), d2h=int(h_out.numel() * 4), step_ms=step_ms,
@@ -273,7 +284,8 @@ def oracle_sample(wl_name: str, budget_s: float = 25.0):
         layers.append(oracle.LayerDef(spec.window, spec.kv_equal, spec.rope_fraction,
                                       oracle.bf16_from_bits(wqkv), oracle.bf16_from_bits(wo)))
     model = oracle.Model(wl.d_model, wl.n_q_heads, wl.n_kv_heads, wl.head_dim,
-                         W.lm_head_weight(wl), layers, wl.rope_theta, wl.rms_eps)
+                         W.lm_head_weight(wl), layers, wl.rope_theta, wl.rms_eps,
+                         W.embedding_weight(wl))
     caches = []
     for l in range(len(wl.layers)):
         lo, k, v = W.context_kv(wl, 0, 0, l, L)
@@ -352,7 +364,7 @@ def main():
                        "context": [int(x) for x in r["lens"]], "layers": len(wl.layers),
                        "d_model": wl.d_model, "vocab": wl.vocab,
                        "l2": f"flushed ({L2_FLUSH_BYTES >> 20} MiB write) before every timed step",
-                       "tokens_per_step": r["tokens_per_step"]},
+                       "tokens_per_step": r["tokens_per_step"], "inputs": r["inputs"]},
             "us_per_step": r["mean_step"] * 1e3,
             "step_hbm": {"bytes": step_bytes, "bytes_with_projections": step_bytes + r["proj_b"],
                          "gbs": step_bytes / step_s / 1e9,

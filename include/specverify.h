@@ -38,7 +38,7 @@
  *     rotated dimensions (n_rot = p*D/2), so per token and KV head it holds
  *     (1+p)*D values instead of 2*D;
  *   - the target layer is x <- x + W_o Attn(RMSNorm(x)) (no MLP), then a
- *     final RMSNorm and the tied LM head; RMSNorm eps from the model, unit
+ *     final RMSNorm and the LM head; RMSNorm eps from the model, unit
  *     gain; fp32 residual stream, bf16 for normalised GEMM inputs, q/k/v after
  *     RoPE, cache entries, attention outputs and the final hidden state;
  *   - argmax ties go to the lowest token id.
@@ -118,7 +118,8 @@ typedef struct spec_model {
                             results do not depend on batch size, k or the GPU */
   float rope_theta;      /* RoPE base (10000) */
   float rms_eps;         /* RMSNorm epsilon (1e-6) */
-  const void* w_lm;      /* [vocab][d_model] bf16: LM head, tied with the token embedding */
+  const void* w_lm;      /* [vocab][d_model] bf16: LM head */
+  const void* w_embed;   /* [vocab][d_model] bf16: token embedding (may equal w_lm: tied) */
   const spec_layer* layers;  /* host array of n_layers */
 } spec_model;
 

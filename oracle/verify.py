@@ -36,7 +36,8 @@ this implementation):
     i < p*D/2 (the highest frequencies) and leaves the rest unchanged;
   * key-equals-value: V is the pre-RoPE key projection;
   * the synthetic target is x <- x + W_o Attn(RMSNorm(x)) per layer (no
-    MLP), then RMSNorm and the tied LM head; RMSNorm eps 1e-6, unit gain;
+    MLP), then RMSNorm and the LM head; RMSNorm eps 1e-6, unit gain; the
+    token embedding is its own table (untied);
   * storage formats: fp32 residual stream; bf16 for normalised GEMM inputs,
     q/k/v after RoPE, cache entries, attention outputs and the final hidden
     state; logits in binary32; argmax ties go to the lowest token id.
@@ -243,10 +244,11 @@ class Model:
     n_q_heads: int
     n_kv_heads: int
     head_dim: int
-    w_lm_bits: np.ndarray        # [V][d] bf16 bits: LM head and (tied) embedding
+    w_lm_bits: np.ndarray        # [V][d] bf16 bits: LM head
     layers: list
     rope_theta: float = 10000.0
     rms_eps: float = 1e-6
+    w_emb_bits: np.ndarray | None = None   # [V][d] token embedding; None: tied to the LM head
 
     @property
     def vocab(self) -> int:
@@ -357,7 +359,8 @@ def verify_forward(model: Model, caches: list, L: int, tokens, lm_rows=None) -> 
     tokens = np.asarray(tokens, dtype=np.int64)
     nq = tokens.shape[0]
     D, Hq, Hkv = model.head_dim, model.n_q_heads, model.n_kv_heads
-    x = bf16_from_bits(model.w_lm_bits[tokens]).astype(np.float32)       # tied embedding rows
+    emb = model.w_lm_bits if model.w_emb_bits is None else model.w_emb_bits
+    x = bf16_from_bits(emb[tokens]).astype(np.float32)                   # embedding rows
     new_entries, attn_out = [], []
     for l, spec in enumerate(model.layers):
         hn = bf16(rmsnorm(x, model.rms_eps))

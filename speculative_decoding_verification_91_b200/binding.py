@@ -54,7 +54,7 @@ class SpecModel(ctypes.Structure):
         ("n_layers", c_int), ("d_model", c_int), ("n_q_heads", c_int), ("n_kv_heads", c_int),
         ("head_dim", c_int), ("vocab", c_int), ("page_size", c_int), ("num_pages", c_int),
         ("split_tokens", c_int), ("rope_theta", c_float), ("rms_eps", c_float),
-        ("w_lm", c_void_p), ("layers", POINTER(SpecLayer)),
+        ("w_lm", c_void_p), ("w_embed", c_void_p), ("layers", POINTER(SpecLayer)),
     ]
 
 

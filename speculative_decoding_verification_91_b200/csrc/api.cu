@@ -62,7 +62,7 @@ int qkv_out(const spec_model* m, const spec_layer& L) {
 }
 
 int check_model(const spec_model* m) {
-  if (!m || !m->layers || !m->w_lm) return SPEC_EINVAL;
+  if (!m || !m->layers || !m->w_lm || !m->w_embed) return SPEC_EINVAL;
   if (m->n_layers < 1 || m->d_model < 8 || m->d_model % 8 || m->n_q_heads < 1 || m->n_kv_heads < 1 ||
       m->n_q_heads % m->n_kv_heads || m->vocab < 1 || m->num_pages < 1)
     return SPEC_EINVAL;
@@ -389,7 +389,7 @@ int spec_verify_step(const spec_model* m, const int32_t* block_table, int max_pa
   uint16_t* attn_out = at<uint16_t>(ws, s.attn_out);
 
   prof_mark(0, st);
-  rc = cuda_status(launch_embed(m->w_lm, m->vocab, d, last_token, drafts, B, q, x, hdr.status, st));
+  rc = cuda_status(launch_embed(m->w_embed, m->vocab, d, last_token, drafts, B, q, x, hdr.status, st));
   if (rc) return rc;
   for (int l = 0; l < m->n_layers; ++l) {
     const spec_layer& L = m->layers[l];

@@ -47,7 +47,7 @@ cudaError_t launch_gemm(const GemmPlan& p, int mode, const void* x, const void* 
                         const GemmBuffers& buf, cudaStream_t st);
 
 // ------------------------------------------------------------- small kernels
-cudaError_t launch_embed(const void* w_lm, int vocab, int d, const int32_t* last_token,
+cudaError_t launch_embed(const void* w_emb, int vocab, int d, const int32_t* last_token,
                          const int32_t* drafts, int B, int q, float* x, unsigned* status,
                          cudaStream_t st);
 cudaError_t launch_rmsnorm(const float* x, int M, int d, float eps, uint16_t* out,

@@ -8,8 +8,8 @@ namespace sv {
 namespace {
 
 // Row m = b*q + i holds token last_token[b] (i = 0) or drafts[b][i-1]; its
-// residual stream starts as the tied embedding row, widened to fp32.
-__global__ void embed_kernel(const uint16_t* __restrict__ w_lm, int vocab, int d,
+// residual stream starts as that token's embedding row, widened to fp32.
+__global__ void embed_kernel(const uint16_t* __restrict__ w_emb, int vocab, int d,
                              const int32_t* __restrict__ last_token,
                              const int32_t* __restrict__ drafts, int q, float* __restrict__ x,
                              unsigned* status) {
@@ -22,7 +22,7 @@ __global__ void embed_kernel(const uint16_t* __restrict__ w_lm, int vocab, int d
     for (int e = threadIdx.x; e < d; e += blockDim.x) row[e] = 0.f;
     return;
   }
-  const uint16_t* src = w_lm + (size_t)tok * d;
+  const uint16_t* src = w_emb + (size_t)tok * d;
   for (int e = threadIdx.x; e < d; e += blockDim.x) row[e] = bf16_to_f32(src[e]);
 }
 
@@ -81,10 +81,10 @@ __global__ void accept_kernel(const int32_t* __restrict__ drafts, const int32_t*
 
 }  // namespace
 
-cudaError_t launch_embed(const void* w_lm, int vocab, int d, const int32_t* last_token,
+cudaError_t launch_embed(const void* w_emb, int vocab, int d, const int32_t* last_token,
                          const int32_t* drafts, int B, int q, float* x, unsigned* status,
                          cudaStream_t st) {
-  embed_kernel<<<B * q, 256, 0, st>>>(static_cast<const uint16_t*>(w_lm), vocab, d, last_token,
+  embed_kernel<<<B * q, 256, 0, st>>>(static_cast<const uint16_t*>(w_emb), vocab, d, last_token,
                                       drafts, q, x, status);
   return cudaGetLastError();
 }

@@ -52,6 +52,7 @@ class Workload:
     seed: int = 0
     steps: int = 1              # verify steps (the loop workload runs many)
     prompt_tokens: int = 0      # >0: context is a prefilled random prompt, not drawn K/V
+    tied_embedding: bool = False
 
     @property
     def q_rows(self) -> int:
@@ -131,8 +132,19 @@ def _w(wl: Workload, name: str, rows: int, cols: int) -> np.ndarray:
 
 
 def lm_head_weight(wl: Workload) -> np.ndarray:
-    """Tied embedding / LM-head matrix, bf16 bits, [vocab][d_model]."""
+    """LM-head matrix, bf16 bits, [vocab][d_model]."""
     return _w(wl, "w_lm", wl.vocab, wl.d_model)
+
+
+def embedding_weight(wl: Workload):
+    """Token embedding, bf16 bits, [vocab][d_model]; None when tied to the LM head.
+
+    Untied by default: with random weights a tied table makes every token's
+    own logit dominate (the model copies its input), which would leave the
+    acceptance path untested by the model's choices."""
+    if wl.tied_embedding:
+        return None
+    return _w(wl, "w_emb", wl.vocab, wl.d_model)
 
 
 def layer_weights(wl: Workload, l: int):

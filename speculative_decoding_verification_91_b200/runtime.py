@@ -39,12 +39,13 @@ class DeviceModel:
 
     def __init__(self, *, d_model, n_q_heads, n_kv_heads, head_dim, vocab, layers, w_lm_bits,
                  layer_weights, num_pages, split_tokens, rope_theta=10000.0, rms_eps=1e-6,
-                 device="cuda", poison=True):
+                 device="cuda", poison=True, w_emb_bits=None):
         self.device = torch.device(device)
         self.d_model, self.n_q_heads, self.n_kv_heads = d_model, n_q_heads, n_kv_heads
         self.head_dim, self.vocab, self.num_pages = head_dim, vocab, num_pages
         self.layers = list(layers)
         self.w_lm = to_device_bf16(w_lm_bits, self.device)
+        self.w_emb = self.w_lm if w_emb_bits is None else to_device_bf16(w_emb_bits, self.device)
         self.w_qkv, self.w_o, self.k_pool, self.v_pool, self.ksb_pool = [], [], [], [], []
         P, H, D = num_pages, n_kv_heads, head_dim
         for (wqkv, wo), spec in zip(layer_weights, self.layers):
@@ -67,7 +68,7 @@ class DeviceModel:
                 int(spec.window), int(spec.kv_equal), float(spec.rope_fraction))
         self.desc = B.SpecModel(len(self.layers), d_model, n_q_heads, n_kv_heads, head_dim, vocab,
                                 B.SPEC_PAGE_SIZE, num_pages, split_tokens, float(rope_theta),
-                                float(rms_eps), self.w_lm.data_ptr(),
+                                float(rms_eps), self.w_lm.data_ptr(), self.w_emb.data_ptr(),
                                 ctypes.cast(self._layers_c, ctypes.POINTER(B.SpecLayer)))
 
     def _pool(self, shape, poison):

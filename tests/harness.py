@@ -30,7 +30,8 @@ def oracle_model(wl: W.Workload) -> oracle.Model:
         layers.append(oracle.LayerDef(spec.window, spec.kv_equal, spec.rope_fraction,
                                       oracle.bf16_from_bits(wqkv), oracle.bf16_from_bits(wo)))
     return oracle.Model(wl.d_model, wl.n_q_heads, wl.n_kv_heads, wl.head_dim,
-                        W.lm_head_weight(wl), layers, wl.rope_theta, wl.rms_eps)
+                        W.lm_head_weight(wl), layers, wl.rope_theta, wl.rms_eps,
+                        W.embedding_weight(wl))
 
 
 def context_caches(wl: W.Workload, model: oracle.Model, b: int, attempt: int, L: int):
