@@ -103,6 +103,7 @@ typedef struct spec_layer {
   int window;           /* 0 = global; else keys t-W < j <= t are visible */
   int kv_equal;         /* 1: value = pre-RoPE key (no v projection, no v_pool) */
   float rope_fraction;  /* fraction of rotary pairs rotated (1.0 or 0.25 here) */
+  int split_tokens;     /* this layer's split-KV chunk, 0 = the model's */
 } spec_layer;
 
 typedef struct spec_model {
@@ -114,10 +115,11 @@ typedef struct spec_model {
   int vocab;
   int page_size;         /* must be SPEC_PAGE_SIZE */
   int num_pages;         /* pages in each layer's pools */
-  int split_tokens;      /* split-KV chunk: a multiple of page_size; fixed per model so that
-                            results do not depend on batch size, k or the GPU */
-  float rope_theta;      /* RoPE base (10000) */
-  float rms_eps;         /* RMSNorm epsilon (1e-6) */
+  int split_tokens;      /* split-KV chunk: a multiple of page_size; fixed per model (and
+                            optionally per layer) so that results do not depend on batch
+                            size, k or the GPU */
+  double rope_theta;     /* RoPE base (10000) */
+  double rms_eps;        /* RMSNorm epsilon (1e-6) */
   const void* w_lm;      /* [vocab][d_model] bf16: LM head */
   const void* w_embed;   /* [vocab][d_model] bf16: token embedding (may equal w_lm: tied) */
   const spec_layer* layers;  /* host array of n_layers */

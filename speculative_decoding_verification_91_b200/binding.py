@@ -46,6 +46,7 @@ class SpecLayer(ctypes.Structure):
         ("w_qkv", c_void_p), ("w_o", c_void_p),
         ("k_pool", c_void_p), ("v_pool", c_void_p), ("ksb_pool", c_void_p),
         ("window", c_int), ("kv_equal", c_int), ("rope_fraction", c_float),
+        ("split_tokens", c_int),
     ]
 
 
@@ -53,7 +54,7 @@ class SpecModel(ctypes.Structure):
     _fields_ = [
         ("n_layers", c_int), ("d_model", c_int), ("n_q_heads", c_int), ("n_kv_heads", c_int),
         ("head_dim", c_int), ("vocab", c_int), ("page_size", c_int), ("num_pages", c_int),
-        ("split_tokens", c_int), ("rope_theta", c_float), ("rms_eps", c_float),
+        ("split_tokens", c_int), ("rope_theta", ctypes.c_double), ("rms_eps", ctypes.c_double),
         ("w_lm", c_void_p), ("w_embed", c_void_p), ("layers", POINTER(SpecLayer)),
     ]
 

@@ -57,6 +57,10 @@ int n_rot_of(const spec_model* m, const spec_layer& L) {
   return (int)lrintf(L.rope_fraction * (float)m->head_dim / 2.0f);
 }
 
+int split_of(const spec_model* m, const spec_layer& L) {
+  return L.split_tokens > 0 ? L.split_tokens : m->split_tokens;
+}
+
 int qkv_out(const spec_model* m, const spec_layer& L) {
   return (m->n_q_heads + m->n_kv_heads + (L.kv_equal ? 0 : m->n_kv_heads)) * m->head_dim;
 }
@@ -69,13 +73,14 @@ int check_model(const spec_model* m) {
   if (m->page_size != SPEC_PAGE_SIZE) return SPEC_EUNSUPPORTED;
   if (m->head_dim != 128 && m->head_dim != 256) return SPEC_EUNSUPPORTED;
   if (m->split_tokens < m->page_size || m->split_tokens % m->page_size) return SPEC_EINVAL;
-  if (!(m->rope_theta > 0.f) || !(m->rms_eps >= 0.f)) return SPEC_EINVAL;
+  if (!(m->rope_theta > 0.0) || !(m->rms_eps >= 0.0)) return SPEC_EINVAL;
   if ((uint64_t)m->num_pages * m->n_kv_heads * m->page_size > 0x7fffffffull) return SPEC_EUNSUPPORTED;
   if (reinterpret_cast<uintptr_t>(m->w_lm) & 15) return SPEC_EINVAL;
   for (int l = 0; l < m->n_layers; ++l) {
     const spec_layer& L = m->layers[l];
     if (!L.w_qkv || !L.w_o || !L.k_pool) return SPEC_EINVAL;
     if (L.window < 0) return SPEC_EINVAL;
+    if (L.split_tokens < 0 || L.split_tokens % m->page_size) return SPEC_EINVAL;
     if (!(L.rope_fraction >= 0.f && L.rope_fraction <= 1.f)) return SPEC_EINVAL;
     const int nr = n_rot_of(m, L);
     if (L.kv_equal) {
@@ -95,10 +100,12 @@ int check_model(const spec_model* m) {
 struct StepLayout {
   size_t x, hn, qkv, qrot, attn_out, attn_part, gemm_part, arg_val, arg_idx, ids, maxv, total;
   int tickets;
+  bool splits_ok;   // every layer's split count fits the combine kernel
 };
 
 StepLayout step_layout(const spec_model* m, int B, int k, int max_pages) {
   StepLayout s{};
+  s.splits_ok = true;
   const int q = k + 1, M = B * q, d = m->d_model, D = m->head_dim;
   int nqkv = 0;
   size_t attn_floats = 0, gemm_floats = 0;
@@ -107,8 +114,9 @@ StepLayout step_layout(const spec_model* m, int B, int k, int max_pages) {
     const spec_layer& L = m->layers[l];
     nqkv = std::max(nqkv, qkv_out(m, L));
     AttnGeom g = plan_attn(B, q, m->n_q_heads, m->n_kv_heads, D, m->page_size, m->num_pages,
-                           max_pages, L.window, L.kv_equal, 2 * n_rot_of(m, L), m->split_tokens);
+                           max_pages, L.window, L.kv_equal, 2 * n_rot_of(m, L), split_of(m, L));
     attn_floats = std::max(attn_floats, attn_partial_floats(g));
+    if (g.n_splits_grid > kMaxSplits) s.splits_ok = false;
     GemmPlan pq = plan_gemm(M, qkv_out(m, L), d, kGemmStore);
     GemmPlan po = plan_gemm(M, d, m->n_q_heads * D, kGemmResidual);
     gemm_floats = std::max({gemm_floats, gemm_partial_floats(pq), gemm_partial_floats(po)});
@@ -226,7 +234,7 @@ size_t spec_layer_pool_bytes(const spec_model* m, int layer, int which) {
 size_t spec_workspace_bytes(const spec_model* m, int max_batch, int max_k, int max_pages) {
   if (!m || !m->layers || max_batch < 1 || max_k < 0 || max_k > SPEC_MAX_K || max_pages < 1) return 0;
   StepLayout s = step_layout(m, max_batch, max_k, max_pages);
-  if (s.tickets > kMaxTickets) return 0;
+  if (s.tickets > kMaxTickets || !s.splits_ok) return 0;
   return s.total;
 }
 
@@ -269,7 +277,7 @@ int spec_cache_write(const spec_model* m, int layer, const int32_t* block_table_
   a.n_kv_heads = m->n_kv_heads;
   a.head_dim = m->head_dim;
   a.n_rot = n_rot_of(m, L);
-  a.theta = m->rope_theta;
+  rope_inv_freq(m->rope_theta, m->head_dim, a.n_rot, a.inv_freq);
   a.page_size = m->page_size;
   a.num_pages = m->num_pages;
   a.max_pages = max_pages;
@@ -299,6 +307,7 @@ int spec_verify_attn(const spec_model* m, int layer, const void* q, const void* 
   if (!L.kv_equal && !v_new) return SPEC_EINVAL;
   const int qn = k + 1, D = m->head_dim;
   StepLayout s = step_layout(m, B, k, max_pages);
+  if (!s.splits_ok) return SPEC_EUNSUPPORTED;
   if (ws_bytes < s.total) return SPEC_EINVAL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   WsHeader hdr = ws_header(ws);
@@ -308,7 +317,7 @@ int spec_verify_attn(const spec_model* m, int layer, const void* q, const void* 
   a.n_kv_heads = m->n_kv_heads;
   a.head_dim = D;
   a.n_rot = n_rot_of(m, L);
-  a.theta = m->rope_theta;
+  rope_inv_freq(m->rope_theta, m->head_dim, a.n_rot, a.inv_freq);
   a.page_size = m->page_size;
   a.num_pages = m->num_pages;
   a.max_pages = max_pages;
@@ -332,7 +341,7 @@ int spec_verify_attn(const spec_model* m, int layer, const void* q, const void* 
   rc = cuda_status(launch_rope_append(a, B, st));
   if (rc) return rc;
   AttnGeom g = plan_attn(B, qn, m->n_q_heads, m->n_kv_heads, D, m->page_size, m->num_pages,
-                         max_pages, L.window, L.kv_equal, 2 * a.n_rot, m->split_tokens);
+                         max_pages, L.window, L.kv_equal, 2 * a.n_rot, split_of(m, L));
   return cuda_status(launch_attention(g, at<uint16_t>(ws, s.qrot), L.k_pool, L.v_pool, L.ksb_pool,
                                       block_table, seq_lens, at<float>(ws, s.attn_part),
                                       static_cast<uint16_t*>(out), hdr.status, st));
@@ -377,7 +386,7 @@ int spec_verify_step(const spec_model* m, const int32_t* block_table, int max_pa
     return SPEC_EINVAL;
   if (B < 1 || k < 0 || k > SPEC_MAX_K || max_pages < 1 || (k > 0 && !drafts)) return SPEC_EINVAL;
   StepLayout s = step_layout(m, B, k, max_pages);
-  if (s.tickets > kMaxTickets) return SPEC_EUNSUPPORTED;
+  if (s.tickets > kMaxTickets || !s.splits_ok) return SPEC_EUNSUPPORTED;
   if (ws_bytes < s.total) return SPEC_EINVAL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   WsHeader hdr = ws_header(ws);
@@ -389,13 +398,16 @@ int spec_verify_step(const spec_model* m, const int32_t* block_table, int max_pa
   uint16_t* attn_out = at<uint16_t>(ws, s.attn_out);
 
   prof_mark(0, st);
-  rc = cuda_status(launch_embed(m->w_embed, m->vocab, d, last_token, drafts, B, q, x, hdr.status, st));
+  rc = cuda_status(launch_embed_norm(m->w_embed, m->vocab, d, last_token, drafts, B, q, m->rms_eps,
+                                     x, hn, hdr.status, st));
   if (rc) return rc;
   for (int l = 0; l < m->n_layers; ++l) {
     const spec_layer& L = m->layers[l];
     const int nqkv = qkv_out(m, L);
-    rc = cuda_status(launch_rmsnorm(x, M, d, m->rms_eps, hn, st));
-    if (rc) return rc;
+    if (l > 0) {
+      rc = cuda_status(launch_rmsnorm(x, M, d, m->rms_eps, hn, st));
+      if (rc) return rc;
+    }
     GemmPlan pq = plan_gemm(M, nqkv, d, kGemmStore);
     GemmBuffers bq{};
     bq.out = qkv;
@@ -410,7 +422,7 @@ int spec_verify_step(const spec_model* m, const int32_t* block_table, int max_pa
     a.n_kv_heads = m->n_kv_heads;
     a.head_dim = D;
     a.n_rot = n_rot_of(m, L);
-    a.theta = m->rope_theta;
+    rope_inv_freq(m->rope_theta, m->head_dim, a.n_rot, a.inv_freq);
     a.page_size = m->page_size;
     a.num_pages = m->num_pages;
     a.max_pages = max_pages;
@@ -436,7 +448,7 @@ int spec_verify_step(const spec_model* m, const int32_t* block_table, int max_pa
     if (rc) return rc;
 
     AttnGeom g = plan_attn(B, q, m->n_q_heads, m->n_kv_heads, D, m->page_size, m->num_pages,
-                           max_pages, L.window, L.kv_equal, 2 * a.n_rot, m->split_tokens);
+                           max_pages, L.window, L.kv_equal, 2 * a.n_rot, split_of(m, L));
     rc = cuda_status(launch_attention(g, qrot, L.k_pool, L.v_pool, L.ksb_pool, block_table, seq_lens,
                                       at<float>(ws, s.attn_part), attn_out, hdr.status, st));
     if (rc) return rc;

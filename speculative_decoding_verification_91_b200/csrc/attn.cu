@@ -36,16 +36,30 @@ __device__ __forceinline__ float load_src(const void* base, long off, int is_f32
                 : bf16_to_f32(static_cast<const uint16_t*>(base)[off]);
 }
 
+// 2*pi split into three parts for Cody-Waite argument reduction (Cody & Waite,
+// "Software Manual for the Elementary Functions", 1980): the first two have
+// 33 significant bits, so k*C1 and k*C2 are exact for |k| < 2^20 (angles up
+// to ~6.5e6 rad, i.e. positions beyond 10^6 for the fastest pair).
+__device__ __forceinline__ double reduce_2pi(double x) {
+  const double C1 = 0x1.921fb54400000p+2, C2 = 0x1.0b4611a600000p-32, C3 = 0x1.3198a2e037073p-67;
+  const double k = rint(x * 0x1.45f306dc9c883p-3);   // x / (2*pi), rounded
+  double r = fma(-k, C1, x);
+  r = fma(-k, C2, r);
+  return fma(-k, C3, r);
+}
+
 __global__ void __launch_bounds__(256) rope_append_kernel(RopeAppend a) {
   __shared__ float cs[128], sn[128];
   const int i = blockIdx.x, b = blockIdx.y;
   const int D = a.head_dim, half = D / 2, n_rot = a.n_rot;
   const int pos = (a.seq_lens ? a.seq_lens[b] : a.pos0) + i;
   for (int j = threadIdx.x; j < n_rot; j += blockDim.x) {
-    const double inv = pow((double)a.theta, -2.0 * j / D);
-    const double ang = (double)pos * inv;
-    cs[j] = (float)cos(ang);
-    sn[j] = (float)sin(ang);
+    // angle = position * theta_j in double (theta_j from the host), reduced to
+    // [-pi, pi] and rounded to binary32 after the trigonometry
+    double sd, cd;
+    sincos(reduce_2pi((double)pos * a.inv_freq[j]), &sd, &cd);
+    cs[j] = (float)cd;
+    sn[j] = (float)sd;
   }
   __syncthreads();
 
@@ -330,7 +344,7 @@ __global__ void __launch_bounds__(kThreads) attn_split_kernel(
           const int j = key0 + warp * 16 + nt * 8 + 2 * t + (e & 1);
           const int p = rpos[mt][e >> 1];
           const bool vis = valid && p >= 0 && j >= klo && j <= p && (a.window == 0 || j > p - a.window);
-          sc[mt][nt][e] = vis ? sc[mt][nt][e] * a.scale_log2 : -INFINITY;
+          sc[mt][nt][e] = vis ? __fmul_rn(sc[mt][nt][e], a.scale_log2) : -INFINITY;
         }
     // ---- row maxima over this warp's keys
 #pragma unroll
@@ -377,7 +391,7 @@ __global__ void __launch_bounds__(kThreads) attn_split_kernel(
         for (int w = 1; w < kCW; ++w) pm = fmaxf(pm, red_max[w * RP + r]);
         const float mn = fmaxf(m_run[mt][h], pm);
         mnew[mt][h] = mn;
-        alpha[mt][h] = (mn == -INFINITY) ? 1.f : exp2f(m_run[mt][h] - mn);
+        alpha[mt][h] = (mn == -INFINITY) ? 1.f : exp2f(__fsub_rn(m_run[mt][h], mn));
       }
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) {
@@ -388,8 +402,8 @@ __global__ void __launch_bounds__(kThreads) attn_split_kernel(
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float x = sc[mt][nt][e];
-          pv[e] = (x == -INFINITY) ? 0.f : exp2f(x - mnew[mt][e >> 1]);
-          rs[e >> 1] += pv[e];
+          pv[e] = (x == -INFINITY) ? 0.f : exp2f(__fsub_rn(x, mnew[mt][e >> 1]));
+          rs[e >> 1] = __fadd_rn(rs[e >> 1], pv[e]);
         }
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -408,8 +422,8 @@ __global__ void __launch_bounds__(kThreads) attn_split_kernel(
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         float v = rs[h];
-        v += __shfl_xor_sync(0xffffffffu, v, 1);
-        v += __shfl_xor_sync(0xffffffffu, v, 2);
+        v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, 1));
+        v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, 2));
         if (t == 0) red_sum[warp * RP + mt * 16 + g + 8 * h] = v;
       }
     }
@@ -423,8 +437,8 @@ __global__ void __launch_bounds__(kThreads) attn_split_kernel(
         const int r = mt * 16 + g + 8 * h;
         float ps = red_sum[r];
 #pragma unroll
-        for (int w = 1; w < kCW; ++w) ps += red_sum[w * RP + r];
-        l_run[mt][h] = l_run[mt][h] * alpha[mt][h] + ps;
+        for (int w = 1; w < kCW; ++w) ps = __fadd_rn(ps, red_sum[w * RP + r]);
+        l_run[mt][h] = __fadd_rn(__fmul_rn(l_run[mt][h], alpha[mt][h]), ps);
         m_run[mt][h] = mnew[mt][h];
       }
 #pragma unroll
@@ -432,7 +446,7 @@ __global__ void __launch_bounds__(kThreads) attn_split_kernel(
 #pragma unroll
       for (int nt = 0; nt < NTO; ++nt)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) o[mt][nt][e] *= alpha[mt][e >> 1];
+        for (int e = 0; e < 4; ++e) o[mt][nt][e] = __fmul_rn(o[mt][nt][e], alpha[mt][e >> 1]);
     if (valid) {
 #pragma unroll
       for (int kk = 0; kk < kPage / 16; ++kk) {
@@ -495,33 +509,69 @@ __global__ void __launch_bounds__(kThreads) attn_split_kernel(
 }
 
 // out[b][i][h] = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s, s ascending.
+// The split weights are formed in parallel into shared memory; each thread
+// then sums its output dimension over the splits in ascending order.
+constexpr int kMaxCombineSplits = kMaxSplits;
 __global__ void attn_combine_kernel(AttnArgs a, int D, uint16_t* __restrict__ out) {
+  __shared__ float wsh[kMaxCombineSplits];
+  __shared__ float lsh[kMaxCombineSplits];
+  __shared__ float red[32];
+  __shared__ float den_sh;
   const int r = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
-  const int d = threadIdx.x;
+  const int tid = threadIdx.x, nthr = blockDim.x;
   const int L = a.seq_lens[b];
   const int gh = r / a.q, i = r % a.q;
   const int h = kvh * a.G + gh;
   uint16_t* dst = out + (((long)b * a.q + i) * a.Hq + h) * D;
   if (L < 0 || L + a.q > a.max_pages * kPage) {
-    for (int e = d; e < D; e += blockDim.x) dst[e] = 0;
+    for (int e = tid; e < D; e += nthr) dst[e] = 0;
     return;
   }
   int klo, khi;
   seq_key_range(L, a.q, a.window, klo, khi);
-  const int ns = khi / a.split - klo / a.split + 1;
+  const int ns = min(khi / a.split - klo / a.split + 1, kMaxCombineSplits);
   const long slot0 = ((long)(b * a.Hkv + kvh) * a.n_splits_grid) * a.rows + r;
-  float M = -INFINITY;
-  for (int s = 0; s < ns; ++s) M = fmaxf(M, __ldcg(a.part_ml + (slot0 + (long)s * a.rows) * 2));
-  for (int e = d; e < D; e += blockDim.x) {
-    float num = 0.f, den = 0.f;
-    for (int s = 0; s < ns; ++s) {
-      const long sl = slot0 + (long)s * a.rows;
-      const float2 ml = __ldcg(reinterpret_cast<const float2*>(a.part_ml + sl * 2));
-      const float w = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - M);
-      num += w * __ldcg(a.part_o + sl * D + e);
-      den += w * ml.y;
+  float mloc = -INFINITY;
+  for (int s = tid; s < ns; s += nthr) {
+    const float2 ml = __ldcg(reinterpret_cast<const float2*>(a.part_ml + (slot0 + (long)s * a.rows) * 2));
+    wsh[s] = ml.x;
+    lsh[s] = ml.y;
+    mloc = fmaxf(mloc, ml.x);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, off));
+  if ((tid & 31) == 0) red[tid >> 5] = mloc;
+  __syncthreads();
+  float M = red[0];
+  for (int w = 1; w < (nthr + 31) / 32; ++w) M = fmaxf(M, red[w]);
+  for (int s = tid; s < ns; s += nthr) {
+    const float m = wsh[s];
+    wsh[s] = (m == -INFINITY) ? 0.f : exp2f(__fsub_rn(m, M));
+  }
+  __syncthreads();
+  if (tid == 0) {
+    float den = 0.f;
+    for (int s = 0; s < ns; ++s) den = __fadd_rn(den, __fmul_rn(wsh[s], lsh[s]));
+    den_sh = den;
+  }
+  __syncthreads();
+  const float den = den_sh;
+  for (int e = tid; e < D; e += nthr) {
+    const float* po = a.part_o + slot0 * D + e;
+    float num = 0.f;
+    int s = 0;
+    for (; s + 4 <= ns; s += 4) {
+      const float o0 = __ldcg(po + (long)(s + 0) * a.rows * D);
+      const float o1 = __ldcg(po + (long)(s + 1) * a.rows * D);
+      const float o2 = __ldcg(po + (long)(s + 2) * a.rows * D);
+      const float o3 = __ldcg(po + (long)(s + 3) * a.rows * D);
+      num = __fadd_rn(num, __fmul_rn(wsh[s + 0], o0));
+      num = __fadd_rn(num, __fmul_rn(wsh[s + 1], o1));
+      num = __fadd_rn(num, __fmul_rn(wsh[s + 2], o2));
+      num = __fadd_rn(num, __fmul_rn(wsh[s + 3], o3));
     }
-    dst[e] = f32_to_bf16(num / den);
+    for (; s < ns; ++s) num = __fadd_rn(num, __fmul_rn(wsh[s], __ldcg(po + (long)s * a.rows * D)));
+    dst[e] = f32_to_bf16(__fdiv_rn(num, den));
   }
 }
 

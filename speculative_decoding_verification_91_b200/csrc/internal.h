@@ -47,11 +47,14 @@ cudaError_t launch_gemm(const GemmPlan& p, int mode, const void* x, const void* 
                         const GemmBuffers& buf, cudaStream_t st);
 
 // ------------------------------------------------------------- small kernels
-cudaError_t launch_embed(const void* w_emb, int vocab, int d, const int32_t* last_token,
-                         const int32_t* drafts, int B, int q, float* x, unsigned* status,
-                         cudaStream_t st);
-cudaError_t launch_rmsnorm(const float* x, int M, int d, float eps, uint16_t* out,
+cudaError_t launch_rmsnorm(const float* x, int M, int d, double eps, uint16_t* out,
                            cudaStream_t st);
+// embedding gather of [last_token, drafts] into x and its RMSNorm into out
+cudaError_t launch_embed_norm(const void* w_emb, int vocab, int d, const int32_t* last_token,
+                              const int32_t* drafts, int B, int q, double eps, float* x,
+                              uint16_t* out, unsigned* status, cudaStream_t st);
+// host: theta_j = base^(-2j/D) for j < n_rot (n_rot <= 128)
+void rope_inv_freq(double base, int head_dim, int n_rot, double* out);
 cudaError_t launch_accept(const int32_t* drafts, const int32_t* target, int B, int k,
                           int32_t* seq_lens, int32_t* accept_len, int32_t* emitted,
                           int32_t* last_token, int32_t* copy_ids, float* copy_max,
@@ -61,7 +64,7 @@ cudaError_t launch_accept(const int32_t* drafts, const int32_t* target, int B, i
 struct RopeAppend {
   // geometry
   int n_q_heads, n_kv_heads, head_dim, n_rot;   // n_rot rotated pairs
-  float theta;
+  double inv_freq[128];                         // theta_j = base^(-2j/D), j < n_rot
   int page_size, num_pages, max_pages;
   // rows: blockIdx.x = i in [0, n_rows), blockIdx.y = sequence b
   int n_rows;
@@ -83,6 +86,7 @@ struct RopeAppend {
 cudaError_t launch_rope_append(const RopeAppend& a, int B, cudaStream_t st);
 
 // ---------------------------------------------------------- split-KV attention
+constexpr int kMaxSplits = 1024;   // splits one combine can merge
 struct AttnGeom {
   int B, q, n_q_heads, n_kv_heads, head_dim, page_size, num_pages, max_pages;
   int window, kv_equal, sb_width, split_tokens;

@@ -1,5 +1,7 @@
 // Small verify-step kernels: token embedding gather, RMSNorm, and the
 // acceptance / bonus-token / commit kernel.
+#include <cmath>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -7,45 +9,54 @@ namespace sv {
 
 namespace {
 
-// Row m = b*q + i holds token last_token[b] (i = 0) or drafts[b][i-1]; its
-// residual stream starts as that token's embedding row, widened to fp32.
-__global__ void embed_kernel(const uint16_t* __restrict__ w_emb, int vocab, int d,
-                             const int32_t* __restrict__ last_token,
-                             const int32_t* __restrict__ drafts, int q, float* __restrict__ x,
-                             unsigned* status) {
-  const int m = blockIdx.x;
-  const int b = m / q, i = m % q;
-  int tok = (i == 0) ? last_token[b] : drafts[b * (q - 1) + (i - 1)];
-  float* row = x + (size_t)m * d;
-  if (tok < 0 || tok >= vocab) {
-    if (threadIdx.x == 0) flag_status(status, SPEC_DEV_BAD_TOKEN);
-    for (int e = threadIdx.x; e < d; e += blockDim.x) row[e] = 0.f;
-    return;
-  }
-  const uint16_t* src = w_emb + (size_t)tok * d;
-  for (int e = threadIdx.x; e < d; e += blockDim.x) row[e] = bf16_to_f32(src[e]);
-}
-
-// out[m] = bf16(x[m] / sqrt(mean(x[m]^2) + eps)); fixed reduction order.
+// out[m] = bf16(x[m] / sqrt(mean(x[m]^2) + eps)).  The mean, square root and
+// division are float64 (then rounded to binary32 and to bf16), so the
+// normalised GEMM input differs from an exact evaluation only when the
+// float64 result sits within a few ulps of a binary32 rounding boundary.
 constexpr int kNormThreads = 256;
-__global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(const float* __restrict__ x, int d,
-                                                               float eps,
-                                                               uint16_t* __restrict__ out) {
-  __shared__ float red[kNormThreads / 32];
-  const int m = blockIdx.x;
-  const float* row = x + (size_t)m * d;
-  float ss = 0.f;
-  for (int e = threadIdx.x; e < d; e += kNormThreads) ss = __fmaf_rn(row[e], row[e], ss);
+__device__ __forceinline__ void norm_row(const float* __restrict__ row, int d, double eps,
+                                         uint16_t* __restrict__ o, double* red) {
+  double ss = 0.0;
+  for (int e = threadIdx.x; e < d; e += kNormThreads) {
+    const double v = row[e];
+    ss = fma(v, v, ss);
+  }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
   __syncthreads();
-  float tot = 0.f;
+  double tot = 0.0;
 #pragma unroll
   for (int w = 0; w < kNormThreads / 32; ++w) tot += red[w];
-  const float inv = 1.0f / sqrtf(tot / (float)d + eps);
-  uint16_t* o = out + (size_t)m * d;
-  for (int e = threadIdx.x; e < d; e += kNormThreads) o[e] = f32_to_bf16(__fmul_rn(row[e], inv));
+  const double rms = sqrt(tot / (double)d + eps);
+  for (int e = threadIdx.x; e < d; e += kNormThreads)
+    o[e] = f32_to_bf16((float)((double)row[e] / rms));
+}
+
+__global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(const float* __restrict__ x, int d,
+                                                               double eps,
+                                                               uint16_t* __restrict__ out) {
+  __shared__ double red[kNormThreads / 32];
+  const int m = blockIdx.x;
+  norm_row(x + (size_t)m * d, d, eps, out + (size_t)m * d, red);
+}
+
+// Embedding gather fused with the first layer's RMSNorm.
+__global__ void __launch_bounds__(kNormThreads) embed_norm_kernel(
+    const uint16_t* __restrict__ w_emb, int vocab, int d, const int32_t* __restrict__ last_token,
+    const int32_t* __restrict__ drafts, int q, double eps, float* __restrict__ x,
+    uint16_t* __restrict__ out, unsigned* status) {
+  __shared__ double red[kNormThreads / 32];
+  const int m = blockIdx.x;
+  const int b = m / q, i = m % q;
+  const int tok = (i == 0) ? last_token[b] : drafts[b * (q - 1) + (i - 1)];
+  float* row = x + (size_t)m * d;
+  const bool ok = tok >= 0 && tok < vocab;
+  if (!ok && threadIdx.x == 0) flag_status(status, SPEC_DEV_BAD_TOKEN);
+  const uint16_t* src = w_emb + (size_t)(ok ? tok : 0) * d;
+  for (int e = threadIdx.x; e < d; e += kNormThreads) row[e] = ok ? bf16_to_f32(src[e]) : 0.f;
+  __syncthreads();
+  norm_row(row, d, eps, out + (size_t)m * d, red);
 }
 
 // One warp per sequence: a = number of leading drafts equal to the target's
@@ -81,18 +92,22 @@ __global__ void accept_kernel(const int32_t* __restrict__ drafts, const int32_t*
 
 }  // namespace
 
-cudaError_t launch_embed(const void* w_emb, int vocab, int d, const int32_t* last_token,
-                         const int32_t* drafts, int B, int q, float* x, unsigned* status,
-                         cudaStream_t st) {
-  embed_kernel<<<B * q, 256, 0, st>>>(static_cast<const uint16_t*>(w_emb), vocab, d, last_token,
-                                      drafts, q, x, status);
+cudaError_t launch_embed_norm(const void* w_emb, int vocab, int d, const int32_t* last_token,
+                              const int32_t* drafts, int B, int q, double eps, float* x,
+                              uint16_t* out, unsigned* status, cudaStream_t st) {
+  embed_norm_kernel<<<B * q, kNormThreads, 0, st>>>(static_cast<const uint16_t*>(w_emb), vocab, d,
+                                                    last_token, drafts, q, eps, x, out, status);
   return cudaGetLastError();
 }
 
-cudaError_t launch_rmsnorm(const float* x, int M, int d, float eps, uint16_t* out,
+cudaError_t launch_rmsnorm(const float* x, int M, int d, double eps, uint16_t* out,
                            cudaStream_t st) {
   rmsnorm_kernel<<<M, kNormThreads, 0, st>>>(x, d, eps, out);
   return cudaGetLastError();
+}
+
+void rope_inv_freq(double base, int head_dim, int n_rot, double* out) {
+  for (int j = 0; j < n_rot && j < 128; ++j) out[j] = std::pow(base, -2.0 * j / head_dim);
 }
 
 cudaError_t launch_accept(const int32_t* drafts, const int32_t* target, int B, int k,

@@ -28,6 +28,7 @@ class LayerSpec:
     window: int = 0            # 0 = global attention; else sliding window (keys incl. self)
     kv_equal: bool = False     # key-equals-value global layer (V = pre-RoPE K)
     rope_fraction: float = 1.0 # fraction of rotary pairs rotated (highest frequencies first)
+    split_tokens: int = 0      # split-KV chunk of this layer (0: the workload's)
 
 
 @dataclass(frozen=True)
@@ -70,7 +71,7 @@ class Workload:
         return dataclasses.replace(self, **kw)
 
 
-LOCAL1024 = LayerSpec(window=1024, kv_equal=False, rope_fraction=1.0)
+LOCAL1024 = LayerSpec(window=1024, kv_equal=False, rope_fraction=1.0, split_tokens=128)
 GLOBAL_KV = LayerSpec(window=0, kv_equal=True, rope_fraction=0.25)
 GLOBAL_FULL = LayerSpec(window=0, kv_equal=False, rope_fraction=1.0)
 
@@ -82,11 +83,11 @@ WORKLOADS = {
     # Batch 1, 8k context, k=4: sliding-window layer + key-equals-value global layer.
     "b1_ctx8k": Workload("b1_ctx8k", batch=1, k=4, d_model=2560, n_q_heads=16, n_kv_heads=8,
                          head_dim=256, vocab=262144, layers=(LOCAL1024, GLOBAL_KV),
-                         ctx_lo=8192, ctx_hi=8192, accept=("geometric", 0.8)),
+                         ctx_lo=8192, ctx_hi=8192, accept=("geometric", 0.8), split_tokens=512),
     # Batch 8 ragged 4k-32k, global key-equals-value layer only.
     "b8_ragged": Workload("b8_ragged", batch=8, k=4, d_model=5376, n_q_heads=32, n_kv_heads=4,
                           head_dim=256, vocab=262144, layers=(GLOBAL_KV,), ctx_lo=4096,
-                          ctx_hi=32768, accept=("geometric", 0.8)),
+                          ctx_hi=32768, accept=("geometric", 0.8), split_tokens=512),
     # Batch 64, k=3, 5 sliding-window layers + 1 key-equals-value global layer.
     "b64_6layer": Workload("b64_6layer", batch=64, k=3, d_model=3840, n_q_heads=16, n_kv_heads=8,
                            head_dim=256, vocab=262144,
@@ -105,12 +106,14 @@ WORKLOADS = {
 # not a multiple of the 64-token page or the split).
 WORKLOADS.update({
     "small_b1": WORKLOADS["b1_ctx8k"].with_(name="small_b1", vocab=9000, ctx_lo=1500, ctx_hi=1500,
-                                              layers=(LayerSpec(window=300), GLOBAL_KV)),
+                                              layers=(LayerSpec(window=300, split_tokens=128),
+                                                      GLOBAL_KV)),
     "small_ragged": WORKLOADS["b8_ragged"].with_(name="small_ragged", batch=4, d_model=1024,
                                                   vocab=5000, ctx_lo=100, ctx_hi=1400),
     "small_b16": WORKLOADS["b64_6layer"].with_(name="small_b16", batch=16, d_model=768,
                                                 vocab=4100, ctx_lo=60, ctx_hi=900,
-                                                layers=(LayerSpec(window=200),) * 2 + (GLOBAL_KV,)),
+                                                layers=(LayerSpec(window=200, split_tokens=64),) * 2
+                                                + (GLOBAL_KV,)),
     "small_loop": WORKLOADS["loop_131k"].with_(name="small_loop", vocab=6000, d_model=512,
                                                 ctx_lo=700, ctx_hi=700, prompt_tokens=700,
                                                 layers=(LayerSpec(window=128),) * 3 + (GLOBAL_KV,),

@@ -28,6 +28,7 @@ class LayerConfig:
     window: int
     kv_equal: bool
     rope_fraction: float
+    split_tokens: int = 0      # 0: the model's split
 
 
 class DeviceModel:
@@ -65,7 +66,8 @@ class DeviceModel:
                 self.w_qkv[l].data_ptr(), self.w_o[l].data_ptr(), self.k_pool[l].data_ptr(),
                 self.v_pool[l].data_ptr() if self.v_pool[l] is not None else None,
                 self.ksb_pool[l].data_ptr() if self.ksb_pool[l] is not None else None,
-                int(spec.window), int(spec.kv_equal), float(spec.rope_fraction))
+                int(spec.window), int(spec.kv_equal), float(spec.rope_fraction),
+                int(spec.split_tokens))
         self.desc = B.SpecModel(len(self.layers), d_model, n_q_heads, n_kv_heads, head_dim, vocab,
                                 B.SPEC_PAGE_SIZE, num_pages, split_tokens, float(rope_theta),
                                 float(rms_eps), self.w_lm.data_ptr(), self.w_emb.data_ptr(),

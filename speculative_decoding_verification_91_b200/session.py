@@ -28,7 +28,8 @@ class WorkloadSession:
         self.dm = DeviceModel(
             d_model=wl.d_model, n_q_heads=wl.n_q_heads, n_kv_heads=wl.n_kv_heads,
             head_dim=wl.head_dim, vocab=wl.vocab,
-            layers=[LayerConfig(s.window, s.kv_equal, s.rope_fraction) for s in wl.layers],
+            layers=[LayerConfig(s.window, s.kv_equal, s.rope_fraction, s.split_tokens)
+                    for s in wl.layers],
             w_lm_bits=W.lm_head_weight(wl), w_emb_bits=W.embedding_weight(wl),
             layer_weights=layer_w, num_pages=self.num_pages,
             split_tokens=wl.split_tokens, rope_theta=wl.rope_theta, rms_eps=wl.rms_eps,

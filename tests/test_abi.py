@@ -46,7 +46,7 @@ def _model(kv_equal=True, D=256, frac=0.25, num_pages=100, n_layers=1):
     layers = (B.SpecLayer * n_layers)()
     for l in range(n_layers):
         layers[l] = B.SpecLayer(FAKE, FAKE, FAKE, None if kv_equal else FAKE, FAKE if kv_equal else None,
-                                0, int(kv_equal), frac)
+                                0, int(kv_equal), frac, 0)
     m = B.SpecModel(n_layers, 2560, 16, 8, D, 262144, 64, num_pages, 256, 10000.0, 1e-6, FAKE, FAKE,
                     ctypes.cast(layers, ctypes.POINTER(B.SpecLayer)))
     m._keep = layers
