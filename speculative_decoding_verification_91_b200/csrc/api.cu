@@ -472,13 +472,23 @@ int spec_verify_step(const spec_model* m, const int32_t* block_table, int max_pa
   bl.maxv = at<float>(ws, s.maxv);
   bl.tickets = hdr.tickets;
   bl.status = hdr.status;
+  bl.acc.B = B;
+  bl.acc.k = k;
+  bl.acc.drafts = drafts;
+  bl.acc.seq_lens = seq_lens;
+  bl.acc.accept_len = accept_len;
+  bl.acc.emitted = emitted;
+  bl.acc.last_token = new_last_token;
+  bl.acc.copy_ids = target_ids;
+  bl.acc.copy_max = target_maxlogit;
   prof_mark(1, st);
   rc = cuda_status(launch_gemm(pl, kGemmArgmax, hn, m->w_lm, bl, st));
   prof_mark(2, st);
   if (rc) return rc;
-  rc = cuda_status(launch_accept(drafts, at<int32_t>(ws, s.ids), B, k, seq_lens, accept_len,
-                                 emitted, new_last_token, target_ids, target_maxlogit,
-                                 at<float>(ws, s.maxv), st));
+  if (pl.mblocks > 1)   // acceptance is fused into the LM head when all rows share one M-block
+    rc = cuda_status(launch_accept(drafts, at<int32_t>(ws, s.ids), B, k, seq_lens, accept_len,
+                                   emitted, new_last_token, target_ids, target_maxlogit,
+                                   at<float>(ws, s.maxv), st));
   prof_mark(3, st);
   prof_step_done();
   return rc;

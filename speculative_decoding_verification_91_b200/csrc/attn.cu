@@ -48,8 +48,13 @@ __device__ __forceinline__ double reduce_2pi(double x) {
   return fma(-k, C3, r);
 }
 
-__global__ void __launch_bounds__(256) rope_append_kernel(RopeAppend a) {
+// One thread per rotated pair (queries, keys) or value pair; grid (rows,
+// sequences, chunks of 256 work items).
+constexpr int kRopeThreads = 256;
+__global__ void __launch_bounds__(kRopeThreads) rope_append_kernel(RopeAppend a) {
   __shared__ float cs[128], sn[128];
+  pdl_trigger();
+  pdl_wait();
   const int i = blockIdx.x, b = blockIdx.y;
   const int D = a.head_dim, half = D / 2, n_rot = a.n_rot;
   const int pos = (a.seq_lens ? a.seq_lens[b] : a.pos0) + i;
@@ -63,42 +68,44 @@ __global__ void __launch_bounds__(256) rope_append_kernel(RopeAppend a) {
   }
   __syncthreads();
 
-  // queries -> rotated bf16 rows
-  if (a.src_q) {
-    const long base = (long)b * a.q_seq_stride + (long)i * a.q_row_stride;
-    uint16_t* qo = a.q_out + ((long)b * a.n_rows + i) * a.n_q_heads * D;
-    for (int idx = threadIdx.x; idx < a.n_q_heads * half; idx += blockDim.x) {
-      const int h = idx / half, j = idx % half;
-      const float x0 = load_src(a.src_q, base + h * D + j, a.src_is_f32);
-      const float x1 = load_src(a.src_q, base + h * D + j + half, a.src_is_f32);
-      float y0 = x0, y1 = x1;
-      if (j < n_rot) {
-        y0 = __fsub_rn(__fmul_rn(x0, cs[j]), __fmul_rn(x1, sn[j]));
-        y1 = __fadd_rn(__fmul_rn(x0, sn[j]), __fmul_rn(x1, cs[j]));
-      }
-      qo[h * D + j] = f32_to_bf16(y0);
-      qo[h * D + j + half] = f32_to_bf16(y1);
+  const int nq = a.src_q ? a.n_q_heads * half : 0;
+  const int nk = a.n_kv_heads * half;
+  const int nv = a.src_v ? a.n_kv_heads * half : 0;
+  const int idx = blockIdx.z * kRopeThreads + threadIdx.x;
+  if (idx >= nq + nk + nv) return;
+
+  if (idx < nq) {  // query pair (h, j)
+    const int h = idx / half, j = idx % half;
+    const long base = (long)b * a.q_seq_stride + (long)i * a.q_row_stride + (long)h * D;
+    const float x0 = load_src(a.src_q, base + j, a.src_is_f32);
+    const float x1 = load_src(a.src_q, base + j + half, a.src_is_f32);
+    float y0 = x0, y1 = x1;
+    if (j < n_rot) {
+      y0 = __fsub_rn(__fmul_rn(x0, cs[j]), __fmul_rn(x1, sn[j]));
+      y1 = __fadd_rn(__fmul_rn(x0, sn[j]), __fmul_rn(x1, cs[j]));
     }
+    uint16_t* qo = a.q_out + (((long)b * a.n_rows + i) * a.n_q_heads + h) * D;
+    qo[j] = f32_to_bf16(y0);
+    qo[j + half] = f32_to_bf16(y1);
+    return;
   }
 
   // cache slot of this position
   if (pos < 0 || pos / a.page_size >= a.max_pages) {
-    if (threadIdx.x == 0) flag_status(a.status, SPEC_DEV_BAD_LENGTH);
+    if (idx == nq) flag_status(a.status, SPEC_DEV_BAD_LENGTH);
     return;
   }
   const int page = a.block_table[(long)b * a.max_pages + pos / a.page_size];
   if (page < 0 || page >= a.num_pages) {
-    if (threadIdx.x == 0) flag_status(a.status, SPEC_DEV_BAD_PAGE);
+    if (idx == nq) flag_status(a.status, SPEC_DEV_BAD_PAGE);
     return;
   }
   const int slot = pos % a.page_size;
-  const int sbw = 2 * n_rot;
-
-  const long kbase = (long)b * a.k_seq_stride + (long)i * a.k_row_stride;
-  for (int idx = threadIdx.x; idx < a.n_kv_heads * half; idx += blockDim.x) {
-    const int h = idx / half, j = idx % half;
-    const float x0 = load_src(a.src_k, kbase + h * D + j, a.src_is_f32);
-    const float x1 = load_src(a.src_k, kbase + h * D + j + half, a.src_is_f32);
+  if (idx < nq + nk) {  // key pair (h, j), plus the side-band of rotated dims
+    const int h = (idx - nq) / half, j = (idx - nq) % half;
+    const long base = (long)b * a.k_seq_stride + (long)i * a.k_row_stride + (long)h * D;
+    const float x0 = load_src(a.src_k, base + j, a.src_is_f32);
+    const float x1 = load_src(a.src_k, base + j + half, a.src_is_f32);
     float y0 = x0, y1 = x1;
     if (j < n_rot) {
       y0 = __fsub_rn(__fmul_rn(x0, cs[j]), __fmul_rn(x1, sn[j]));
@@ -108,17 +115,19 @@ __global__ void __launch_bounds__(256) rope_append_kernel(RopeAppend a) {
     a.k_pool[row * D + j] = f32_to_bf16(y0);
     a.k_pool[row * D + j + half] = f32_to_bf16(y1);
     if (a.ksb_pool && j < n_rot) {
+      const int sbw = 2 * n_rot;
       a.ksb_pool[row * sbw + j] = f32_to_bf16(x0);
       a.ksb_pool[row * sbw + n_rot + j] = f32_to_bf16(x1);
     }
+    return;
   }
-  if (a.src_v) {
-    const long vbase = (long)b * a.v_seq_stride + (long)i * a.v_row_stride;
-    for (int idx = threadIdx.x; idx < a.n_kv_heads * D; idx += blockDim.x) {
-      const int h = idx / D, e = idx % D;
-      const long row = ((long)page * a.n_kv_heads + h) * a.page_size + slot;
-      a.v_pool[row * D + e] = f32_to_bf16(load_src(a.src_v, vbase + h * D + e, a.src_is_f32));
-    }
+  {  // value pair: elements e, e+1 of head h
+    const int w = idx - nq - nk;
+    const int h = w / half, e = (w % half) * 2;
+    const long base = (long)b * a.v_seq_stride + (long)i * a.v_row_stride + (long)h * D + e;
+    const long row = ((long)page * a.n_kv_heads + h) * a.page_size + slot;
+    a.v_pool[row * D + e] = f32_to_bf16(load_src(a.src_v, base, a.src_is_f32));
+    a.v_pool[row * D + e + 1] = f32_to_bf16(load_src(a.src_v, base + 1, a.src_is_f32));
   }
 }
 
@@ -183,6 +192,8 @@ __global__ void __launch_bounds__(kThreads) attn_split_kernel(
   uint64_t* empty = full + C::kStages;
   volatile int* fail = reinterpret_cast<volatile int*>(empty + C::kStages);
 
+  pdl_trigger();
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.z, kvh = blockIdx.y % a.Hkv, rb = blockIdx.y / a.Hkv;
   const int L = a.seq_lens[b];
@@ -517,6 +528,8 @@ __global__ void attn_combine_kernel(AttnArgs a, int D, uint16_t* __restrict__ ou
   __shared__ float lsh[kMaxCombineSplits];
   __shared__ float red[32];
   __shared__ float den_sh;
+  pdl_trigger();
+  pdl_wait();
   const int r = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, nthr = blockDim.x;
   const int L = a.seq_lens[b];
@@ -582,9 +595,8 @@ cudaError_t launch_split(const AttnGeom& g, const CUtensorMap& tk, const CUtenso
   const int smem = ACfg<D, MT, KVEQ>::kSmem;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(g.n_splits_grid, g.n_kv_heads * g.row_blocks, g.B);
-  kern<<<grid, kThreads, smem, st>>>(tk, tv, a);
-  return cudaGetLastError();
+  return launch_k(kern, dim3(g.n_splits_grid, g.n_kv_heads * g.row_blocks, g.B), dim3(kThreads),
+                  smem, st, tk, tv, a);
 }
 
 template <int D, bool KVEQ>
@@ -603,8 +615,11 @@ cudaError_t launch_mt(int mt, const AttnGeom& g, const CUtensorMap& tk, const CU
 
 cudaError_t launch_rope_append(const RopeAppend& a, int B, cudaStream_t st) {
   if (a.n_rows <= 0 || B <= 0) return cudaSuccess;
-  rope_append_kernel<<<dim3(a.n_rows, B), 256, 0, st>>>(a);
-  return cudaGetLastError();
+  const int half = a.head_dim / 2;
+  const int items = (a.src_q ? a.n_q_heads * half : 0) + a.n_kv_heads * half +
+                    (a.src_v ? a.n_kv_heads * half : 0);
+  return launch_k(rope_append_kernel, dim3(a.n_rows, B, (items + kRopeThreads - 1) / kRopeThreads),
+                  dim3(kRopeThreads), 0, st, a);
 }
 
 AttnGeom plan_attn(int B, int q, int Hq, int Hkv, int D, int page, int num_pages, int max_pages,
@@ -682,9 +697,8 @@ cudaError_t launch_attention(const AttnGeom& g, const uint16_t* qrot, const void
     return cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) return e;
-  attn_combine_kernel<<<dim3(g.rows, g.n_kv_heads, g.B), std::min(g.head_dim, 256), 0, st>>>(
-      a, g.head_dim, out);
-  return cudaGetLastError();
+  return launch_k(attn_combine_kernel, dim3(g.rows, g.n_kv_heads, g.B),
+                  dim3(std::min(g.head_dim, 256)), 0, st, a, g.head_dim, out);
 }
 
 }  // namespace sv

@@ -1,13 +1,16 @@
 // Streaming skinny GEMM for the verify step: Y = X . W^T where X holds the
 // few verify rows (M = B*(k+1), tens of rows) and W is a large bf16 weight
 // matrix read once from HBM.  Used for the QKV projection, the output
-// projection (+ residual) and the tied LM head with a fused argmax.
+// projection (+ residual) and the LM head with a fused argmax (and, when all
+// rows fit one M-block, the acceptance of every sequence).
 //
 // Design (sm_100a):
 //   * one producer warp issues TMA tile loads (W box 128 rows x 64 k, X box
 //     (8*NT) rows x 64 k, both 128-byte swizzled) into a ring of stages
 //     guarded by mbarriers; W uses an evict-first L2 policy (read once), X
-//     evict-last (re-read by every CTA);
+//     evict-last (re-read by every CTA).  W does not depend on earlier
+//     kernels, so the first ring of W tiles is requested before the
+//     programmatic-launch wait and overlaps the previous kernel's tail;
 //   * four consumer warps each own 32 W rows of the 128-row tile and all
 //     M-block rows: swap-AB mma.sync m16n8k16 (W rows are the MMA's M side,
 //     the verify rows its N side), fp32 accumulators in registers;
@@ -52,7 +55,28 @@ struct Args {
   float* maxv;
   unsigned* tickets;
   unsigned* status;
+  AcceptFuse acc;   // acc.B > 0: the argmax's last CTA also runs the acceptance
 };
+
+// Acceptance of sequence b from the argmax ids of its k+1 rows (one warp).
+__device__ __forceinline__ void accept_one(const AcceptFuse& f, int b, const int32_t* tg, int lane) {
+  const int k = f.k, q = k + 1;
+  const bool match = lane < k && f.drafts[(size_t)b * k + lane] == tg[lane];
+  const unsigned mism = ~__ballot_sync(0xffffffffu, match);   // bit i: draft i not accepted
+  const int a = min(__ffs(mism) - 1, k);
+  if (lane < q) {
+    int v = -1;
+    if (lane < a) v = f.drafts[(size_t)b * k + lane];
+    else if (lane == a) v = tg[a];
+    f.emitted[(size_t)b * q + lane] = v;
+  }
+  __syncwarp();
+  if (lane == 0) {
+    f.accept_len[b] = a;
+    f.last_token[b] = tg[a];
+    f.seq_lens[b] += a + 1;
+  }
+}
 
 template <int NT, int MODE>
 __global__ void __launch_bounds__(kThreads) stream_gemm_kernel(
@@ -69,6 +93,7 @@ __global__ void __launch_bounds__(kThreads) stream_gemm_kernel(
   int* flag = red_i + kConsumerWarps * MP;
   volatile int* fail = flag + 1;  // set by any consumer warp whose wait ran out
 
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_tile = blockIdx.x, split = blockIdx.y, mblk = blockIdx.z;
   const int m0 = mblk * kMBlock;
@@ -93,10 +118,20 @@ __global__ void __launch_bounds__(kThreads) stream_gemm_kernel(
       prefetch_tmap(&tx);
       const uint64_t pol_w = policy_evict_first();
       const uint64_t pol_x = policy_evict_last();
-      int issued = 0;
-      for (int it = 0; it < nk; ++it) {
+      const int pre = min(nk, C::kStages);
+      for (int it = 0; it < pre; ++it) {   // weights only: independent of earlier kernels
+        mbar_arrive_expect_tx(&full[it], C::kStageBytes);
+        tma_load_2d(smem + it * C::kStageBytes, &tw, &full[it], (kc0 + it) * kTileK,
+                    n_tile * kTileN, pol_w);
+      }
+      pdl_wait();
+      for (int it = 0; it < pre; ++it)
+        tma_load_2d(smem + it * C::kStageBytes + C::kWBytes, &tx, &full[it], (kc0 + it) * kTileK, m0,
+                    pol_x);
+      int issued = pre;
+      for (int it = pre; it < nk; ++it) {
         const int s = it % C::kStages;
-        if (it >= C::kStages && !mbar_wait(&empty[s], ((it / C::kStages) - 1) & 1, a.status)) break;
+        if (!mbar_wait(&empty[s], ((it / C::kStages) - 1) & 1, a.status)) break;
         uint8_t* st = smem + s * C::kStageBytes;
         mbar_arrive_expect_tx(&full[s], C::kStageBytes);
         const int kx = (kc0 + it) * kTileK;
@@ -219,13 +254,15 @@ __global__ void __launch_bounds__(kThreads) stream_gemm_kernel(
     named_bar(1, kConsumerWarps * 32);
     if (!*flag) return;
     __threadfence();
-    // ---- last CTA of this M-block: reduce over all tiles, lowest index wins ties
+    // ---- last CTA of this M-block: each warp reduces whole rows over all
+    //      tiles (lanes stride the tiles), lowest index wins ties
     const int mcount = min(kMBlock, a.M - m0);
-    for (int mm = 0; mm < mcount; ++mm) {
+    int* ids_s = red_i;   // reused: final ids of this block's rows (mcount <= MP)
+    for (int mm = warp; mm < mcount; mm += kConsumerWarps) {
       const int m = m0 + mm;
       float bv = -INFINITY;
       int bi = 0x7fffffff;
-      for (int tile = ctid; tile < a.n_tiles; tile += kConsumerWarps * 32) {
+      for (int tile = lane; tile < a.n_tiles; tile += 32) {
         const float v = __ldcg(&a.arg_val[(size_t)tile * a.M + m]);
         const int i = __ldcg(&a.arg_idx[(size_t)tile * a.M + m]);
         if (better(v, i, bv, bi)) {
@@ -243,22 +280,19 @@ __global__ void __launch_bounds__(kThreads) stream_gemm_kernel(
         }
       }
       if (lane == 0) {
-        red_v[warp] = bv;
-        red_i[warp] = bi;
-      }
-      named_bar(1, kConsumerWarps * 32);
-      if (ctid == 0) {
-        for (int w = 1; w < kConsumerWarps; ++w)
-          if (better(red_v[w], red_i[w], bv, bi)) {
-            bv = red_v[w];
-            bi = red_i[w];
-          }
         a.ids[m] = bi;
         if (a.maxv) a.maxv[m] = bv;
+        ids_s[mm] = bi;
+        if (a.acc.copy_ids) a.acc.copy_ids[m] = bi;
+        if (a.acc.copy_max) a.acc.copy_max[m] = bv;
       }
-      named_bar(1, kConsumerWarps * 32);
     }
     if (ctid == 0) a.tickets[mblk] = 0u;
+    if (a.acc.B > 0) {                 // all rows are in this block (M <= 64)
+      named_bar(1, kConsumerWarps * 32);
+      for (int b = warp; b < a.acc.B; b += kConsumerWarps)
+        accept_one(a.acc, b, ids_s + b * (a.acc.k + 1), lane);
+    }
     return;
   }
 
@@ -334,9 +368,7 @@ cudaError_t launch_nt(const GemmPlan& p, const CUtensorMap& tw, const CUtensorMa
   const int smem = Cfg<NT>::kSmem;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.n_tiles, p.splits, p.mblocks);
-  kern<<<grid, kThreads, smem, st>>>(tw, tx, a);
-  return cudaGetLastError();
+  return launch_k(kern, dim3(p.n_tiles, p.splits, p.mblocks), dim3(kThreads), smem, st, tw, tx, a);
 }
 
 template <int MODE>
@@ -404,6 +436,8 @@ cudaError_t launch_gemm(const GemmPlan& p, int mode, const void* x, const void* 
   a.maxv = b.maxv;
   a.tickets = b.tickets;
   a.status = b.status;
+  a.acc = b.acc;
+  if (mode != kGemmArgmax || p.mblocks != 1) a.acc.B = 0;
   switch (mode) {
     case kGemmStore: return launch_mode<kGemmStore>(p, tw, tx, a, st);
     case kGemmResidual: return launch_mode<kGemmResidual>(p, tw, tx, a, st);

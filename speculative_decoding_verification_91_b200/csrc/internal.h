@@ -33,6 +33,18 @@ size_t gemm_partial_floats(const GemmPlan& p);   // split-K partial sums
 size_t gemm_argmax_entries(const GemmPlan& p);   // per-tile argmax partials
 int gemm_tickets(const GemmPlan& p);
 
+// Acceptance fused into the LM-head argmax (B = 0: not fused).
+struct AcceptFuse {
+  int B = 0, k = 0;
+  const int32_t* drafts = nullptr;   // [B][k]
+  int32_t* seq_lens = nullptr;
+  int32_t* accept_len = nullptr;
+  int32_t* emitted = nullptr;        // [B][k+1]
+  int32_t* last_token = nullptr;
+  int32_t* copy_ids = nullptr;       // optional copies of every row's argmax / logit
+  float* copy_max = nullptr;
+};
+
 struct GemmBuffers {
   float* out;          // kGemmStore: [M][N]; kGemmResidual: [M][N] updated in place
   float* partial;      // gemm_partial_floats()
@@ -42,6 +54,7 @@ struct GemmBuffers {
   float* maxv;         // kGemmArgmax: [M] or null
   unsigned* tickets;   // gemm_tickets() counters, zero on entry, zero on exit
   unsigned* status;
+  AcceptFuse acc;      // kGemmArgmax with a single M-block only
 };
 cudaError_t launch_gemm(const GemmPlan& p, int mode, const void* x, const void* w,
                         const GemmBuffers& buf, cudaStream_t st);

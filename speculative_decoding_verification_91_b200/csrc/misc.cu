@@ -1,6 +1,7 @@
 // Small verify-step kernels: token embedding gather, RMSNorm, and the
 // acceptance / bonus-token / commit kernel.
 #include <cmath>
+#include <cstdlib>
 
 #include "common.cuh"
 #include "internal.h"
@@ -37,6 +38,8 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(const float* __re
                                                                double eps,
                                                                uint16_t* __restrict__ out) {
   __shared__ double red[kNormThreads / 32];
+  pdl_trigger();
+  pdl_wait();
   const int m = blockIdx.x;
   norm_row(x + (size_t)m * d, d, eps, out + (size_t)m * d, red);
 }
@@ -47,6 +50,8 @@ __global__ void __launch_bounds__(kNormThreads) embed_norm_kernel(
     const int32_t* __restrict__ drafts, int q, double eps, float* __restrict__ x,
     uint16_t* __restrict__ out, unsigned* status) {
   __shared__ double red[kNormThreads / 32];
+  pdl_trigger();
+  pdl_wait();
   const int m = blockIdx.x;
   const int b = m / q, i = m % q;
   const int tok = (i == 0) ? last_token[b] : drafts[b * (q - 1) + (i - 1)];
@@ -66,6 +71,8 @@ __global__ void accept_kernel(const int32_t* __restrict__ drafts, const int32_t*
                               int B, int k, int32_t* seq_lens, int32_t* accept_len,
                               int32_t* emitted, int32_t* last_token, int32_t* copy_ids,
                               float* copy_max, const float* maxv) {
+  pdl_trigger();
+  pdl_wait();
   const int b = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (b >= B) return;
@@ -95,15 +102,22 @@ __global__ void accept_kernel(const int32_t* __restrict__ drafts, const int32_t*
 cudaError_t launch_embed_norm(const void* w_emb, int vocab, int d, const int32_t* last_token,
                               const int32_t* drafts, int B, int q, double eps, float* x,
                               uint16_t* out, unsigned* status, cudaStream_t st) {
-  embed_norm_kernel<<<B * q, kNormThreads, 0, st>>>(static_cast<const uint16_t*>(w_emb), vocab, d,
-                                                    last_token, drafts, q, eps, x, out, status);
-  return cudaGetLastError();
+  return launch_k(embed_norm_kernel, dim3(B * q), dim3(kNormThreads), 0, st,
+                  static_cast<const uint16_t*>(w_emb), vocab, d, last_token, drafts, q, eps, x, out,
+                  status);
 }
 
 cudaError_t launch_rmsnorm(const float* x, int M, int d, double eps, uint16_t* out,
                            cudaStream_t st) {
-  rmsnorm_kernel<<<M, kNormThreads, 0, st>>>(x, d, eps, out);
-  return cudaGetLastError();
+  return launch_k(rmsnorm_kernel, dim3(M), dim3(kNormThreads), 0, st, x, d, eps, out);
+}
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* v = getenv("SPECVERIFY_NO_PDL");
+    return !(v && v[0] == '1');
+  }();
+  return on;
 }
 
 void rope_inv_freq(double base, int head_dim, int n_rot, double* out) {
@@ -115,9 +129,8 @@ cudaError_t launch_accept(const int32_t* drafts, const int32_t* target, int B, i
                           int32_t* last_token, int32_t* copy_ids, float* copy_max,
                           const float* maxv, cudaStream_t st) {
   const int warps = 4;
-  accept_kernel<<<(B + warps - 1) / warps, warps * 32, 0, st>>>(
-      drafts, target, B, k, seq_lens, accept_len, emitted, last_token, copy_ids, copy_max, maxv);
-  return cudaGetLastError();
+  return launch_k(accept_kernel, dim3((B + warps - 1) / warps), dim3(warps * 32), 0, st, drafts,
+                  target, B, k, seq_lens, accept_len, emitted, last_token, copy_ids, copy_max, maxv);
 }
 
 }  // namespace sv

@@ -247,7 +247,7 @@ def test_step_is_invariant_to_k(name):
     same argmax logits and the same cache entries (fixed split boundaries,
     M-independent reduction orders)."""
     base = W.get_workload(name)
-    g0 = WorkloadSession(base.with_(k=0))
+    g0 = WorkloadSession(base.with_(k=0), extra_tokens=8)      # pages for three k=0 steps
     Bn = base.batch
     last = np.array([W.last_token(base, b, 0) for b in range(Bn)], dtype=np.int32)
     tokens, maxes = [], []
@@ -266,6 +266,7 @@ def test_step_is_invariant_to_k(name):
     s8.set_inputs(last, drafts)
     s8.step()
     o8 = s8.outputs()
+    assert g0.ws.device_status() == 0 and s8.ws.device_status() == 0
     for b in range(Bn):
         assert o8["accept_len"][b] >= 3
         for i in range(3):
