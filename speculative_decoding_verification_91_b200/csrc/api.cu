@@ -98,7 +98,8 @@ int check_model(const spec_model* m) {
 
 // Workspace layout of one verify step for (B, k, max_pages).
 struct StepLayout {
-  size_t x, hn, qkv, qrot, attn_out, attn_part, gemm_part, arg_val, arg_idx, ids, maxv, total;
+  size_t x, hn, qrot, attn_out, attn_part, gemm_part, arg_val, arg_idx, ids, maxv, rope_tab,
+      total;
   int tickets;
   bool splits_ok;   // every layer's split count fits the combine kernel
 };
@@ -107,17 +108,15 @@ StepLayout step_layout(const spec_model* m, int B, int k, int max_pages) {
   StepLayout s{};
   s.splits_ok = true;
   const int q = k + 1, M = B * q, d = m->d_model, D = m->head_dim;
-  int nqkv = 0;
   size_t attn_floats = 0, gemm_floats = 0;
   int tickets = 0;
   for (int l = 0; l < m->n_layers; ++l) {
     const spec_layer& L = m->layers[l];
-    nqkv = std::max(nqkv, qkv_out(m, L));
     AttnGeom g = plan_attn(B, q, m->n_q_heads, m->n_kv_heads, D, m->page_size, m->num_pages,
                            max_pages, L.window, L.kv_equal, 2 * n_rot_of(m, L), split_of(m, L));
     attn_floats = std::max(attn_floats, attn_partial_floats(g));
     if (g.n_splits_grid > kMaxSplits) s.splits_ok = false;
-    GemmPlan pq = plan_gemm(M, qkv_out(m, L), d, kGemmStore);
+    GemmPlan pq = plan_gemm(M, qkv_out(m, L), d, kGemmQkvRope);
     GemmPlan po = plan_gemm(M, d, m->n_q_heads * D, kGemmResidual);
     gemm_floats = std::max({gemm_floats, gemm_partial_floats(pq), gemm_partial_floats(po)});
     tickets = std::max({tickets, gemm_tickets(pq), gemm_tickets(po)});
@@ -127,7 +126,6 @@ StepLayout step_layout(const spec_model* m, int B, int k, int max_pages) {
   size_t off = kWsHeaderBytes;
   s.x = off;         off = up(off + (size_t)M * d * 4);
   s.hn = off;        off = up(off + (size_t)M * d * 2);
-  s.qkv = off;       off = up(off + (size_t)M * nqkv * 4);
   s.qrot = off;      off = up(off + (size_t)M * m->n_q_heads * D * 2);
   s.attn_out = off;  off = up(off + (size_t)M * m->n_q_heads * D * 2);
   s.attn_part = off; off = up(off + attn_floats * 4);
@@ -136,6 +134,7 @@ StepLayout step_layout(const spec_model* m, int B, int k, int max_pages) {
   s.arg_idx = off;   off = up(off + gemm_argmax_entries(pl) * 4);
   s.ids = off;       off = up(off + (size_t)M * 4);
   s.maxv = off;      off = up(off + (size_t)M * 4);
+  s.rope_tab = off;  off = up(off + (size_t)M * (D / 2) * 8);
   s.total = off;
   s.tickets = tickets;
   return s;
@@ -393,13 +392,15 @@ int spec_verify_step(const spec_model* m, const int32_t* block_table, int max_pa
   const int q = k + 1, M = B * q, d = m->d_model, D = m->head_dim;
   float* x = at<float>(ws, s.x);
   uint16_t* hn = at<uint16_t>(ws, s.hn);
-  float* qkv = at<float>(ws, s.qkv);
   uint16_t* qrot = at<uint16_t>(ws, s.qrot);
   uint16_t* attn_out = at<uint16_t>(ws, s.attn_out);
 
   prof_mark(0, st);
+  double inv_freq[128];
+  rope_inv_freq(m->rope_theta, D, D / 2, inv_freq);
+  float2* rope_tab = at<float2>(ws, s.rope_tab);
   rc = cuda_status(launch_embed_norm(m->w_embed, m->vocab, d, last_token, drafts, B, q, m->rms_eps,
-                                     x, hn, hdr.status, st));
+                                     x, hn, hdr.status, seq_lens, inv_freq, D / 2, rope_tab, st));
   if (rc) return rc;
   for (int l = 0; l < m->n_layers; ++l) {
     const spec_layer& L = m->layers[l];
@@ -408,47 +409,32 @@ int spec_verify_step(const spec_model* m, const int32_t* block_table, int max_pa
       rc = cuda_status(launch_rmsnorm(x, M, d, m->rms_eps, hn, st));
       if (rc) return rc;
     }
-    GemmPlan pq = plan_gemm(M, nqkv, d, kGemmStore);
+    // QKV projection with RoPE and the cache append in its epilogue
+    GemmPlan pq = plan_gemm(M, nqkv, d, kGemmQkvRope);
     GemmBuffers bq{};
-    bq.out = qkv;
     bq.partial = at<float>(ws, s.gemm_part);
     bq.tickets = hdr.tickets;
     bq.status = hdr.status;
-    rc = cuda_status(launch_gemm(pq, kGemmStore, hn, L.w_qkv, bq, st));
+    RopeFuse& f = bq.rope;
+    f.n_q_heads = m->n_q_heads;
+    f.n_kv_heads = m->n_kv_heads;
+    f.head_dim = D;
+    f.n_rot = n_rot_of(m, L);
+    f.q = q;
+    f.page_size = m->page_size;
+    f.num_pages = m->num_pages;
+    f.max_pages = max_pages;
+    f.seq_lens = seq_lens;
+    f.block_table = block_table;
+    f.rope_tab = rope_tab;
+    f.q_out = qrot;
+    f.k_pool = static_cast<uint16_t*>(L.k_pool);
+    f.v_pool = static_cast<uint16_t*>(L.v_pool);
+    f.ksb_pool = static_cast<uint16_t*>(L.ksb_pool);
+    rc = cuda_status(launch_gemm(pq, kGemmQkvRope, hn, L.w_qkv, bq, st));
     if (rc) return rc;
-
-    RopeAppend a{};
-    a.n_q_heads = m->n_q_heads;
-    a.n_kv_heads = m->n_kv_heads;
-    a.head_dim = D;
-    a.n_rot = n_rot_of(m, L);
-    rope_inv_freq(m->rope_theta, m->head_dim, a.n_rot, a.inv_freq);
-    a.page_size = m->page_size;
-    a.num_pages = m->num_pages;
-    a.max_pages = max_pages;
-    a.n_rows = q;
-    a.seq_lens = seq_lens;
-    a.block_table = block_table;
-    a.src_is_f32 = 1;
-    a.src_q = qkv;
-    a.q_row_stride = nqkv;
-    a.q_seq_stride = (long)nqkv * q;
-    a.src_k = qkv + (size_t)m->n_q_heads * D;
-    a.k_row_stride = nqkv;
-    a.k_seq_stride = (long)nqkv * q;
-    a.src_v = L.kv_equal ? nullptr : qkv + (size_t)(m->n_q_heads + m->n_kv_heads) * D;
-    a.v_row_stride = nqkv;
-    a.v_seq_stride = (long)nqkv * q;
-    a.q_out = qrot;
-    a.k_pool = static_cast<uint16_t*>(L.k_pool);
-    a.v_pool = static_cast<uint16_t*>(L.v_pool);
-    a.ksb_pool = static_cast<uint16_t*>(L.ksb_pool);
-    a.status = hdr.status;
-    rc = cuda_status(launch_rope_append(a, B, st));
-    if (rc) return rc;
-
     AttnGeom g = plan_attn(B, q, m->n_q_heads, m->n_kv_heads, D, m->page_size, m->num_pages,
-                           max_pages, L.window, L.kv_equal, 2 * a.n_rot, split_of(m, L));
+                           max_pages, L.window, L.kv_equal, 2 * f.n_rot, split_of(m, L));
     rc = cuda_status(launch_attention(g, qrot, L.k_pool, L.v_pool, L.ksb_pool, block_table, seq_lens,
                                       at<float>(ws, s.attn_part), attn_out, hdr.status, st));
     if (rc) return rc;

@@ -36,18 +36,6 @@ __device__ __forceinline__ float load_src(const void* base, long off, int is_f32
                 : bf16_to_f32(static_cast<const uint16_t*>(base)[off]);
 }
 
-// 2*pi split into three parts for Cody-Waite argument reduction (Cody & Waite,
-// "Software Manual for the Elementary Functions", 1980): the first two have
-// 33 significant bits, so k*C1 and k*C2 are exact for |k| < 2^20 (angles up
-// to ~6.5e6 rad, i.e. positions beyond 10^6 for the fastest pair).
-__device__ __forceinline__ double reduce_2pi(double x) {
-  const double C1 = 0x1.921fb54400000p+2, C2 = 0x1.0b4611a600000p-32, C3 = 0x1.3198a2e037073p-67;
-  const double k = rint(x * 0x1.45f306dc9c883p-3);   // x / (2*pi), rounded
-  double r = fma(-k, C1, x);
-  r = fma(-k, C2, r);
-  return fma(-k, C3, r);
-}
-
 // One thread per rotated pair (queries, keys) or value pair; grid (rows,
 // sequences, chunks of 256 work items).
 constexpr int kRopeThreads = 256;
@@ -61,10 +49,9 @@ __global__ void __launch_bounds__(kRopeThreads) rope_append_kernel(RopeAppend a)
   for (int j = threadIdx.x; j < n_rot; j += blockDim.x) {
     // angle = position * theta_j in double (theta_j from the host), reduced to
     // [-pi, pi] and rounded to binary32 after the trigonometry
-    double sd, cd;
-    sincos(reduce_2pi((double)pos * a.inv_freq[j]), &sd, &cd);
-    cs[j] = (float)cd;
-    sn[j] = (float)sd;
+    const float2 c = rope_cs(pos, a.inv_freq[j]);
+    cs[j] = c.x;
+    sn[j] = c.y;
   }
   __syncthreads();
 
@@ -150,7 +137,11 @@ struct ACfg {
   static constexpr int kPBytes = 2 * kRowsPad * 128;   // P = P_hi + P_lo, both bf16
   static constexpr int kRedBytes = 2 * kCW * kRowsPad * 4;
   static constexpr int kFixed = 1024 + kQBytes + kPBytes + kRedBytes + 256;
-  static constexpr int kStagesRaw = (kSmemBudget - kFixed) / kStageBytes;
+  // Prefer a footprint that lets two CTAs share an SM (two pages in flight
+  // per SM hide the per-page latency chain); else use the whole budget.
+  static constexpr int kStagesHalf = (kSmemBudget / 2 - 1024 - kFixed) / kStageBytes;
+  static constexpr int kStagesRaw =
+      kStagesHalf >= 2 ? kStagesHalf : (kSmemBudget - kFixed) / kStageBytes;
   static constexpr int kStages = kStagesRaw > 4 ? 4 : kStagesRaw;
   static constexpr int kSmem = kFixed + kStages * kStageBytes;
   static_assert(kStages >= 2, "attention tile does not fit in shared memory");

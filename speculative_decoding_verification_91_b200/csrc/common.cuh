@@ -186,6 +186,32 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
+// 2*pi split into three parts for Cody-Waite argument reduction (Cody & Waite,
+// "Software Manual for the Elementary Functions", 1980): the first two have
+// 33 significant bits, so k*C1 and k*C2 are exact for |k| < 2^20 (angles up
+// to ~6.5e6 rad, i.e. positions beyond 10^6 for the fastest pair).
+__device__ __forceinline__ double reduce_2pi(double x) {
+  const double C1 = 0x1.921fb54400000p+2, C2 = 0x1.0b4611a600000p-32, C3 = 0x1.3198a2e037073p-67;
+  const double k = rint(x * 0x1.45f306dc9c883p-3);   // x / (2*pi), rounded
+  double r = fma(-k, C1, x);
+  r = fma(-k, C2, r);
+  return fma(-k, C3, r);
+}
+
+// (cos, sin) of position * theta in double, rounded to binary32.
+__device__ __forceinline__ float2 rope_cs(int pos, double theta) {
+  double sd, cd;
+  sincos(reduce_2pi((double)pos * theta), &sd, &cd);
+  return make_float2((float)cd, (float)sd);
+}
+
+// Rotate the pair (x0, x1) = (dim j, dim j + D/2) by (c, s) in binary32 with
+// every product and sum rounded on its own.
+__device__ __forceinline__ void rope_pair(float x0, float x1, float c, float s, float& y0, float& y1) {
+  y0 = __fsub_rn(__fmul_rn(x0, c), __fmul_rn(x1, s));
+  y1 = __fadd_rn(__fmul_rn(x0, s), __fmul_rn(x1, c));
+}
+
 // Argmax candidate order: larger value wins; equal values -> lower index.
 __device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
   return v > bv || (v == bv && i < bi);
@@ -210,5 +236,10 @@ cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
   cfg.numAttrs = pdl_enabled() ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
+
+// Fixed-size copy of the host theta table into a kernel parameter.
+struct InvFreq {
+  double v[128];
+};
 
 }  // namespace sv

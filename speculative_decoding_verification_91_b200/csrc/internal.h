@@ -18,7 +18,7 @@ bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64
 // --------------------------------------------------------- streaming GEMM
 // Y = X . W^T with X [M][K] bf16 (row-major), W [N][K] bf16 (row-major),
 // fp32 accumulation, W streamed once per M-block by TMA.
-enum GemmMode { kGemmStore = 0, kGemmResidual = 1, kGemmArgmax = 2 };
+enum GemmMode { kGemmStore = 0, kGemmResidual = 1, kGemmArgmax = 2, kGemmQkvRope = 3 };
 
 struct GemmPlan {
   int M, N, K;
@@ -45,6 +45,21 @@ struct AcceptFuse {
   float* copy_max = nullptr;
 };
 
+// RoPE + cache append fused into the QKV projection's epilogue: the last CTA
+// to finish a head (all its splits and column tiles) rotates each pair and
+// writes queries (workspace), keys / values / side-band (cache pools).
+struct RopeFuse {
+  int n_q_heads = 0, n_kv_heads = 0, head_dim = 0, n_rot = 0, q = 0;
+  int page_size = 0, num_pages = 0, max_pages = 0;
+  const int32_t* seq_lens = nullptr;
+  const int32_t* block_table = nullptr;
+  const float2* rope_tab = nullptr;  // [M][head_dim/2] (cos, sin) of each row's position
+  uint16_t* q_out = nullptr;         // [M][Hq][D]
+  uint16_t* k_pool = nullptr;
+  uint16_t* v_pool = nullptr;        // null on key-equals-value layers
+  uint16_t* ksb_pool = nullptr;      // key-equals-value side-band
+};
+
 struct GemmBuffers {
   float* out;          // kGemmStore: [M][N]; kGemmResidual: [M][N] updated in place
   float* partial;      // gemm_partial_floats()
@@ -55,6 +70,7 @@ struct GemmBuffers {
   unsigned* tickets;   // gemm_tickets() counters, zero on entry, zero on exit
   unsigned* status;
   AcceptFuse acc;      // kGemmArgmax with a single M-block only
+  RopeFuse rope;       // kGemmQkvRope
 };
 cudaError_t launch_gemm(const GemmPlan& p, int mode, const void* x, const void* w,
                         const GemmBuffers& buf, cudaStream_t st);
@@ -62,10 +78,13 @@ cudaError_t launch_gemm(const GemmPlan& p, int mode, const void* x, const void* 
 // ------------------------------------------------------------- small kernels
 cudaError_t launch_rmsnorm(const float* x, int M, int d, double eps, uint16_t* out,
                            cudaStream_t st);
-// embedding gather of [last_token, drafts] into x and its RMSNorm into out
+// embedding gather of [last_token, drafts] into x and its RMSNorm into out;
+// also the (cos, sin) table of every row's position for pairs j < half
+// (rope_tab [B*q][half], theta_j = inv_freq[j]); rope_tab may be null
 cudaError_t launch_embed_norm(const void* w_emb, int vocab, int d, const int32_t* last_token,
                               const int32_t* drafts, int B, int q, double eps, float* x,
-                              uint16_t* out, unsigned* status, cudaStream_t st);
+                              uint16_t* out, unsigned* status, const int32_t* seq_lens,
+                              const double* inv_freq, int half, float2* rope_tab, cudaStream_t st);
 // host: theta_j = base^(-2j/D) for j < n_rot (n_rot <= 128)
 void rope_inv_freq(double base, int head_dim, int n_rot, double* out);
 cudaError_t launch_accept(const int32_t* drafts, const int32_t* target, int B, int k,

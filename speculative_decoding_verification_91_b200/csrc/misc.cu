@@ -44,16 +44,23 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(const float* __re
   norm_row(x + (size_t)m * d, d, eps, out + (size_t)m * d, red);
 }
 
-// Embedding gather fused with the first layer's RMSNorm.
+// Embedding gather fused with the first layer's RMSNorm and with the
+// (cos, sin) table of the row's position for every rotary pair.
 __global__ void __launch_bounds__(kNormThreads) embed_norm_kernel(
     const uint16_t* __restrict__ w_emb, int vocab, int d, const int32_t* __restrict__ last_token,
     const int32_t* __restrict__ drafts, int q, double eps, float* __restrict__ x,
-    uint16_t* __restrict__ out, unsigned* status) {
+    uint16_t* __restrict__ out, unsigned* status, const int32_t* __restrict__ seq_lens,
+    InvFreq inv_freq, int half, float2* __restrict__ rope_tab) {
   __shared__ double red[kNormThreads / 32];
   pdl_trigger();
   pdl_wait();
   const int m = blockIdx.x;
   const int b = m / q, i = m % q;
+  if (rope_tab) {
+    const int pos = seq_lens[b] + i;
+    for (int j = threadIdx.x; j < half; j += kNormThreads)
+      rope_tab[(size_t)m * half + j] = rope_cs(pos, inv_freq.v[j]);
+  }
   const int tok = (i == 0) ? last_token[b] : drafts[b * (q - 1) + (i - 1)];
   float* row = x + (size_t)m * d;
   const bool ok = tok >= 0 && tok < vocab;
@@ -101,10 +108,13 @@ __global__ void accept_kernel(const int32_t* __restrict__ drafts, const int32_t*
 
 cudaError_t launch_embed_norm(const void* w_emb, int vocab, int d, const int32_t* last_token,
                               const int32_t* drafts, int B, int q, double eps, float* x,
-                              uint16_t* out, unsigned* status, cudaStream_t st) {
+                              uint16_t* out, unsigned* status, const int32_t* seq_lens,
+                              const double* inv_freq, int half, float2* rope_tab, cudaStream_t st) {
+  InvFreq f{};
+  for (int j = 0; j < half && j < 128; ++j) f.v[j] = inv_freq[j];
   return launch_k(embed_norm_kernel, dim3(B * q), dim3(kNormThreads), 0, st,
                   static_cast<const uint16_t*>(w_emb), vocab, d, last_token, drafts, q, eps, x, out,
-                  status);
+                  status, seq_lens, f, half, rope_tab);
 }
 
 cudaError_t launch_rmsnorm(const float* x, int M, int d, double eps, uint16_t* out,

@@ -83,7 +83,7 @@ WORKLOADS = {
     # Batch 1, 8k context, k=4: sliding-window layer + key-equals-value global layer.
     "b1_ctx8k": Workload("b1_ctx8k", batch=1, k=4, d_model=2560, n_q_heads=16, n_kv_heads=8,
                          head_dim=256, vocab=262144, layers=(LOCAL1024, GLOBAL_KV),
-                         ctx_lo=8192, ctx_hi=8192, accept=("geometric", 0.8), split_tokens=512),
+                         ctx_lo=8192, ctx_hi=8192, accept=("geometric", 0.8), split_tokens=256),
     # Batch 8 ragged 4k-32k, global key-equals-value layer only.
     "b8_ragged": Workload("b8_ragged", batch=8, k=4, d_model=5376, n_q_heads=32, n_kv_heads=4,
                           head_dim=256, vocab=262144, layers=(GLOBAL_KV,), ctx_lo=4096,
