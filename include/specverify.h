@@ -214,6 +214,35 @@ int spec_verify_step(const spec_model* m, const int32_t* block_table, int max_pa
                      int32_t* new_last_token, int32_t* target_ids, float* target_maxlogit,
                      void* ws, size_t ws_bytes, void* stream);
 
+/* LM head + argmax without a workspace, for callers that cannot allocate
+ * device memory.  The pages have no counterpart: this is a deployment aid.
+ *
+ * Who needs it: callers that have no way to hand the library a workspace --
+ * a runtime whose device memory plan is fixed before decoding starts and
+ * forbids allocation on the decode path, a plugin that a host framework
+ * gives only its input and output tensors, a latency-critical loop that
+ * cannot take cudaMalloc's implicit device synchronisation.
+ *
+ * Same operation, arguments and errors as spec_lmhead_argmax, minus the
+ * workspace.  Its scratch (argmax partials, a completion counter, a status
+ * word) is a file-scope __device__ array inside the library, of about 1 MiB,
+ * that every GPU which loads the library holds until the process exits.
+ * Limits: M <= SPEC_NOALLOC_MAX_ROWS and ceil(V / 128) * M <=
+ * SPEC_NOALLOC_MAX_TILE_ROWS (so V = 262,144 allows M <= 64); larger
+ * problems return SPEC_EUNSUPPORTED and launch nothing.
+ *
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  Each call clears the counter and status word
+ * (an async memset on `stream`) and allocates nothing.  All calls share the
+ * one array, which keeps the last call's contents: calls that overlap on the
+ * GPU (different streams, or concurrent host threads on one device) race and
+ * must be serialised by the caller. */
+#define SPEC_NOALLOC_MAX_ROWS 64
+#define SPEC_NOALLOC_MAX_TILE_ROWS 131072
+int spec_lmhead_argmax_noalloc(const void* h, const void* w, int M, int d, int V, int32_t* ids,
+                               float* maxlogit, void* stream);
+
 /* Timing hook (no counterpart in the pages; measurement only).
  * spec_profile_start(n): the next n spec_verify_step calls record CUDA events
  * (created and owned by the library) on their stream around the whole step

@@ -32,7 +32,10 @@ EXPORTED = [
     "spec_lmhead_workspace_bytes", "spec_workspace_init", "spec_read_device_status",
     "spec_cache_write", "spec_verify_attn", "spec_lmhead_argmax", "spec_accept_commit",
     "spec_verify_step", "spec_profile_start", "spec_profile_collect",
+    "spec_lmhead_argmax_noalloc",
 ]
+SPEC_NOALLOC_MAX_ROWS = 64
+SPEC_NOALLOC_MAX_TILE_ROWS = 131072
 
 
 class SpecError(RuntimeError):
@@ -98,6 +101,8 @@ def lib():
         L.spec_verify_step.argtypes = [pm, c_void_p, c_int, c_void_p, c_void_p, c_int, c_int,
                                        c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                        c_void_p, c_size_t, c_void_p]
+        L.spec_lmhead_argmax_noalloc.argtypes = [c_void_p, c_void_p, c_int, c_int, c_int, c_void_p,
+                                                 c_void_p, c_void_p]
         L.spec_profile_start.argtypes = [c_int]
         L.spec_profile_collect.argtypes = [POINTER(c_float), POINTER(c_float), c_int]
         for name in EXPORTED[4:]:
@@ -204,3 +209,15 @@ def spec_profile_collect(n_steps: int):
     b = (c_float * n_steps)()
     _check(lib().spec_profile_collect(a, b, n_steps), "spec_profile_collect")
     return list(a), list(b)
+
+
+def spec_lmhead_argmax_noalloc(h, w, M, d, V, ids, maxlogit, stream=None) -> int:
+    """spec_lmhead_argmax without a workspace: the scratch is a fixed device
+    array inside the library, for callers that cannot allocate device memory.
+    Raises SpecError(SPEC_EUNSUPPORTED) when M > 64 or ceil(V/128)*M > 131072."""
+    rc = lib().spec_lmhead_argmax_noalloc(_p(h), _p(w), M, d, V, _p(ids), _p(maxlogit), _s(stream))
+    if rc == SPEC_EUNSUPPORTED:
+        raise SpecError(rc, f"spec_lmhead_argmax_noalloc: M={M}, V={V} exceeds the fixed scratch "
+                            f"(M <= {SPEC_NOALLOC_MAX_ROWS}, ceil(V/128)*M <= "
+                            f"{SPEC_NOALLOC_MAX_TILE_ROWS})")
+    return _check(rc, "spec_lmhead_argmax_noalloc")

@@ -1,0 +1,79 @@
+// LM head + argmax for callers that cannot allocate device memory.
+//
+// spec_lmhead_argmax needs a caller-provided workspace for its per-tile
+// argmax partials and its completion counter.  Some callers have no way to
+// provide one: code that runs where device allocation is not permitted or
+// not wanted (an inference runtime whose memory plan is fixed before the
+// first token and forbids allocations on the decode path, a plugin handed
+// only its input and output tensors by a host framework that owns every
+// allocation, a latency-critical loop that cannot afford cudaMalloc's
+// implicit device synchronisation).  spec_lmhead_argmax_noalloc serves them:
+// its scratch is a file-scope __device__ array below, loaded with the
+// library, so the call itself allocates nothing.
+#include <mutex>
+
+#include "../../include/specverify.h"
+#include "common.cuh"
+#include "internal.h"
+
+namespace sv {
+namespace {
+
+constexpr size_t kNoAllocHeader = kWsHeaderBytes;                       // status + counters
+constexpr size_t kNoAllocEntries = (size_t)SPEC_NOALLOC_MAX_TILE_ROWS;  // tiles x rows
+constexpr size_t kNoAllocBytes = kNoAllocHeader + 2 * kNoAllocEntries * 4;
+
+// One copy per GPU that loads the library; it stays allocated until exit.
+__device__ __align__(256) uint8_t g_lmhead_scratch[kNoAllocBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_setup_mutex;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device.  In host code
+// `g_lmhead_scratch` names a host-side stand-in, not device memory, so the
+// address must come from cudaGetSymbolAddress, once per device, with that
+// device current.
+int scratch_for_current_device(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SPEC_ECUDA;
+  std::lock_guard<std::mutex> lock(g_setup_mutex);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_lmhead_scratch) != cudaSuccess || !p) return SPEC_ECUDA;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return SPEC_OK;
+}
+
+}  // namespace
+}  // namespace sv
+
+using namespace sv;
+
+extern "C" int spec_lmhead_argmax_noalloc(const void* h, const void* w, int M, int d, int V,
+                                          int32_t* ids, float* maxlogit, void* stream) {
+  if (!h || !w || !ids || M < 1 || V < 1 || d < 8 || d % 8) return SPEC_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(h) & 15) || (reinterpret_cast<uintptr_t>(w) & 15)) return SPEC_EINVAL;
+  GemmPlan p = plan_gemm(M, V, d, kGemmArgmax);
+  // The fixed scratch holds one M-block of rows and ceil(V/128) * M partials.
+  if (M > SPEC_NOALLOC_MAX_ROWS || gemm_argmax_entries(p) > kNoAllocEntries) return SPEC_EUNSUPPORTED;
+  void* scratch = nullptr;
+  int rc = scratch_for_current_device(&scratch);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // The array keeps the previous call's contents: the status word and the
+  // completion counter must start at zero.
+  if (cudaMemsetAsync(scratch, 0, kNoAllocHeader, st) != cudaSuccess) return SPEC_ECUDA;
+  WsHeader hdr = ws_header(scratch);
+  GemmBuffers b{};
+  b.arg_val = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + kNoAllocHeader);
+  b.arg_idx = reinterpret_cast<int*>(static_cast<uint8_t*>(scratch) + kNoAllocHeader +
+                                     kNoAllocEntries * 4);
+  b.ids = ids;
+  b.maxv = maxlogit;
+  b.tickets = hdr.tickets;
+  b.status = hdr.status;
+  return launch_gemm(p, kGemmArgmax, h, w, b, st) == cudaSuccess ? SPEC_OK : SPEC_ECUDA;
+}
