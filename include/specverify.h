@@ -214,6 +214,21 @@ int spec_verify_step(const spec_model* m, const int32_t* block_table, int max_pa
                      int32_t* new_last_token, int32_t* target_ids, float* target_maxlogit,
                      void* ws, size_t ws_bytes, void* stream);
 
+/* Prefill: the target forward over n new tokens per sequence at positions
+ * L..L+n-1 (L = seq_lens[b]) through the same kernels as the verify step, so
+ * the cache holds exactly what a token-by-token decode would have written
+ * ("Gemma 4 拆解" §4.2: the target's prefilled cache that the drafter and the
+ * verify step share).  All n rows are committed: seq_lens[b] += n.  The
+ * argmax of each sequence's last row (the first token after the chunk) goes
+ * to next_token[b], its logit to next_maxlogit[b] (may be NULL).
+ *   tokens [B][n] int32, n in [1, SPEC_MAX_PREFILL]; the workspace comes
+ *   from spec_prefill_workspace_bytes(m, >= B, >= n, >= max_pages). */
+#define SPEC_MAX_PREFILL 256
+size_t spec_prefill_workspace_bytes(const spec_model* m, int max_batch, int max_n, int max_pages);
+int spec_prefill(const spec_model* m, const int32_t* block_table, int max_pages,
+                 const int32_t* tokens, int B, int n, int32_t* seq_lens, int32_t* next_token,
+                 float* next_maxlogit, void* ws, size_t ws_bytes, void* stream);
+
 /* LM head + argmax without a workspace, for callers that cannot allocate
  * device memory.  The pages have no counterpart: this is a deployment aid.
  *

@@ -32,8 +32,9 @@ EXPORTED = [
     "spec_lmhead_workspace_bytes", "spec_workspace_init", "spec_read_device_status",
     "spec_cache_write", "spec_verify_attn", "spec_lmhead_argmax", "spec_accept_commit",
     "spec_verify_step", "spec_profile_start", "spec_profile_collect",
-    "spec_lmhead_argmax_noalloc",
+    "spec_lmhead_argmax_noalloc", "spec_prefill_workspace_bytes", "spec_prefill",
 ]
+SPEC_MAX_PREFILL = 256
 SPEC_NOALLOC_MAX_ROWS = 64
 SPEC_NOALLOC_MAX_TILE_ROWS = 131072
 
@@ -103,10 +104,15 @@ def lib():
                                        c_void_p, c_size_t, c_void_p]
         L.spec_lmhead_argmax_noalloc.argtypes = [c_void_p, c_void_p, c_int, c_int, c_int, c_void_p,
                                                  c_void_p, c_void_p]
+        L.spec_prefill_workspace_bytes.restype = c_size_t
+        L.spec_prefill_workspace_bytes.argtypes = [pm, c_int, c_int, c_int]
+        L.spec_prefill.argtypes = [pm, c_void_p, c_int, c_void_p, c_int, c_int, c_void_p, c_void_p,
+                                   c_void_p, c_void_p, c_size_t, c_void_p]
         L.spec_profile_start.argtypes = [c_int]
         L.spec_profile_collect.argtypes = [POINTER(c_float), POINTER(c_float), c_int]
         for name in EXPORTED[4:]:
-            getattr(L, name).restype = c_int
+            if name != "spec_prefill_workspace_bytes":
+                getattr(L, name).restype = c_int
         _lib = L
     return _lib
 
@@ -221,3 +227,14 @@ def spec_lmhead_argmax_noalloc(h, w, M, d, V, ids, maxlogit, stream=None) -> int
                             f"(M <= {SPEC_NOALLOC_MAX_ROWS}, ceil(V/128)*M <= "
                             f"{SPEC_NOALLOC_MAX_TILE_ROWS})")
     return _check(rc, "spec_lmhead_argmax_noalloc")
+
+
+def spec_prefill_workspace_bytes(model: SpecModel, max_batch: int, max_n: int, max_pages: int) -> int:
+    return int(lib().spec_prefill_workspace_bytes(ctypes.byref(model), max_batch, max_n, max_pages))
+
+
+def spec_prefill(model, block_table, max_pages, tokens, B, n, seq_lens, next_token, next_maxlogit,
+                 ws, ws_bytes, stream=None) -> int:
+    return _check(lib().spec_prefill(ctypes.byref(model), _p(block_table), max_pages, _p(tokens), B, n,
+                                     _p(seq_lens), _p(next_token), _p(next_maxlogit), _p(ws),
+                                     ws_bytes, _s(stream)), "spec_prefill")

@@ -33,12 +33,15 @@ void resolve_encode() {
 }  // namespace
 
 bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
-                       uint32_t box_rows, uint32_t box_cols) {
+                       uint32_t box_rows, uint32_t box_cols, uint64_t row_stride) {
   std::call_once(g_encode_once, resolve_encode);
   if (!g_encode || !base) return false;
-  if ((reinterpret_cast<uintptr_t>(base) & 15) || (cols * 2) % 16 || box_cols * 2 > 128) return false;
+  if (row_stride == 0) row_stride = cols;
+  if ((reinterpret_cast<uintptr_t>(base) & 15) || (row_stride * 2) % 16 || box_cols * 2 > 128 ||
+      row_stride < cols)
+    return false;
   cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * 2};
+  cuuint64_t strides[1] = {row_stride * 2};
   cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
@@ -96,7 +99,8 @@ int check_model(const spec_model* m) {
   return SPEC_OK;
 }
 
-// Workspace layout of one verify step for (B, k, max_pages).
+// Workspace layout of one forward over q rows per sequence (q = k + 1 for a
+// verify step, q = n for a prefill chunk) for (B, q, max_pages).
 struct StepLayout {
   size_t x, hn, qrot, attn_out, attn_part, gemm_part, arg_val, arg_idx, ids, maxv, rope_tab,
       total;
@@ -104,10 +108,10 @@ struct StepLayout {
   bool splits_ok;   // every layer's split count fits the combine kernel
 };
 
-StepLayout step_layout(const spec_model* m, int B, int k, int max_pages) {
+StepLayout step_layout(const spec_model* m, int B, int q, int max_pages) {
   StepLayout s{};
   s.splits_ok = true;
-  const int q = k + 1, M = B * q, d = m->d_model, D = m->head_dim;
+  const int M = B * q, d = m->d_model, D = m->head_dim;
   size_t attn_floats = 0, gemm_floats = 0;
   int tickets = 0;
   for (int l = 0; l < m->n_layers; ++l) {
@@ -166,6 +170,135 @@ void prof_release() {
   g_prof.ev.clear();
   g_prof.n = g_prof.used = 0;
   g_prof.on = false;
+}
+
+// Inputs and outputs of one forward: a verify step (last_token/drafts ->
+// acceptance outputs) or a prefill chunk (tokens -> next_token).
+struct ForwardIo {
+  const int32_t* last_token = nullptr;
+  const int32_t* drafts = nullptr;
+  int32_t* accept_len = nullptr;
+  int32_t* emitted = nullptr;
+  int32_t* new_last_token = nullptr;
+  int32_t* target_ids = nullptr;
+  float* target_maxlogit = nullptr;
+  const int32_t* tokens = nullptr;     // prefill: [B][q]
+  int32_t* next_token = nullptr;       // prefill: [B]
+  float* next_maxlogit = nullptr;
+};
+
+// embed -> per layer (RMSNorm, QKV + RoPE + cache append, split-KV attention,
+// O-proj + residual) -> final RMSNorm -> LM head argmax -> acceptance (verify)
+// or commit of all q rows (prefill).
+int run_forward(const spec_model* m, const int32_t* block_table, int max_pages, int B, int q,
+                int32_t* seq_lens, const ForwardIo& io, void* ws, size_t ws_bytes,
+                cudaStream_t st) {
+  const bool prefill = io.tokens != nullptr;
+  StepLayout s = step_layout(m, B, q, max_pages);
+  if (s.tickets > kMaxTickets || !s.splits_ok) return SPEC_EUNSUPPORTED;
+  if (ws_bytes < s.total) return SPEC_EINVAL;
+  WsHeader hdr = ws_header(ws);
+  const int k = q - 1, M = B * q, d = m->d_model, D = m->head_dim;
+  float* x = at<float>(ws, s.x);
+  uint16_t* hn = at<uint16_t>(ws, s.hn);
+  uint16_t* qrot = at<uint16_t>(ws, s.qrot);
+  uint16_t* attn_out = at<uint16_t>(ws, s.attn_out);
+  int rc;
+
+  prof_mark(0, st);
+  double inv_freq[128];
+  rope_inv_freq(m->rope_theta, D, D / 2, inv_freq);
+  float2* rope_tab = at<float2>(ws, s.rope_tab);
+  rc = cuda_status(launch_embed_norm(m->w_embed, m->vocab, d, io.last_token, io.drafts, io.tokens,
+                                     B, q, m->rms_eps, x, hn, hdr.status, seq_lens, inv_freq, D / 2,
+                                     rope_tab, st));
+  if (rc) return rc;
+  for (int l = 0; l < m->n_layers; ++l) {
+    const spec_layer& L = m->layers[l];
+    const int nqkv = qkv_out(m, L);
+    if (l > 0) {
+      rc = cuda_status(launch_rmsnorm(x, M, d, m->rms_eps, hn, st));
+      if (rc) return rc;
+    }
+    // QKV projection with RoPE and the cache append in its epilogue
+    GemmPlan pq = plan_gemm(M, nqkv, d, kGemmQkvRope);
+    GemmBuffers bq{};
+    bq.partial = at<float>(ws, s.gemm_part);
+    bq.tickets = hdr.tickets;
+    bq.status = hdr.status;
+    RopeFuse& f = bq.rope;
+    f.n_q_heads = m->n_q_heads;
+    f.n_kv_heads = m->n_kv_heads;
+    f.head_dim = D;
+    f.n_rot = n_rot_of(m, L);
+    f.q = q;
+    f.page_size = m->page_size;
+    f.num_pages = m->num_pages;
+    f.max_pages = max_pages;
+    f.seq_lens = seq_lens;
+    f.block_table = block_table;
+    f.rope_tab = rope_tab;
+    f.q_out = qrot;
+    f.k_pool = static_cast<uint16_t*>(L.k_pool);
+    f.v_pool = static_cast<uint16_t*>(L.v_pool);
+    f.ksb_pool = static_cast<uint16_t*>(L.ksb_pool);
+    rc = cuda_status(launch_gemm(pq, kGemmQkvRope, hn, L.w_qkv, bq, st));
+    if (rc) return rc;
+    AttnGeom g = plan_attn(B, q, m->n_q_heads, m->n_kv_heads, D, m->page_size, m->num_pages,
+                           max_pages, L.window, L.kv_equal, 2 * f.n_rot, split_of(m, L));
+    rc = cuda_status(launch_attention(g, qrot, L.k_pool, L.v_pool, L.ksb_pool, block_table, seq_lens,
+                                      at<float>(ws, s.attn_part), attn_out, hdr.status, st));
+    if (rc) return rc;
+    GemmPlan po = plan_gemm(M, d, m->n_q_heads * D, kGemmResidual);
+    GemmBuffers bo{};
+    bo.out = x;
+    bo.partial = at<float>(ws, s.gemm_part);
+    bo.tickets = hdr.tickets;
+    bo.status = hdr.status;
+    rc = cuda_status(launch_gemm(po, kGemmResidual, attn_out, L.w_o, bo, st));
+    if (rc) return rc;
+  }
+  rc = cuda_status(launch_rmsnorm(x, M, d, m->rms_eps, hn, st));
+  if (rc) return rc;
+  // LM head: every row (verify) or each sequence's last row (prefill)
+  GemmPlan pl = plan_gemm(prefill ? B : M, m->vocab, d, kGemmArgmax);
+  GemmBuffers bl{};
+  bl.arg_val = at<float>(ws, s.arg_val);
+  bl.arg_idx = at<int>(ws, s.arg_idx);
+  bl.ids = at<int32_t>(ws, s.ids);
+  bl.maxv = at<float>(ws, s.maxv);
+  bl.tickets = hdr.tickets;
+  bl.status = hdr.status;
+  const uint16_t* lm_x = hn;
+  if (prefill) {
+    pl.x_row_stride = q * d;
+    lm_x = hn + (size_t)(q - 1) * d;
+  } else {
+    bl.acc.B = B;
+    bl.acc.k = k;
+    bl.acc.drafts = io.drafts;
+    bl.acc.seq_lens = seq_lens;
+    bl.acc.accept_len = io.accept_len;
+    bl.acc.emitted = io.emitted;
+    bl.acc.last_token = io.new_last_token;
+    bl.acc.copy_ids = io.target_ids;
+    bl.acc.copy_max = io.target_maxlogit;
+  }
+  prof_mark(1, st);
+  rc = cuda_status(launch_gemm(pl, kGemmArgmax, lm_x, m->w_lm, bl, st));
+  prof_mark(2, st);
+  if (rc) return rc;
+  if (prefill) {
+    rc = cuda_status(launch_prefill_commit(at<int32_t>(ws, s.ids), at<float>(ws, s.maxv), B, q,
+                                           seq_lens, io.next_token, io.next_maxlogit, st));
+  } else if (pl.mblocks > 1) {  // acceptance is fused into the LM head for a single M-block
+    rc = cuda_status(launch_accept(io.drafts, at<int32_t>(ws, s.ids), B, k, seq_lens, io.accept_len,
+                                   io.emitted, io.new_last_token, io.target_ids,
+                                   io.target_maxlogit, at<float>(ws, s.maxv), st));
+  }
+  prof_mark(3, st);
+  prof_step_done();
+  return rc;
 }
 
 }  // namespace
@@ -232,7 +365,7 @@ size_t spec_layer_pool_bytes(const spec_model* m, int layer, int which) {
 
 size_t spec_workspace_bytes(const spec_model* m, int max_batch, int max_k, int max_pages) {
   if (!m || !m->layers || max_batch < 1 || max_k < 0 || max_k > SPEC_MAX_K || max_pages < 1) return 0;
-  StepLayout s = step_layout(m, max_batch, max_k, max_pages);
+  StepLayout s = step_layout(m, max_batch, max_k + 1, max_pages);
   if (s.tickets > kMaxTickets || !s.splits_ok) return 0;
   return s.total;
 }
@@ -305,7 +438,7 @@ int spec_verify_attn(const spec_model* m, int layer, const void* q, const void* 
   const spec_layer& L = m->layers[layer];
   if (!L.kv_equal && !v_new) return SPEC_EINVAL;
   const int qn = k + 1, D = m->head_dim;
-  StepLayout s = step_layout(m, B, k, max_pages);
+  StepLayout s = step_layout(m, B, k + 1, max_pages);
   if (!s.splits_ok) return SPEC_EUNSUPPORTED;
   if (ws_bytes < s.total) return SPEC_EINVAL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -384,100 +517,39 @@ int spec_verify_step(const spec_model* m, const int32_t* block_table, int max_pa
   if (!block_table || !last_token || !seq_lens || !accept_len || !emitted || !new_last_token || !ws)
     return SPEC_EINVAL;
   if (B < 1 || k < 0 || k > SPEC_MAX_K || max_pages < 1 || (k > 0 && !drafts)) return SPEC_EINVAL;
-  StepLayout s = step_layout(m, B, k, max_pages);
-  if (s.tickets > kMaxTickets || !s.splits_ok) return SPEC_EUNSUPPORTED;
-  if (ws_bytes < s.total) return SPEC_EINVAL;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  WsHeader hdr = ws_header(ws);
-  const int q = k + 1, M = B * q, d = m->d_model, D = m->head_dim;
-  float* x = at<float>(ws, s.x);
-  uint16_t* hn = at<uint16_t>(ws, s.hn);
-  uint16_t* qrot = at<uint16_t>(ws, s.qrot);
-  uint16_t* attn_out = at<uint16_t>(ws, s.attn_out);
+  ForwardIo io{};
+  io.last_token = last_token;
+  io.drafts = drafts;
+  io.accept_len = accept_len;
+  io.emitted = emitted;
+  io.new_last_token = new_last_token;
+  io.target_ids = target_ids;
+  io.target_maxlogit = target_maxlogit;
+  return run_forward(m, block_table, max_pages, B, k + 1, seq_lens, io, ws, ws_bytes,
+                     static_cast<cudaStream_t>(stream));
+}
 
-  prof_mark(0, st);
-  double inv_freq[128];
-  rope_inv_freq(m->rope_theta, D, D / 2, inv_freq);
-  float2* rope_tab = at<float2>(ws, s.rope_tab);
-  rc = cuda_status(launch_embed_norm(m->w_embed, m->vocab, d, last_token, drafts, B, q, m->rms_eps,
-                                     x, hn, hdr.status, seq_lens, inv_freq, D / 2, rope_tab, st));
-  if (rc) return rc;
-  for (int l = 0; l < m->n_layers; ++l) {
-    const spec_layer& L = m->layers[l];
-    const int nqkv = qkv_out(m, L);
-    if (l > 0) {
-      rc = cuda_status(launch_rmsnorm(x, M, d, m->rms_eps, hn, st));
-      if (rc) return rc;
-    }
-    // QKV projection with RoPE and the cache append in its epilogue
-    GemmPlan pq = plan_gemm(M, nqkv, d, kGemmQkvRope);
-    GemmBuffers bq{};
-    bq.partial = at<float>(ws, s.gemm_part);
-    bq.tickets = hdr.tickets;
-    bq.status = hdr.status;
-    RopeFuse& f = bq.rope;
-    f.n_q_heads = m->n_q_heads;
-    f.n_kv_heads = m->n_kv_heads;
-    f.head_dim = D;
-    f.n_rot = n_rot_of(m, L);
-    f.q = q;
-    f.page_size = m->page_size;
-    f.num_pages = m->num_pages;
-    f.max_pages = max_pages;
-    f.seq_lens = seq_lens;
-    f.block_table = block_table;
-    f.rope_tab = rope_tab;
-    f.q_out = qrot;
-    f.k_pool = static_cast<uint16_t*>(L.k_pool);
-    f.v_pool = static_cast<uint16_t*>(L.v_pool);
-    f.ksb_pool = static_cast<uint16_t*>(L.ksb_pool);
-    rc = cuda_status(launch_gemm(pq, kGemmQkvRope, hn, L.w_qkv, bq, st));
-    if (rc) return rc;
-    AttnGeom g = plan_attn(B, q, m->n_q_heads, m->n_kv_heads, D, m->page_size, m->num_pages,
-                           max_pages, L.window, L.kv_equal, 2 * f.n_rot, split_of(m, L));
-    rc = cuda_status(launch_attention(g, qrot, L.k_pool, L.v_pool, L.ksb_pool, block_table, seq_lens,
-                                      at<float>(ws, s.attn_part), attn_out, hdr.status, st));
-    if (rc) return rc;
+size_t spec_prefill_workspace_bytes(const spec_model* m, int max_batch, int max_n, int max_pages) {
+  if (!m || !m->layers || max_batch < 1 || max_n < 1 || max_n > SPEC_MAX_PREFILL || max_pages < 1)
+    return 0;
+  StepLayout s = step_layout(m, max_batch, max_n, max_pages);
+  if (s.tickets > kMaxTickets || !s.splits_ok) return 0;
+  return s.total;
+}
 
-    GemmPlan po = plan_gemm(M, d, m->n_q_heads * D, kGemmResidual);
-    GemmBuffers bo{};
-    bo.out = x;
-    bo.partial = at<float>(ws, s.gemm_part);
-    bo.tickets = hdr.tickets;
-    bo.status = hdr.status;
-    rc = cuda_status(launch_gemm(po, kGemmResidual, attn_out, L.w_o, bo, st));
-    if (rc) return rc;
-  }
-  rc = cuda_status(launch_rmsnorm(x, M, d, m->rms_eps, hn, st));
+int spec_prefill(const spec_model* m, const int32_t* block_table, int max_pages,
+                 const int32_t* tokens, int B, int n, int32_t* seq_lens, int32_t* next_token,
+                 float* next_maxlogit, void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_model(m);
   if (rc) return rc;
-  GemmPlan pl = plan_gemm(M, m->vocab, d, kGemmArgmax);
-  GemmBuffers bl{};
-  bl.arg_val = at<float>(ws, s.arg_val);
-  bl.arg_idx = at<int>(ws, s.arg_idx);
-  bl.ids = at<int32_t>(ws, s.ids);
-  bl.maxv = at<float>(ws, s.maxv);
-  bl.tickets = hdr.tickets;
-  bl.status = hdr.status;
-  bl.acc.B = B;
-  bl.acc.k = k;
-  bl.acc.drafts = drafts;
-  bl.acc.seq_lens = seq_lens;
-  bl.acc.accept_len = accept_len;
-  bl.acc.emitted = emitted;
-  bl.acc.last_token = new_last_token;
-  bl.acc.copy_ids = target_ids;
-  bl.acc.copy_max = target_maxlogit;
-  prof_mark(1, st);
-  rc = cuda_status(launch_gemm(pl, kGemmArgmax, hn, m->w_lm, bl, st));
-  prof_mark(2, st);
-  if (rc) return rc;
-  if (pl.mblocks > 1)   // acceptance is fused into the LM head when all rows share one M-block
-    rc = cuda_status(launch_accept(drafts, at<int32_t>(ws, s.ids), B, k, seq_lens, accept_len,
-                                   emitted, new_last_token, target_ids, target_maxlogit,
-                                   at<float>(ws, s.maxv), st));
-  prof_mark(3, st);
-  prof_step_done();
-  return rc;
+  if (!block_table || !tokens || !seq_lens || !next_token || !ws) return SPEC_EINVAL;
+  if (B < 1 || n < 1 || n > SPEC_MAX_PREFILL || max_pages < 1) return SPEC_EINVAL;
+  ForwardIo io{};
+  io.tokens = tokens;
+  io.next_token = next_token;
+  io.next_maxlogit = next_maxlogit;
+  return run_forward(m, block_table, max_pages, B, n, seq_lens, io, ws, ws_bytes,
+                     static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -519,7 +519,8 @@ cudaError_t launch_gemm(const GemmPlan& p, int mode, const void* x, const void* 
                         const GemmBuffers& b, cudaStream_t st) {
   CUtensorMap tw, tx;
   if (!make_tmap_bf16_2d(&tw, w, p.N, p.K, kTileN, kTileK)) return cudaErrorInvalidValue;
-  if (!make_tmap_bf16_2d(&tx, x, p.M, p.K, p.nt * 8, kTileK)) return cudaErrorInvalidValue;
+  if (!make_tmap_bf16_2d(&tx, x, p.M, p.K, p.nt * 8, kTileK, p.x_row_stride))
+    return cudaErrorInvalidValue;
   Args a{};
   a.M = p.M;
   a.N = p.N;

@@ -13,7 +13,7 @@ namespace sv {
 // swizzle, zero fill outside the tensor.  Returns false if the driver call
 // fails (the caller reports SPEC_ECUDA) or the layout is not encodable.
 bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
-                       uint32_t box_rows, uint32_t box_cols);
+                       uint32_t box_rows, uint32_t box_cols, uint64_t row_stride = 0);
 
 // --------------------------------------------------------- streaming GEMM
 // Y = X . W^T with X [M][K] bf16 (row-major), W [N][K] bf16 (row-major),
@@ -27,6 +27,7 @@ struct GemmPlan {
   int splits;    // split-K factor (1 for argmax)
   int mblocks;   // ceil(M / 64)
   int nt;        // n8 tiles per M-block: ceil(min(M, 64) / 8)
+  int x_row_stride = 0;   // elements between X rows (0: K)
 };
 GemmPlan plan_gemm(int M, int N, int K, int mode);
 size_t gemm_partial_floats(const GemmPlan& p);   // split-K partial sums
@@ -81,10 +82,17 @@ cudaError_t launch_rmsnorm(const float* x, int M, int d, double eps, uint16_t* o
 // embedding gather of [last_token, drafts] into x and its RMSNorm into out;
 // also the (cos, sin) table of every row's position for pairs j < half
 // (rope_tab [B*q][half], theta_j = inv_freq[j]); rope_tab may be null
+// Row m = b*q + i takes tokens_flat[m] when tokens_flat is set (prefill), else
+// last_token[b] (i = 0) / drafts[b][i-1] (verify).
 cudaError_t launch_embed_norm(const void* w_emb, int vocab, int d, const int32_t* last_token,
-                              const int32_t* drafts, int B, int q, double eps, float* x,
-                              uint16_t* out, unsigned* status, const int32_t* seq_lens,
-                              const double* inv_freq, int half, float2* rope_tab, cudaStream_t st);
+                              const int32_t* drafts, const int32_t* tokens_flat, int B, int q,
+                              double eps, float* x, uint16_t* out, unsigned* status,
+                              const int32_t* seq_lens, const double* inv_freq, int half,
+                              float2* rope_tab, cudaStream_t st);
+// Prefill commit: seq_lens[b] += n; next_token[b] = ids[b]; next_max[b] = maxv[b] (if set).
+cudaError_t launch_prefill_commit(const int32_t* ids, const float* maxv, int B, int n,
+                                  int32_t* seq_lens, int32_t* next_token, float* next_max,
+                                  cudaStream_t st);
 // host: theta_j = base^(-2j/D) for j < n_rot (n_rot <= 128)
 void rope_inv_freq(double base, int head_dim, int n_rot, double* out);
 cudaError_t launch_accept(const int32_t* drafts, const int32_t* target, int B, int k,

@@ -48,9 +48,10 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(const float* __re
 // (cos, sin) table of the row's position for every rotary pair.
 __global__ void __launch_bounds__(kNormThreads) embed_norm_kernel(
     const uint16_t* __restrict__ w_emb, int vocab, int d, const int32_t* __restrict__ last_token,
-    const int32_t* __restrict__ drafts, int q, double eps, float* __restrict__ x,
-    uint16_t* __restrict__ out, unsigned* status, const int32_t* __restrict__ seq_lens,
-    InvFreq inv_freq, int half, float2* __restrict__ rope_tab) {
+    const int32_t* __restrict__ drafts, const int32_t* __restrict__ tokens_flat, int q, double eps,
+    float* __restrict__ x, uint16_t* __restrict__ out, unsigned* status,
+    const int32_t* __restrict__ seq_lens, InvFreq inv_freq, int half,
+    float2* __restrict__ rope_tab) {
   __shared__ double red[kNormThreads / 32];
   pdl_trigger();
   pdl_wait();
@@ -61,7 +62,8 @@ __global__ void __launch_bounds__(kNormThreads) embed_norm_kernel(
     for (int j = threadIdx.x; j < half; j += kNormThreads)
       rope_tab[(size_t)m * half + j] = rope_cs(pos, inv_freq.v[j]);
   }
-  const int tok = (i == 0) ? last_token[b] : drafts[b * (q - 1) + (i - 1)];
+  const int tok = tokens_flat ? tokens_flat[m]
+                              : ((i == 0) ? last_token[b] : drafts[b * (q - 1) + (i - 1)]);
   float* row = x + (size_t)m * d;
   const bool ok = tok >= 0 && tok < vocab;
   if (!ok && threadIdx.x == 0) flag_status(status, SPEC_DEV_BAD_TOKEN);
@@ -107,14 +109,34 @@ __global__ void accept_kernel(const int32_t* __restrict__ drafts, const int32_t*
 }  // namespace
 
 cudaError_t launch_embed_norm(const void* w_emb, int vocab, int d, const int32_t* last_token,
-                              const int32_t* drafts, int B, int q, double eps, float* x,
-                              uint16_t* out, unsigned* status, const int32_t* seq_lens,
-                              const double* inv_freq, int half, float2* rope_tab, cudaStream_t st) {
+                              const int32_t* drafts, const int32_t* tokens_flat, int B, int q,
+                              double eps, float* x, uint16_t* out, unsigned* status,
+                              const int32_t* seq_lens, const double* inv_freq, int half,
+                              float2* rope_tab, cudaStream_t st) {
   InvFreq f{};
   for (int j = 0; j < half && j < 128; ++j) f.v[j] = inv_freq[j];
   return launch_k(embed_norm_kernel, dim3(B * q), dim3(kNormThreads), 0, st,
-                  static_cast<const uint16_t*>(w_emb), vocab, d, last_token, drafts, q, eps, x, out,
-                  status, seq_lens, f, half, rope_tab);
+                  static_cast<const uint16_t*>(w_emb), vocab, d, last_token, drafts, tokens_flat, q,
+                  eps, x, out, status, seq_lens, f, half, rope_tab);
+}
+
+__global__ void prefill_commit_kernel(const int32_t* __restrict__ ids, const float* __restrict__ maxv,
+                                      int B, int n, int32_t* seq_lens, int32_t* next_token,
+                                      float* next_max) {
+  pdl_trigger();
+  pdl_wait();
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= B) return;
+  seq_lens[b] += n;
+  next_token[b] = ids[b];
+  if (next_max) next_max[b] = maxv[b];
+}
+
+cudaError_t launch_prefill_commit(const int32_t* ids, const float* maxv, int B, int n,
+                                  int32_t* seq_lens, int32_t* next_token, float* next_max,
+                                  cudaStream_t st) {
+  return launch_k(prefill_commit_kernel, dim3((B + 127) / 128), dim3(128), 0, st, ids, maxv, B, n,
+                  seq_lens, next_token, next_max);
 }
 
 cudaError_t launch_rmsnorm(const float* x, int M, int d, double eps, uint16_t* out,

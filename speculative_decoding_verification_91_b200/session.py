@@ -73,14 +73,78 @@ class WorkloadSession:
     def reset_lengths(self):
         self.seq_lens.copy_(self.seq_lens0)
 
-    def step(self, stream=None, with_targets=True):
+    def step(self, stream=None, with_targets=True, k=None):
+        """One spec_verify_step with this session's inputs (k defaults to the
+        workload's; any k up to it fits the workspace)."""
         wl = self.wl
+        k = wl.k if k is None else k
         B.spec_verify_step(self.dm.desc, self.block_table, self.max_pages, self.last_token,
-                           self.drafts if wl.k > 0 else None, wl.batch, wl.k, self.seq_lens,
+                           self.drafts if k > 0 else None, wl.batch, k, self.seq_lens,
                            self.accept_len, self.emitted, self.new_last,
                            self.target_ids if with_targets else None,
                            self.target_max if with_targets else None,
                            self.ws.buf, self.ws.nbytes, stream)
+
+    # ---------------------------------------------------------------- prefill
+
+    def prefill(self, tokens: np.ndarray, chunk: int = 256):
+        """Prefill tokens [B][n] from the current lengths through spec_prefill
+        in chunks; returns (next_token [B], its logit [B]) after the last chunk."""
+        tokens = np.asarray(tokens, dtype=np.int32)
+        Bn, n = tokens.shape
+        chunk = min(chunk, B.SPEC_MAX_PREFILL)
+        if not hasattr(self, "pws"):
+            nb = B.spec_prefill_workspace_bytes(self.dm.desc, self.wl.batch, chunk, self.max_pages)
+            from .runtime import Workspace
+            self.pws = Workspace(nb, self.device)
+        nxt = torch.zeros(Bn, dtype=torch.int32, device=self.device)
+        nmax = torch.zeros(Bn, dtype=torch.float32, device=self.device)
+        dev_tok = torch.from_numpy(tokens).to(self.device)
+        for c0 in range(0, n, chunk):
+            c = min(chunk, n - c0)
+            part = dev_tok[:, c0:c0 + c].contiguous()
+            B.spec_prefill(self.dm.desc, self.block_table, self.max_pages, part, Bn, c, self.seq_lens,
+                           nxt, nmax, self.pws.buf, self.pws.nbytes)
+        torch.cuda.synchronize(self.device)
+        return nxt.cpu().numpy(), nmax.cpu().numpy()
+
+    # ---------------------------------------------------------------- loops
+
+    def greedy(self, last: np.ndarray, n_tokens: int):
+        """k = 0 verify steps: one token per step.  Returns tokens [B][n] and
+        the max logit of every step."""
+        toks = np.zeros((self.wl.batch, n_tokens), dtype=np.int64)
+        maxes = np.zeros((self.wl.batch, n_tokens), dtype=np.float32)
+        cur = np.asarray(last, dtype=np.int32)
+        for t in range(n_tokens):
+            self.last_token.copy_(torch.from_numpy(cur))
+            self.step(k=0)
+            o = self.outputs()
+            toks[:, t] = o["target_ids"][:, 0]
+            maxes[:, t] = o["target_max"][:, 0]
+            cur = o["new_last"].astype(np.int32)
+        return toks, maxes
+
+    def speculative(self, last: np.ndarray, n_steps: int, drafter):
+        """n_steps verify steps of k drafts each; drafter(step, emitted_b,
+        b) -> k drafts for sequence b given its emitted tokens so far.
+        Returns (emitted streams per sequence, accept lengths [steps][B])."""
+        wl = self.wl
+        streams = [[] for _ in range(wl.batch)]
+        accepts = []
+        cur = np.asarray(last, dtype=np.int32)
+        for st in range(n_steps):
+            d = np.stack([np.asarray(drafter(st, streams[b], b), dtype=np.int32)
+                          for b in range(wl.batch)])
+            self.set_inputs(cur, d)
+            self.step()
+            o = self.outputs()
+            for b in range(wl.batch):
+                a = int(o["accept_len"][b])
+                streams[b].extend(int(t) for t in o["emitted"][b][:a + 1])
+            accepts.append(o["accept_len"].copy())
+            cur = o["new_last"].astype(np.int32)
+        return streams, np.array(accepts)
 
     def outputs(self):
         torch.cuda.synchronize(self.device)
