@@ -110,5 +110,15 @@ def test_speculative_loop_equals_greedy(name):
     assert s.ws.device_status() == 0
     got = [int(nxt[0])] + spec[0]
     assert got == stream[:len(got)]
-    assert accepts.max() == wl.k and accepts.min() == 0   # full accepts and immediate rejections
+    # every step accepts exactly the drafts designed to be right (the leading
+    # run of coin flips below p), so acceptance and rollback were both exercised
+    designed = []
+    for st in range(steps):
+        flips, _ = W.loop_draft_flips(wl, st)
+        r = 0
+        while r < wl.k and flips[r] < wl.accept[1]:
+            r += 1
+        designed.append(r)
+    assert accepts[:, 0].tolist() == designed
+    assert min(designed) == 0 and max(designed) >= 4
     assert int(s.seq_lens[0].item()) == L0 + len(spec[0])
