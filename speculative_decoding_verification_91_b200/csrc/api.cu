@@ -242,7 +242,7 @@ int run_forward(const spec_model* m, const int32_t* block_table, int max_pages, 
     f.k_pool = static_cast<uint16_t*>(L.k_pool);
     f.v_pool = static_cast<uint16_t*>(L.v_pool);
     f.ksb_pool = static_cast<uint16_t*>(L.ksb_pool);
-    rc = cuda_status(launch_gemm(pq, kGemmQkvRope, hn, L.w_qkv, bq, st));
+    rc = cuda_status(launch_gemm_any(pq, kGemmQkvRope, hn, L.w_qkv, bq, st));
     if (rc) return rc;
     AttnGeom g = plan_attn(B, q, m->n_q_heads, m->n_kv_heads, D, m->page_size, m->num_pages,
                            max_pages, L.window, L.kv_equal, 2 * f.n_rot, split_of(m, L));
@@ -255,7 +255,7 @@ int run_forward(const spec_model* m, const int32_t* block_table, int max_pages, 
     bo.partial = at<float>(ws, s.gemm_part);
     bo.tickets = hdr.tickets;
     bo.status = hdr.status;
-    rc = cuda_status(launch_gemm(po, kGemmResidual, attn_out, L.w_o, bo, st));
+    rc = cuda_status(launch_gemm_any(po, kGemmResidual, attn_out, L.w_o, bo, st));
     if (rc) return rc;
   }
   rc = cuda_status(launch_rmsnorm(x, M, d, m->rms_eps, hn, st));
@@ -285,13 +285,14 @@ int run_forward(const spec_model* m, const int32_t* block_table, int max_pages, 
     bl.acc.copy_max = io.target_maxlogit;
   }
   prof_mark(1, st);
-  rc = cuda_status(launch_gemm(pl, kGemmArgmax, lm_x, m->w_lm, bl, st));
+  rc = cuda_status(launch_gemm_any(pl, kGemmArgmax, lm_x, m->w_lm, bl, st));
   prof_mark(2, st);
   if (rc) return rc;
   if (prefill) {
     rc = cuda_status(launch_prefill_commit(at<int32_t>(ws, s.ids), at<float>(ws, s.maxv), B, q,
                                            seq_lens, io.next_token, io.next_maxlogit, st));
-  } else if (pl.mblocks > 1) {  // acceptance is fused into the LM head for a single M-block
+  } else if (pl.mblocks > 1 && !tc_supported(pl.M)) {
+    // acceptance is fused into the LM head when all rows share one block
     rc = cuda_status(launch_accept(io.drafts, at<int32_t>(ws, s.ids), B, k, seq_lens, io.accept_len,
                                    io.emitted, io.new_last_token, io.target_ids,
                                    io.target_maxlogit, at<float>(ws, s.maxv), st));
@@ -495,7 +496,7 @@ int spec_lmhead_argmax(const void* h, const void* w, int M, int d, int V, int32_
   b.maxv = maxlogit;
   b.tickets = hdr.tickets;
   b.status = hdr.status;
-  return cuda_status(launch_gemm(p, kGemmArgmax, h, w, b, static_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_gemm_any(p, kGemmArgmax, h, w, b, static_cast<cudaStream_t>(stream)));
 }
 
 int spec_accept_commit(const int32_t* drafts, const int32_t* target, int B, int k,

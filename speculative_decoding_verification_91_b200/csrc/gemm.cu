@@ -23,14 +23,13 @@
 #include <algorithm>
 
 #include "common.cuh"
+#include "gemm_epi.cuh"
 #include "internal.h"
 
 namespace sv {
 
 namespace {
 
-constexpr int kTileN = 128;
-constexpr int kTileK = 64;
 constexpr int kConsumerWarps = 4;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kMBlock = 64;
@@ -44,126 +43,6 @@ struct Cfg {
   static constexpr int kRedBytes = 2 * kConsumerWarps * NT * 8 * 4;
   static constexpr int kSmem = 1024 + kStages * kStageBytes + 2 * kStages * 8 + kRedBytes + 64;
 };
-
-struct Args {
-  int M, N, K, kchunks, splits, n_tiles;
-  float* out;
-  float* partial;
-  float* arg_val;
-  int* arg_idx;
-  int32_t* ids;
-  float* maxv;
-  unsigned* tickets;
-  unsigned* status;
-  AcceptFuse acc;   // acc.B > 0: the argmax's last CTA also runs the acceptance
-  RopeFuse rope;    // kGemmQkvRope
-};
-
-// Acceptance of sequence b from the argmax ids of its k+1 rows (one warp).
-__device__ __forceinline__ void accept_one(const AcceptFuse& f, int b, const int32_t* tg, int lane) {
-  const int k = f.k, q = k + 1;
-  const bool match = lane < k && f.drafts[(size_t)b * k + lane] == tg[lane];
-  const unsigned mism = ~__ballot_sync(0xffffffffu, match);   // bit i: draft i not accepted
-  const int a = min(__ffs(mism) - 1, k);
-  if (lane < q) {
-    int v = -1;
-    if (lane < a) v = f.drafts[(size_t)b * k + lane];
-    else if (lane == a) v = tg[a];
-    f.emitted[(size_t)b * q + lane] = v;
-  }
-  __syncwarp();
-  if (lane == 0) {
-    f.accept_len[b] = a;
-    f.last_token[b] = tg[a];
-    f.seq_lens[b] += a + 1;
-  }
-}
-
-// QKV projection epilogue: after this CTA published its split partial, the
-// last CTA to finish a head (all splits of its D/128 column tiles) sums the
-// partials in split order, rotates each (j, j + D/2) pair of query and key
-// heads at its row's position and writes queries to the workspace and keys,
-// values and the key-equals-value side-band to the cache pools.
-template <int MP>
-__device__ __forceinline__ void rope_epilogue(const Args& a, int n_tile, int mblk, int m0, int ctid,
-                                              int* flag) {
-  const RopeFuse& f = a.rope;
-  const int D = f.head_dim, half = D / 2, tph = D / kTileN;
-  const int head = n_tile / tph, n_heads = a.N / D;
-  if (ctid == 0) {
-    const unsigned prev = atomicAdd(&a.tickets[mblk * n_heads + head], 1u);
-    *flag = (prev == (unsigned)(a.splits * tph - 1));
-  }
-  named_bar(1, kConsumerWarps * 32);
-  if (!*flag) return;
-  __threadfence();
-  const int mcount = min(MP, a.M - m0);
-  const size_t split_stride = (size_t)a.n_tiles * kTileN * MP;
-  const float* base = a.partial + (size_t)mblk * a.splits * a.n_tiles * kTileN * MP;
-  for (int item = ctid; item < half * mcount; item += kConsumerWarps * 32) {
-    const int mm = item / half, j = item % half;
-    const int f0 = head * D + j, f1 = f0 + half;
-    const float* p0 = base + ((size_t)(f0 / kTileN) * kTileN + f0 % kTileN) * MP + mm;
-    const float* p1 = base + ((size_t)(f1 / kTileN) * kTileN + f1 % kTileN) * MP + mm;
-    float x0 = 0.f, x1 = 0.f;
-    int sp = 0;
-    for (; sp + 4 <= a.splits; sp += 4) {
-      float u[4], v[4];
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        u[w] = __ldcg(p0 + (size_t)(sp + w) * split_stride);
-        v[w] = __ldcg(p1 + (size_t)(sp + w) * split_stride);
-      }
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        x0 = __fadd_rn(x0, u[w]);
-        x1 = __fadd_rn(x1, v[w]);
-      }
-    }
-    for (; sp < a.splits; ++sp) {
-      x0 = __fadd_rn(x0, __ldcg(p0 + (size_t)sp * split_stride));
-      x1 = __fadd_rn(x1, __ldcg(p1 + (size_t)sp * split_stride));
-    }
-    const int m = m0 + mm, b = m / f.q, i = m % f.q;
-    const bool rot = j < f.n_rot && head < f.n_q_heads + f.n_kv_heads;
-    float y0 = x0, y1 = x1;
-    if (rot) {
-      const float2 cs = f.rope_tab[(size_t)m * half + j];
-      rope_pair(x0, x1, cs.x, cs.y, y0, y1);
-    }
-    if (head < f.n_q_heads) {
-      uint16_t* qo = f.q_out + ((size_t)m * f.n_q_heads + head) * D;
-      qo[j] = f32_to_bf16(y0);
-      qo[j + half] = f32_to_bf16(y1);
-      continue;
-    }
-    const int pos = f.seq_lens[b] + i;
-    if (pos < 0 || pos / f.page_size >= f.max_pages) {
-      flag_status(a.status, SPEC_DEV_BAD_LENGTH);
-      continue;
-    }
-    const int page = f.block_table[(size_t)b * f.max_pages + pos / f.page_size];
-    if (page < 0 || page >= f.num_pages) {
-      flag_status(a.status, SPEC_DEV_BAD_PAGE);
-      continue;
-    }
-    const int kvh = head < f.n_q_heads + f.n_kv_heads ? head - f.n_q_heads
-                                                      : head - f.n_q_heads - f.n_kv_heads;
-    const size_t row = ((size_t)page * f.n_kv_heads + kvh) * f.page_size + pos % f.page_size;
-    if (head < f.n_q_heads + f.n_kv_heads) {
-      f.k_pool[row * D + j] = f32_to_bf16(y0);
-      f.k_pool[row * D + j + half] = f32_to_bf16(y1);
-      if (f.ksb_pool && j < f.n_rot) {
-        f.ksb_pool[row * 2 * f.n_rot + j] = f32_to_bf16(x0);
-        f.ksb_pool[row * 2 * f.n_rot + f.n_rot + j] = f32_to_bf16(x1);
-      }
-    } else {
-      f.v_pool[row * D + j] = f32_to_bf16(x0);
-      f.v_pool[row * D + j + half] = f32_to_bf16(x1);
-    }
-  }
-  if (ctid == 0) a.tickets[mblk * n_heads + head] = 0u;
-}
 
 template <int NT, int MODE>
 __global__ void __launch_bounds__(kThreads) stream_gemm_kernel(
@@ -332,55 +211,7 @@ __global__ void __launch_bounds__(kThreads) stream_gemm_kernel(
       a.arg_val[o] = bv;
       a.arg_idx[o] = bi;
     }
-    __threadfence();
-    named_bar(1, kConsumerWarps * 32);
-    if (ctid == 0) {
-      const unsigned prev = atomicAdd(&a.tickets[mblk], 1u);
-      *flag = (prev == (unsigned)(a.n_tiles - 1));
-    }
-    named_bar(1, kConsumerWarps * 32);
-    if (!*flag) return;
-    __threadfence();
-    // ---- last CTA of this M-block: each warp reduces whole rows over all
-    //      tiles (lanes stride the tiles), lowest index wins ties
-    const int mcount = min(kMBlock, a.M - m0);
-    int* ids_s = red_i;   // reused: final ids of this block's rows (mcount <= MP)
-    for (int mm = warp; mm < mcount; mm += kConsumerWarps) {
-      const int m = m0 + mm;
-      float bv = -INFINITY;
-      int bi = 0x7fffffff;
-#pragma unroll 8
-      for (int tile = lane; tile < a.n_tiles; tile += 32) {
-        const float v = __ldcg(&a.arg_val[(size_t)tile * a.M + m]);
-        const int i = __ldcg(&a.arg_idx[(size_t)tile * a.M + m]);
-        if (better(v, i, bv, bi)) {
-          bv = v;
-          bi = i;
-        }
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-        if (better(ov, oi, bv, bi)) {
-          bv = ov;
-          bi = oi;
-        }
-      }
-      if (lane == 0) {
-        a.ids[m] = bi;
-        if (a.maxv) a.maxv[m] = bv;
-        ids_s[mm] = bi;
-        if (a.acc.copy_ids) a.acc.copy_ids[m] = bi;
-        if (a.acc.copy_max) a.acc.copy_max[m] = bv;
-      }
-    }
-    if (ctid == 0) a.tickets[mblk] = 0u;
-    if (a.acc.B > 0) {                 // all rows are in this block (M <= 64)
-      named_bar(1, kConsumerWarps * 32);
-      for (int b = warp; b < a.acc.B; b += kConsumerWarps)
-        accept_one(a.acc, b, ids_s + b * (a.acc.k + 1), lane);
-    }
+    argmax_finish(a, a.n_tiles, mblk, m0, kMBlock, ctid, flag, red_i);
     return;
   }
 
@@ -420,45 +251,10 @@ __global__ void __launch_bounds__(kThreads) stream_gemm_kernel(
   __threadfence();
   named_bar(1, kConsumerWarps * 32);
   if (MODE == kGemmQkvRope) {
-    rope_epilogue<MP>(a, n_tile, mblk, m0, ctid, flag);
+    rope_epilogue(a, MP, n_tile, mblk, m0, ctid, flag);
     return;
   }
-  if (ctid == 0) {
-    unsigned* tk = &a.tickets[mblk * a.n_tiles + n_tile];
-    const unsigned prev = atomicAdd(tk, 1u);
-    *flag = (prev == (unsigned)(a.splits - 1));
-  }
-  named_bar(1, kConsumerWarps * 32);
-  if (!*flag) return;
-  __threadfence();
-  // last split of this tile: sum partials in split order, then the epilogue.
-  // Work item = (output feature r, row mm); the split loads of an item are
-  // issued together (independent) and then added in split order.
-  const int mcount = min(MP, a.M - m0);
-  const size_t split_stride = (size_t)a.n_tiles * kTileN * MP;
-  const float* base = a.partial + ((size_t)mblk * a.splits * a.n_tiles + n_tile) * kTileN * MP;
-  for (int item = ctid; item < kTileN * mcount; item += kConsumerWarps * 32) {
-    const int mm = item / kTileN, r = item % kTileN;
-    const int n = n_tile * kTileN + r;
-    if (n >= a.N) continue;
-    const float* p = base + (size_t)r * MP + mm;
-    float s = 0.f;
-    int sp = 0;
-    for (; sp + 8 <= a.splits; sp += 8) {
-      float v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = __ldcg(p + (size_t)(sp + u) * split_stride);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) s = __fadd_rn(s, v[u]);
-    }
-    for (; sp < a.splits; ++sp) s = __fadd_rn(s, __ldcg(p + (size_t)sp * split_stride));
-    float* dst = a.out + (size_t)(m0 + mm) * a.N + n;
-    if (MODE == kGemmResidual)
-      *dst = __fadd_rn(*dst, s);
-    else
-      *dst = s;
-  }
-  if (ctid == 0) a.tickets[mblk * a.n_tiles + n_tile] = 0u;
+  splitk_finish<MODE>(a, MP, n_tile, mblk, m0, ctid, flag);
 }
 
 template <int NT, int MODE>

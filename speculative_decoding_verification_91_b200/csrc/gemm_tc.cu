@@ -1,0 +1,370 @@
+// Streaming GEMM on the 5th-generation tensor cores (tcgen05 + TMEM) for
+// verify steps with many rows (M = B*(k+1) up to 256, e.g. batch 64 x 4
+// rows): Y = X . W^T with W [N][K] streamed once from HBM and every verify
+// row in the MMA's N dimension, so the weights are read once whatever M is.
+//
+// One CTA per (128-row weight tile, K split); 6 warps:
+//   warp 0   TMA producer: W box 128 x 64 and X box NP x 64 (128-byte
+//            swizzle) into a ring of stages (mbarrier full/empty); the first
+//            ring of W tiles is requested before the programmatic-launch wait;
+//   warp 1   allocates the TMEM accumulator (128 lanes x NP fp32 columns) and
+//            one elected thread issues tcgen05.mma kind::f16 (A = W tile,
+//            B = X tile, both K-major SW128 shared-memory descriptors), 4 MMAs
+//            of K = 16 per stage; tcgen05.commit releases each stage and, after
+//            the last, signals the accumulator;
+//   warps 2-5 read the accumulator with tcgen05.ld (warp w owns TMEM lanes
+//            32*(w%4)..: one weight row per thread) and run the epilogue:
+//            per-tile argmax over the 128 rows of every verify row, or the
+//            split-K partial tile for the store / residual / RoPE epilogues.
+//
+// Every wait is bounded; the CTA always reaches its final barrier and frees
+// its TMEM, also after a timeout.
+#include <algorithm>
+#include <cstdlib>
+
+#include "common.cuh"
+#include "gemm_epi.cuh"
+#include "internal.h"
+
+namespace sv {
+
+namespace {
+
+constexpr int kTcThreads = 192;
+constexpr int kTcEpiWarp0 = 2;
+constexpr uint32_t kABytes = kTileN * 128;   // 16 KB weight tile per stage
+
+// ---- tcgen05 PTX wrappers -------------------------------------------------
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(dst_smem)),
+               "r"(ncols));
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols));
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// D[tmem] (+)= A[smem desc] . B[smem desc]^T, kind::f16 (bf16 in, fp32 accumulate)
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// mbarrier arrives once all tcgen05 operations issued so far by this thread completed
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+// 32 lanes x 32 consecutive fp32 columns: thread t gets lane (quadrant + t)
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+        "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+        "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, rows of 128 B in
+// 1024-byte atoms of 8 rows (stride byte offset 1024, leading byte offset 16),
+// descriptor version 1, base offset 0 (stage buffers are 1024-aligned).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr) {
+  return (uint64_t)((smem_addr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// Instruction descriptor, kind::f16: D fp32, A and B bf16, both K-major, M = 128, N = np.
+__device__ __forceinline__ uint32_t idesc_bf16(int np) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(np >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+
+// barriers, TMEM slot, flags, then red_v / red_i [4][256] for the argmax
+constexpr uint32_t kTailBytes = 256u + 2u * 4u * 256u * 4u;
+
+struct TcLayout {
+  int stages;
+  uint32_t stage_bytes;   // kABytes + np * 128
+  uint32_t smem;          // dynamic shared memory bytes
+};
+
+__host__ __device__ inline TcLayout tc_layout(int np) {
+  TcLayout t{};
+  t.stage_bytes = kABytes + (uint32_t)np * 128u;
+  // two CTAs per SM when the ring fits 2 stages in ~110 KB, else one
+  const uint32_t budget = 110u * 1024u;
+  int s = (int)((budget - 1024u - kTailBytes) / t.stage_bytes);
+  s = s < 2 ? 2 : (s > 6 ? 6 : s);
+  t.stages = s;
+  t.smem = 1024u + (uint32_t)s * t.stage_bytes + kTailBytes;
+  return t;
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kTcThreads, 2) tc_gemm_kernel(
+    const __grid_constant__ CUtensorMap tw, const __grid_constant__ CUtensorMap tx, Args a) {
+  const int np = a.np;
+  const TcLayout L = tc_layout(np);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* tail = smem + L.stages * L.stage_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(tail);
+  uint64_t* empty = full + L.stages;
+  uint64_t* acc_full = empty + L.stages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+  int* flag = reinterpret_cast<int*>(tmem_slot + 1);
+  volatile int* fail = flag + 1;
+  float* red_v = reinterpret_cast<float*>(smem + L.stages * L.stage_bytes + 256);   // [4][256]
+  int* red_i = reinterpret_cast<int*>(red_v + 4 * 256);                              // [4][256]
+
+  pdl_trigger();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_tile = blockIdx.x, split = blockIdx.y;
+  const int kc0 = (int)((long)split * a.kchunks / a.splits);
+  const int kc1 = (int)((long)(split + 1) * a.kchunks / a.splits);
+  const int nk = kc1 - kc0;
+  const uint32_t ncols = np <= 32 ? 32u : (np <= 64 ? 64u : (np <= 128 ? 128u : 256u));
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < L.stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    *fail = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, ncols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tw);
+      prefetch_tmap(&tx);
+      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_x = policy_evict_last();
+      const int pre = min(nk, L.stages);
+      for (int it = 0; it < pre; ++it) {
+        mbar_arrive_expect_tx(&full[it], L.stage_bytes);
+        tma_load_2d(smem + it * L.stage_bytes, &tw, &full[it], (kc0 + it) * kTileK, n_tile * kTileN,
+                    pol_w);
+      }
+      pdl_wait();
+      for (int it = 0; it < pre; ++it)
+        tma_load_2d(smem + it * L.stage_bytes + kABytes, &tx, &full[it], (kc0 + it) * kTileK, 0, pol_x);
+      int issued = pre;
+      for (int it = pre; it < nk; ++it) {
+        const int s = it % L.stages;
+        if (*fail || !mbar_wait(&empty[s], ((it / L.stages) - 1) & 1, a.status)) {
+          *fail = 1;
+          break;
+        }
+        uint8_t* st = smem + s * L.stage_bytes;
+        mbar_arrive_expect_tx(&full[s], L.stage_bytes);
+        const int kx = (kc0 + it) * kTileK;
+        tma_load_2d(st, &tw, &full[s], kx, n_tile * kTileN, pol_w);
+        tma_load_2d(st + kABytes, &tx, &full[s], kx, 0, pol_x);
+        issued = it + 1;
+      }
+      for (int it = (issued > L.stages ? issued - L.stages : 0); it < issued; ++it)
+        mbar_wait(&full[it % L.stages], (it / L.stages) & 1, a.status);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(np);
+      int done = 0;
+      for (int it = 0; it < nk; ++it) {
+        const int s = it % L.stages;
+        if (*fail || !mbar_wait(&full[s], (it / L.stages) & 1, a.status)) {
+          *fail = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(smem + s * L.stage_bytes);
+        const uint32_t b_addr = a_addr + kABytes;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)   // K = 16 per MMA: +32 bytes inside the swizzled rows
+          umma_bf16(tmem, sw128_desc(a_addr + kk * 32), sw128_desc(b_addr + kk * 32), idesc,
+                    (it > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(&empty[s]);
+        done = it + 1;
+      }
+      umma_commit(acc_full);             // fires once every MMA issued above has completed
+      // the accumulator must be complete before the CTA may free its TMEM
+      mbar_wait(acc_full, 0, a.status);
+      (void)done;
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int ctid = threadIdx.x - kTcEpiWarp0 * 32;      // 0..127
+    const int quad = warp & 3;                             // TMEM lanes 32*quad ..
+    const int row = quad * 32 + lane;                      // weight row within the tile
+    const bool ok = mbar_wait(acc_full, 0, a.status);
+    tc_fence_after();
+    if (!ok) *fail = 1;
+    named_bar(1, kEpiThreads);
+    if (!*fail) {
+      const uint32_t tq = tmem + ((uint32_t)(quad * 32) << 16);
+      if (MODE == kGemmArgmax) {
+        // per verify row (column): max over this tile's 128 weight rows
+        const int n = n_tile * kTileN + row;
+        for (int c0 = 0; c0 < np; c0 += 32) {
+          float v[32];
+          int id[32];
+          tmem_ld32(tq + c0, v);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            id[j] = n;
+            if (n >= a.N) v[j] = -INFINITY;
+          }
+          // transpose-reduce: after the 5 rounds lane l holds column c0 + l
+#pragma unroll
+          for (int r = 0; r < 5; ++r) {
+            const int off = 16 >> r, half = 16 >> r;
+            const bool up = (lane & off) != 0;
+#pragma unroll
+            for (int j = 0; j < half; ++j) {
+              const float sv = up ? v[j] : v[j + half];
+              const int si = up ? id[j] : id[j + half];
+              const float kv = up ? v[j + half] : v[j];
+              const int ki = up ? id[j + half] : id[j];
+              const float ov = __shfl_xor_sync(0xffffffffu, sv, off);
+              const int oi = __shfl_xor_sync(0xffffffffu, si, off);
+              const bool take = better(ov, oi, kv, ki);
+              v[j] = take ? ov : kv;
+              id[j] = take ? oi : ki;
+            }
+          }
+          if (c0 + lane < np) {
+            red_v[quad * 256 + c0 + lane] = v[0];
+            red_i[quad * 256 + c0 + lane] = id[0];
+          }
+        }
+        named_bar(1, kEpiThreads);
+        for (int c = ctid; c < np && c < a.M; c += kEpiThreads) {
+          float bv = red_v[c];
+          int bi = red_i[c];
+          for (int q2 = 1; q2 < 4; ++q2)
+            if (better(red_v[q2 * 256 + c], red_i[q2 * 256 + c], bv, bi)) {
+              bv = red_v[q2 * 256 + c];
+              bi = red_i[q2 * 256 + c];
+            }
+          a.arg_val[(size_t)n_tile * a.M + c] = bv;
+          a.arg_idx[(size_t)n_tile * a.M + c] = bi;
+        }
+      } else {
+        // split-K partial tile [128 rows][np], then the shared epilogues
+        float* mine = a.partial + ((size_t)split * a.n_tiles + n_tile) * kTileN * np;
+        for (int c0 = 0; c0 < np; c0 += 32) {
+          float v[32];
+          tmem_ld32(tq + c0, v);
+#pragma unroll
+          for (int j = 0; j < 32; j += 4)
+            if (c0 + j < np)   // np is a multiple of 16: a float4 is wholly inside or outside
+              __stcg(reinterpret_cast<float4*>(mine + (size_t)row * np + c0 + j),
+                     make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]));
+        }
+      }
+    }
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, ncols);
+  if (warp < kTcEpiWarp0 || *fail) return;
+
+  // ---- cross-CTA completion (epilogue warps only)
+  const int ctid = threadIdx.x - kTcEpiWarp0 * 32;
+  if (MODE == kGemmArgmax) {
+    argmax_finish(a, a.n_tiles, 0, 0, np, ctid, flag, red_i);
+    return;
+  }
+  __threadfence();
+  named_bar(1, kEpiThreads);
+  if (MODE == kGemmQkvRope) {
+    rope_epilogue(a, np, n_tile, 0, 0, ctid, flag);
+    return;
+  }
+  splitk_finish<MODE>(a, np, n_tile, 0, 0, ctid, flag);
+}
+
+template <int MODE>
+cudaError_t launch_tc_mode(const GemmPlan& p, const CUtensorMap& tw, const CUtensorMap& tx,
+                           const Args& a, cudaStream_t st) {
+  auto kern = tc_gemm_kernel<MODE>;
+  const TcLayout L = tc_layout(a.np);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.smem);
+  if (e != cudaSuccess) return e;
+  return launch_k(kern, dim3(p.n_tiles, p.splits, 1), dim3(kTcThreads), L.smem, st, tw, tx, a);
+}
+
+}  // namespace
+
+bool tc_supported(int M) {
+  static const bool on = [] {
+    const char* v = getenv("SPECVERIFY_NO_TC");
+    return !(v && v[0] == '1');
+  }();
+  return on && M > 64 && M <= 256;
+}
+
+int tc_np(int M) { return (M + 15) / 16 * 16; }
+
+cudaError_t launch_gemm_tc(const GemmPlan& p, int mode, const void* x, const void* w,
+                           const GemmBuffers& b, cudaStream_t st) {
+  const int np = tc_np(p.M);
+  if (!tc_supported(p.M)) return cudaErrorInvalidValue;
+  CUtensorMap tw, tx;
+  if (!make_tmap_bf16_2d(&tw, w, p.N, p.K, kTileN, kTileK)) return cudaErrorInvalidValue;
+  if (!make_tmap_bf16_2d(&tx, x, p.M, p.K, np, kTileK, p.x_row_stride)) return cudaErrorInvalidValue;
+  Args a{};
+  a.M = p.M;
+  a.N = p.N;
+  a.K = p.K;
+  a.kchunks = p.kchunks;
+  a.splits = p.splits;
+  a.n_tiles = p.n_tiles;
+  a.np = np;
+  a.out = b.out;
+  a.partial = b.partial;
+  a.arg_val = b.arg_val;
+  a.arg_idx = b.arg_idx;
+  a.ids = b.ids;
+  a.maxv = b.maxv;
+  a.tickets = b.tickets;
+  a.status = b.status;
+  a.acc = b.acc;
+  a.rope = b.rope;
+  if (mode != kGemmArgmax) a.acc.B = 0;
+  switch (mode) {
+    case kGemmStore: return launch_tc_mode<kGemmStore>(p, tw, tx, a, st);
+    case kGemmResidual: return launch_tc_mode<kGemmResidual>(p, tw, tx, a, st);
+    case kGemmArgmax: return launch_tc_mode<kGemmArgmax>(p, tw, tx, a, st);
+    case kGemmQkvRope: return launch_tc_mode<kGemmQkvRope>(p, tw, tx, a, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace sv

@@ -75,6 +75,18 @@ struct GemmBuffers {
 };
 cudaError_t launch_gemm(const GemmPlan& p, int mode, const void* x, const void* w,
                         const GemmBuffers& buf, cudaStream_t st);
+// The same GEMMs on tcgen05 / TMEM for 64 < M <= 256 rows: every row sits in
+// the MMA's N dimension, so the weights stream once.  tc_supported() is false
+// outside that range or when SPECVERIFY_NO_TC=1.
+bool tc_supported(int M);
+cudaError_t launch_gemm_tc(const GemmPlan& p, int mode, const void* x, const void* w,
+                           const GemmBuffers& buf, cudaStream_t st);
+// tcgen05 path when it applies, else the mma.sync path
+inline cudaError_t launch_gemm_any(const GemmPlan& p, int mode, const void* x, const void* w,
+                                   const GemmBuffers& buf, cudaStream_t st) {
+  return tc_supported(p.M) ? launch_gemm_tc(p, mode, x, w, buf, st)
+                           : launch_gemm(p, mode, x, w, buf, st);
+}
 
 // ------------------------------------------------------------- small kernels
 cudaError_t launch_rmsnorm(const float* x, int M, int d, double eps, uint16_t* out,

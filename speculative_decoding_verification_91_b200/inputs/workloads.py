@@ -114,6 +114,11 @@ WORKLOADS.update({
                                                 vocab=4100, ctx_lo=60, ctx_hi=900,
                                                 layers=(LayerSpec(window=200, split_tokens=64),) * 2
                                                 + (GLOBAL_KV,)),
+    # 32 sequences x 4 rows = 128 verify rows: the many-row (tensor-memory) GEMM path
+    "small_b32": WORKLOADS["b64_6layer"].with_(name="small_b32", batch=32, d_model=768,
+                                                vocab=4100, ctx_lo=60, ctx_hi=700,
+                                                layers=(LayerSpec(window=200, split_tokens=64),
+                                                        GLOBAL_KV)),
     "small_loop": WORKLOADS["loop_131k"].with_(name="small_loop", vocab=6000, d_model=512,
                                                 ctx_lo=700, ctx_hi=700, prompt_tokens=700,
                                                 layers=(LayerSpec(window=128),) * 3 + (GLOBAL_KV,),

@@ -68,7 +68,8 @@ def test_accept_commit_matches_oracle(k):
 # ---------------------------------------------------------------- LM head
 
 @pytest.mark.parametrize("M,d,V", [(1, 512, 4096), (5, 2560, 9000), (9, 256, 1000),
-                                   (40, 1024, 5000), (100, 512, 3000), (64, 2048, 131)])
+                                   (40, 1024, 5000), (100, 512, 3000), (64, 2048, 131),
+                                   (256, 1024, 5000), (72, 3840, 1000)])
 def test_lmhead_argmax_matches_oracle(M, d, V):
     h = gen.normal_bf16(1, f"test/lm/h/{M}/{d}", 0, M * d, 1.0).reshape(M, d)
     w = gen.normal_bf16(1, f"test/lm/w/{d}/{V}", 0, V * d, 0.02).reshape(V, d)
@@ -193,7 +194,7 @@ def _run_step(wl, cases):
     return s, s.outputs()
 
 
-@pytest.mark.parametrize("name", ["tiny", "small_b1", "small_ragged", "small_b16"])
+@pytest.mark.parametrize("name", ["tiny", "small_b1", "small_ragged", "small_b16", "small_b32"])
 def test_verify_step_matches_oracle(name):
     wl = W.get_workload(name)
     model = harness.oracle_model(wl)
