@@ -309,8 +309,50 @@ def oracle_sample(wl_name: str, budget_s: float = 25.0):
     return tokens / dt, dt / n, threads, desc
 
 
+def run_lmhead_only(args):
+    """--workload lmhead:M,d,V: the LM head + argmax kernel alone on random bf16
+    inputs, L2 flushed before every launch; reports its roofline."""
+    import torch
+    from speculative_decoding_verification_91_b200 import binding as B
+    from speculative_decoding_verification_91_b200.inputs import gen
+    from speculative_decoding_verification_91_b200.runtime import Workspace, to_device_bf16
+    M, d, V = (int(x) for x in args.workload.split(":")[1].split(","))
+    torch.cuda.set_device(0)
+    h = to_device_bf16(gen.normal_bf16(0, "bench/lm/h", 0, M * d, 1.0), "cuda")
+    w = to_device_bf16(gen.normal_bf16(0, "bench/lm/w", 0, V * d, 0.02), "cuda")
+    ws = Workspace(B.spec_lmhead_workspace_bytes(M, V))
+    ids = torch.zeros(M, dtype=torch.int32, device="cuda")
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    for _ in range(args.warmup):
+        B.spec_lmhead_argmax(h, w, M, d, V, ids, None, ws.buf, ws.nbytes)
+    t0 = [ev() for _ in range(args.steps)]
+    t1 = [ev() for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        t0[i].record()
+        B.spec_lmhead_argmax(h, w, M, d, V, ids, None, ws.buf, ws.nbytes)
+        t1[i].record()
+    torch.cuda.synchronize()
+    us = float(np.mean([a.elapsed_time(b) for a, b in zip(t0, t1)])) * 1e3
+    byts = V * d * 2 + M * d * 2
+    flops = 2.0 * M * d * V
+    peak, kind = measured_peaks()
+    tf = None
+    mp = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(mp):
+        tf = json.load(open(mp)).get("bf16_tflops")
+    print(json.dumps({"kernel": "lmhead_argmax", "M": M, "d": d, "V": V, "us": us,
+                      "gbs": byts / us / 1e3, "frac_hbm": byts / us / 1e3 / peak,
+                      "tflops": flops / us / 1e6,
+                      "frac_tensor": (flops / us / 1e6 / tf) if tf else None}), flush=True)
+
+
 def main():
     args = parse()
+    if args.workload.startswith("lmhead:"):
+        run_lmhead_only(args)
+        return
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
