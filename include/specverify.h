@@ -140,8 +140,9 @@ size_t spec_workspace_bytes(const spec_model* m, int max_batch, int max_k, int m
 /* Workspace bytes spec_lmhead_argmax needs on its own for M rows and vocab V. */
 size_t spec_lmhead_workspace_bytes(int M, int V);
 
-/* Clears the workspace's counters and status word (async memset).  Call once
- * after allocating a workspace; every kernel leaves its counters at zero. */
+/* Clears the whole workspace (async memset): counters, status word and the
+ * argmax keys must start at zero.  Call once after allocating a workspace;
+ * every kernel leaves them at zero again. */
 int spec_workspace_init(void* ws, size_t ws_bytes, void* stream);
 
 /* Reads and clears the device status word (synchronises the stream).
@@ -239,9 +240,10 @@ int spec_prefill(const spec_model* m, const int32_t* block_table, int max_pages,
  * cannot take cudaMalloc's implicit device synchronisation.
  *
  * Same operation, arguments and errors as spec_lmhead_argmax, minus the
- * workspace.  Its scratch (argmax partials, a completion counter, a status
- * word) is a file-scope __device__ array inside the library, of about 1 MiB,
- * that every GPU which loads the library holds until the process exits.
+ * workspace.  Its scratch (one argmax key per row, a completion counter, a
+ * status word) is a file-scope __device__ array inside the library, of about
+ * 4.5 KiB, that every GPU which loads the library holds until the process
+ * exits.
  * Limits: M <= SPEC_NOALLOC_MAX_ROWS and ceil(V / 128) * M <=
  * SPEC_NOALLOC_MAX_TILE_ROWS (so V = 262,144 allows M <= 64); larger
  * problems return SPEC_EUNSUPPORTED and launch nothing.
@@ -249,7 +251,7 @@ int spec_prefill(const spec_model* m, const int32_t* block_table, int max_pages,
  * The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current; make that first call
  * before any stream capture.  Each call clears the counter and status word
- * (an async memset on `stream`) and allocates nothing.  All calls share the
+ * and keys (an async memset on `stream`) and allocates nothing.  All calls share the
  * one array, which keeps the last call's contents: calls that overlap on the
  * GPU (different streams, or concurrent host threads on one device) race and
  * must be serialised by the caller. */

@@ -102,7 +102,7 @@ int check_model(const spec_model* m) {
 // Workspace layout of one forward over q rows per sequence (q = k + 1 for a
 // verify step, q = n for a prefill chunk) for (B, q, max_pages).
 struct StepLayout {
-  size_t x, hn, qrot, attn_out, attn_part, gemm_part, arg_val, arg_idx, ids, maxv, rope_tab,
+  size_t x, hn, qrot, attn_out, attn_part, gemm_part, arg_keys, ids, maxv, rope_tab,
       total;
   int tickets;
   bool splits_ok;   // every layer's split count fits the combine kernel
@@ -134,8 +134,7 @@ StepLayout step_layout(const spec_model* m, int B, int q, int max_pages) {
   s.attn_out = off;  off = up(off + (size_t)M * m->n_q_heads * D * 2);
   s.attn_part = off; off = up(off + attn_floats * 4);
   s.gemm_part = off; off = up(off + gemm_floats * 4);
-  s.arg_val = off;   off = up(off + gemm_argmax_entries(pl) * 4);
-  s.arg_idx = off;   off = up(off + gemm_argmax_entries(pl) * 4);
+  s.arg_keys = off;  off = up(off + gemm_argmax_entries(pl) * 8);
   s.ids = off;       off = up(off + (size_t)M * 4);
   s.maxv = off;      off = up(off + (size_t)M * 4);
   s.rope_tab = off;  off = up(off + (size_t)M * (D / 2) * 8);
@@ -263,8 +262,7 @@ int run_forward(const spec_model* m, const int32_t* block_table, int max_pages, 
   // LM head: every row (verify) or each sequence's last row (prefill)
   GemmPlan pl = plan_gemm(prefill ? B : M, m->vocab, d, kGemmArgmax);
   GemmBuffers bl{};
-  bl.arg_val = at<float>(ws, s.arg_val);
-  bl.arg_idx = at<int>(ws, s.arg_idx);
+  bl.arg_keys = at<unsigned long long>(ws, s.arg_keys);
   bl.ids = at<int32_t>(ws, s.ids);
   bl.maxv = at<float>(ws, s.maxv);
   bl.tickets = hdr.tickets;
@@ -374,12 +372,12 @@ size_t spec_workspace_bytes(const spec_model* m, int max_batch, int max_k, int m
 size_t spec_lmhead_workspace_bytes(int M, int V) {
   if (M < 1 || V < 1) return 0;
   GemmPlan p = plan_gemm(M, V, 64, kGemmArgmax);
-  return kWsHeaderBytes + up(gemm_argmax_entries(p) * 4) * 2;
+  return kWsHeaderBytes + up(gemm_argmax_entries(p) * 8);
 }
 
 int spec_workspace_init(void* ws, size_t ws_bytes, void* stream) {
   if (!ws || ws_bytes < kWsHeaderBytes) return SPEC_EINVAL;
-  return cuda_status(cudaMemsetAsync(ws, 0, kWsHeaderBytes, static_cast<cudaStream_t>(stream)));
+  return cuda_status(cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream)));
 }
 
 int spec_read_device_status(void* ws, size_t ws_bytes, void* stream, unsigned* status) {
@@ -490,8 +488,7 @@ int spec_lmhead_argmax(const void* h, const void* w, int M, int d, int V, int32_
   if (ws_bytes < need) return SPEC_EINVAL;
   WsHeader hdr = ws_header(ws);
   GemmBuffers b{};
-  b.arg_val = at<float>(ws, kWsHeaderBytes);
-  b.arg_idx = at<int>(ws, kWsHeaderBytes + up(gemm_argmax_entries(p) * 4));
+  b.arg_keys = at<unsigned long long>(ws, kWsHeaderBytes);
   b.ids = ids;
   b.maxv = maxlogit;
   b.tickets = hdr.tickets;

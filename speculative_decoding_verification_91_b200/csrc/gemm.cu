@@ -207,9 +207,7 @@ __global__ void __launch_bounds__(kThreads) stream_gemm_kernel(
           bi = i;
         }
       }
-      const size_t o = (size_t)n_tile * a.M + m0 + ctid;
-      a.arg_val[o] = bv;
-      a.arg_idx[o] = bi;
+      atomicMax(&a.arg_keys[m0 + ctid], pack_arg(bv, bi));
     }
     argmax_finish(a, a.n_tiles, mblk, m0, kMBlock, ctid, flag, red_i);
     return;
@@ -308,7 +306,7 @@ GemmPlan plan_gemm(int M, int N, int K, int mode) {
 size_t gemm_partial_floats(const GemmPlan& p) {
   return (size_t)p.mblocks * p.splits * p.n_tiles * kTileN * (p.nt * 8);
 }
-size_t gemm_argmax_entries(const GemmPlan& p) { return (size_t)p.n_tiles * p.M; }
+size_t gemm_argmax_entries(const GemmPlan& p) { return (size_t)p.M; }
 int gemm_tickets(const GemmPlan& p) { return p.mblocks * p.n_tiles; }
 
 cudaError_t launch_gemm(const GemmPlan& p, int mode, const void* x, const void* w,
@@ -326,8 +324,7 @@ cudaError_t launch_gemm(const GemmPlan& p, int mode, const void* x, const void* 
   a.n_tiles = p.n_tiles;
   a.out = b.out;
   a.partial = b.partial;
-  a.arg_val = b.arg_val;
-  a.arg_idx = b.arg_idx;
+  a.arg_keys = b.arg_keys;
   a.ids = b.ids;
   a.maxv = b.maxv;
   a.tickets = b.tickets;

@@ -18,8 +18,7 @@ struct Args {
   int np;           // tcgen05 kernel: padded token count (MMA N)
   float* out;
   float* partial;
-  float* arg_val;
-  int* arg_idx;
+  unsigned long long* arg_keys;   // [M] packed (value, id) keys, zero between launches
   int32_t* ids;
   float* maxv;
   unsigned* tickets;
@@ -48,61 +47,56 @@ __device__ __forceinline__ void accept_one(const AcceptFuse& f, int b, const int
   }
 }
 
-// After this CTA wrote its per-tile argmax partials (rows m0..): the last CTA
-// of the M-block reduces every row over all tiles (each warp whole rows,
-// lanes striding the tiles; lowest index wins ties) and, when fused, runs the
-// acceptance of every sequence.  ids_s: shared scratch of >= mrows ints.
+// Argmax candidates are published as one 64-bit key per row and merged with
+// atomicMax: the key orders by value (order-preserving binary32 bits) and, for
+// equal values, by the lower token id (id stored as 0xFFFFFFFF - id).  The
+// maximum of a set of keys does not depend on the order of the atomics, so
+// the result is deterministic.  A zero key is below every real candidate.
+__device__ __forceinline__ unsigned long long pack_arg(float v, int idx) {
+  uint32_t u = __float_as_uint(v);
+  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return ((unsigned long long)u << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)idx);
+}
+__device__ __forceinline__ void unpack_arg(unsigned long long key, float& v, int& idx) {
+  const uint32_t hi = (uint32_t)(key >> 32);
+  v = __uint_as_float((hi & 0x80000000u) ? (hi & 0x7FFFFFFFu) : ~hi);
+  idx = (int)(0xFFFFFFFFu - (uint32_t)(key & 0xFFFFFFFFull));
+}
+
+// After this CTA merged its per-tile candidates into the row keys: the last
+// CTA of the M-block turns the keys of its rows into ids / max logits, clears
+// them for the next launch and, when fused, runs the acceptance of every
+// sequence.  ids_s: shared scratch of >= mrows ints.
 __device__ __forceinline__ void argmax_finish(const Args& a, int n_parts, int mblk, int m0,
                                               int mrows, int ctid, int* flag, int* ids_s) {
   const int warp = ctid >> 5, lane = ctid & 31;
-    __threadfence();
+  __threadfence();
+  named_bar(1, kEpiThreads);
+  if (ctid == 0) {
+    const unsigned prev = atomicAdd(&a.tickets[mblk], 1u);
+    *flag = (prev == (unsigned)(n_parts - 1));
+  }
+  named_bar(1, kEpiThreads);
+  if (!*flag) return;
+  __threadfence();
+  const int mcount = min(mrows, a.M - m0);
+  for (int mm = ctid; mm < mcount; mm += kEpiThreads) {
+    const int m = m0 + mm;
+    float bv;
+    int bi;
+    unpack_arg(atomicExch(&a.arg_keys[m], 0ull), bv, bi);
+    a.ids[m] = bi;
+    if (a.maxv) a.maxv[m] = bv;
+    ids_s[mm] = bi;
+    if (a.acc.copy_ids) a.acc.copy_ids[m] = bi;
+    if (a.acc.copy_max) a.acc.copy_max[m] = bv;
+  }
+  if (ctid == 0) a.tickets[mblk] = 0u;
+  if (a.acc.B > 0) {                 // all rows are in this block
     named_bar(1, kEpiThreads);
-    if (ctid == 0) {
-      const unsigned prev = atomicAdd(&a.tickets[mblk], 1u);
-      *flag = (prev == (unsigned)(n_parts - 1));
-    }
-    named_bar(1, kEpiThreads);
-    if (!*flag) return;
-    __threadfence();
-    // ---- last CTA of this M-block: each warp reduces whole rows over all
-    //      tiles (lanes stride the tiles), lowest index wins ties
-    const int mcount = min(mrows, a.M - m0);
-    for (int mm = warp; mm < mcount; mm += kEpiThreads / 32) {
-      const int m = m0 + mm;
-      float bv = -INFINITY;
-      int bi = 0x7fffffff;
-#pragma unroll 8
-      for (int tile = lane; tile < n_parts; tile += 32) {
-        const float v = __ldcg(&a.arg_val[(size_t)tile * a.M + m]);
-        const int i = __ldcg(&a.arg_idx[(size_t)tile * a.M + m]);
-        if (better(v, i, bv, bi)) {
-          bv = v;
-          bi = i;
-        }
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-        if (better(ov, oi, bv, bi)) {
-          bv = ov;
-          bi = oi;
-        }
-      }
-      if (lane == 0) {
-        a.ids[m] = bi;
-        if (a.maxv) a.maxv[m] = bv;
-        ids_s[mm] = bi;
-        if (a.acc.copy_ids) a.acc.copy_ids[m] = bi;
-        if (a.acc.copy_max) a.acc.copy_max[m] = bv;
-      }
-    }
-    if (ctid == 0) a.tickets[mblk] = 0u;
-    if (a.acc.B > 0) {                 // all rows are in this block
-      named_bar(1, kEpiThreads);
-      for (int b = warp; b < a.acc.B; b += kEpiThreads / 32)
-        accept_one(a.acc, b, ids_s + b * (a.acc.k + 1), lane);
-    }
+    for (int b = warp; b < a.acc.B; b += kEpiThreads / 32)
+      accept_one(a.acc, b, ids_s + b * (a.acc.k + 1), lane);
+  }
 }
 
 // QKV projection epilogue: after this CTA published its split partial, the

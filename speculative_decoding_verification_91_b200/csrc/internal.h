@@ -31,7 +31,7 @@ struct GemmPlan {
 };
 GemmPlan plan_gemm(int M, int N, int K, int mode);
 size_t gemm_partial_floats(const GemmPlan& p);   // split-K partial sums
-size_t gemm_argmax_entries(const GemmPlan& p);   // per-tile argmax partials
+size_t gemm_argmax_entries(const GemmPlan& p);   // argmax keys (one per row)
 int gemm_tickets(const GemmPlan& p);
 
 // Acceptance fused into the LM-head argmax (B = 0: not fused).
@@ -64,8 +64,7 @@ struct RopeFuse {
 struct GemmBuffers {
   float* out;          // kGemmStore: [M][N]; kGemmResidual: [M][N] updated in place
   float* partial;      // gemm_partial_floats()
-  float* arg_val;      // gemm_argmax_entries()
-  int* arg_idx;
+  unsigned long long* arg_keys;   // gemm_argmax_entries() keys, zero on entry and exit
   int32_t* ids;        // kGemmArgmax: [M]
   float* maxv;         // kGemmArgmax: [M] or null
   unsigned* tickets;   // gemm_tickets() counters, zero on entry, zero on exit

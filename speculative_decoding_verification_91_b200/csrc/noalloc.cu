@@ -20,8 +20,8 @@ namespace sv {
 namespace {
 
 constexpr size_t kNoAllocHeader = kWsHeaderBytes;                       // status + counters
-constexpr size_t kNoAllocEntries = (size_t)SPEC_NOALLOC_MAX_TILE_ROWS;  // tiles x rows
-constexpr size_t kNoAllocBytes = kNoAllocHeader + 2 * kNoAllocEntries * 4;
+constexpr size_t kNoAllocEntries = (size_t)SPEC_NOALLOC_MAX_ROWS;       // argmax keys (one per row)
+constexpr size_t kNoAllocBytes = kNoAllocHeader + kNoAllocEntries * 8;
 
 // One copy per GPU that loads the library; it stays allocated until exit.
 __device__ __align__(256) uint8_t g_lmhead_scratch[kNoAllocBytes];
@@ -57,20 +57,19 @@ extern "C" int spec_lmhead_argmax_noalloc(const void* h, const void* w, int M, i
   if (!h || !w || !ids || M < 1 || V < 1 || d < 8 || d % 8) return SPEC_EINVAL;
   if ((reinterpret_cast<uintptr_t>(h) & 15) || (reinterpret_cast<uintptr_t>(w) & 15)) return SPEC_EINVAL;
   GemmPlan p = plan_gemm(M, V, d, kGemmArgmax);
-  // The fixed scratch holds one M-block of rows and ceil(V/128) * M partials.
-  if (M > SPEC_NOALLOC_MAX_ROWS || gemm_argmax_entries(p) > kNoAllocEntries) return SPEC_EUNSUPPORTED;
+  // The fixed scratch holds one key per row; the tile count is bounded as documented.
+  if (M > SPEC_NOALLOC_MAX_ROWS || (size_t)p.n_tiles * M > (size_t)SPEC_NOALLOC_MAX_TILE_ROWS)
+    return SPEC_EUNSUPPORTED;
   void* scratch = nullptr;
   int rc = scratch_for_current_device(&scratch);
   if (rc) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // The array keeps the previous call's contents: the status word and the
-  // completion counter must start at zero.
-  if (cudaMemsetAsync(scratch, 0, kNoAllocHeader, st) != cudaSuccess) return SPEC_ECUDA;
+  // The array keeps the previous call's contents: the status word, the
+  // completion counter and the argmax keys must start at zero.
+  if (cudaMemsetAsync(scratch, 0, kNoAllocBytes, st) != cudaSuccess) return SPEC_ECUDA;
   WsHeader hdr = ws_header(scratch);
   GemmBuffers b{};
-  b.arg_val = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + kNoAllocHeader);
-  b.arg_idx = reinterpret_cast<int*>(static_cast<uint8_t*>(scratch) + kNoAllocHeader +
-                                     kNoAllocEntries * 4);
+  b.arg_keys = reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(scratch) + kNoAllocHeader);
   b.ids = ids;
   b.maxv = maxlogit;
   b.tickets = hdr.tickets;
