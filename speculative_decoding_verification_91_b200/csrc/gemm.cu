@@ -33,6 +33,7 @@ namespace {
 constexpr int kConsumerWarps = 4;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kMBlock = 64;
+constexpr int kFusedTailMaxRows = 16;   // up to this many rows the last CTA runs the epilogue
 
 template <int NT>
 struct Cfg {
@@ -233,8 +234,8 @@ __global__ void __launch_bounds__(kThreads) stream_gemm_kernel(
         }
     return;
   }
-  // split-K: publish this split's partial tile [128][MP]
-  float* mine = a.partial + (((size_t)mblk * a.splits + split) * a.n_tiles + n_tile) * kTileN * MP;
+  // split-K: publish this split's partial tile (128 features x this block's rows)
+  float* mine = a.partial + ((size_t)split * a.n_tiles + n_tile) * kTileN * a.ldp + m0;
 #pragma unroll
   for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
@@ -243,9 +244,10 @@ __global__ void __launch_bounds__(kThreads) stream_gemm_kernel(
       for (int h = 0; h < 2; ++h) {
         const int r = warp * 32 + mt * 16 + g + h * 8;
         const int c = nt * 8 + 2 * t;
-        __stcg(reinterpret_cast<float2*>(mine + (size_t)r * MP + c),
+        __stcg(reinterpret_cast<float2*>(mine + (size_t)r * a.ldp + c),
                make_float2(acc[mt][nt][h * 2], acc[mt][nt][h * 2 + 1]));
       }
+  if (a.grid_reduce) return;   // splitk_reduce_kernel finishes
   __threadfence();
   named_bar(1, kConsumerWarps * 32);
   if (MODE == kGemmQkvRope) {
@@ -253,6 +255,103 @@ __global__ void __launch_bounds__(kThreads) stream_gemm_kernel(
     return;
   }
   splitk_finish<MODE>(a, MP, n_tile, mblk, m0, ctid, flag);
+}
+
+// Split-K sum (in split order) + epilogue over the whole grid, one output
+// per thread, 32x32 tiles transposed through shared memory so that both the
+// partial reads (along rows) and the output writes (along features) coalesce.
+//   store / residual: tile = 32 features x 32 rows, out[m][n] (+)= sum
+//   QKV + RoPE: tile = 32 pairs (j, j + D/2) of one head x 32 rows
+template <int MODE>
+__global__ void __launch_bounds__(256) splitk_reduce_kernel(Args a) {
+  __shared__ float t0[32][33], t1[32][33];
+  pdl_trigger();
+  pdl_wait();
+  const int ld = a.ldp, tx = threadIdx.x, ty = threadIdx.y;   // 32 x 8
+  const int m_base = blockIdx.y * 32;
+  const size_t split_stride = (size_t)a.n_tiles * kTileN * ld;
+  if (MODE != kGemmQkvRope) {
+    const int n_base = blockIdx.x * 32;
+    for (int r = ty; r < 32; r += 8) {             // r: feature within the tile
+      const int n = n_base + r, m = m_base + tx;
+      float s = 0.f;
+      if (n < a.N && m < a.M) {
+        const float* p = a.partial + (size_t)n * ld + m;
+        for (int sp = 0; sp < a.splits; ++sp) s = __fadd_rn(s, __ldcg(p + (size_t)sp * split_stride));
+      }
+      t0[r][tx] = s;
+    }
+    __syncthreads();
+    for (int r = ty; r < 32; r += 8) {             // r: row within the tile
+      const int n = n_base + tx, m = m_base + r;
+      if (n < a.N && m < a.M) {
+        float* dst = a.out + (size_t)m * a.N + n;
+        *dst = (MODE == kGemmResidual) ? __fadd_rn(*dst, t0[tx][r]) : t0[tx][r];
+      }
+    }
+    return;
+  }
+  const RopeFuse& f = a.rope;
+  const int D = f.head_dim, half = D / 2;
+  const int pairs_per_head = half / 32;
+  const int head = blockIdx.x / pairs_per_head, j0 = (blockIdx.x % pairs_per_head) * 32;
+  for (int r = ty; r < 32; r += 8) {               // r: pair within the tile
+    const int m = m_base + tx, j = j0 + r;
+    float x0 = 0.f, x1 = 0.f;
+    if (m < a.M) {
+      const float* p0 = a.partial + (size_t)(head * D + j) * ld + m;
+      const float* p1 = a.partial + (size_t)(head * D + j + half) * ld + m;
+      for (int sp = 0; sp < a.splits; ++sp) {
+        x0 = __fadd_rn(x0, __ldcg(p0 + (size_t)sp * split_stride));
+        x1 = __fadd_rn(x1, __ldcg(p1 + (size_t)sp * split_stride));
+      }
+    }
+    t0[r][tx] = x0;
+    t1[r][tx] = x1;
+  }
+  __syncthreads();
+  for (int r = ty; r < 32; r += 8) {               // r: row within the tile
+    const int m = m_base + r, j = j0 + tx;
+    if (m >= a.M) continue;
+    const float x0 = t0[tx][r], x1 = t1[tx][r];
+    const int b = m / f.q, i = m % f.q;
+    const bool rot = j < f.n_rot && head < f.n_q_heads + f.n_kv_heads;
+    float y0 = x0, y1 = x1;
+    if (rot) {
+      const float2 cs = f.rope_tab[(size_t)m * half + j];
+      rope_pair(x0, x1, cs.x, cs.y, y0, y1);
+    }
+    if (head < f.n_q_heads) {
+      uint16_t* qo = f.q_out + ((size_t)m * f.n_q_heads + head) * D;
+      qo[j] = f32_to_bf16(y0);
+      qo[j + half] = f32_to_bf16(y1);
+      continue;
+    }
+    const int pos = f.seq_lens[b] + i;
+    if (pos < 0 || pos / f.page_size >= f.max_pages) {
+      flag_status(a.status, SPEC_DEV_BAD_LENGTH);
+      continue;
+    }
+    const int page = f.block_table[(size_t)b * f.max_pages + pos / f.page_size];
+    if (page < 0 || page >= f.num_pages) {
+      flag_status(a.status, SPEC_DEV_BAD_PAGE);
+      continue;
+    }
+    const int kvh = head < f.n_q_heads + f.n_kv_heads ? head - f.n_q_heads
+                                                      : head - f.n_q_heads - f.n_kv_heads;
+    const size_t row = ((size_t)page * f.n_kv_heads + kvh) * f.page_size + pos % f.page_size;
+    if (head < f.n_q_heads + f.n_kv_heads) {
+      f.k_pool[row * D + j] = f32_to_bf16(y0);
+      f.k_pool[row * D + j + half] = f32_to_bf16(y1);
+      if (f.ksb_pool && j < f.n_rot) {
+        f.ksb_pool[row * 2 * f.n_rot + j] = f32_to_bf16(x0);
+        f.ksb_pool[row * 2 * f.n_rot + f.n_rot + j] = f32_to_bf16(x1);
+      }
+    } else {
+      f.v_pool[row * D + j] = f32_to_bf16(x0);
+      f.v_pool[row * D + j + half] = f32_to_bf16(x1);
+    }
+  }
 }
 
 template <int NT, int MODE>
@@ -283,6 +382,9 @@ cudaError_t launch_mode(const GemmPlan& p, const CUtensorMap& tw, const CUtensor
 
 }  // namespace
 
+// partial row stride of the mma.sync path (the tcgen05 path uses its padded N <= this)
+static int mma_ldp(const GemmPlan& p) { return p.mblocks > 1 ? p.mblocks * kMBlock : p.nt * 8; }
+
 GemmPlan plan_gemm(int M, int N, int K, int mode) {
   GemmPlan p{};
   p.M = M;
@@ -304,7 +406,7 @@ GemmPlan plan_gemm(int M, int N, int K, int mode) {
 }
 
 size_t gemm_partial_floats(const GemmPlan& p) {
-  return (size_t)p.mblocks * p.splits * p.n_tiles * kTileN * (p.nt * 8);
+  return (size_t)p.splits * p.n_tiles * kTileN * mma_ldp(p);
 }
 size_t gemm_argmax_entries(const GemmPlan& p) { return (size_t)p.M; }
 int gemm_tickets(const GemmPlan& p) { return p.mblocks * p.n_tiles; }
@@ -331,12 +433,36 @@ cudaError_t launch_gemm(const GemmPlan& p, int mode, const void* x, const void* 
   a.status = b.status;
   a.acc = b.acc;
   a.rope = b.rope;
+  a.ldp = mma_ldp(p);
+  // more than a few rows: reduce the split partials with the whole grid
+  a.grid_reduce = (mode != kGemmArgmax && p.M > kFusedTailMaxRows) ? 1 : 0;
   if (mode != kGemmArgmax || p.mblocks != 1) a.acc.B = 0;
   switch (mode) {
-    case kGemmStore: return launch_mode<kGemmStore>(p, tw, tx, a, st);
-    case kGemmResidual: return launch_mode<kGemmResidual>(p, tw, tx, a, st);
     case kGemmArgmax: return launch_mode<kGemmArgmax>(p, tw, tx, a, st);
-    case kGemmQkvRope: return launch_mode<kGemmQkvRope>(p, tw, tx, a, st);
+  }
+  cudaError_t e = cudaErrorInvalidValue;
+  switch (mode) {
+    case kGemmStore: e = launch_mode<kGemmStore>(p, tw, tx, a, st); break;
+    case kGemmResidual: e = launch_mode<kGemmResidual>(p, tw, tx, a, st); break;
+    case kGemmQkvRope: e = launch_mode<kGemmQkvRope>(p, tw, tx, a, st); break;
+  }
+  if (e != cudaSuccess || !a.grid_reduce) return e;
+  return launch_splitk_reduce(a, mode, st);
+}
+
+cudaError_t launch_splitk_reduce(const Args& a, int mode, cudaStream_t st) {
+  const int mt = (a.M + 31) / 32;
+  switch (mode) {
+    case kGemmStore:
+      return launch_k(splitk_reduce_kernel<kGemmStore>, dim3((a.N + 31) / 32, mt), dim3(32, 8), 0, st, a);
+    case kGemmResidual:
+      return launch_k(splitk_reduce_kernel<kGemmResidual>, dim3((a.N + 31) / 32, mt), dim3(32, 8), 0, st,
+                      a);
+    case kGemmQkvRope: {
+      const int D = a.rope.head_dim;
+      return launch_k(splitk_reduce_kernel<kGemmQkvRope>, dim3((a.N / D) * (D / 2 / 32), mt),
+                      dim3(32, 8), 0, st, a);
+    }
   }
   return cudaErrorInvalidValue;
 }

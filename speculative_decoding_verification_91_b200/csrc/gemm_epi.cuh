@@ -16,6 +16,8 @@ constexpr int kEpiThreads = 128;
 struct Args {
   int M, N, K, kchunks, splits, n_tiles;
   int np;           // tcgen05 kernel: padded token count (MMA N)
+  int ldp;          // partials: element (split s, feature f, row m) at (s*n_tiles*128 + f)*ldp + m
+  int grid_reduce;  // 1: the split partials are reduced by splitk_reduce_kernel, not the last CTA
   float* out;
   float* partial;
   unsigned long long* arg_keys;   // [M] packed (value, id) keys, zero between launches
@@ -117,13 +119,12 @@ __device__ __forceinline__ void rope_epilogue(const Args& a, int MP, int n_tile,
   if (!*flag) return;
   __threadfence();
   const int mcount = min(MP, a.M - m0);
-  const size_t split_stride = (size_t)a.n_tiles * kTileN * MP;
-  const float* base = a.partial + (size_t)mblk * a.splits * a.n_tiles * kTileN * MP;
+  const size_t split_stride = (size_t)a.n_tiles * kTileN * a.ldp;
   for (int item = ctid; item < half * mcount; item += kEpiThreads) {
     const int mm = item / half, j = item % half;
     const int f0 = head * D + j, f1 = f0 + half;
-    const float* p0 = base + ((size_t)(f0 / kTileN) * kTileN + f0 % kTileN) * MP + mm;
-    const float* p1 = base + ((size_t)(f1 / kTileN) * kTileN + f1 % kTileN) * MP + mm;
+    const float* p0 = a.partial + (size_t)f0 * a.ldp + m0 + mm;
+    const float* p1 = a.partial + (size_t)f1 * a.ldp + m0 + mm;
     float x0 = 0.f, x1 = 0.f;
     int sp = 0;
     for (; sp + 4 <= a.splits; sp += 4) {
@@ -201,13 +202,13 @@ __device__ __forceinline__ void splitk_finish(const Args& a, int MP, int n_tile,
   // Work item = (output feature r, row mm); the split loads of an item are
   // issued together (independent) and then added in split order.
   const int mcount = min(MP, a.M - m0);
-  const size_t split_stride = (size_t)a.n_tiles * kTileN * MP;
-  const float* base = a.partial + ((size_t)mblk * a.splits * a.n_tiles + n_tile) * kTileN * MP;
+  const size_t split_stride = (size_t)a.n_tiles * kTileN * a.ldp;
+  const float* base = a.partial + (size_t)n_tile * kTileN * a.ldp + m0;
   for (int item = ctid; item < kTileN * mcount; item += kEpiThreads) {
     const int mm = item / kTileN, r = item % kTileN;
     const int n = n_tile * kTileN + r;
     if (n >= a.N) continue;
-    const float* p = base + (size_t)r * MP + mm;
+    const float* p = base + (size_t)r * a.ldp + mm;
     float s = 0.f;
     int sp = 0;
     for (; sp + 8 <= a.splits; sp += 8) {
@@ -226,5 +227,9 @@ __device__ __forceinline__ void splitk_finish(const Args& a, int MP, int n_tile,
   }
   if (ctid == 0) a.tickets[mblk * a.n_tiles + n_tile] = 0u;
 }
+
+// Grid-wide split-K sum + epilogue (store / residual / QKV + RoPE) for
+// problems whose rows are too many for one CTA per tile to finish quickly.
+cudaError_t launch_splitk_reduce(const Args& a, int mode, cudaStream_t st);
 
 }  // namespace sv

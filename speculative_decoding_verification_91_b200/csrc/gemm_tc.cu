@@ -275,14 +275,14 @@ __global__ void __launch_bounds__(kTcThreads, 2) tc_gemm_kernel(
         }
       } else {
         // split-K partial tile [128 rows][np], then the shared epilogues
-        float* mine = a.partial + ((size_t)split * a.n_tiles + n_tile) * kTileN * np;
+        float* mine = a.partial + ((size_t)split * a.n_tiles + n_tile) * kTileN * a.ldp;
         for (int c0 = 0; c0 < np; c0 += 32) {
           float v[32];
           tmem_ld32(tq + c0, v);
 #pragma unroll
           for (int j = 0; j < 32; j += 4)
             if (c0 + j < np)   // np is a multiple of 16: a float4 is wholly inside or outside
-              __stcg(reinterpret_cast<float4*>(mine + (size_t)row * np + c0 + j),
+              __stcg(reinterpret_cast<float4*>(mine + (size_t)row * a.ldp + c0 + j),
                      make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]));
         }
       }
@@ -295,108 +295,11 @@ __global__ void __launch_bounds__(kTcThreads, 2) tc_gemm_kernel(
   if (warp < kTcEpiWarp0 || *fail) return;
 
   // ---- cross-CTA completion of the argmax (epilogue warps only); the other
-  //      modes finish in tc_reduce_kernel, which sums the split partials with
+  //      modes finish in splitk_reduce_kernel, which sums the split partials with
   //      the whole grid instead of one CTA per tile
   if (MODE == kGemmArgmax) {
     const int ctid = threadIdx.x - kTcEpiWarp0 * 32;
     argmax_finish(a, a.n_tiles, 0, 0, np, ctid, flag, red_i);
-  }
-}
-
-// Split-K sum (in split order) + epilogue for the many-row GEMM, one output
-// per thread, 32x32 tiles transposed through shared memory so that both the
-// partial reads (along rows) and the output writes (along features) coalesce.
-//   store / residual: tile = 32 features x 32 rows, out[m][n] (+)= sum
-//   QKV + RoPE: tile = 32 pairs (j, j + D/2) of one head x 32 rows
-template <int MODE>
-__global__ void __launch_bounds__(256) tc_reduce_kernel(Args a) {
-  __shared__ float t0[32][33], t1[32][33];
-  pdl_trigger();
-  pdl_wait();
-  const int np = a.np, tx = threadIdx.x, ty = threadIdx.y;   // 32 x 8
-  const int m_base = blockIdx.y * 32;
-  const size_t split_stride = (size_t)a.n_tiles * kTileN * np;
-  if (MODE != kGemmQkvRope) {
-    const int n_base = blockIdx.x * 32;
-    for (int r = ty; r < 32; r += 8) {             // r: feature within the tile
-      const int n = n_base + r, m = m_base + tx;
-      float s = 0.f;
-      if (n < a.N && m < a.M) {
-        const float* p = a.partial + (size_t)n * np + m;
-        for (int sp = 0; sp < a.splits; ++sp) s = __fadd_rn(s, __ldcg(p + (size_t)sp * split_stride));
-      }
-      t0[r][tx] = s;
-    }
-    __syncthreads();
-    for (int r = ty; r < 32; r += 8) {             // r: row within the tile
-      const int n = n_base + tx, m = m_base + r;
-      if (n < a.N && m < a.M) {
-        float* dst = a.out + (size_t)m * a.N + n;
-        *dst = (MODE == kGemmResidual) ? __fadd_rn(*dst, t0[tx][r]) : t0[tx][r];
-      }
-    }
-    return;
-  }
-  const RopeFuse& f = a.rope;
-  const int D = f.head_dim, half = D / 2;
-  const int pairs_per_head = half / 32;
-  const int head = blockIdx.x / pairs_per_head, j0 = (blockIdx.x % pairs_per_head) * 32;
-  for (int r = ty; r < 32; r += 8) {               // r: pair within the tile
-    const int m = m_base + tx, j = j0 + r;
-    float x0 = 0.f, x1 = 0.f;
-    if (m < a.M) {
-      const float* p0 = a.partial + (size_t)(head * D + j) * np + m;
-      const float* p1 = a.partial + (size_t)(head * D + j + half) * np + m;
-      for (int sp = 0; sp < a.splits; ++sp) {
-        x0 = __fadd_rn(x0, __ldcg(p0 + (size_t)sp * split_stride));
-        x1 = __fadd_rn(x1, __ldcg(p1 + (size_t)sp * split_stride));
-      }
-    }
-    t0[r][tx] = x0;
-    t1[r][tx] = x1;
-  }
-  __syncthreads();
-  for (int r = ty; r < 32; r += 8) {               // r: row within the tile
-    const int m = m_base + r, j = j0 + tx;
-    if (m >= a.M) continue;
-    const float x0 = t0[tx][r], x1 = t1[tx][r];
-    const int b = m / f.q, i = m % f.q;
-    const bool rot = j < f.n_rot && head < f.n_q_heads + f.n_kv_heads;
-    float y0 = x0, y1 = x1;
-    if (rot) {
-      const float2 cs = f.rope_tab[(size_t)m * half + j];
-      rope_pair(x0, x1, cs.x, cs.y, y0, y1);
-    }
-    if (head < f.n_q_heads) {
-      uint16_t* qo = f.q_out + ((size_t)m * f.n_q_heads + head) * D;
-      qo[j] = f32_to_bf16(y0);
-      qo[j + half] = f32_to_bf16(y1);
-      continue;
-    }
-    const int pos = f.seq_lens[b] + i;
-    if (pos < 0 || pos / f.page_size >= f.max_pages) {
-      flag_status(a.status, SPEC_DEV_BAD_LENGTH);
-      continue;
-    }
-    const int page = f.block_table[(size_t)b * f.max_pages + pos / f.page_size];
-    if (page < 0 || page >= f.num_pages) {
-      flag_status(a.status, SPEC_DEV_BAD_PAGE);
-      continue;
-    }
-    const int kvh = head < f.n_q_heads + f.n_kv_heads ? head - f.n_q_heads
-                                                      : head - f.n_q_heads - f.n_kv_heads;
-    const size_t row = ((size_t)page * f.n_kv_heads + kvh) * f.page_size + pos % f.page_size;
-    if (head < f.n_q_heads + f.n_kv_heads) {
-      f.k_pool[row * D + j] = f32_to_bf16(y0);
-      f.k_pool[row * D + j + half] = f32_to_bf16(y1);
-      if (f.ksb_pool && j < f.n_rot) {
-        f.ksb_pool[row * 2 * f.n_rot + j] = f32_to_bf16(x0);
-        f.ksb_pool[row * 2 * f.n_rot + f.n_rot + j] = f32_to_bf16(x1);
-      }
-    } else {
-      f.v_pool[row * D + j] = f32_to_bf16(x0);
-      f.v_pool[row * D + j + half] = f32_to_bf16(x1);
-    }
   }
 }
 
@@ -409,12 +312,7 @@ cudaError_t launch_tc_mode(const GemmPlan& p, const CUtensorMap& tw, const CUten
   if (e != cudaSuccess) return e;
   e = launch_k(kern, dim3(p.n_tiles, p.splits, 1), dim3(kTcThreads), L.smem, st, tw, tx, a);
   if (e != cudaSuccess || MODE == kGemmArgmax) return e;
-  const int mt = (p.M + 31) / 32;
-  if (MODE == kGemmQkvRope) {
-    const int D = a.rope.head_dim;
-    return launch_k(tc_reduce_kernel<MODE>, dim3((p.N / D) * (D / 2 / 32), mt), dim3(32, 8), 0, st, a);
-  }
-  return launch_k(tc_reduce_kernel<MODE>, dim3((p.N + 31) / 32, mt), dim3(32, 8), 0, st, a);
+  return launch_splitk_reduce(a, MODE, st);
 }
 
 }  // namespace
@@ -444,6 +342,8 @@ cudaError_t launch_gemm_tc(const GemmPlan& p, int mode, const void* x, const voi
   a.splits = p.splits;
   a.n_tiles = p.n_tiles;
   a.np = np;
+  a.ldp = np;
+  a.grid_reduce = 1;
   a.out = b.out;
   a.partial = b.partial;
   a.arg_keys = b.arg_keys;

@@ -89,10 +89,13 @@ WORKLOADS = {
                           head_dim=256, vocab=262144, layers=(GLOBAL_KV,), ctx_lo=4096,
                           ctx_hi=32768, accept=("geometric", 0.8), split_tokens=512),
     # Batch 64, k=3, 5 sliding-window layers + 1 key-equals-value global layer.
+    # (64 sequences x 8 KV heads already fill the GPU: long splits keep the
+    #  split-combine traffic small)
     "b64_6layer": Workload("b64_6layer", batch=64, k=3, d_model=3840, n_q_heads=16, n_kv_heads=8,
                            head_dim=256, vocab=262144,
-                           layers=(LOCAL1024,) * 5 + (GLOBAL_KV,), ctx_lo=1024, ctx_hi=16384,
-                           accept=("geometric_per_seq", 0.5, 0.9)),
+                           layers=(LOCAL1024.__class__(window=1024, split_tokens=1024),) * 5
+                           + (GLOBAL_KV,), ctx_lo=1024, ctx_hi=16384,
+                           accept=("geometric_per_seq", 0.5, 0.9), split_tokens=2048),
     # Speculative loop: 4 layers (3 sliding + 1 global K=V), 131072-token prompt, k=8, 512 steps.
     "loop_131k": Workload("loop_131k", batch=1, k=8, d_model=2048, n_q_heads=8, n_kv_heads=2,
                           head_dim=256, vocab=262144, layers=(LOCAL1024,) * 3 + (GLOBAL_KV,),
