@@ -249,6 +249,13 @@ def run_cuda(args, rank, world, local_rank):
     got_acc = h_out[Bn * (k + 1):Bn * (k + 2)].numpy()
     assert np.array_equal(got_acc, out["accept_len"]), "e2e step disagrees with the device-timed step"
 
+    # per-launch breakdown of one extra step (events serialise the launches)
+    flush.zero_()
+    sess.reset_lengths()
+    B.spec_profile_launches(256)
+    sess.step(stream=stream, with_targets=False)
+    launch_ms = B.spec_profile_launches_collect(256)
+
     mean_step = float(np.mean(step_ms))
     mean_lm = float(np.mean(lm_ms))
     mean_e2e = float(np.mean(e2e_ms))
@@ -262,7 +269,7 @@ def run_cuda(args, rank, world, local_rank):
                 mean_lm=mean_lm, mean_e2e=mean_e2e, kv_b=kv_b, lm_b=lm_b, proj_b=proj_b,
                 launches=launches_per_step * args.steps, clocks=clocks.summary(),
                 h2d=int(h_in.numel() * 4), d2h=int(h_out.numel() * 4), step_ms=step_ms,
-                M=wl.batch * wl.q_rows)
+                M=wl.batch * wl.q_rows, launch_us=[round(x * 1e3, 1) for x in launch_ms])
 
 
 # --------------------------------------------------------------------------
@@ -419,6 +426,7 @@ def main():
             "e2e": {"value": r["tokens_per_step"] * world / (r["mean_e2e"] / 1e3), "unit": "tokens/s",
                     "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
             "gpu_launches": r["launches"],
+            "launch_breakdown_us": r["launch_us"],
             "clocks": r["clocks"],
         }
         if not args.no_cpu_baseline and world == 1:

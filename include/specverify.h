@@ -270,6 +270,13 @@ int spec_lmhead_argmax_noalloc(const void* h, const void* w, int M, int d, int V
  * were recorded. */
 int spec_profile_start(int n_steps);
 int spec_profile_collect(float* step_ms, float* lmhead_ms, int n_steps);
+/* Per-launch timing of the next spec_verify_step / spec_prefill call: an event
+ * after every kernel launch of that call (at most max_marks).  The events
+ * serialise the launches (no programmatic overlap), so the sum exceeds a
+ * normal step; the intervals show each kernel's own time.  collect writes
+ * the intervals in launch order, in milliseconds. */
+int spec_profile_launches(int max_marks);
+int spec_profile_launches_collect(float* ms, int max_marks, int* n_intervals);
 
 #ifdef __cplusplus
 }

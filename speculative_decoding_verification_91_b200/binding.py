@@ -33,6 +33,7 @@ EXPORTED = [
     "spec_cache_write", "spec_verify_attn", "spec_lmhead_argmax", "spec_accept_commit",
     "spec_verify_step", "spec_profile_start", "spec_profile_collect",
     "spec_lmhead_argmax_noalloc", "spec_prefill_workspace_bytes", "spec_prefill",
+    "spec_profile_launches", "spec_profile_launches_collect",
 ]
 SPEC_MAX_PREFILL = 256
 SPEC_NOALLOC_MAX_ROWS = 64
@@ -108,6 +109,8 @@ def lib():
         L.spec_prefill_workspace_bytes.argtypes = [pm, c_int, c_int, c_int]
         L.spec_prefill.argtypes = [pm, c_void_p, c_int, c_void_p, c_int, c_int, c_void_p, c_void_p,
                                    c_void_p, c_void_p, c_size_t, c_void_p]
+        L.spec_profile_launches.argtypes = [c_int]
+        L.spec_profile_launches_collect.argtypes = [POINTER(c_float), c_int, POINTER(c_int)]
         L.spec_profile_start.argtypes = [c_int]
         L.spec_profile_collect.argtypes = [POINTER(c_float), POINTER(c_float), c_int]
         for name in EXPORTED[4:]:
@@ -238,3 +241,16 @@ def spec_prefill(model, block_table, max_pages, tokens, B, n, seq_lens, next_tok
     return _check(lib().spec_prefill(ctypes.byref(model), _p(block_table), max_pages, _p(tokens), B, n,
                                      _p(seq_lens), _p(next_token), _p(next_maxlogit), _p(ws),
                                      ws_bytes, _s(stream)), "spec_prefill")
+
+
+def spec_profile_launches(max_marks: int = 256) -> int:
+    return _check(lib().spec_profile_launches(max_marks), "spec_profile_launches")
+
+
+def spec_profile_launches_collect(max_marks: int = 256):
+    """Per-launch intervals (ms, launch order) of the profiled call."""
+    buf = (c_float * max_marks)()
+    n = c_int(0)
+    _check(lib().spec_profile_launches_collect(buf, max_marks, ctypes.byref(n)),
+           "spec_profile_launches_collect")
+    return list(buf[:n.value])

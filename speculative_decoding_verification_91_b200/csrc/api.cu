@@ -164,6 +164,18 @@ inline void prof_mark(int which, cudaStream_t st) {
 inline void prof_step_done() {
   if (g_prof.on && g_prof.used < g_prof.n) ++g_prof.used;
 }
+// Per-launch timing of one step (diagnostics): an event after every launch.
+struct ProfDetail {
+  std::vector<cudaEvent_t> ev;
+  int used = 0;
+  bool on = false;
+};
+ProfDetail g_detail;
+inline void detail_mark(cudaStream_t st) {
+  if (g_detail.on && g_detail.used < (int)g_detail.ev.size())
+    cudaEventRecord(g_detail.ev[g_detail.used++], st);
+}
+
 void prof_release() {
   for (cudaEvent_t e : g_prof.ev) cudaEventDestroy(e);
   g_prof.ev.clear();
@@ -205,6 +217,7 @@ int run_forward(const spec_model* m, const int32_t* block_table, int max_pages, 
   int rc;
 
   prof_mark(0, st);
+  detail_mark(st);
   double inv_freq[128];
   rope_inv_freq(m->rope_theta, D, D / 2, inv_freq);
   float2* rope_tab = at<float2>(ws, s.rope_tab);
@@ -212,12 +225,14 @@ int run_forward(const spec_model* m, const int32_t* block_table, int max_pages, 
                                      B, q, m->rms_eps, x, hn, hdr.status, seq_lens, inv_freq, D / 2,
                                      rope_tab, st));
   if (rc) return rc;
+  detail_mark(st);
   for (int l = 0; l < m->n_layers; ++l) {
     const spec_layer& L = m->layers[l];
     const int nqkv = qkv_out(m, L);
     if (l > 0) {
       rc = cuda_status(launch_rmsnorm(x, M, d, m->rms_eps, hn, st));
       if (rc) return rc;
+      detail_mark(st);
     }
     // QKV projection with RoPE and the cache append in its epilogue
     GemmPlan pq = plan_gemm(M, nqkv, d, kGemmQkvRope);
@@ -243,11 +258,14 @@ int run_forward(const spec_model* m, const int32_t* block_table, int max_pages, 
     f.ksb_pool = static_cast<uint16_t*>(L.ksb_pool);
     rc = cuda_status(launch_gemm_any(pq, kGemmQkvRope, hn, L.w_qkv, bq, st));
     if (rc) return rc;
+    detail_mark(st);
     AttnGeom g = plan_attn(B, q, m->n_q_heads, m->n_kv_heads, D, m->page_size, m->num_pages,
                            max_pages, L.window, L.kv_equal, 2 * f.n_rot, split_of(m, L));
     rc = cuda_status(launch_attention(g, qrot, L.k_pool, L.v_pool, L.ksb_pool, block_table, seq_lens,
-                                      at<float>(ws, s.attn_part), attn_out, hdr.status, st));
+                                      at<float>(ws, s.attn_part), attn_out, hdr.status, st,
+                                      g_detail.on ? detail_mark : nullptr));
     if (rc) return rc;
+    detail_mark(st);
     GemmPlan po = plan_gemm(M, d, m->n_q_heads * D, kGemmResidual);
     GemmBuffers bo{};
     bo.out = x;
@@ -256,9 +274,11 @@ int run_forward(const spec_model* m, const int32_t* block_table, int max_pages, 
     bo.status = hdr.status;
     rc = cuda_status(launch_gemm_any(po, kGemmResidual, attn_out, L.w_o, bo, st));
     if (rc) return rc;
+    detail_mark(st);
   }
   rc = cuda_status(launch_rmsnorm(x, M, d, m->rms_eps, hn, st));
   if (rc) return rc;
+  detail_mark(st);
   // LM head: every row (verify) or each sequence's last row (prefill)
   GemmPlan pl = plan_gemm(prefill ? B : M, m->vocab, d, kGemmArgmax);
   GemmBuffers bl{};
@@ -285,6 +305,7 @@ int run_forward(const spec_model* m, const int32_t* block_table, int max_pages, 
   prof_mark(1, st);
   rc = cuda_status(launch_gemm_any(pl, kGemmArgmax, lm_x, m->w_lm, bl, st));
   prof_mark(2, st);
+  detail_mark(st);
   if (rc) return rc;
   if (prefill) {
     rc = cuda_status(launch_prefill_commit(at<int32_t>(ws, s.ids), at<float>(ws, s.maxv), B, q,
@@ -296,6 +317,8 @@ int run_forward(const spec_model* m, const int32_t* block_table, int max_pages, 
                                    io.target_maxlogit, at<float>(ws, s.maxv), st));
   }
   prof_mark(3, st);
+  detail_mark(st);
+  g_detail.on = false;
   prof_step_done();
   return rc;
 }
@@ -318,6 +341,32 @@ int spec_profile_start(int n_steps) {
     }
   g_prof.n = n_steps;
   g_prof.on = true;
+  return SPEC_OK;
+}
+
+int spec_profile_launches(int max_marks) {
+  if (max_marks < 2 || max_marks > 4096) return SPEC_EINVAL;
+  for (cudaEvent_t e : g_detail.ev) cudaEventDestroy(e);
+  g_detail.ev.assign(max_marks, nullptr);
+  for (auto& e : g_detail.ev)
+    if (cudaEventCreate(&e) != cudaSuccess) return SPEC_ECUDA;
+  g_detail.used = 0;
+  g_detail.on = true;
+  return SPEC_OK;
+}
+
+int spec_profile_launches_collect(float* ms, int max_marks, int* n_intervals) {
+  if (!ms || !n_intervals || g_detail.used < 2) return SPEC_EINVAL;
+  int n = 0;
+  if (cudaEventSynchronize(g_detail.ev[g_detail.used - 1]) != cudaSuccess) return SPEC_ECUDA;
+  for (int i = 1; i < g_detail.used && i - 1 < max_marks; ++i, ++n)
+    if (cudaEventElapsedTime(&ms[i - 1], g_detail.ev[i - 1], g_detail.ev[i]) != cudaSuccess)
+      return SPEC_ECUDA;
+  *n_intervals = n;
+  for (cudaEvent_t e : g_detail.ev) cudaEventDestroy(e);
+  g_detail.ev.clear();
+  g_detail.used = 0;
+  g_detail.on = false;
   return SPEC_OK;
 }
 

@@ -649,7 +649,7 @@ size_t attn_partial_floats(const AttnGeom& g) {
 cudaError_t launch_attention(const AttnGeom& g, const uint16_t* qrot, const void* k_pool,
                              const void* v_pool, const void* ksb_pool, const int32_t* block_table,
                              const int32_t* seq_lens, float* part, uint16_t* out, unsigned* status,
-                             cudaStream_t st) {
+                             cudaStream_t st, void (*mark)(cudaStream_t)) {
   const uint64_t rows = (uint64_t)g.num_pages * g.n_kv_heads * g.page_size;
   CUtensorMap tk, tv;
   if (!make_tmap_bf16_2d(&tk, k_pool, rows, g.head_dim, 64, 64)) return cudaErrorInvalidValue;
@@ -688,6 +688,7 @@ cudaError_t launch_attention(const AttnGeom& g, const uint16_t* qrot, const void
     return cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) return e;
+  if (mark) mark(st);
   return launch_k(attn_combine_kernel, dim3(g.rows, g.n_kv_heads, g.B),
                   dim3(std::min(g.head_dim, 256)), 0, st, a, g.head_dim, out);
 }

@@ -21,6 +21,7 @@
 //   * argmax epilogue: per-tile (max, index) per row, ties to the lowest
 //     index, reduced across tiles by the last CTA; logits never reach HBM.
 #include <algorithm>
+#include <cstdlib>
 
 #include "common.cuh"
 #include "gemm_epi.cuh"
@@ -397,8 +398,14 @@ GemmPlan plan_gemm(int M, int N, int K, int mode) {
   if (mode == kGemmArgmax) {
     p.splits = 1;
   } else {
-    // about 256 CTAs per M-block, at least 4 K chunks each; depends on N, K only
-    int s = (256 + p.n_tiles - 1) / p.n_tiles;
+    // about one CTA per SM per M-block, at least 4 K chunks each; depends
+    // on N, K only (SPECVERIFY_SPLIT_TARGET overrides the target, for tuning)
+    static const int target = [] {
+      const char* v = getenv("SPECVERIFY_SPLIT_TARGET");
+      const int t = v ? atoi(v) : 0;
+      return t > 0 ? t : 148;   // one CTA per SM of a B200
+    }();
+    int s = (target + p.n_tiles - 1) / p.n_tiles;
     s = std::min(s, std::max(1, p.kchunks / 4));
     p.splits = std::max(1, s);
   }

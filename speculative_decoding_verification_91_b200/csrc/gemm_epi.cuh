@@ -120,30 +120,39 @@ __device__ __forceinline__ void rope_epilogue(const Args& a, int MP, int n_tile,
   __threadfence();
   const int mcount = min(MP, a.M - m0);
   const size_t split_stride = (size_t)a.n_tiles * kTileN * a.ldp;
-  for (int item = ctid; item < half * mcount; item += kEpiThreads) {
+  const int n_items = half * mcount;
+  for (int it0 = ctid; it0 < n_items; it0 += 2 * kEpiThreads) {
+   float xs0[2] = {0.f, 0.f}, xs1[2] = {0.f, 0.f};
+   for (int sp0 = 0; sp0 < a.splits; sp0 += 8) {
+    float u0[2][8], u1[2][8];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int item = it0 + u * kEpiThreads;
+      const int mm = item / half, j = item % half;
+      const int f0 = head * D + j, f1 = f0 + half;
+      const float* p0 = a.partial + (size_t)f0 * a.ldp + m0 + mm;
+      const float* p1 = a.partial + (size_t)f1 * a.ldp + m0 + mm;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) {
+        const bool ok = item < n_items && sp0 + w < a.splits;
+        u0[u][w] = ok ? __ldcg(p0 + (size_t)(sp0 + w) * split_stride) : 0.f;
+        u1[u][w] = ok ? __ldcg(p1 + (size_t)(sp0 + w) * split_stride) : 0.f;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+#pragma unroll
+      for (int w = 0; w < 8; ++w)
+        if (sp0 + w < a.splits) {
+          xs0[u] = __fadd_rn(xs0[u], u0[u][w]);
+          xs1[u] = __fadd_rn(xs1[u], u1[u][w]);
+        }
+   }
+   for (int u = 0; u < 2; ++u) {
+    const int item = it0 + u * kEpiThreads;
+    if (item >= n_items) break;
     const int mm = item / half, j = item % half;
-    const int f0 = head * D + j, f1 = f0 + half;
-    const float* p0 = a.partial + (size_t)f0 * a.ldp + m0 + mm;
-    const float* p1 = a.partial + (size_t)f1 * a.ldp + m0 + mm;
-    float x0 = 0.f, x1 = 0.f;
-    int sp = 0;
-    for (; sp + 4 <= a.splits; sp += 4) {
-      float u[4], v[4];
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        u[w] = __ldcg(p0 + (size_t)(sp + w) * split_stride);
-        v[w] = __ldcg(p1 + (size_t)(sp + w) * split_stride);
-      }
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        x0 = __fadd_rn(x0, u[w]);
-        x1 = __fadd_rn(x1, v[w]);
-      }
-    }
-    for (; sp < a.splits; ++sp) {
-      x0 = __fadd_rn(x0, __ldcg(p0 + (size_t)sp * split_stride));
-      x1 = __fadd_rn(x1, __ldcg(p1 + (size_t)sp * split_stride));
-    }
+    const float x0 = xs0[u], x1 = xs1[u];
     const int m = m0 + mm, b = m / f.q, i = m % f.q;
     const bool rot = j < f.n_rot && head < f.n_q_heads + f.n_kv_heads;
     float y0 = x0, y1 = x1;
@@ -181,6 +190,7 @@ __device__ __forceinline__ void rope_epilogue(const Args& a, int MP, int n_tile,
       f.v_pool[row * D + j] = f32_to_bf16(x0);
       f.v_pool[row * D + j + half] = f32_to_bf16(x1);
     }
+   }
   }
   if (ctid == 0) a.tickets[mblk * n_heads + head] = 0u;
 }
@@ -204,26 +214,41 @@ __device__ __forceinline__ void splitk_finish(const Args& a, int MP, int n_tile,
   const int mcount = min(MP, a.M - m0);
   const size_t split_stride = (size_t)a.n_tiles * kTileN * a.ldp;
   const float* base = a.partial + (size_t)n_tile * kTileN * a.ldp + m0;
-  for (int item = ctid; item < kTileN * mcount; item += kEpiThreads) {
-    const int mm = item / kTileN, r = item % kTileN;
-    const int n = n_tile * kTileN + r;
-    if (n >= a.N) continue;
-    const float* p = base + (size_t)r * a.ldp + mm;
-    float s = 0.f;
-    int sp = 0;
-    for (; sp + 8 <= a.splits; sp += 8) {
-      float v[8];
+  const int n_items = kTileN * mcount;
+  // four items per thread at a time, their split loads issued together
+  for (int it0 = ctid; it0 < n_items; it0 += 4 * kEpiThreads) {
+    float s[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int sp0 = 0; sp0 < a.splits; sp0 += 8) {
+      float v[4][8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = __ldcg(p + (size_t)(sp + u) * split_stride);
+      for (int u = 0; u < 4; ++u) {
+        const int item = it0 + u * kEpiThreads;
+        const int mm = item / kTileN, r = item % kTileN;
+        const float* p = base + (size_t)r * a.ldp + mm;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) s = __fadd_rn(s, v[u]);
+        for (int w = 0; w < 8; ++w)
+          v[u][w] = (item < n_items && sp0 + w < a.splits) ? __ldcg(p + (size_t)(sp0 + w) * split_stride)
+                                                           : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int w = 0; w < 8; ++w)
+          if (sp0 + w < a.splits) s[u] = __fadd_rn(s[u], v[u][w]);
     }
-    for (; sp < a.splits; ++sp) s = __fadd_rn(s, __ldcg(p + (size_t)sp * split_stride));
-    float* dst = a.out + (size_t)(m0 + mm) * a.N + n;
-    if (MODE == kGemmResidual)
-      *dst = __fadd_rn(*dst, s);
-    else
-      *dst = s;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int item = it0 + u * kEpiThreads;
+      if (item >= n_items) continue;
+      const int mm = item / kTileN, r = item % kTileN;
+      const int n = n_tile * kTileN + r;
+      if (n >= a.N) continue;
+      float* dst = a.out + (size_t)(m0 + mm) * a.N + n;
+      if (MODE == kGemmResidual)
+        *dst = __fadd_rn(*dst, s[u]);
+      else
+        *dst = s[u];
+    }
   }
   if (ctid == 0) a.tickets[mblk * a.n_tiles + n_tile] = 0u;
 }

@@ -151,6 +151,6 @@ size_t attn_partial_floats(const AttnGeom& g);
 cudaError_t launch_attention(const AttnGeom& g, const uint16_t* qrot, const void* k_pool,
                              const void* v_pool, const void* ksb_pool, const int32_t* block_table,
                              const int32_t* seq_lens, float* part, uint16_t* out, unsigned* status,
-                             cudaStream_t st);
+                             cudaStream_t st, void (*mark)(cudaStream_t) = nullptr);
 
 }  // namespace sv

@@ -55,13 +55,19 @@ __global__ void __launch_bounds__(kNormThreads) embed_norm_kernel(
   __shared__ double red[kNormThreads / 32];
   pdl_trigger();
   pdl_wait();
+  const int n_rows = gridDim.x - (rope_tab ? (int)(((size_t)gridDim.x) / 2) : 0);
+  if ((int)blockIdx.x >= n_rows) {
+    // blocks past the rows: the (cos, sin) table, one (row, pair) per thread,
+    // in parallel with the gather and normalisation of the other blocks
+    const size_t idx = (size_t)(blockIdx.x - n_rows) * kNormThreads + threadIdx.x;
+    if (idx < (size_t)n_rows * half) {
+      const int m = (int)(idx / half), j = (int)(idx % half);
+      rope_tab[idx] = rope_cs(seq_lens[m / q] + m % q, inv_freq.v[j]);
+    }
+    return;
+  }
   const int m = blockIdx.x;
   const int b = m / q, i = m % q;
-  if (rope_tab) {
-    const int pos = seq_lens[b] + i;
-    for (int j = threadIdx.x; j < half; j += kNormThreads)
-      rope_tab[(size_t)m * half + j] = rope_cs(pos, inv_freq.v[j]);
-  }
   const int tok = tokens_flat ? tokens_flat[m]
                               : ((i == 0) ? last_token[b] : drafts[b * (q - 1) + (i - 1)]);
   float* row = x + (size_t)m * d;
@@ -115,7 +121,11 @@ cudaError_t launch_embed_norm(const void* w_emb, int vocab, int d, const int32_t
                               float2* rope_tab, cudaStream_t st) {
   InvFreq f{};
   for (int j = 0; j < half && j < 128; ++j) f.v[j] = inv_freq[j];
-  return launch_k(embed_norm_kernel, dim3(B * q), dim3(kNormThreads), 0, st,
+  // rows, then as many blocks again for the RoPE table (table blocks <= rows
+  // since half <= kNormThreads); the kernel splits the grid in two halves
+  const int rows = B * q;
+  const int tab_blocks = rope_tab ? rows : 0;
+  return launch_k(embed_norm_kernel, dim3(rows + tab_blocks), dim3(kNormThreads), 0, st,
                   static_cast<const uint16_t*>(w_emb), vocab, d, last_token, drafts, tokens_flat, q,
                   eps, x, out, status, seq_lens, f, half, rope_tab);
 }
