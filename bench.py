@@ -48,6 +48,10 @@ def parse():
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
     ap.add_argument("--workload", default="b1_ctx8k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", action="store_true",
+                    help="shrink the vocabulary to 4096 (attention and projection shapes kept) "
+                         "so that a profiler capture of the layer kernels holds little device "
+                         "memory; random drafts; not a benchmark number")
     return ap.parse_args()
 
 
@@ -163,19 +167,51 @@ def algorithmic_bytes(wl, lens):
     return int(kv), int(lm), int(proj)
 
 
+def launch_labels(wl):
+    """Names of the intervals spec_profile_launches reports for one step, in
+    launch order (a GEMM and its split-K reduce share one interval)."""
+    names = ["embed_norm"]
+    for l, spec in enumerate(wl.layers):
+        kind = "global" if spec.window == 0 else "local"
+        if l > 0:
+            names.append(f"L{l}.rmsnorm")
+        names += [f"L{l}.qkv_rope", f"L{l}.attn_split[{kind}]", f"L{l}.attn_combine", f"L{l}.o_proj"]
+    return names + ["final_rmsnorm", "lm_head_argmax", "accept"]
+
+
+def attention_bytes(wl, lens, layer):
+    spec = wl.layers[layer]
+    per = (wl.head_dim * (1 + spec.rope_fraction) if spec.kv_equal else 2 * wl.head_dim) * 2
+    kv = 0
+    for L in lens:
+        hi = L + wl.k + 1
+        lo = 0 if spec.window == 0 else max(0, L - spec.window + 1)
+        kv += (hi - lo) * wl.n_kv_heads * per
+    return int(kv)
+
+
 def run_cuda(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
     from speculative_decoding_verification_91_b200 import binding as B
+    from speculative_decoding_verification_91_b200.inputs import gen
     from speculative_decoding_verification_91_b200.inputs import workloads as W
     from speculative_decoding_verification_91_b200.session import WorkloadSession
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     wl = W.get_workload(args.workload)
+    if args.profile_case:
+        wl = wl.with_(vocab=4096)
     B.lib()
     fixture = os.path.join(ROOT, "tests", "golden", f"verify_{wl.name}.json")
-    if os.path.exists(fixture):
+    if args.profile_case:
+        sess = WorkloadSession(wl, device=dev, poison=False)
+        last = np.array([W.last_token(wl, b, 0) for b in range(wl.batch)], dtype=np.int32)
+        drafts = np.stack([gen.randint(wl.seed, f"{wl.name}/profile_drafts", b * wl.k, wl.k, 0, wl.vocab)
+                           for b in range(wl.batch)]).astype(np.int32)
+        inputs = "profile case: vocabulary 4096, random drafts"
+    elif os.path.exists(fixture):
         # margin-guarded inputs shared with the parity tests
         with open(fixture) as f:
             seqs = json.load(f)["sequences"]
@@ -210,12 +246,14 @@ def run_cuda(args, rank, world, local_rank):
         dist.barrier()
     torch.cuda.synchronize(dev)
     B.spec_profile_start(args.steps)
+    n_launch0 = B.spec_launch_count()
     with ClockSampler(local_rank) as clocks:
         for i in range(args.steps):
             flush.zero_()
             sess.reset_lengths()
             sess.step(stream=stream, with_targets=False)
         torch.cuda.synchronize(dev)
+    n_launches = B.spec_launch_count() - n_launch0
     step_ms, lm_ms = B.spec_profile_collect(args.steps)
     if world > 1:
         dist.barrier()
@@ -264,10 +302,9 @@ def run_cuda(args, rank, world, local_rank):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         mean_step, mean_e2e, mean_lm = [float(v) for v in t.tolist()]
     kv_b, lm_b, proj_b = algorithmic_bytes(wl, sess.lens)
-    launches_per_step = 4 + 6 * len(wl.layers)
     return dict(wl=wl, lens=sess.lens, tokens_per_step=tokens_per_step, mean_step=mean_step, inputs=inputs,
                 mean_lm=mean_lm, mean_e2e=mean_e2e, kv_b=kv_b, lm_b=lm_b, proj_b=proj_b,
-                launches=launches_per_step * args.steps, clocks=clocks.summary(),
+                launches=n_launches, clocks=clocks.summary(),
                 h2d=int(h_in.numel() * 4), d2h=int(h_out.numel() * 4), step_ms=step_ms,
                 M=wl.batch * wl.q_rows, launch_us=[round(x * 1e3, 1) for x in launch_ms])
 
@@ -355,6 +392,23 @@ def run_lmhead_only(args):
                       "frac_tensor": (flops / us / 1e6 / tf) if tf else None}), flush=True)
 
 
+def attention_roofline(wl, r, peak):
+    """Per layer: visible KV bytes / (split + combine interval) of the
+    per-launch breakdown (launches serialised by events there, so slightly
+    pessimistic)."""
+    labels = launch_labels(wl)
+    if len(labels) != len(r["launch_us"]):
+        return None
+    us = dict(zip(labels, r["launch_us"]))
+    out = []
+    for l, spec in enumerate(wl.layers):
+        t = [v for k, v in us.items() if k.startswith(f"L{l}.attn_split")][0] + us[f"L{l}.attn_combine"]
+        b = attention_bytes(wl, r["lens"], l)
+        out.append({"layer": l, "kind": "global" if spec.window == 0 else "local", "bytes": b,
+                    "us": t, "gbs": b / t / 1e3, "frac_of_measured": b / t / 1e3 / peak})
+    return out
+
+
 def main():
     args = parse()
     if args.workload.startswith("lmhead:"):
@@ -426,7 +480,9 @@ def main():
             "e2e": {"value": r["tokens_per_step"] * world / (r["mean_e2e"] / 1e3), "unit": "tokens/s",
                     "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
             "gpu_launches": r["launches"],
-            "launch_breakdown_us": r["launch_us"],
+            "launch_breakdown_us": dict(zip(launch_labels(wl), r["launch_us"]))
+            if len(launch_labels(wl)) == len(r["launch_us"]) else r["launch_us"],
+            "attention_hbm": attention_roofline(wl, r, peak),
             "clocks": r["clocks"],
         }
         if not args.no_cpu_baseline and world == 1:

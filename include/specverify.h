@@ -278,6 +278,11 @@ int spec_profile_collect(float* step_ms, float* lmhead_ms, int n_steps);
 int spec_profile_launches(int max_marks);
 int spec_profile_launches_collect(float* ms, int max_marks, int* n_intervals);
 
+/* Number of kernels the library has launched successfully since it was
+ * loaded (all devices and threads; a relaxed atomic counter).  The
+ * difference across a region counts that region's launches. */
+unsigned long long spec_launch_count(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -33,7 +33,7 @@ EXPORTED = [
     "spec_cache_write", "spec_verify_attn", "spec_lmhead_argmax", "spec_accept_commit",
     "spec_verify_step", "spec_profile_start", "spec_profile_collect",
     "spec_lmhead_argmax_noalloc", "spec_prefill_workspace_bytes", "spec_prefill",
-    "spec_profile_launches", "spec_profile_launches_collect",
+    "spec_profile_launches", "spec_profile_launches_collect", "spec_launch_count",
 ]
 SPEC_MAX_PREFILL = 256
 SPEC_NOALLOC_MAX_ROWS = 64
@@ -116,6 +116,8 @@ def lib():
         for name in EXPORTED[4:]:
             if name != "spec_prefill_workspace_bytes":
                 getattr(L, name).restype = c_int
+        L.spec_launch_count.argtypes = []
+        L.spec_launch_count.restype = ctypes.c_ulonglong
         _lib = L
     return _lib
 
@@ -245,6 +247,11 @@ def spec_prefill(model, block_table, max_pages, tokens, B, n, seq_lens, next_tok
 
 def spec_profile_launches(max_marks: int = 256) -> int:
     return _check(lib().spec_profile_launches(max_marks), "spec_profile_launches")
+
+
+def spec_launch_count() -> int:
+    """Kernels the library has launched since it was loaded."""
+    return int(lib().spec_launch_count())
 
 
 def spec_profile_launches_collect(max_marks: int = 256):

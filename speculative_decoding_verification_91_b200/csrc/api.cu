@@ -5,6 +5,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 #include <vector>
 
@@ -13,6 +14,9 @@
 #include "internal.h"
 
 namespace sv {
+
+std::atomic<unsigned long long> g_launch_count{0};
+void count_launch() { g_launch_count.fetch_add(1, std::memory_order_relaxed); }
 
 // ------------------------------------------------------------------ TMA maps
 namespace {
@@ -368,6 +372,10 @@ int spec_profile_launches_collect(float* ms, int max_marks, int* n_intervals) {
   g_detail.used = 0;
   g_detail.on = false;
   return SPEC_OK;
+}
+
+unsigned long long spec_launch_count(void) {
+  return g_launch_count.load(std::memory_order_relaxed);
 }
 
 int spec_profile_collect(float* step_ms, float* lmhead_ms, int n_steps) {

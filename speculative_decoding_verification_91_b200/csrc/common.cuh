@@ -221,6 +221,8 @@ __device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
 // the kernel may start while its predecessor in the stream drains.  Disabled
 // (plain stream order) when the environment sets SPECVERIFY_NO_PDL=1.
 bool pdl_enabled();
+// Kernels this library has launched successfully (all go through launch_k).
+void count_launch();
 template <typename... KArgs, typename... Args>
 cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
                      Args&&... args) {
@@ -234,7 +236,9 @@ cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl_enabled() ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+  if (e == cudaSuccess) count_launch();
+  return e;
 }
 
 // Fixed-size copy of the host theta table into a kernel parameter.
