@@ -48,11 +48,38 @@ def parse():
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
     ap.add_argument("--workload", default="b1_ctx8k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="verify-step time over batch x k on the b1_ctx8k model; one JSON line")
     ap.add_argument("--profile-case", action="store_true",
                     help="shrink the vocabulary to 4096 (attention and projection shapes kept) "
                          "so that a profiler capture of the layer kernels holds little device "
                          "memory; random drafts; not a benchmark number")
     return ap.parse_args()
+
+
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def kernel_sources_sha1(files):
+    import hashlib
+    h = hashlib.sha1()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def measured_traffic(key):
+    """DRAM bytes (read + write) per launch of a kernel from a committed ncu
+    capture, if the sources it was built from are unchanged; else None."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            entry = json.load(f)[key]
+        if kernel_sources_sha1(entry["sources"]) != entry["sources_sha1"]:
+            return None
+        return entry["dram_bytes_per_launch"]
+    except (OSError, KeyError, ValueError):
+        return None
 
 
 def measured_peaks():
@@ -190,6 +217,21 @@ def attention_bytes(wl, lens, layer):
     return int(kv)
 
 
+def reduce_over_ranks(times, tokens, world, device):
+    """Whole-job figures of a multi-rank run: every time is the maximum over
+    the ranks (the job is as slow as its slowest rank) and the emitted tokens
+    are summed over the ranks.  One all-reduce each; every rank calls it."""
+    if world == 1:
+        return [float(t) for t in times], int(tokens)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x) for x in times], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    n = torch.tensor([float(tokens)], dtype=torch.float64, device=device)
+    dist.all_reduce(n, op=dist.ReduceOp.SUM)
+    return [float(v) for v in t.tolist()], int(round(n.item()))
+
+
 def run_cuda(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -297,12 +339,11 @@ def run_cuda(args, rank, world, local_rank):
     mean_step = float(np.mean(step_ms))
     mean_lm = float(np.mean(lm_ms))
     mean_e2e = float(np.mean(e2e_ms))
-    if world > 1:
-        t = torch.tensor([mean_step, mean_e2e, mean_lm], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        mean_step, mean_e2e, mean_lm = [float(v) for v in t.tolist()]
+    (mean_step, mean_e2e, mean_lm), tokens_all = reduce_over_ranks(
+        [mean_step, mean_e2e, mean_lm], tokens_per_step, world, dev)
     kv_b, lm_b, proj_b = algorithmic_bytes(wl, sess.lens)
-    return dict(wl=wl, lens=sess.lens, tokens_per_step=tokens_per_step, mean_step=mean_step, inputs=inputs,
+    return dict(wl=wl, lens=sess.lens, tokens_per_step=tokens_per_step, tokens_all=tokens_all,
+                mean_step=mean_step, inputs=inputs,
                 mean_lm=mean_lm, mean_e2e=mean_e2e, kv_b=kv_b, lm_b=lm_b, proj_b=proj_b,
                 launches=n_launches, clocks=clocks.summary(),
                 h2d=int(h_in.numel() * 4), d2h=int(h_out.numel() * 4), step_ms=step_ms,
@@ -409,8 +450,82 @@ def attention_roofline(wl, r, peak):
     return out
 
 
+SWEEP_B = (1, 2, 4, 8, 16, 32, 64)
+SWEEP_K = (0, 1, 2, 4, 8, 16)
+
+
+def expected_tokens(alpha, k):
+    """Emitted tokens per verify step when every draft is right with
+    probability alpha independently: sum_{i=0..k} alpha^i."""
+    return sum(alpha ** i for i in range(k + 1))
+
+
+def run_sweep(args):
+    """--sweep: the fused verify step over batch sizes B and draft counts k on
+    the b1_ctx8k model (2 layers, d_model 2560, vocab 262,144, every sequence
+    at context 8192).  One session sized for the largest B and k; smaller
+    configurations use its first B sequences.  The cache pages are zero (the
+    step time does not depend on their values); L2 is flushed before every
+    timed step.  Reports us per step, its ratio to the k = 0 step (a plain
+    decode step through the same kernels) and the speed-up over decoding
+    that i.i.d. acceptance alpha = 0.8 would give."""
+    import torch
+    from speculative_decoding_verification_91_b200 import binding as B
+    from speculative_decoding_verification_91_b200.inputs import workloads as W
+    from speculative_decoding_verification_91_b200.session import WorkloadSession
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    wl = W.get_workload("b1_ctx8k").with_(name="sweep", batch=max(SWEEP_B), k=max(SWEEP_K))
+    sess = WorkloadSession(wl, device=dev, poison=False, fill_context=False)
+    for pools in (sess.dm.k_pool, sess.dm.v_pool, sess.dm.ksb_pool):
+        for p in pools:
+            if p is not None:
+                p.zero_()
+    sess.set_inputs(np.zeros(wl.batch, np.int32), np.ones((wl.batch, wl.k), np.int32))
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    d = sess.dm.desc
+
+    def step(Bn, k):
+        B.spec_verify_step(d, sess.block_table, sess.max_pages, sess.last_token,
+                           sess.drafts if k > 0 else None, Bn, k, sess.seq_lens, sess.accept_len,
+                           sess.emitted, sess.new_last, None, None, sess.ws.buf, sess.ws.nbytes, stream)
+
+    steps = max(3, min(args.steps, 50))
+    out = []
+    with ClockSampler(0) as clocks:
+        for Bn in SWEEP_B:
+            t0 = None
+            for k in SWEEP_K:
+                for _ in range(max(3, args.warmup)):
+                    sess.reset_lengths()
+                    step(Bn, k)
+                torch.cuda.synchronize(dev)
+                B.spec_profile_start(steps)
+                for _ in range(steps):
+                    flush.zero_()
+                    sess.reset_lengths()
+                    step(Bn, k)
+                torch.cuda.synchronize(dev)
+                ms, _ = B.spec_profile_collect(steps)
+                us = float(np.mean(ms)) * 1e3
+                t0 = us if k == 0 else t0
+                ratio = us / t0
+                out.append({"B": Bn, "k": k, "rows": Bn * (k + 1), "us_per_step": round(us, 1),
+                            "vs_k0": round(ratio, 3),
+                            "speedup_at_alpha_0.8": round(expected_tokens(0.8, k) / ratio, 3)})
+    if sess.ws.device_status(stream) != 0:
+        raise RuntimeError("device status flagged during the sweep")
+    print(json.dumps({"sweep": "verify step, batch x k", "workload": "b1_ctx8k model, context 8192",
+                      "steps_per_point": steps, "l2": "flushed before every timed step",
+                      "points": out, "clocks": clocks.summary()}), flush=True)
+
+
 def main():
     args = parse()
+    if args.sweep:
+        run_sweep(args)
+        return
     if args.workload.startswith("lmhead:"):
         run_lmhead_only(args)
         return
@@ -454,7 +569,7 @@ def main():
         peak, peak_kind = measured_peaks()
         step_s = r["mean_step"] / 1e3
         lm_s = r["mean_lm"] / 1e3
-        value = r["tokens_per_step"] * world / step_s
+        value = r["tokens_all"] / step_s
         lm_bytes = r["lm_b"] + r["M"] * wl.d_model * 2
         achieved = lm_bytes / lm_s / 1e9
         step_bytes = r["kv_b"] + r["lm_b"]
@@ -475,9 +590,10 @@ def main():
                          "frac_of_measured": step_bytes / step_s / 1e9 / peak},
             "roofline": {"kernel": "stream_gemm_kernel<argmax> (LM head + argmax)", "bound": "hbm",
                          "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "peak_kind": peak_kind, "traffic": None,
+                         "frac": achieved / peak, "peak_kind": peak_kind,
+                         "traffic": measured_traffic(f"lm_head_argmax/{wl.name}"),
                          "bytes_per_launch": lm_bytes, "us_per_launch": r["mean_lm"] * 1e3},
-            "e2e": {"value": r["tokens_per_step"] * world / (r["mean_e2e"] / 1e3), "unit": "tokens/s",
+            "e2e": {"value": r["tokens_all"] / (r["mean_e2e"] / 1e3), "unit": "tokens/s",
                     "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
             "gpu_launches": r["launches"],
             "launch_breakdown_us": dict(zip(launch_labels(wl), r["launch_us"]))

@@ -510,73 +510,127 @@ __global__ void __launch_bounds__(kThreads) attn_split_kernel(
     }
 }
 
-// out[b][i][h] = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s, s ascending.
-// The split weights are formed in parallel into shared memory; each thread
-// then sums its output dimension over the splits in ascending order.
+// out[b][i][h] = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s.
+// The split maxima and weighted denominators are butterfly reductions over a
+// warp's lanes; the numerator is summed over four contiguous quarters of the
+// splits, each in ascending order (lane: 8 output dims), and the quarters are
+// added in order.  That tree depends only on the split count, i.e. on the
+// sequence length, and is the same in both thread mappings:
+//   warp_per_row = 1: one warp per query row (4 rows per CTA), the warp
+//                     walks the four quarters itself (few splits, many rows);
+//   warp_per_row = 0: one CTA of four warps per query row, warp w sums
+//                     quarter w (many splits, few rows).
+constexpr int kCombineWarps = 4;
 constexpr int kMaxCombineSplits = kMaxSplits;
-__global__ void attn_combine_kernel(AttnArgs a, int D, uint16_t* __restrict__ out) {
-  __shared__ float wsh[kMaxCombineSplits];
-  __shared__ float lsh[kMaxCombineSplits];
-  __shared__ float red[32];
-  __shared__ float den_sh;
+__global__ void __launch_bounds__(kCombineWarps * 32) attn_combine_kernel(AttnArgs a, int D, int n_items,
+                                                                          int warp_per_row,
+                                                                          uint16_t* __restrict__ out) {
+  __shared__ float msh[kCombineWarps][kMaxCombineSplits];
+  __shared__ float lsh[kCombineWarps][kMaxCombineSplits];
+  __shared__ float part[kCombineWarps][256];
   pdl_trigger();
   pdl_wait();
-  const int r = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
-  const int tid = threadIdx.x, nthr = blockDim.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
+  const int item = warp_per_row ? blockIdx.x * kCombineWarps + warp : blockIdx.x;
+  if (item >= n_items) return;   // (warp_per_row only: whole warps leave, no CTA barrier follows)
+  const int r = item % a.rows, kvh = (item / a.rows) % a.Hkv, b = item / (a.rows * a.Hkv);
   const int L = a.seq_lens[b];
   const int gh = r / a.q, i = r % a.q;
   const int h = kvh * a.G + gh;
   uint16_t* dst = out + (((long)b * a.q + i) * a.Hq + h) * D;
   if (L < 0 || L + a.q > a.max_pages * kPage) {
-    for (int e = tid; e < D; e += nthr) dst[e] = 0;
+    if (warp_per_row || warp == 0)
+      for (int e = lane; e < D; e += 32) dst[e] = 0;
     return;
   }
   int klo, khi;
   seq_key_range(L, a.q, a.window, klo, khi);
   const int ns = min(khi / a.split - klo / a.split + 1, kMaxCombineSplits);
   const long slot0 = ((long)(b * a.Hkv + kvh) * a.n_splits_grid) * a.rows + r;
-  float mloc = -INFINITY;
-  for (int s = tid; s < ns; s += nthr) {
+  float* m_s = msh[warp_per_row ? warp : 0];
+  float* l_s = lsh[warp_per_row ? warp : 0];
+  const int t0 = warp_per_row ? lane : tid, nt = warp_per_row ? 32 : kCombineWarps * 32;
+  for (int s = t0; s < ns; s += nt) {
     const float2 ml = __ldcg(reinterpret_cast<const float2*>(a.part_ml + (slot0 + (long)s * a.rows) * 2));
-    wsh[s] = ml.x;
-    lsh[s] = ml.y;
-    mloc = fmaxf(mloc, ml.x);
+    m_s[s] = ml.x;
+    l_s[s] = ml.y;
   }
+  if (warp_per_row) __syncwarp(); else __syncthreads();
+  // every warp of the row forms the same maximum and denominator
+  float mloc = -INFINITY;
+  for (int s = lane; s < ns; s += 32) mloc = fmaxf(mloc, m_s[s]);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, off));
-  if ((tid & 31) == 0) red[tid >> 5] = mloc;
-  __syncthreads();
-  float M = red[0];
-  for (int w = 1; w < (nthr + 31) / 32; ++w) M = fmaxf(M, red[w]);
-  for (int s = tid; s < ns; s += nthr) {
-    const float m = wsh[s];
-    wsh[s] = (m == -INFINITY) ? 0.f : exp2f(__fsub_rn(m, M));
+  const float M = mloc;
+  float den = 0.f;
+  for (int s = lane; s < ns; s += 32) {
+    const float m = m_s[s];
+    den = __fadd_rn(den, __fmul_rn((m == -INFINITY) ? 0.f : exp2f(__fsub_rn(m, M)), l_s[s]));
   }
-  __syncthreads();
-  if (tid == 0) {
-    float den = 0.f;
-    for (int s = 0; s < ns; ++s) den = __fadd_rn(den, __fmul_rn(wsh[s], lsh[s]));
-    den_sh = den;
-  }
-  __syncthreads();
-  const float den = den_sh;
-  for (int e = tid; e < D; e += nthr) {
-    const float* po = a.part_o + slot0 * D + e;
-    float num = 0.f;
-    int s = 0;
-    for (; s + 4 <= ns; s += 4) {
-      const float o0 = __ldcg(po + (long)(s + 0) * a.rows * D);
-      const float o1 = __ldcg(po + (long)(s + 1) * a.rows * D);
-      const float o2 = __ldcg(po + (long)(s + 2) * a.rows * D);
-      const float o3 = __ldcg(po + (long)(s + 3) * a.rows * D);
-      num = __fadd_rn(num, __fmul_rn(wsh[s + 0], o0));
-      num = __fadd_rn(num, __fmul_rn(wsh[s + 1], o1));
-      num = __fadd_rn(num, __fmul_rn(wsh[s + 2], o2));
-      num = __fadd_rn(num, __fmul_rn(wsh[s + 3], o3));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) den = __fadd_rn(den, __shfl_xor_sync(0xffffffffu, den, off));
+
+  const int per_q = (ns + 3) / 4;
+  const int per_lane = D / 32;   // 8 (D = 256) or 4 (D = 128)
+  const float* po = a.part_o + slot0 * D + lane * per_lane;
+  const long sstride = (long)a.rows * D;
+  // sum of quarter q of the splits for this lane's dims, ascending, four
+  // splits' loads in flight per step
+  auto quarter = [&](int q, float (&acc)[8]) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+    const int s_lo = q * per_q, s_hi = min(ns, s_lo + per_q);
+    constexpr int U = 4;
+    for (int s0 = s_lo; s0 < s_hi; s0 += U) {
+      float4 x[U][2];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const bool in = s0 + u < s_hi;
+        const float* pp = po + (s0 + u) * sstride;
+        x[u][0] = in ? __ldcg(reinterpret_cast<const float4*>(pp)) : make_float4(0, 0, 0, 0);
+        x[u][1] = (in && per_lane == 8) ? __ldcg(reinterpret_cast<const float4*>(pp + 4))
+                                        : make_float4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        if (s0 + u >= s_hi) break;
+        const float m = m_s[s0 + u];
+        const float ws = (m == -INFINITY) ? 0.f : exp2f(__fsub_rn(m, M));
+        const float xs[8] = {x[u][0].x, x[u][0].y, x[u][0].z, x[u][0].w,
+                             x[u][1].x, x[u][1].y, x[u][1].z, x[u][1].w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = __fadd_rn(acc[e], __fmul_rn(ws, xs[e]));
+      }
     }
-    for (; s < ns; ++s) num = __fadd_rn(num, __fmul_rn(wsh[s], __ldcg(po + (long)s * a.rows * D)));
-    dst[e] = f32_to_bf16(__fdiv_rn(num, den));
+  };
+  float num[8];
+  if (warp_per_row) {
+    quarter(0, num);
+#pragma unroll 1
+    for (int q = 1; q < 4; ++q) {
+      float acc[8];
+      quarter(q, acc);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) num[e] = __fadd_rn(num[e], acc[e]);
+    }
+  } else {
+    float acc[8];
+    quarter(warp, acc);
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if (e < per_lane) part[warp][lane * per_lane + e] = acc[e];
+    __syncthreads();
+    if (warp != 0) return;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      if (e >= per_lane) break;
+      const int d = lane * per_lane + e;
+      num[e] = __fadd_rn(__fadd_rn(__fadd_rn(part[0][d], part[1][d]), part[2][d]), part[3][d]);
+    }
   }
+#pragma unroll
+  for (int e = 0; e < 8; ++e)
+    if (e < per_lane) dst[lane * per_lane + e] = f32_to_bf16(__fdiv_rn(num[e], den));
 }
 
 template <int D, int MT, bool KVEQ>
@@ -680,7 +734,10 @@ cudaError_t launch_attention(const AttnGeom& g, const uint16_t* qrot, const void
   a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)g.head_dim));
   const int mt = std::min(4, (g.rows + 15) / 16);
   cudaError_t e;
-  if (g.head_dim == 256) {
+  if (attn_tc_supported(g)) {
+    e = launch_attn_tc(g, tk, tv, qrot, block_table, seq_lens, a.part_o, a.part_ml, status,
+                       a.scale_log2, st);
+  } else if (g.head_dim == 256) {
     e = g.kv_equal ? launch_mt<256, true>(mt, g, tk, tv, a, st) : launch_mt<256, false>(mt, g, tk, tv, a, st);
   } else if (g.head_dim == 128) {
     e = g.kv_equal ? launch_mt<128, true>(mt, g, tk, tv, a, st) : launch_mt<128, false>(mt, g, tk, tv, a, st);
@@ -689,8 +746,12 @@ cudaError_t launch_attention(const AttnGeom& g, const uint16_t* qrot, const void
   }
   if (e != cudaSuccess) return e;
   if (mark) mark(st);
-  return launch_k(attn_combine_kernel, dim3(g.rows, g.n_kv_heads, g.B),
-                  dim3(std::min(g.head_dim, 256)), 0, st, a, g.head_dim, out);
+  // few splits: a warp per row; many: four warps per row (same arithmetic)
+  const int items = g.B * g.n_kv_heads * g.rows;
+  const int wpr = g.n_splits_grid <= 16 ? 1 : 0;
+  return launch_k(attn_combine_kernel,
+                  dim3(wpr ? (items + kCombineWarps - 1) / kCombineWarps : items),
+                  dim3(kCombineWarps * 32), 0, st, a, g.head_dim, items, wpr, out);
 }
 
 }  // namespace sv

@@ -412,11 +412,19 @@ GemmPlan plan_gemm(int M, int N, int K, int mode) {
   return p;
 }
 
+// Split-K partial floats of either path: the tensor-memory kernel writes
+// rows padded to 16 (tc_np), the mma.sync kernel to its M-block width.
 size_t gemm_partial_floats(const GemmPlan& p) {
-  return (size_t)p.splits * p.n_tiles * kTileN * mma_ldp(p);
+  const size_t ldp = tc_supported(p.M) ? std::max<size_t>(mma_ldp(p), (size_t)tc_np(p.M)) : mma_ldp(p);
+  return (size_t)p.splits * p.n_tiles * kTileN * ldp;
 }
 size_t gemm_argmax_entries(const GemmPlan& p) { return (size_t)p.M; }
-int gemm_tickets(const GemmPlan& p) { return p.mblocks * p.n_tiles; }
+// Completion counters the fused last-CTA epilogue needs: one per (M-block,
+// tile) when it runs (few rows), none when the grid-wide reduce does the
+// epilogue (more rows).
+int gemm_tickets(const GemmPlan& p) {
+  return p.M > kFusedTailMaxRows ? 0 : p.mblocks * p.n_tiles;
+}
 
 cudaError_t launch_gemm(const GemmPlan& p, int mode, const void* x, const void* w,
                         const GemmBuffers& b, cudaStream_t st) {

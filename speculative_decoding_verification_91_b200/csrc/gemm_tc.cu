@@ -25,6 +25,7 @@
 #include "common.cuh"
 #include "gemm_epi.cuh"
 #include "internal.h"
+#include "tc_common.cuh"
 
 namespace sv {
 
@@ -33,67 +34,6 @@ namespace {
 constexpr int kTcThreads = 192;
 constexpr int kTcEpiWarp0 = 2;
 constexpr uint32_t kABytes = kTileN * 128;   // 16 KB weight tile per stage
-
-// ---- tcgen05 PTX wrappers -------------------------------------------------
-__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                   smem_u32(dst_smem)),
-               "r"(ncols));
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
-}
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols));
-}
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-// D[tmem] (+)= A[smem desc] . B[smem desc]^T, kind::f16 (bf16 in, fp32 accumulate)
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                          uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// mbarrier arrives once all tcgen05 operations issued so far by this thread completed
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   smem_u32(bar))
-               : "memory");
-}
-// 32 lanes x 32 consecutive fp32 columns: thread t gets lane (quadrant + t)
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
-      "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
-        "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
-        "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-// Shared-memory matrix descriptor: K-major, 128-byte swizzle, rows of 128 B in
-// 1024-byte atoms of 8 rows (stride byte offset 1024, leading byte offset 16),
-// descriptor version 1, base offset 0 (stage buffers are 1024-aligned).
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr) {
-  return (uint64_t)((smem_addr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
-         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
-// Instruction descriptor, kind::f16: D fp32, A and B bf16, both K-major, M = 128, N = np.
-__device__ __forceinline__ uint32_t idesc_bf16(int np) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(np >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
-}
 
 // barriers, TMEM slot, flags, then red_v / red_i [4][256] for the argmax
 constexpr uint32_t kTailBytes = 256u + 2u * 4u * 256u * 4u;
@@ -317,12 +257,21 @@ cudaError_t launch_tc_mode(const GemmPlan& p, const CUtensorMap& tw, const CUten
 
 }  // namespace
 
+// Row counts for the tensor-memory GEMM: above 32 (up to there the mma.sync
+// kernel streams the weights at the same HBM speed; at 40 and 64 rows it
+// becomes compute-bound: LM head at d 2560, 64 rows 442 us vs 230 us here)
+// and up to 256 (one TMEM accumulator of N = 256 columns).
+// SPECVERIFY_TC_MIN_ROWS overrides the lower bound (>= 16),
+// SPECVERIFY_NO_TC=1 turns the path off.
 bool tc_supported(int M) {
-  static const bool on = [] {
+  static const int min_rows = [] {
     const char* v = getenv("SPECVERIFY_NO_TC");
-    return !(v && v[0] == '1');
+    if (v && v[0] == '1') return 1 << 30;
+    const char* m = getenv("SPECVERIFY_TC_MIN_ROWS");
+    const int r = m ? atoi(m) : 32;
+    return r < 16 ? 16 : r;
   }();
-  return on && M > 64 && M <= 256;
+  return M > min_rows && M <= 256;
 }
 
 int tc_np(int M) { return (M + 15) / 16 * 16; }

@@ -74,10 +74,12 @@ struct GemmBuffers {
 };
 cudaError_t launch_gemm(const GemmPlan& p, int mode, const void* x, const void* w,
                         const GemmBuffers& buf, cudaStream_t st);
-// The same GEMMs on tcgen05 / TMEM for 64 < M <= 256 rows: every row sits in
+// The same GEMMs on tcgen05 / TMEM for 32 < M <= 256 rows: every row sits in
 // the MMA's N dimension, so the weights stream once.  tc_supported() is false
-// outside that range or when SPECVERIFY_NO_TC=1.
+// outside that range (SPECVERIFY_TC_MIN_ROWS moves the lower bound) or when
+// SPECVERIFY_NO_TC=1.
 bool tc_supported(int M);
+int tc_np(int M);   // rows of the tensor-memory GEMM (M rounded up to 16)
 cudaError_t launch_gemm_tc(const GemmPlan& p, int mode, const void* x, const void* w,
                            const GemmBuffers& buf, cudaStream_t st);
 // tcgen05 path when it applies, else the mma.sync path
@@ -148,6 +150,11 @@ struct AttnGeom {
 AttnGeom plan_attn(int B, int q, int Hq, int Hkv, int D, int page, int num_pages, int max_pages,
                    int window, int kv_equal, int sb_width, int split_tokens);
 size_t attn_partial_floats(const AttnGeom& g);
+bool attn_tc_supported(const AttnGeom& g);
+cudaError_t launch_attn_tc(const AttnGeom& g, const CUtensorMap& tk, const CUtensorMap& tv,
+                           const uint16_t* qrot, const int32_t* block_table, const int32_t* seq_lens,
+                           float* part_o, float* part_ml, unsigned* status, float scale_log2,
+                           cudaStream_t st);
 cudaError_t launch_attention(const AttnGeom& g, const uint16_t* qrot, const void* k_pool,
                              const void* v_pool, const void* ksb_pool, const int32_t* block_table,
                              const int32_t* seq_lens, float* part, uint16_t* out, unsigned* status,
