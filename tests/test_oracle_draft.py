@@ -1,0 +1,157 @@
+"""Pins of the drafter oracle (CPU only).
+
+The drafter's cross-attention is checked against torch's scaled-dot-product
+attention with an explicit visibility mask, its position convention by the
+window edge (one visible key gives that key's value exactly, none gives
+zero), the input concatenation and projections against torch's linear
+layers in the degenerate case where every block adds nothing, and the
+autoregressive loop against single steps.
+"""
+import copy
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import draft as OD
+from oracle import verify as OV
+
+D, HKV, HQD, DM, DD, V = 16, 2, 4, 32, 16, 50
+
+
+def _rng(seed=0):
+    return np.random.default_rng(seed)
+
+
+def _bits(x):
+    return OV.bits_from_bf16(x)
+
+
+def _model(window, kv_equal, frac, seed=0):
+    r = _rng(seed)
+    layer = OV.LayerDef(window, kv_equal, frac, np.zeros((1, DM), np.float32),
+                        np.zeros((DM, 1), np.float32))
+    return OV.Model(DM, 4, HKV, D, _bits(r.standard_normal((V, DM)) * 0.3), [layer])
+
+
+def _cache(model, L, seed=1):
+    r = _rng(seed)
+    spec = model.layers[0]
+    k_raw = OV.bf16(r.standard_normal((L, HKV, D)))
+    v_raw = None if spec.kv_equal else OV.bf16(r.standard_normal((L, HKV, D)))
+    return OV.cache_from_raw(model, 0, 0, k_raw, v_raw)
+
+
+def _drafter(seed=2, zero_o=False, n_blocks=2):
+    r = _rng(seed)
+    blocks = [OD.DraftBlockDef(0, OV.bf16(r.standard_normal((HQD * D, DD)) * 0.3),
+                               np.zeros((DD, HQD * D), np.float32) if zero_o
+                               else OV.bf16(r.standard_normal((DD, HQD * D)) * 0.1))
+              for _ in range(n_blocks)]
+    return OD.Drafter(DD, HQD, _bits(r.standard_normal((V, DD))),
+                      OV.bf16(r.standard_normal((DD, DM + DD)) * 0.2),
+                      OV.bf16(r.standard_normal((DM, DD)) * 0.3), blocks)
+
+
+def _sdpa(q, k, v, mask, scale):
+    t = lambda a: torch.from_numpy(np.asarray(a, np.float64))[None, None]
+    return torch.nn.functional.scaled_dot_product_attention(
+        t(q), t(k), t(v), attn_mask=torch.from_numpy(mask)[None, None], scale=scale)[0, 0].numpy()
+
+
+@pytest.mark.parametrize("window,kv_equal,frac,s", [(0, False, 1.0, 0), (0, True, 0.25, 2),
+                                                    (7, False, 1.0, 0), (7, False, 1.0, 3),
+                                                    (12, True, 0.25, 1)])
+def test_cross_attention_is_masked_sdpa(window, kv_equal, frac, s):
+    model, L = _model(window, kv_equal, frac), 20
+    cache, dr = _cache(model, L), _drafter()
+    q_pre = OV.f32(_rng(5).standard_normal((HQD, D)))
+    pos = L + s
+    got = OD.cross_attention(model, dr, dr.blocks[0], cache, L, pos, q_pre)
+    q_rot = OV.bf16(OV.rope(q_pre[None], [pos], D, model.rope_theta, frac))[0]
+    kpos = np.arange(L)
+    mask = (kpos <= pos) & ((kpos > pos - window) if window else True)
+    G = HQD // HKV
+    for h in range(HQD):
+        want = _sdpa(q_rot[h][None], cache.k[:, h // G], cache.values()[:, h // G], mask[None],
+                     1.0 / np.sqrt(D))[0]
+        np.testing.assert_array_equal(got[h], OV.bf16(want))
+
+
+def test_query_position_is_committed_length_plus_step():
+    # window 3, cache positions 0..4 (L = 5): step 1 sits at 6 and sees only
+    # key 4, so its output is that key's value exactly; step 0 (position 5)
+    # also sees key 3
+    model, L = _model(3, False, 1.0), 5
+    cache, dr = _cache(model, L), _drafter()
+    q_pre = OV.f32(_rng(6).standard_normal((HQD, D)))
+    out1 = OD.cross_attention(model, dr, dr.blocks[0], cache, L, L + 1, q_pre)
+    G = HQD // HKV
+    for h in range(HQD):
+        np.testing.assert_array_equal(out1[h], cache.v[4, h // G])
+    out0 = OD.cross_attention(model, dr, dr.blocks[0], cache, L, L, q_pre)
+    assert not np.array_equal(out0, out1)
+
+
+def test_no_visible_key_gives_zero():
+    model, L = _model(1, False, 1.0), 6       # window 1 at position L + 1: nothing cached
+    cache, dr = _cache(model, L), _drafter()
+    out = OD.cross_attention(model, dr, dr.blocks[0], cache, L, L + 1,
+                             OV.f32(_rng(7).standard_normal((HQD, D))))
+    assert np.array_equal(out, np.zeros_like(out))
+
+
+def test_projections_and_unembed_when_blocks_add_nothing():
+    # every W_o = 0: h = W_up (W_down [bf16(prev) || emb(tok)]) and the draft
+    # is the LM head's argmax on RMSNorm(h); torch linear layers, rms_norm
+    # and argmax give the same
+    model, L = _model(0, False, 1.0), 9
+    cache, dr = _cache(model, L), _drafter(zero_o=True)
+    prev = OV.f32(_rng(8).standard_normal(DM))
+    tok = 17
+    st = OD.draft_step(model, dr, [cache], L, 0, prev, tok)
+    t = lambda a: torch.from_numpy(np.asarray(a, np.float64))
+    u = torch.cat([t(OV.bf16(prev)), t(OV.bf16_from_bits(dr.w_emb_bits[tok]))])
+    x = torch.nn.functional.linear(u, t(dr.w_down)).float().double()
+    h = torch.nn.functional.linear(x, t(dr.w_up)).float()
+    np.testing.assert_array_equal(st.h, h.numpy())
+    hn = torch.nn.functional.rms_norm(h.double(), (DM,), eps=model.rms_eps)
+    hn = hn.float().to(torch.bfloat16).double()
+    logits = torch.nn.functional.linear(hn, t(OV.bf16_from_bits(model.w_lm_bits))).float()
+    assert st.token == int(torch.argmax(logits))
+    assert st.top1 == pytest.approx(float(logits.max()), rel=1e-6)
+
+
+def test_draft_is_autoregressive_and_reads_only():
+    model, L = _model(7, True, 0.25), 15
+    cache, dr = _cache(model, L), _drafter(n_blocks=3)
+    before = copy.deepcopy(cache)
+    prev = OV.f32(_rng(9).standard_normal(DM))
+    steps = OD.draft(model, dr, [cache], L, prev, 3, 4)
+    assert len(steps) == 4
+    hidden, tok = prev, 3
+    for s, st in enumerate(steps):
+        one = OD.draft_step(model, dr, [cache], L, s, hidden, tok)
+        assert one.token == st.token and np.array_equal(one.h, st.h)
+        hidden, tok = one.h, one.token
+    shorter = OD.draft(model, dr, [cache], L, prev, 3, 2)
+    assert [x.token for x in shorter] == [x.token for x in steps[:2]]
+    assert OD.draft(model, dr, [cache], L, prev, 3, 0) == []
+    for a, b in ((cache.k, before.k), (cache.kpre, before.kpre)):
+        assert np.array_equal(a, b)
+
+
+def test_draft_step_queries_sit_at_L_plus_s():
+    # window 2: step 2 sits at L + 2 and no cached key (< L) is in its window,
+    # so its blocks add nothing and it equals the same drafter with W_o = 0;
+    # step 0 (position L) sees key L - 1 and does not
+    model, L = _model(2, False, 1.0), 11
+    cache = _cache(model, L)
+    dr, dr0 = _drafter(seed=4), _drafter(seed=4, zero_o=True)
+    prev = OV.f32(_rng(10).standard_normal(DM))
+    a2 = OD.draft_step(model, dr, [cache], L, 2, prev, 5)
+    b2 = OD.draft_step(model, dr0, [cache], L, 2, prev, 5)
+    assert np.array_equal(a2.h, b2.h)
+    a0 = OD.draft_step(model, dr, [cache], L, 0, prev, 5)
+    b0 = OD.draft_step(model, dr0, [cache], L, 0, prev, 5)
+    assert not np.array_equal(a0.h, b0.h)
