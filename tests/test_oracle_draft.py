@@ -44,10 +44,11 @@ def _cache(model, L, seed=1):
 
 def _drafter(seed=2, zero_o=False, n_blocks=2):
     r = _rng(seed)
-    blocks = [OD.DraftBlockDef(0, OV.bf16(r.standard_normal((HQD * D, DD)) * 0.3),
-                               np.zeros((DD, HQD * D), np.float32) if zero_o
-                               else OV.bf16(r.standard_normal((DD, HQD * D)) * 0.1))
-              for _ in range(n_blocks)]
+    blocks = []
+    for _ in range(n_blocks):
+        w_q = OV.bf16(r.standard_normal((HQD * D, DD)) * 0.3)
+        w_o = OV.bf16(r.standard_normal((DD, HQD * D)) * 0.1)   # drawn either way: same stream
+        blocks.append(OD.DraftBlockDef(0, w_q, np.zeros_like(w_o) if zero_o else w_o))
     return OD.Drafter(DD, HQD, _bits(r.standard_normal((V, DD))),
                       OV.bf16(r.standard_normal((DD, DM + DD)) * 0.2),
                       OV.bf16(r.standard_normal((DM, DD)) * 0.3), blocks)
