@@ -36,11 +36,13 @@ the block internals from their sketch):
     cache holds positions < L only (the drafter writes nothing), so key j is
     visible iff j < L, and on a window-W block also j > L + s - W.  A query
     that sees no key gets a zero attention output;
-  * the concatenation order is [target activation, token embedding]; the
-    activation is rounded to bf16 as a GEMM input; the up-projection's
-    output (binary32) is both the next step's activation and, after the
-    target's final RMSNorm (rounded to bf16), the input of the target's LM
-    head; argmax ties go to the lowest token id.
+  * the concatenation order is [target activation, token embedding]; every
+    projection reads bf16 (the activation and the residual stream are
+    rounded to bf16 where they enter a projection, as the target's GEMM
+    inputs are); the up-projection's output (binary32) is both the next
+    step's activation and, after the target's final RMSNorm (rounded to
+    bf16), the input of the target's LM head; argmax ties go to the lowest
+    token id.
 """
 from __future__ import annotations
 
@@ -122,7 +124,7 @@ def draft_step(model: Model, drafter: Drafter, caches: list, L: int, s: int, pre
         o = cross_attention(model, drafter, blk, caches[blk.target_layer], L, L + s, q_pre)
         y = f32(o.reshape(-1).astype(np.float64) @ blk.w_o.astype(np.float64).T)
         x = f32(x.astype(np.float64) + y.astype(np.float64))
-    h = f32(x.astype(np.float64) @ drafter.w_up.astype(np.float64).T)
+    h = f32(bf16(x).astype(np.float64) @ drafter.w_up.astype(np.float64).T)
     hn = bf16(rmsnorm(h, model.rms_eps))
     g, t1, t2 = lm_head_top2(hn[None], model.w_lm_bits)
     return DraftStep(h, int(g[0]), float(t1[0]), float(t2[0]))

@@ -103,7 +103,7 @@ def test_no_visible_key_gives_zero():
 
 
 def test_projections_and_unembed_when_blocks_add_nothing():
-    # every W_o = 0: h = W_up (W_down [bf16(prev) || emb(tok)]) and the draft
+    # every W_o = 0: h = W_up bf16(W_down [bf16(prev) || emb(tok)]) and the draft
     # is the LM head's argmax on RMSNorm(h); torch linear layers, rms_norm
     # and argmax give the same
     model, L = _model(0, False, 1.0), 9
@@ -113,8 +113,8 @@ def test_projections_and_unembed_when_blocks_add_nothing():
     st = OD.draft_step(model, dr, [cache], L, 0, prev, tok)
     t = lambda a: torch.from_numpy(np.asarray(a, np.float64))
     u = torch.cat([t(OV.bf16(prev)), t(OV.bf16_from_bits(dr.w_emb_bits[tok]))])
-    x = torch.nn.functional.linear(u, t(dr.w_down)).float().double()
-    h = torch.nn.functional.linear(x, t(dr.w_up)).float()
+    x = torch.nn.functional.linear(u, t(dr.w_down)).float()
+    h = torch.nn.functional.linear(x.to(torch.bfloat16).double(), t(dr.w_up)).float()
     np.testing.assert_array_equal(st.h, h.numpy())
     hn = torch.nn.functional.rms_norm(h.double(), (DM,), eps=model.rms_eps)
     hn = hn.float().to(torch.bfloat16).double()
