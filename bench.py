@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
     ap.add_argument("--workload", default="b1_ctx8k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--draft", action="store_true",
+                    help="time the MTP drafter (spec_draft, k steps) on the workload; one JSON line")
     ap.add_argument("--sweep", action="store_true",
                     help="verify-step time over batch x k on the b1_ctx8k model; one JSON line")
     ap.add_argument("--profile-case", action="store_true",
@@ -521,8 +523,69 @@ def run_sweep(args):
                       "points": out, "clocks": clocks.summary()}), flush=True)
 
 
+def run_draft_bench(args):
+    """--draft: k drafter steps (spec_draft) for the workload's batch on its
+    target cache: 4 blocks (3 sliding-window, 1 global) of width 256, each
+    step ending in the target's LM head over the full vocabulary.  Inputs
+    resident; L2 flushed before every timed call; CUDA events on the stream."""
+    import torch
+    from speculative_decoding_verification_91_b200 import binding as B
+    from speculative_decoding_verification_91_b200.inputs import workloads as W
+    from speculative_decoding_verification_91_b200.runtime import DeviceDrafter, Workspace, to_device_bf16
+    from speculative_decoding_verification_91_b200.session import WorkloadSession
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    wl = W.get_workload(args.workload)
+    sess = WorkloadSession(wl, device=dev, poison=False)
+    dd, hq, targets = W.drafter_spec(wl)
+    emb, down, upw, blocks = W.drafter_weights(wl)
+    dr = DeviceDrafter(d_draft=dd, n_q_heads=hq, w_emb_bits=emb, w_down_bits=down, w_up_bits=upw,
+                       blocks=blocks, device=dev)
+    Bn, k = wl.batch, max(1, wl.k)
+    hidden = to_device_bf16(np.stack([W.drafter_inputs(wl, b, 0)[0] for b in range(Bn)]), dev)
+    toks = torch.tensor([W.drafter_inputs(wl, b, 0)[1] for b in range(Bn)], dtype=torch.int32, device=dev)
+    ws = Workspace(B.spec_draft_workspace_bytes(sess.dm.desc, dr.desc, Bn, sess.max_pages), dev)
+    drafts = torch.zeros(Bn * k, dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def call():
+        B.spec_draft(sess.dm.desc, dr.desc, sess.block_table, sess.max_pages, sess.seq_lens, hidden,
+                     toks, Bn, k, drafts, None, ws.buf, ws.nbytes, stream)
+
+    for _ in range(max(3, args.warmup)):
+        call()
+    torch.cuda.synchronize(dev)
+    steps = max(3, min(args.steps, 200))
+    e0 = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    e1 = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    n0 = B.spec_launch_count()
+    with ClockSampler(0) as clocks:
+        for i in range(steps):
+            flush.zero_()
+            e0[i].record(stream)
+            call()
+            e1[i].record(stream)
+        torch.cuda.synchronize(dev)
+    launches = B.spec_launch_count() - n0
+    if ws.device_status(stream) != 0:
+        raise RuntimeError("device status flagged during the drafter calls")
+    us = float(np.mean([a.elapsed_time(b) for a, b in zip(e0, e1)])) * 1e3
+    lm_bytes = wl.vocab * wl.d_model * 2
+    print(json.dumps({"kernel": "spec_draft", "workload": wl.name, "batch": Bn, "k": k,
+                      "d_draft": dd, "blocks_target_layers": targets,
+                      "us_per_call": us, "us_per_draft_step": us / k,
+                      "drafted_tokens_per_s": Bn * k / (us / 1e6),
+                      "lm_head_bytes_per_step": lm_bytes,
+                      "gpu_launches_per_call": launches / steps,
+                      "l2": "flushed before every timed call", "clocks": clocks.summary()}), flush=True)
+
+
 def main():
     args = parse()
+    if args.draft:
+        run_draft_bench(args)
+        return
     if args.sweep:
         run_sweep(args)
         return

@@ -230,6 +230,63 @@ int spec_prefill(const spec_model* m, const int32_t* block_table, int max_pages,
                  const int32_t* tokens, int B, int n, int32_t* seq_lens, int32_t* next_token,
                  float* next_maxlogit, void* ws, size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * MTP drafter on the target's shared KV cache ("Gemma 4 拆解 | 多模态怎么塞进端侧，
+ * MTP drafter 又是怎么自带投机采样的" §4.2: the drafter's input is the target's
+ * last-layer activation plus the embedding of the previous token, projected
+ * down to the drafter width; its blocks (three sliding-window, one global)
+ * attend to the target's cache instead of keeping one of their own, so it
+ * needs no prefill; its output is projected back up and the target's
+ * unembedding picks the next draft token; k tokens are drafted one after the
+ * other).
+ *
+ * Each block is x <- x + W_o CrossAttn(RMSNorm(x)) with n_q_heads heads of
+ * the target's head_dim over the cache of target layer `target_layer`, read
+ * as stored (post-RoPE keys; values or the key-equals-value side-band) with
+ * that layer's window and RoPE fraction.  Draft step s of sequence b sits at
+ * position seq_lens[b] + s and sees the cached keys j < seq_lens[b] (window
+ * layers: also j > seq_lens[b] + s - window); a query that sees no key gets
+ * a zero attention output.  The up-projection's output (binary32) is the
+ * next step's activation; the target's final RMSNorm and LM head turn it
+ * into the draft token (argmax, ties to the lowest id).  Every projection
+ * input is bf16.  The drafter writes nothing to the cache and does not
+ * change seq_lens.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  const void* w_q;     /* bf16 [n_q_heads * head_dim][d_draft] */
+  const void* w_o;     /* bf16 [d_draft][n_q_heads * head_dim] */
+  int target_layer;    /* target layer whose cache this block reads */
+} spec_draft_block;
+
+typedef struct {
+  int d_draft;         /* drafter width, multiple of 8 */
+  int n_q_heads;       /* query heads per block, multiple of the target's n_kv_heads */
+  int n_blocks;        /* 1..16 */
+  const void* w_embed; /* bf16 [vocab][d_draft]: the drafter's own token embedding */
+  const void* w_down;  /* bf16 [d_draft][d_model + d_draft]: input [activation || embedding] */
+  const void* w_up;    /* bf16 [d_model][d_draft] */
+  const spec_draft_block* blocks;
+} spec_drafter;
+
+/* Workspace bytes of spec_draft for up to B sequences (0 if unsupported). */
+size_t spec_draft_workspace_bytes(const spec_model* m, const spec_drafter* d, int B, int max_pages);
+
+/* k drafter steps for B sequences.
+ *   block_table [B][max_pages], seq_lens [B]: the target's committed cache
+ *     (device, read only);
+ *   prev_hidden: bf16 [B][d_model], the target's last-layer activation for
+ *     the last accepted token (device);
+ *   prev_token [B]: that token (device);
+ *   drafts [B][k] (out, device), draft_maxlogit [B][k] (out, device, or NULL).
+ * ws: caller-owned device workspace of spec_draft_workspace_bytes, set up
+ * once with spec_workspace_init.  Host-detectable errors return before any
+ * launch; a bad token id sets SPEC_DEV_BAD_TOKEN (read with
+ * spec_read_device_status).  k = 0 launches nothing. */
+int spec_draft(const spec_model* m, const spec_drafter* d, const int32_t* block_table, int max_pages,
+               const int32_t* seq_lens, const void* prev_hidden, const int32_t* prev_token, int B,
+               int k, int32_t* drafts, float* draft_maxlogit, void* ws, size_t ws_bytes,
+               void* stream);
+
 /* LM head + argmax without a workspace, for callers that cannot allocate
  * device memory.  The pages have no counterpart: this is a deployment aid.
  *

@@ -34,6 +34,7 @@ EXPORTED = [
     "spec_verify_step", "spec_profile_start", "spec_profile_collect",
     "spec_lmhead_argmax_noalloc", "spec_prefill_workspace_bytes", "spec_prefill",
     "spec_profile_launches", "spec_profile_launches_collect", "spec_launch_count",
+    "spec_draft_workspace_bytes", "spec_draft",
 ]
 SPEC_MAX_PREFILL = 256
 SPEC_NOALLOC_MAX_ROWS = 64
@@ -61,6 +62,18 @@ class SpecModel(ctypes.Structure):
         ("head_dim", c_int), ("vocab", c_int), ("page_size", c_int), ("num_pages", c_int),
         ("split_tokens", c_int), ("rope_theta", ctypes.c_double), ("rms_eps", ctypes.c_double),
         ("w_lm", c_void_p), ("w_embed", c_void_p), ("layers", POINTER(SpecLayer)),
+    ]
+
+
+class SpecDraftBlock(ctypes.Structure):
+    _fields_ = [("w_q", c_void_p), ("w_o", c_void_p), ("target_layer", c_int)]
+
+
+class SpecDrafter(ctypes.Structure):
+    _fields_ = [
+        ("d_draft", c_int), ("n_q_heads", c_int), ("n_blocks", c_int),
+        ("w_embed", c_void_p), ("w_down", c_void_p), ("w_up", c_void_p),
+        ("blocks", POINTER(SpecDraftBlock)),
     ]
 
 
@@ -113,9 +126,14 @@ def lib():
         L.spec_profile_launches_collect.argtypes = [POINTER(c_float), c_int, POINTER(c_int)]
         L.spec_profile_start.argtypes = [c_int]
         L.spec_profile_collect.argtypes = [POINTER(c_float), POINTER(c_float), c_int]
+        pd = POINTER(SpecDrafter)
+        L.spec_draft_workspace_bytes.argtypes = [pm, pd, c_int, c_int]
+        L.spec_draft.argtypes = [pm, pd, c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_int, c_int,
+                                 c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]
         for name in EXPORTED[4:]:
-            if name != "spec_prefill_workspace_bytes":
+            if name not in ("spec_prefill_workspace_bytes", "spec_draft_workspace_bytes"):
                 getattr(L, name).restype = c_int
+        L.spec_draft_workspace_bytes.restype = c_size_t
         L.spec_launch_count.argtypes = []
         L.spec_launch_count.restype = ctypes.c_ulonglong
         _lib = L
@@ -261,3 +279,15 @@ def spec_profile_launches_collect(max_marks: int = 256):
     _check(lib().spec_profile_launches_collect(buf, max_marks, ctypes.byref(n)),
            "spec_profile_launches_collect")
     return list(buf[:n.value])
+
+
+def spec_draft_workspace_bytes(model, drafter, B: int, max_pages: int) -> int:
+    return int(lib().spec_draft_workspace_bytes(ctypes.byref(model), ctypes.byref(drafter), B, max_pages))
+
+
+def spec_draft(model, drafter, block_table, max_pages, seq_lens, prev_hidden, prev_token, B, k,
+               drafts, draft_maxlogit, ws, ws_bytes, stream=None) -> int:
+    return _check(lib().spec_draft(ctypes.byref(model), ctypes.byref(drafter), _p(block_table),
+                                   max_pages, _p(seq_lens), _p(prev_hidden), _p(prev_token), B, k,
+                                   _p(drafts), _p(draft_maxlogit), _p(ws), ws_bytes, _s(stream)),
+                  "spec_draft")

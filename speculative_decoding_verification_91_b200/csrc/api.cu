@@ -327,6 +327,164 @@ int run_forward(const spec_model* m, const int32_t* block_table, int max_pages, 
   return rc;
 }
 
+// ---------------------------------------------------------------- drafter
+
+int check_drafter(const spec_model* m, const spec_drafter* d) {
+  if (!d || !d->blocks || !d->w_embed || !d->w_down || !d->w_up) return SPEC_EINVAL;
+  if (d->d_draft < 8 || d->d_draft % 8 || d->n_q_heads < 1 || d->n_q_heads % m->n_kv_heads ||
+      d->n_blocks < 1 || d->n_blocks > 16)
+    return SPEC_EINVAL;
+  const void* ptrs[3] = {d->w_embed, d->w_down, d->w_up};
+  for (const void* p : ptrs)
+    if (reinterpret_cast<uintptr_t>(p) & 15) return SPEC_EINVAL;
+  for (int i = 0; i < d->n_blocks; ++i) {
+    const spec_draft_block& b = d->blocks[i];
+    if (!b.w_q || !b.w_o || b.target_layer < 0 || b.target_layer >= m->n_layers) return SPEC_EINVAL;
+    if ((reinterpret_cast<uintptr_t>(b.w_q) & 15) || (reinterpret_cast<uintptr_t>(b.w_o) & 15))
+      return SPEC_EINVAL;
+  }
+  return SPEC_OK;
+}
+
+// Workspace of one drafter call for B sequences (q = 1 row each).
+struct DraftLayout {
+  size_t u, x, hn, qrot, attn_out, attn_part, gemm_part, h, arg_keys, ids, maxv, rope_tab, total;
+  int tickets;
+  bool splits_ok;
+};
+
+DraftLayout draft_layout(const spec_model* m, const spec_drafter* d, int B, int max_pages) {
+  DraftLayout s{};
+  s.splits_ok = true;
+  const int D = m->head_dim, dm = m->d_model, dd = d->d_draft, nq = d->n_q_heads * D;
+  size_t attn = 0;
+  for (int i = 0; i < d->n_blocks; ++i) {
+    const spec_layer& L = m->layers[d->blocks[i].target_layer];
+    AttnGeom g = plan_attn(B, 1, d->n_q_heads, m->n_kv_heads, D, m->page_size, m->num_pages,
+                           max_pages, L.window, L.kv_equal, 2 * n_rot_of(m, L), split_of(m, L));
+    attn = std::max(attn, attn_partial_floats(g));
+    if (g.n_splits_grid > kMaxSplits) s.splits_ok = false;
+  }
+  const GemmPlan ps[4] = {plan_gemm(B, dd, dm + dd, kGemmStore), plan_gemm(B, nq, dd, kGemmQkvRope),
+                          plan_gemm(B, dd, nq, kGemmResidual), plan_gemm(B, dm, dd, kGemmStore)};
+  size_t gp = 0;
+  int tickets = plan_gemm(B, m->vocab, dm, kGemmArgmax).mblocks;
+  for (const GemmPlan& p : ps) {
+    gp = std::max(gp, gemm_partial_floats(p));
+    tickets = std::max(tickets, gemm_tickets(p));
+  }
+  size_t off = kWsHeaderBytes;
+  s.u = off;         off = up(off + (size_t)B * (dm + dd) * 2);
+  s.x = off;         off = up(off + (size_t)B * dd * 4);
+  s.hn = off;        off = up(off + (size_t)B * std::max(dd, dm) * 2);
+  s.qrot = off;      off = up(off + (size_t)B * nq * 2);
+  s.attn_out = off;  off = up(off + (size_t)B * nq * 2);
+  s.attn_part = off; off = up(off + attn * 4);
+  s.gemm_part = off; off = up(off + gp * 4);
+  s.h = off;         off = up(off + (size_t)B * dm * 4);
+  s.arg_keys = off;  off = up(off + (size_t)B * 8);
+  s.ids = off;       off = up(off + (size_t)B * 4);
+  s.maxv = off;      off = up(off + (size_t)B * 4);
+  s.rope_tab = off;  off = up(off + (size_t)B * (D / 2) * 8);
+  s.total = off;
+  s.tickets = tickets;
+  return s;
+}
+
+// k drafter steps: [activation || embedding] -> down -> blocks (RMSNorm, query
+// projection + RoPE at position L + s, cross-attention over the target
+// layer's cache, output projection + residual) -> bf16 -> up -> final RMSNorm
+// -> LM head argmax -> drafts[:, s].
+int run_draft(const spec_model* m, const spec_drafter* d, const int32_t* block_table, int max_pages,
+              const int32_t* seq_lens, const void* prev_hidden, const int32_t* prev_token, int B, int k,
+              int32_t* drafts, float* draft_max, void* ws, size_t ws_bytes, cudaStream_t st) {
+  DraftLayout s = draft_layout(m, d, B, max_pages);
+  if (s.tickets > kMaxTickets || !s.splits_ok) return SPEC_EUNSUPPORTED;
+  if (ws_bytes < s.total) return SPEC_EINVAL;
+  WsHeader hdr = ws_header(ws);
+  const int D = m->head_dim, dm = m->d_model, dd = d->d_draft, nq = d->n_q_heads * D, half = D / 2;
+  uint16_t* u = at<uint16_t>(ws, s.u);
+  float* x = at<float>(ws, s.x);
+  uint16_t* hn = at<uint16_t>(ws, s.hn);
+  uint16_t* qrot = at<uint16_t>(ws, s.qrot);
+  uint16_t* attn_out = at<uint16_t>(ws, s.attn_out);
+  float* h = at<float>(ws, s.h);
+  int32_t* ids = at<int32_t>(ws, s.ids);
+  float* maxv = at<float>(ws, s.maxv);
+  float2* rope_tab = at<float2>(ws, s.rope_tab);
+  double inv_freq[128];
+  rope_inv_freq(m->rope_theta, D, half, inv_freq);
+  auto bufs = [&]() {
+    GemmBuffers b{};
+    b.partial = at<float>(ws, s.gemm_part);
+    b.tickets = hdr.tickets;
+    b.status = hdr.status;
+    return b;
+  };
+  int rc;
+  for (int step = 0; step < k; ++step) {
+    rc = cuda_status(launch_draft_input(step == 0 ? static_cast<const uint16_t*>(prev_hidden) : nullptr,
+                                        step == 0 ? nullptr : h, dm, step == 0 ? prev_token : ids,
+                                        d->w_embed, m->vocab, dd, u, hdr.status, seq_lens, step,
+                                        inv_freq, half, rope_tab, B, st));
+    if (rc) return rc;
+    GemmBuffers bd = bufs();
+    bd.out = x;
+    rc = cuda_status(launch_gemm_any(plan_gemm(B, dd, dm + dd, kGemmStore), kGemmStore, u, d->w_down, bd, st));
+    if (rc) return rc;
+    for (int i = 0; i < d->n_blocks; ++i) {
+      const spec_draft_block& blk = d->blocks[i];
+      const spec_layer& L = m->layers[blk.target_layer];
+      rc = cuda_status(launch_rmsnorm(x, B, dd, m->rms_eps, hn, st));
+      if (rc) return rc;
+      GemmBuffers bq = bufs();
+      RopeFuse& f = bq.rope;
+      f.n_q_heads = d->n_q_heads;     // every projected head is a query head: the cache is not written
+      f.n_kv_heads = m->n_kv_heads;
+      f.head_dim = D;
+      f.n_rot = n_rot_of(m, L);
+      f.q = 1;
+      f.page_size = m->page_size;
+      f.num_pages = m->num_pages;
+      f.max_pages = max_pages;
+      f.seq_lens = seq_lens;
+      f.block_table = block_table;
+      f.rope_tab = rope_tab;
+      f.q_out = qrot;
+      rc = cuda_status(launch_gemm_any(plan_gemm(B, nq, dd, kGemmQkvRope), kGemmQkvRope, hn, blk.w_q, bq, st));
+      if (rc) return rc;
+      AttnGeom g = plan_attn(B, 1, d->n_q_heads, m->n_kv_heads, D, m->page_size, m->num_pages,
+                             max_pages, L.window, L.kv_equal, 2 * f.n_rot, split_of(m, L));
+      g.qpos_off = step;   // the query sits at L + step ...
+      g.kend_off = -1;     // ... over the cached keys j < L
+      rc = cuda_status(launch_attention(g, qrot, L.k_pool, L.v_pool, L.ksb_pool, block_table, seq_lens,
+                                        at<float>(ws, s.attn_part), attn_out, hdr.status, st));
+      if (rc) return rc;
+      GemmBuffers bo = bufs();
+      bo.out = x;
+      rc = cuda_status(launch_gemm_any(plan_gemm(B, dd, nq, kGemmResidual), kGemmResidual, attn_out, blk.w_o, bo, st));
+      if (rc) return rc;
+    }
+    rc = cuda_status(launch_to_bf16(x, (size_t)B * dd, hn, st));
+    if (rc) return rc;
+    GemmBuffers bu = bufs();
+    bu.out = h;
+    rc = cuda_status(launch_gemm_any(plan_gemm(B, dm, dd, kGemmStore), kGemmStore, hn, d->w_up, bu, st));
+    if (rc) return rc;
+    rc = cuda_status(launch_rmsnorm(h, B, dm, m->rms_eps, hn, st));
+    if (rc) return rc;
+    GemmBuffers bl = bufs();
+    bl.arg_keys = at<unsigned long long>(ws, s.arg_keys);
+    bl.ids = ids;
+    bl.maxv = maxv;
+    rc = cuda_status(launch_gemm_any(plan_gemm(B, m->vocab, dm, kGemmArgmax), kGemmArgmax, hn, m->w_lm, bl, st));
+    if (rc) return rc;
+    rc = cuda_status(launch_draft_collect(ids, maxv, B, k, step, drafts, draft_max, st));
+    if (rc) return rc;
+  }
+  return SPEC_OK;
+}
+
 }  // namespace
 }  // namespace sv
 
@@ -605,6 +763,28 @@ int spec_prefill(const spec_model* m, const int32_t* block_table, int max_pages,
   io.next_maxlogit = next_maxlogit;
   return run_forward(m, block_table, max_pages, B, n, seq_lens, io, ws, ws_bytes,
                      static_cast<cudaStream_t>(stream));
+}
+
+size_t spec_draft_workspace_bytes(const spec_model* m, const spec_drafter* d, int B, int max_pages) {
+  if (check_model(m) || check_drafter(m, d) || B < 1 || max_pages < 1) return 0;
+  DraftLayout s = draft_layout(m, d, B, max_pages);
+  if (s.tickets > kMaxTickets || !s.splits_ok) return 0;
+  return s.total;
+}
+
+int spec_draft(const spec_model* m, const spec_drafter* d, const int32_t* block_table, int max_pages,
+               const int32_t* seq_lens, const void* prev_hidden, const int32_t* prev_token, int B,
+               int k, int32_t* drafts, float* draft_maxlogit, void* ws, size_t ws_bytes,
+               void* stream) {
+  int rc = check_model(m);
+  if (rc) return rc;
+  rc = check_drafter(m, d);
+  if (rc) return rc;
+  if (!block_table || !seq_lens || !prev_hidden || !prev_token || !drafts || !ws) return SPEC_EINVAL;
+  if (B < 1 || k < 0 || max_pages < 1) return SPEC_EINVAL;
+  if (k == 0) return SPEC_OK;
+  return run_draft(m, d, block_table, max_pages, seq_lens, prev_hidden, prev_token, B, k, drafts,
+                   draft_maxlogit, ws, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

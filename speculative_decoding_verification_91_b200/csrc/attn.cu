@@ -149,6 +149,8 @@ struct ACfg {
 
 struct AttnArgs {
   int q, Hq, Hkv, G, max_pages, num_pages, window, split, n_splits_grid, rows, n_rot;
+  int qpos_off;   // row i of a sequence sits at position L + qpos_off + i
+  int kend_off;   // its last cached key is at position L + kend_off
   const uint16_t* qrot;
   const int32_t* block_table;
   const int32_t* seq_lens;
@@ -158,9 +160,13 @@ struct AttnArgs {
   float scale_log2;
 };
 
-__device__ __forceinline__ void seq_key_range(int L, int q, int window, int& klo, int& khi) {
-  klo = window > 0 ? max(0, L - window + 1) : 0;
-  khi = L + q - 1;
+// Keys any row of a sequence may see: from the first row's window start
+// (global layers: 0) to the last cached key.  Verify rows: positions L..L+q-1
+// after appending their own keys (qpos_off 0, kend_off q-1); drafter rows:
+// position L + s over the cache [0, L) (qpos_off s, kend_off -1).
+__device__ __forceinline__ void seq_key_range(int L, const AttnArgs& a, int& klo, int& khi) {
+  klo = a.window > 0 ? max(0, L + a.qpos_off - a.window + 1) : 0;
+  khi = L + a.kend_off;
 }
 
 template <int D, int MT, bool KVEQ>
@@ -194,7 +200,7 @@ __global__ void __launch_bounds__(kThreads) attn_split_kernel(
     return;
   }
   int klo, khi;
-  seq_key_range(L, a.q, a.window, klo, khi);
+  seq_key_range(L, a, klo, khi);
   const int s_abs = klo / a.split + blockIdx.x;
   if (s_abs * a.split > khi) return;  // beyond this sequence's last split
   const int lo = max(s_abs * a.split, klo);
@@ -275,7 +281,7 @@ __global__ void __launch_bounds__(kThreads) attn_split_kernel(
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int r = mt * 16 + g + 8 * h;
-      rpos[mt][h] = (r < nrows) ? L + (r0 + r) % a.q : -1;
+      rpos[mt][h] = (r < nrows) ? L + a.qpos_off + (r0 + r) % a.q : -1;
     }
 
   float m_run[MT][2], l_run[MT][2];
@@ -345,7 +351,8 @@ __global__ void __launch_bounds__(kThreads) attn_split_kernel(
         for (int e = 0; e < 4; ++e) {
           const int j = key0 + warp * 16 + nt * 8 + 2 * t + (e & 1);
           const int p = rpos[mt][e >> 1];
-          const bool vis = valid && p >= 0 && j >= klo && j <= p && (a.window == 0 || j > p - a.window);
+          const bool vis = valid && p >= 0 && j >= klo && j <= p && j <= khi &&
+                           (a.window == 0 || j > p - a.window);
           sc[mt][nt][e] = vis ? __fmul_rn(sc[mt][nt][e], a.scale_log2) : -INFINITY;
         }
     // ---- row maxima over this warp's keys
@@ -512,14 +519,16 @@ __global__ void __launch_bounds__(kThreads) attn_split_kernel(
 
 // out[b][i][h] = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s.
 // The split maxima and weighted denominators are butterfly reductions over a
-// warp's lanes; the numerator is summed over four contiguous quarters of the
-// splits, each in ascending order (lane: 8 output dims), and the quarters are
-// added in order.  That tree depends only on the split count, i.e. on the
-// sequence length, and is the same in both thread mappings:
-//   warp_per_row = 1: one warp per query row (4 rows per CTA), the warp
-//                     walks the four quarters itself (few splits, many rows);
-//   warp_per_row = 0: one CTA of four warps per query row, warp w sums
-//                     quarter w (many splits, few rows).
+// warp's lanes.  The numerator is summed in four parts: part v takes the
+// splits s with (s / 4) % 4 == v in ascending order (lane: 8 output dims),
+// and the parts are added in order.  The grouping is by absolute split
+// index, so splits past a row's own keys (more of them for larger k) only
+// append exact zeros: a row's result does not depend on k.  Both thread
+// mappings compute exactly this:
+//   warp_per_row = 1: one warp per query row (4 rows per CTA) walks the four
+//                     parts itself (few splits, many rows);
+//   warp_per_row = 0: one CTA of four warps per query row, warp v sums part
+//                     v (many splits, few rows).
 constexpr int kCombineWarps = 4;
 constexpr int kMaxCombineSplits = kMaxSplits;
 __global__ void __launch_bounds__(kCombineWarps * 32) attn_combine_kernel(AttnArgs a, int D, int n_items,
@@ -544,8 +553,8 @@ __global__ void __launch_bounds__(kCombineWarps * 32) attn_combine_kernel(AttnAr
     return;
   }
   int klo, khi;
-  seq_key_range(L, a.q, a.window, klo, khi);
-  const int ns = min(khi / a.split - klo / a.split + 1, kMaxCombineSplits);
+  seq_key_range(L, a, klo, khi);
+  const int ns = khi < klo ? 0 : min(khi / a.split - klo / a.split + 1, kMaxCombineSplits);
   const long slot0 = ((long)(b * a.Hkv + kvh) * a.n_splits_grid) * a.rows + r;
   float* m_s = msh[warp_per_row ? warp : 0];
   float* l_s = lsh[warp_per_row ? warp : 0];
@@ -569,23 +578,26 @@ __global__ void __launch_bounds__(kCombineWarps * 32) attn_combine_kernel(AttnAr
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) den = __fadd_rn(den, __shfl_xor_sync(0xffffffffu, den, off));
+  if (!(den > 0.f)) {   // the row sees no key (drafter rows past a short window): zero output
+    if (warp_per_row || warp == 0)
+      for (int e = lane; e < D; e += 32) dst[e] = 0;
+    return;
+  }
 
-  const int per_q = (ns + 3) / 4;
   const int per_lane = D / 32;   // 8 (D = 256) or 4 (D = 128)
   const float* po = a.part_o + slot0 * D + lane * per_lane;
   const long sstride = (long)a.rows * D;
-  // sum of quarter q of the splits for this lane's dims, ascending, four
-  // splits' loads in flight per step
-  auto quarter = [&](int q, float (&acc)[8]) {
+  // part v: chunks of four splits c = v, v + 4, v + 8, ..., ascending, the
+  // chunk's four loads in flight together
+  auto part_sum = [&](int v, float (&acc)[8]) {
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-    const int s_lo = q * per_q, s_hi = min(ns, s_lo + per_q);
     constexpr int U = 4;
-    for (int s0 = s_lo; s0 < s_hi; s0 += U) {
+    for (int s0 = v * U; s0 < ns; s0 += 4 * U) {
       float4 x[U][2];
 #pragma unroll
       for (int u = 0; u < U; ++u) {
-        const bool in = s0 + u < s_hi;
+        const bool in = s0 + u < ns;
         const float* pp = po + (s0 + u) * sstride;
         x[u][0] = in ? __ldcg(reinterpret_cast<const float4*>(pp)) : make_float4(0, 0, 0, 0);
         x[u][1] = (in && per_lane == 8) ? __ldcg(reinterpret_cast<const float4*>(pp + 4))
@@ -593,7 +605,7 @@ __global__ void __launch_bounds__(kCombineWarps * 32) attn_combine_kernel(AttnAr
       }
 #pragma unroll
       for (int u = 0; u < U; ++u) {
-        if (s0 + u >= s_hi) break;
+        if (s0 + u >= ns) break;
         const float m = m_s[s0 + u];
         const float ws = (m == -INFINITY) ? 0.f : exp2f(__fsub_rn(m, M));
         const float xs[8] = {x[u][0].x, x[u][0].y, x[u][0].z, x[u][0].w,
@@ -605,17 +617,17 @@ __global__ void __launch_bounds__(kCombineWarps * 32) attn_combine_kernel(AttnAr
   };
   float num[8];
   if (warp_per_row) {
-    quarter(0, num);
+    part_sum(0, num);
 #pragma unroll 1
     for (int q = 1; q < 4; ++q) {
       float acc[8];
-      quarter(q, acc);
+      part_sum(q, acc);
 #pragma unroll
       for (int e = 0; e < 8; ++e) num[e] = __fadd_rn(num[e], acc[e]);
     }
   } else {
     float acc[8];
-    quarter(warp, acc);
+    part_sum(warp, acc);
 #pragma unroll
     for (int e = 0; e < 8; ++e)
       if (e < per_lane) part[warp][lane * per_lane + e] = acc[e];
@@ -683,6 +695,8 @@ AttnGeom plan_attn(int B, int q, int Hq, int Hkv, int D, int page, int num_pages
   g.sb_width = sb_width;
   g.split_tokens = split_tokens;
   g.rows = (Hq / Hkv) * q;
+  g.qpos_off = 0;
+  g.kend_off = q - 1;
   const int mt = std::min(4, (g.rows + 15) / 16);
   g.row_blocks = (g.rows + mt * 16 - 1) / (mt * 16);
   if (window > 0) {
@@ -721,6 +735,8 @@ cudaError_t launch_attention(const AttnGeom& g, const uint16_t* qrot, const void
   a.num_pages = g.num_pages;
   a.window = g.window;
   a.split = g.split_tokens;
+  a.qpos_off = g.qpos_off;
+  a.kend_off = g.kend_off;
   a.n_splits_grid = g.n_splits_grid;
   a.rows = g.rows;
   a.n_rot = g.sb_width / 2;

@@ -548,7 +548,8 @@ bool attn_tc_supported(const AttnGeom& g) {
     const char* off = getenv("SPECVERIFY_NO_TC");
     return v && v[0] == '1' && !(off && off[0] == '1');
   }();
-  return on && g.head_dim == kDim && g.page_size == kPg && g.split_tokens % kBlk == 0 &&
+  return on && g.qpos_off == 0 && g.kend_off == g.q - 1 &&   // verify rows only
+         g.head_dim == kDim && g.page_size == kPg && g.split_tokens % kBlk == 0 &&
          g.split_tokens <= kPg * kMaxSplitPages && (!g.kv_equal || g.sb_width == 64);
 }
 

@@ -90,6 +90,14 @@ inline cudaError_t launch_gemm_any(const GemmPlan& p, int mode, const void* x, c
 }
 
 // ------------------------------------------------------------- small kernels
+cudaError_t launch_draft_input(const uint16_t* prev_bf16, const float* prev_f32, int d_model,
+                               const int32_t* token, const void* w_emb, int vocab, int d_draft,
+                               uint16_t* u, unsigned* status, const int32_t* seq_lens, int pos_off,
+                               const double* inv_freq, int half, float2* rope_tab, int B,
+                               cudaStream_t st);
+cudaError_t launch_draft_collect(const int32_t* ids, const float* maxv, int B, int k, int s,
+                                 int32_t* drafts, float* draft_max, cudaStream_t st);
+cudaError_t launch_to_bf16(const float* x, size_t n, uint16_t* out, cudaStream_t st);
 cudaError_t launch_rmsnorm(const float* x, int M, int d, double eps, uint16_t* out,
                            cudaStream_t st);
 // embedding gather of [last_token, drafts] into x and its RMSNorm into out;
@@ -145,6 +153,8 @@ struct AttnGeom {
   int window, kv_equal, sb_width, split_tokens;
   int n_splits_grid;   // CTAs per (sequence, kv head, row block)
   int rows;            // G * q
+  int qpos_off;        // row i at position L + qpos_off + i (verify: 0)
+  int kend_off;        // last visible cached key at L + kend_off (verify: q - 1)
   int row_blocks;      // ceil(rows / 64)
 };
 AttnGeom plan_attn(int B, int q, int Hq, int Hkv, int D, int page, int num_pages, int max_pages,

@@ -1,5 +1,6 @@
 // Small verify-step kernels: token embedding gather, RMSNorm, and the
 // acceptance / bonus-token / commit kernel.
+#include <algorithm>
 #include <cmath>
 #include <cstdlib>
 
@@ -112,6 +113,59 @@ __global__ void accept_kernel(const int32_t* __restrict__ drafts, const int32_t*
   }
 }
 
+// Drafter step input: row b = [target activation (bf16) || drafter embedding
+// of the token] (the GEMM input of the down-projection).  Step 0 reads the
+// caller's activation (bf16) and token; later steps the previous step's
+// up-projection output (binary32, rounded here) and its argmax token.
+// Blocks past the B rows fill the (cos, sin) table of position
+// seq_lens[b] + pos_off for every rotary pair, as embed_norm_kernel does.
+__global__ void __launch_bounds__(kNormThreads) draft_input_kernel(
+    const uint16_t* __restrict__ prev_bf16, const float* __restrict__ prev_f32, int d_model,
+    const int32_t* __restrict__ token, const uint16_t* __restrict__ w_emb, int vocab, int d_draft,
+    uint16_t* __restrict__ u, unsigned* status, const int32_t* __restrict__ seq_lens, int pos_off,
+    InvFreq inv_freq, int half, float2* __restrict__ rope_tab, int B) {
+  pdl_trigger();
+  pdl_wait();
+  if ((int)blockIdx.x >= B) {
+    const size_t idx = (size_t)(blockIdx.x - B) * kNormThreads + threadIdx.x;
+    if (idx < (size_t)B * half) {
+      const int b = (int)(idx / half), j = (int)(idx % half);
+      rope_tab[idx] = rope_cs(seq_lens[b] + pos_off, inv_freq.v[j]);
+    }
+    return;
+  }
+  const int b = blockIdx.x;
+  const int width = d_model + d_draft;
+  uint16_t* row = u + (size_t)b * width;
+  for (int e = threadIdx.x; e < d_model; e += kNormThreads)
+    row[e] = prev_bf16 ? prev_bf16[(size_t)b * d_model + e] : f32_to_bf16(prev_f32[(size_t)b * d_model + e]);
+  const int tok = token[b];
+  const bool ok = tok >= 0 && tok < vocab;
+  if (!ok && threadIdx.x == 0) flag_status(status, SPEC_DEV_BAD_TOKEN);
+  const uint16_t* src = w_emb + (size_t)(ok ? tok : 0) * d_draft;
+  for (int e = threadIdx.x; e < d_draft; e += kNormThreads) row[d_model + e] = ok ? src[e] : 0;
+}
+
+// drafts[b][s] = argmax of step s, draft_max[b][s] its logit
+__global__ void draft_collect_kernel(const int32_t* __restrict__ ids, const float* __restrict__ maxv,
+                                     int B, int k, int s, int32_t* __restrict__ drafts,
+                                     float* __restrict__ draft_max) {
+  pdl_trigger();
+  pdl_wait();
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= B) return;
+  drafts[(size_t)b * k + s] = ids[b];
+  if (draft_max) draft_max[(size_t)b * k + s] = maxv[b];
+}
+
+// out[i] = bf16(x[i]): a binary32 activation entering a projection
+__global__ void to_bf16_kernel(const float* __restrict__ x, size_t n, uint16_t* __restrict__ out) {
+  pdl_trigger();
+  pdl_wait();
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+    out[i] = f32_to_bf16(x[i]);
+}
+
 }  // namespace
 
 cudaError_t launch_embed_norm(const void* w_emb, int vocab, int d, const int32_t* last_token,
@@ -173,6 +227,30 @@ cudaError_t launch_accept(const int32_t* drafts, const int32_t* target, int B, i
   const int warps = 4;
   return launch_k(accept_kernel, dim3((B + warps - 1) / warps), dim3(warps * 32), 0, st, drafts,
                   target, B, k, seq_lens, accept_len, emitted, last_token, copy_ids, copy_max, maxv);
+}
+
+cudaError_t launch_draft_input(const uint16_t* prev_bf16, const float* prev_f32, int d_model,
+                               const int32_t* token, const void* w_emb, int vocab, int d_draft,
+                               uint16_t* u, unsigned* status, const int32_t* seq_lens, int pos_off,
+                               const double* inv_freq, int half, float2* rope_tab, int B,
+                               cudaStream_t st) {
+  InvFreq f{};
+  for (int j = 0; j < half && j < 128; ++j) f.v[j] = inv_freq[j];
+  const int tab_blocks = (B * half + kNormThreads - 1) / kNormThreads;
+  return launch_k(draft_input_kernel, dim3(B + tab_blocks), dim3(kNormThreads), 0, st, prev_bf16,
+                  prev_f32, d_model, token, static_cast<const uint16_t*>(w_emb), vocab, d_draft, u,
+                  status, seq_lens, pos_off, f, half, rope_tab, B);
+}
+
+cudaError_t launch_draft_collect(const int32_t* ids, const float* maxv, int B, int k, int s,
+                                 int32_t* drafts, float* draft_max, cudaStream_t st) {
+  return launch_k(draft_collect_kernel, dim3((B + 127) / 128), dim3(128), 0, st, ids, maxv, B, k, s,
+                  drafts, draft_max);
+}
+
+cudaError_t launch_to_bf16(const float* x, size_t n, uint16_t* out, cudaStream_t st) {
+  const int blocks = (int)std::min<size_t>((n + 255) / 256, 1024);
+  return launch_k(to_bf16_kernel, dim3(blocks), dim3(256), 0, st, x, n, out);
 }
 
 }  // namespace sv

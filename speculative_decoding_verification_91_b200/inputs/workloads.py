@@ -158,6 +158,44 @@ def embedding_weight(wl: Workload):
     return _w(wl, "w_emb", wl.vocab, wl.d_model)
 
 
+DRAFT_WIDTH = 256       # drafter block width of the small models' drafters
+DRAFT_BLOCKS = 4        # three sliding-window blocks, then one global block
+
+
+def drafter_spec(wl: Workload):
+    """(d_draft, n_q_heads, target layer of each block): the sliding-window
+    blocks read the target's last sliding-window layer, the global block its
+    last global layer (either kind stands in when the target lacks the
+    other)."""
+    local = [l for l, s in enumerate(wl.layers) if s.window > 0]
+    glob = [l for l, s in enumerate(wl.layers) if s.window == 0]
+    last_local = local[-1] if local else glob[-1]
+    last_global = glob[-1] if glob else local[-1]
+    targets = [last_local] * (DRAFT_BLOCKS - 1) + [last_global]
+    return min(DRAFT_WIDTH, wl.d_model), wl.n_q_heads, targets
+
+
+def drafter_weights(wl: Workload):
+    """Drafter weights, bf16 bits: (embedding [vocab][d_draft], W_down
+    [d_draft][d_model + d_draft], W_up [d_model][d_draft], blocks [(W_q
+    [Hq*D][d_draft], W_o [d_draft][Hq*D], target layer)])."""
+    dd, hq, targets = drafter_spec(wl)
+    nq = hq * wl.head_dim
+    emb = _w(wl, "draft/w_emb", wl.vocab, dd)
+    down = _w(wl, "draft/w_down", dd, wl.d_model + dd)
+    upw = _w(wl, "draft/w_up", wl.d_model, dd)
+    blocks = [(_w(wl, f"draft/b{i}/w_q", nq, dd), _w(wl, f"draft/b{i}/w_o", dd, nq), t)
+              for i, t in enumerate(targets)]
+    return emb, down, upw, blocks
+
+
+def drafter_inputs(wl: Workload, b: int, attempt: int):
+    """(target activation bf16 bits [d_model], previous token) of sequence b."""
+    key = f"{wl.name}/draft_in/b{b}/a{attempt}"
+    return (gen.normal_bf16(wl.seed, key + "/h", 0, wl.d_model, 1.0),
+            int(gen.randint(wl.seed, key + "/tok", 0, 1, 0, wl.vocab)[0]))
+
+
 def layer_weights(wl: Workload, l: int):
     """(W_qkv [Nqkv][d], W_o [d][Hq*D]) bf16 bits, rows = output features.
 

@@ -101,3 +101,26 @@ class Workspace:
 
     def device_status(self, stream=None) -> int:
         return B.spec_read_device_status(self.buf, self.nbytes, stream)
+
+
+class DeviceDrafter:
+    """Weights of one synthetic MTP drafter on one GPU and its spec_drafter
+    descriptor.  blocks: (w_q bits, w_o bits, target layer) per block."""
+
+    def __init__(self, *, d_draft, n_q_heads, w_emb_bits, w_down_bits, w_up_bits, blocks,
+                 device="cuda"):
+        self.device = torch.device(device)
+        self.d_draft, self.n_q_heads = d_draft, n_q_heads
+        self.w_emb = to_device_bf16(w_emb_bits, self.device)
+        self.w_down = to_device_bf16(w_down_bits, self.device)
+        self.w_up = to_device_bf16(w_up_bits, self.device)
+        self.w_q = [to_device_bf16(b[0], self.device) for b in blocks]
+        self.w_o = [to_device_bf16(b[1], self.device) for b in blocks]
+        self.target_layers = [int(b[2]) for b in blocks]
+        self._blocks_c = (B.SpecDraftBlock * len(blocks))()
+        for i in range(len(blocks)):
+            self._blocks_c[i] = B.SpecDraftBlock(self.w_q[i].data_ptr(), self.w_o[i].data_ptr(),
+                                                 self.target_layers[i])
+        self.desc = B.SpecDrafter(d_draft, n_q_heads, len(blocks), self.w_emb.data_ptr(),
+                                  self.w_down.data_ptr(), self.w_up.data_ptr(),
+                                  ctypes.cast(self._blocks_c, ctypes.POINTER(B.SpecDraftBlock)))

@@ -92,3 +92,26 @@ def guarded_sequence(wl, model, b, L, max_attempts=40, start=0) -> SeqCase:
         if case.guarded:
             return case
     raise RuntimeError(f"no margin-safe draw for sequence {b} in {max_attempts} attempts")
+
+
+def oracle_drafter(wl: W.Workload):
+    """The drafter of a workload as the oracle sees it (weights as values)."""
+    from oracle import draft as OD
+    dd, hq, _ = W.drafter_spec(wl)
+    emb, down, upw, blocks = W.drafter_weights(wl)
+    return OD.Drafter(dd, hq, emb, oracle.bf16_from_bits(down), oracle.bf16_from_bits(upw),
+                      [OD.DraftBlockDef(t, oracle.bf16_from_bits(q), oracle.bf16_from_bits(o))
+                       for q, o, t in blocks])
+
+
+def guarded_draft_inputs(wl, model, drafter, caches, b, L, k, max_attempts=40):
+    """Redraw sequence b's drafter inputs (target activation, token) until every
+    one of the k oracle draft steps has a safe top-2 margin.  Returns
+    (attempt, activation bits, token, oracle steps)."""
+    from oracle import draft as OD
+    for t in range(max_attempts):
+        h_bits, tok = W.drafter_inputs(wl, b, t)
+        steps = OD.draft(model, drafter, caches, L, oracle.bf16_from_bits(h_bits), tok, k)
+        if all(margin_ok(st.top1, st.top2) for st in steps):
+            return t, h_bits, tok, steps
+    raise RuntimeError(f"no margin-safe drafter inputs for sequence {b}")

@@ -109,3 +109,32 @@ def test_unsupported_shapes_are_reported(lib):
     m3.page_size = 32
     assert lib.spec_verify_step(ctypes.byref(m3), FAKE, 10, FAKE, FAKE, 1, 4, FAKE, FAKE, FAKE, FAKE,
                                 None, None, FAKE, 1 << 30, None) == B.SPEC_EUNSUPPORTED
+
+
+def _drafter(n_q_heads=16, target=0, d_draft=256):
+    blocks = (B.SpecDraftBlock * 4)(*[B.SpecDraftBlock(FAKE, FAKE, target) for _ in range(4)])
+    d = B.SpecDrafter(d_draft, n_q_heads, 4, FAKE, FAKE, FAKE,
+                      ctypes.cast(blocks, ctypes.POINTER(B.SpecDraftBlock)))
+    d._keep = blocks
+    return d
+
+
+def test_drafter_workspace_and_validation(lib):
+    m = _model()
+    d = _drafter()
+    ws = B.spec_draft_workspace_bytes(m, d, 4, 520)
+    assert ws > 4096
+    assert B.spec_draft_workspace_bytes(m, d, 8, 520) > ws
+    assert B.spec_draft_workspace_bytes(m, _drafter(n_q_heads=12), 4, 520) == 0   # not a multiple of Hkv
+    assert B.spec_draft_workspace_bytes(m, _drafter(target=5), 4, 520) == 0       # no such target layer
+    assert B.spec_draft_workspace_bytes(m, _drafter(d_draft=250), 4, 520) == 0
+    pm, pd = ctypes.byref(m), ctypes.byref(d)
+    # missing pointers, negative k, workspace too small: rejected before any launch
+    assert lib.spec_draft(pm, pd, None, 10, FAKE, FAKE, FAKE, 1, 4, FAKE, None, FAKE, 1 << 30,
+                          None) == B.SPEC_EINVAL
+    assert lib.spec_draft(pm, pd, FAKE, 10, FAKE, FAKE, FAKE, 1, -1, FAKE, None, FAKE, 1 << 30,
+                          None) == B.SPEC_EINVAL
+    assert lib.spec_draft(pm, pd, FAKE, 10, FAKE, FAKE, FAKE, 1, 4, FAKE, None, FAKE, 100,
+                          None) == B.SPEC_EINVAL
+    assert lib.spec_draft(pm, ctypes.byref(_drafter(n_q_heads=12)), FAKE, 10, FAKE, FAKE, FAKE, 1, 4,
+                          FAKE, None, FAKE, 1 << 30, None) == B.SPEC_EINVAL
