@@ -17,6 +17,10 @@ Pages this follows (title and section):
      picks the next draft token; k tokens are drafted autoregressively.
      §4.2 (figure): the blocks attend to the target's last prefilled local
      and global layers.
+     §4.3: for small drafters the projection onto the whole vocabulary is
+     replaced by a top-k over token clusters: the clusters' centroids are
+     scored first and only the tokens of the best clusters (~4096) get real
+     logits.
 [P5] "Gemma 4 与 Gemini Nano：端侧智能的架构拆解" §草稿模型: the drafter reuses
      the base model's KV cache.
 
@@ -42,7 +46,12 @@ the block internals from their sketch):
     inputs are); the up-projection's output (binary32) is both the next
     step's activation and, after the target's final RMSNorm (rounded to
     bf16), the input of the target's LM head; argmax ties go to the lowest
-    token id.
+    token id;
+  * cheap unembedding: every token belongs to exactly one cluster; a
+    cluster's logit is h . centroid with the centroid a bf16 row of the
+    tables; the n_select best clusters are kept (ties: lower cluster id);
+    their tokens are scored with the target's LM-head rows and the argmax
+    over those candidates is the draft token (ties: lowest token id).
 """
 from __future__ import annotations
 
@@ -53,7 +62,8 @@ import numpy as np
 from .verify import (LayerCache, Model, attend, bf16, bf16_from_bits, f32, lm_head_top2, rmsnorm,
                      rope)
 
-__all__ = ["DraftBlockDef", "Drafter", "cross_attention", "draft_step", "draft"]
+__all__ = ["DraftBlockDef", "Drafter", "ClusterTables", "cheap_unembed", "cross_attention",
+           "draft_step", "draft"]
 
 
 @dataclass
@@ -104,6 +114,48 @@ def cross_attention(model: Model, drafter: Drafter, blk: DraftBlockDef, cache: L
 
 
 @dataclass
+class ClusterTables:
+    """Token clusters for the cheap unembedding ([P1] §4.3).
+
+    cluster_tokens [C][S]: token ids of each cluster (-1 pads a short last
+    cluster; every token sits in exactly one cluster); centroids_bits
+    [C][d_model] bf16 bits; n_select: clusters whose tokens are scored."""
+    cluster_tokens: np.ndarray
+    centroids_bits: np.ndarray
+    n_select: int
+
+
+def cheap_unembed(h, w_lm_bits, tables: ClusterTables):
+    """Argmax over the tokens of the best-scoring clusters instead of the
+    whole vocabulary ([P1] §4.3 `cheap_unembed`).
+
+    h [M][d] (bf16 values).  Each cluster logit is h . centroid (float64,
+    rounded to binary32); the n_select clusters with the largest logits are
+    kept (equal logits: lower cluster id first); every token of those
+    clusters gets its logit h . W_v (float64, rounded to binary32) and the
+    largest wins (equal logits: lowest token id).  Returns (ids [M], top1
+    [M], top2 [M]) over the candidates."""
+    h = np.asarray(h, dtype=np.float64)
+    cent = bf16_from_bits(tables.centroids_bits).astype(np.float64)
+    C = cent.shape[0]
+    M = h.shape[0]
+    ids = np.zeros(M, dtype=np.int64)
+    top1, top2 = np.zeros(M), np.zeros(M)
+    for m in range(M):
+        cl = f32(h[m] @ cent.T).astype(np.float64)
+        order = sorted(range(C), key=lambda c: (-cl[c], c))
+        sel = order[:tables.n_select]
+        cand = np.sort(np.concatenate([tables.cluster_tokens[c] for c in sel]))
+        cand = cand[cand >= 0]
+        lg = f32(h[m] @ bf16_from_bits(w_lm_bits[cand]).astype(np.float64).T).astype(np.float64)
+        j = int(np.argmax(lg))                 # first maximum: candidates are in id order
+        ids[m], top1[m] = cand[j], lg[j]
+        rest = np.delete(lg, j)
+        top2[m] = rest.max() if rest.size else -np.inf
+    return ids, top1, top2
+
+
+@dataclass
 class DraftStep:
     h: np.ndarray                # up-projection output (binary32) [d_model]
     token: int                   # argmax of the target's LM head on RMSNorm(h)
@@ -112,8 +164,10 @@ class DraftStep:
 
 
 def draft_step(model: Model, drafter: Drafter, caches: list, L: int, s: int, prev_hidden,
-               prev_token: int) -> DraftStep:
-    """One drafter forward ([P1] §4.2 `draft_one_step`) at position L + s."""
+               prev_token: int, tables: ClusterTables | None = None) -> DraftStep:
+    """One drafter forward ([P1] §4.2 `draft_one_step`) at position L + s; the
+    draft token comes from the full LM head, or from the cheap clustered
+    unembedding ([P1] §4.3) when cluster tables are given."""
     D = model.head_dim
     tok = bf16_from_bits(drafter.w_emb_bits[int(prev_token)]).astype(np.float64)
     u = np.concatenate([bf16(prev_hidden).astype(np.float64), tok])
@@ -126,19 +180,22 @@ def draft_step(model: Model, drafter: Drafter, caches: list, L: int, s: int, pre
         x = f32(x.astype(np.float64) + y.astype(np.float64))
     h = f32(bf16(x).astype(np.float64) @ drafter.w_up.astype(np.float64).T)
     hn = bf16(rmsnorm(h, model.rms_eps))
-    g, t1, t2 = lm_head_top2(hn[None], model.w_lm_bits)
+    if tables is None:
+        g, t1, t2 = lm_head_top2(hn[None], model.w_lm_bits)
+    else:
+        g, t1, t2 = cheap_unembed(hn[None], model.w_lm_bits, tables)
     return DraftStep(h, int(g[0]), float(t1[0]), float(t2[0]))
 
 
 def draft(model: Model, drafter: Drafter, caches: list, L: int, prev_hidden, prev_token: int,
-          k: int) -> list:
+          k: int, tables: ClusterTables | None = None) -> list:
     """k autoregressive drafter steps ([P1] §4.2 `draft`): step s reads the
     previous step's up-projection output and draft token.  Returns the list
     of DraftStep."""
     out = []
     hidden, tok = np.asarray(prev_hidden, dtype=np.float32), int(prev_token)
     for s in range(k):
-        st = draft_step(model, drafter, caches, L, s, hidden, tok)
+        st = draft_step(model, drafter, caches, L, s, hidden, tok, tables)
         out.append(st)
         hidden, tok = st.h, st.token
     return out

@@ -156,3 +156,60 @@ def test_draft_step_queries_sit_at_L_plus_s():
     a0 = OD.draft_step(model, dr, [cache], L, 0, prev, 5)
     b0 = OD.draft_step(model, dr0, [cache], L, 0, prev, 5)
     assert not np.array_equal(a0.h, b0.h)
+
+
+# ---------------------------------------------------------------- cheap unembedding
+
+def _tables(V, S, d, n_select, seed=3):
+    r = _rng(seed)
+    perm = r.permutation(V)
+    C = -(-V // S)
+    toks = np.full((C, S), -1, np.int64)
+    toks.reshape(-1)[:V] = perm
+    cent = _bits(r.standard_normal((C, d)))
+    return OD.ClusterTables(toks, cent, n_select)
+
+
+def test_cheap_unembed_over_every_cluster_is_the_full_argmax():
+    r = _rng(11)
+    V, d = 1000, 24
+    w = _bits(r.standard_normal((V, d)))
+    h = OV.bf16(r.standard_normal((5, d)))
+    t = _tables(V, 16, d, n_select=-(-V // 16))
+    ids, t1, _ = OD.cheap_unembed(h, w, t)
+    fids, ft1, _ = OV.lm_head_top2(h, w)
+    assert np.array_equal(ids, fids) and np.array_equal(t1, ft1)
+
+
+@pytest.mark.parametrize("n_select", [1, 3, 7])
+def test_cheap_unembed_keeps_the_best_clusters(n_select):
+    # reference: cluster logits by torch matmul, kept set by a stable
+    # lexicographic sort (logit descending, id ascending), argmax over the
+    # kept tokens by torch (first maximum in token-id order)
+    r = _rng(12 + n_select)
+    V, S, d = 203, 8, 12          # 26 clusters, the last one 3 tokens short
+    w = _bits(r.standard_normal((V, d)))
+    t = _tables(V, S, d, n_select)
+    t.centroids_bits[5] = t.centroids_bits[9]          # a tie between two clusters
+    h = OV.bf16(r.standard_normal((6, d)))
+    ids, t1, _ = OD.cheap_unembed(h, w, t)
+    tt = lambda a: torch.from_numpy(np.asarray(a, np.float64))
+    cl = torch.nn.functional.linear(tt(h), tt(OV.bf16_from_bits(t.centroids_bits))).float().numpy()
+    for m in range(h.shape[0]):
+        order = np.lexsort((np.arange(cl.shape[1]), -cl[m].astype(np.float64)))
+        cand = np.sort(t.cluster_tokens[order[:n_select]].reshape(-1))
+        cand = cand[cand >= 0]
+        lg = torch.nn.functional.linear(tt(h[m]), tt(OV.bf16_from_bits(w[cand]))).float()
+        j = int(torch.argmax(lg))
+        assert ids[m] == cand[j] and t1[m] == float(lg[j])
+
+
+def test_draft_step_with_clusters_uses_them():
+    model, L = _model(0, False, 1.0), 9
+    cache, dr = _cache(model, L), _drafter()
+    prev = OV.f32(_rng(13).standard_normal(DM))
+    full = OD.draft_step(model, dr, [cache], L, 0, prev, 4)
+    every = OD.draft_step(model, dr, [cache], L, 0, prev, 4, _tables(V, 5, DM, n_select=V // 5))
+    assert (every.token, every.top1) == (full.token, full.top1)
+    one = OD.draft_step(model, dr, [cache], L, 0, prev, 4, _tables(V, 5, DM, n_select=1))
+    assert np.array_equal(one.h, full.h)
