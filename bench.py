@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--draft", action="store_true",
                     help="time the MTP drafter (spec_draft, k steps) on the workload; one JSON line")
+    ap.add_argument("--clusters", action="store_true",
+                    help="with --draft: the cheap clustered unembedding picks each draft token")
     ap.add_argument("--sweep", action="store_true",
                     help="verify-step time over batch x k on the b1_ctx8k model; one JSON line")
     ap.add_argument("--profile-case", action="store_true",
@@ -531,7 +533,8 @@ def run_draft_bench(args):
     import torch
     from speculative_decoding_verification_91_b200 import binding as B
     from speculative_decoding_verification_91_b200.inputs import workloads as W
-    from speculative_decoding_verification_91_b200.runtime import DeviceDrafter, Workspace, to_device_bf16
+    from speculative_decoding_verification_91_b200.runtime import (DeviceClusters, DeviceDrafter,
+                                                                    Workspace, to_device_bf16)
     from speculative_decoding_verification_91_b200.session import WorkloadSession
     torch.cuda.set_device(0)
     dev = torch.device("cuda", 0)
@@ -539,8 +542,13 @@ def run_draft_bench(args):
     sess = WorkloadSession(wl, device=dev, poison=False)
     dd, hq, targets = W.drafter_spec(wl)
     emb, down, upw, blocks = W.drafter_weights(wl)
+    cl = None
+    if args.clusters:
+        cl_tokens, cent, wc, n_sel = W.cluster_tables(wl)
+        cl = DeviceClusters(cluster_tokens=cl_tokens, centroid_bits=cent, clustered_bits=wc,
+                            n_select=n_sel, device=dev)
     dr = DeviceDrafter(d_draft=dd, n_q_heads=hq, w_emb_bits=emb, w_down_bits=down, w_up_bits=upw,
-                       blocks=blocks, device=dev)
+                       blocks=blocks, device=dev, clusters=cl)
     Bn, k = wl.batch, max(1, wl.k)
     hidden = to_device_bf16(np.stack([W.drafter_inputs(wl, b, 0)[0] for b in range(Bn)]), dev)
     toks = torch.tensor([W.drafter_inputs(wl, b, 0)[1] for b in range(Bn)], dtype=torch.int32, device=dev)
@@ -572,7 +580,37 @@ def run_draft_bench(args):
         raise RuntimeError("device status flagged during the drafter calls")
     us = float(np.mean([a.elapsed_time(b) for a, b in zip(e0, e1)])) * 1e3
     lm_bytes = wl.vocab * wl.d_model * 2
+    unembed = None
+    if cl is not None:
+        # the unembedding alone: clusters vs the full LM head, same rows
+        hrows = torch.randn(Bn, wl.d_model, device=dev).to(torch.bfloat16)
+        ids = torch.zeros(Bn, dtype=torch.int32, device=dev)
+        wsc = Workspace(B.spec_cluster_unembed_workspace_bytes(Bn, wl.d_model, cl.desc), dev)
+        wsl = Workspace(B.spec_lmhead_workspace_bytes(Bn, wl.vocab), dev)
+        def t_of(fn, n=50):
+            for _ in range(3):
+                fn()
+            a = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+            z = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+            for i in range(n):
+                flush.zero_()
+                a[i].record(stream)
+                fn()
+                z[i].record(stream)
+            torch.cuda.synchronize(dev)
+            return float(np.mean([x.elapsed_time(y) for x, y in zip(a, z)])) * 1e3
+        t_cl = t_of(lambda: B.spec_cluster_unembed(hrows, Bn, wl.d_model, cl.desc, ids, None, wsc.buf,
+                                                    wsc.nbytes, stream))
+        t_lm = t_of(lambda: B.spec_lmhead_argmax(hrows, sess.dm.w_lm, Bn, wl.d_model, wl.vocab, ids,
+                                                  None, wsl.buf, wsl.nbytes, stream))
+        C, S = cl_tokens.shape
+        cand_bytes = Bn * n_sel * S * wl.d_model * 2 + C * wl.d_model * 2
+        unembed = {"clusters": C, "cluster_size": S, "n_select": n_sel,
+                   "us_cluster_unembed": t_cl, "us_full_lm_head": t_lm,
+                   "bytes_cluster_unembed": cand_bytes, "bytes_full_lm_head": lm_bytes}
     print(json.dumps({"kernel": "spec_draft", "workload": wl.name, "batch": Bn, "k": k,
+                      "unembed": "clusters" if cl is not None else "full LM head",
+                      "unembed_alone": unembed,
                       "d_draft": dd, "blocks_target_layers": targets,
                       "us_per_call": us, "us_per_draft_step": us / k,
                       "drafted_tokens_per_s": Bn * k / (us / 1e6),

@@ -258,6 +258,32 @@ typedef struct {
   int target_layer;    /* target layer whose cache this block reads */
 } spec_draft_block;
 
+/* Token clusters for the cheap unembedding ("Gemma 4 拆解 ..." §4.3: score the
+ * clusters' centroids, keep the best few, and take the argmax over their
+ * tokens only, ~4096 candidates instead of the whole vocabulary).  A
+ * cluster's logit is h . centroid; the n_select largest are kept (equal
+ * logits: lower cluster id); every token of those clusters is scored with
+ * its LM-head row and the largest logit wins (equal logits: lowest token
+ * id).  All pointers are device memory owned by the caller. */
+typedef struct {
+  int n_clusters;                 /* C, 1..8192 */
+  int cluster_size;               /* S, tokens per cluster, 1..4096 */
+  int n_select;                   /* clusters kept per row, 1..C */
+  const void* centroids;          /* bf16 [C][d_model] */
+  const int32_t* cluster_tokens;  /* [C][S] token ids; -1 pads a short cluster */
+  const void* w_clustered;        /* bf16 [C*S][d_model]: row c*S+i = LM-head row of
+                                     cluster_tokens[c][i] (rows of pads are never read) */
+} spec_clusters;
+
+/* Workspace bytes of spec_cluster_unembed for M rows of width d (0 if unsupported). */
+size_t spec_cluster_unembed_workspace_bytes(int M, int d, const spec_clusters* t);
+
+/* ids[M] (and maxlogit[M], or NULL) = the cheap clustered argmax of h
+ * (bf16 [M][d], device).  ws: spec_cluster_unembed_workspace_bytes, set up
+ * once with spec_workspace_init. */
+int spec_cluster_unembed(const void* h, int M, int d, const spec_clusters* t, int32_t* ids,
+                         float* maxlogit, void* ws, size_t ws_bytes, void* stream);
+
 typedef struct {
   int d_draft;         /* drafter width, multiple of 8 */
   int n_q_heads;       /* query heads per block, multiple of the target's n_kv_heads */
@@ -266,6 +292,8 @@ typedef struct {
   const void* w_down;  /* bf16 [d_draft][d_model + d_draft]: input [activation || embedding] */
   const void* w_up;    /* bf16 [d_model][d_draft] */
   const spec_draft_block* blocks;
+  const spec_clusters* clusters; /* NULL: the target's full LM head picks each draft token;
+                                    else the cheap clustered unembedding does */
 } spec_drafter;
 
 /* Workspace bytes of spec_draft for up to B sequences (0 if unsupported). */

@@ -35,6 +35,7 @@ EXPORTED = [
     "spec_lmhead_argmax_noalloc", "spec_prefill_workspace_bytes", "spec_prefill",
     "spec_profile_launches", "spec_profile_launches_collect", "spec_launch_count",
     "spec_draft_workspace_bytes", "spec_draft",
+    "spec_cluster_unembed_workspace_bytes", "spec_cluster_unembed",
 ]
 SPEC_MAX_PREFILL = 256
 SPEC_NOALLOC_MAX_ROWS = 64
@@ -69,11 +70,18 @@ class SpecDraftBlock(ctypes.Structure):
     _fields_ = [("w_q", c_void_p), ("w_o", c_void_p), ("target_layer", c_int)]
 
 
+class SpecClusters(ctypes.Structure):
+    _fields_ = [
+        ("n_clusters", c_int), ("cluster_size", c_int), ("n_select", c_int),
+        ("centroids", c_void_p), ("cluster_tokens", c_void_p), ("w_clustered", c_void_p),
+    ]
+
+
 class SpecDrafter(ctypes.Structure):
     _fields_ = [
         ("d_draft", c_int), ("n_q_heads", c_int), ("n_blocks", c_int),
         ("w_embed", c_void_p), ("w_down", c_void_p), ("w_up", c_void_p),
-        ("blocks", POINTER(SpecDraftBlock)),
+        ("blocks", POINTER(SpecDraftBlock)), ("clusters", POINTER(SpecClusters)),
     ]
 
 
@@ -130,10 +138,17 @@ def lib():
         L.spec_draft_workspace_bytes.argtypes = [pm, pd, c_int, c_int]
         L.spec_draft.argtypes = [pm, pd, c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_int, c_int,
                                  c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]
+        pc = POINTER(SpecClusters)
+        L.spec_cluster_unembed_workspace_bytes.argtypes = [c_int, c_int, pc]
+        L.spec_cluster_unembed.argtypes = [c_void_p, c_int, c_int, pc, c_void_p, c_void_p, c_void_p,
+                                           c_size_t, c_void_p]
+        sizes = ("spec_prefill_workspace_bytes", "spec_draft_workspace_bytes",
+                 "spec_cluster_unembed_workspace_bytes")
         for name in EXPORTED[4:]:
-            if name not in ("spec_prefill_workspace_bytes", "spec_draft_workspace_bytes"):
+            if name not in sizes:
                 getattr(L, name).restype = c_int
-        L.spec_draft_workspace_bytes.restype = c_size_t
+        for name in sizes:
+            getattr(L, name).restype = c_size_t
         L.spec_launch_count.argtypes = []
         L.spec_launch_count.restype = ctypes.c_ulonglong
         _lib = L
@@ -291,3 +306,13 @@ def spec_draft(model, drafter, block_table, max_pages, seq_lens, prev_hidden, pr
                                    max_pages, _p(seq_lens), _p(prev_hidden), _p(prev_token), B, k,
                                    _p(drafts), _p(draft_maxlogit), _p(ws), ws_bytes, _s(stream)),
                   "spec_draft")
+
+
+def spec_cluster_unembed_workspace_bytes(M: int, d: int, clusters) -> int:
+    return int(lib().spec_cluster_unembed_workspace_bytes(M, d, ctypes.byref(clusters)))
+
+
+def spec_cluster_unembed(h, M, d, clusters, ids, maxlogit, ws, ws_bytes, stream=None) -> int:
+    return _check(lib().spec_cluster_unembed(_p(h), M, d, ctypes.byref(clusters), _p(ids),
+                                             _p(maxlogit), _p(ws), ws_bytes, _s(stream)),
+                  "spec_cluster_unembed")

@@ -327,6 +327,62 @@ int run_forward(const spec_model* m, const int32_t* block_table, int max_pages, 
   return rc;
 }
 
+// ---------------------------------------------------------------- clusters
+
+constexpr int kMaxClusterCount = 8192;   // keys of one row sorted in shared memory
+
+int check_clusters(const spec_clusters* t, int d) {
+  if (!t || !t->centroids || !t->cluster_tokens || !t->w_clustered) return SPEC_EINVAL;
+  if (t->n_clusters < 1 || t->cluster_size < 1 || t->n_select < 1 || t->n_select > t->n_clusters)
+    return SPEC_EINVAL;
+  if (t->n_clusters > kMaxClusterCount || t->cluster_size > 4096) return SPEC_EUNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(t->centroids) & 15) || (reinterpret_cast<uintptr_t>(t->w_clustered) & 15))
+    return SPEC_EINVAL;
+  if (d < 8 || d % 8) return SPEC_EINVAL;
+  return SPEC_OK;
+}
+
+ClusterArgs cluster_args(const spec_clusters* t) {
+  ClusterArgs c{};
+  c.n_clusters = t->n_clusters;
+  c.cluster_size = t->cluster_size;
+  c.n_select = t->n_select;
+  c.centroids = t->centroids;
+  c.cluster_tokens = t->cluster_tokens;
+  c.w_clustered = t->w_clustered;
+  return c;
+}
+
+// Scratch of one cheap unembedding of M rows: cluster logits, the centroid
+// GEMM's split-K partials, the selected clusters, the per-row argmax keys.
+struct ClusterLayout {
+  size_t logits, part, sel, keys, bytes;
+  int tickets;
+};
+ClusterLayout cluster_layout(int M, int d, const spec_clusters* t, size_t base) {
+  ClusterLayout c{};
+  GemmPlan p = plan_gemm(M, t->n_clusters, d, kGemmStore);
+  size_t off = base;
+  c.logits = off; off = up(off + cluster_logit_floats(M, t->n_clusters) * 4);
+  c.part = off;   off = up(off + gemm_partial_floats(p) * 4);
+  c.sel = off;    off = up(off + (size_t)M * t->n_select * 4);
+  c.keys = off;   off = up(off + (size_t)M * 8);
+  c.bytes = off - base;
+  c.tickets = gemm_tickets(p);
+  return c;
+}
+
+cudaError_t run_clusters(const spec_clusters* t, const uint16_t* h, int M, int d, int32_t* ids,
+                         float* maxv, void* ws, const ClusterLayout& c, cudaStream_t st) {
+  WsHeader hdr = ws_header(ws);
+  GemmBuffers b{};
+  b.partial = at<float>(ws, c.part);
+  b.tickets = hdr.tickets;
+  b.status = hdr.status;
+  return launch_cluster_unembed(cluster_args(t), h, M, d, ids, maxv, at<float>(ws, c.logits),
+                                at<int32_t>(ws, c.sel), at<unsigned long long>(ws, c.keys), b, st);
+}
+
 // ---------------------------------------------------------------- drafter
 
 int check_drafter(const spec_model* m, const spec_drafter* d) {
@@ -337,6 +393,10 @@ int check_drafter(const spec_model* m, const spec_drafter* d) {
   const void* ptrs[3] = {d->w_embed, d->w_down, d->w_up};
   for (const void* p : ptrs)
     if (reinterpret_cast<uintptr_t>(p) & 15) return SPEC_EINVAL;
+  if (d->clusters) {
+    const int rc = check_clusters(d->clusters, m->d_model);
+    if (rc) return rc;
+  }
   for (int i = 0; i < d->n_blocks; ++i) {
     const spec_draft_block& b = d->blocks[i];
     if (!b.w_q || !b.w_o || b.target_layer < 0 || b.target_layer >= m->n_layers) return SPEC_EINVAL;
@@ -349,6 +409,7 @@ int check_drafter(const spec_model* m, const spec_drafter* d) {
 // Workspace of one drafter call for B sequences (q = 1 row each).
 struct DraftLayout {
   size_t u, x, hn, qrot, attn_out, attn_part, gemm_part, h, arg_keys, ids, maxv, rope_tab, total;
+  ClusterLayout cl;
   int tickets;
   bool splits_ok;
 };
@@ -386,6 +447,11 @@ DraftLayout draft_layout(const spec_model* m, const spec_drafter* d, int B, int 
   s.ids = off;       off = up(off + (size_t)B * 4);
   s.maxv = off;      off = up(off + (size_t)B * 4);
   s.rope_tab = off;  off = up(off + (size_t)B * (D / 2) * 8);
+  if (d->clusters) {
+    s.cl = cluster_layout(B, dm, d->clusters, off);
+    off += s.cl.bytes;
+    tickets = std::max(tickets, s.cl.tickets);
+  }
   s.total = off;
   s.tickets = tickets;
   return s;
@@ -473,11 +539,15 @@ int run_draft(const spec_model* m, const spec_drafter* d, const int32_t* block_t
     if (rc) return rc;
     rc = cuda_status(launch_rmsnorm(h, B, dm, m->rms_eps, hn, st));
     if (rc) return rc;
-    GemmBuffers bl = bufs();
-    bl.arg_keys = at<unsigned long long>(ws, s.arg_keys);
-    bl.ids = ids;
-    bl.maxv = maxv;
-    rc = cuda_status(launch_gemm_any(plan_gemm(B, m->vocab, dm, kGemmArgmax), kGemmArgmax, hn, m->w_lm, bl, st));
+    if (d->clusters) {         // cheap unembedding over the best token clusters
+      rc = cuda_status(run_clusters(d->clusters, hn, B, dm, ids, maxv, ws, s.cl, st));
+    } else {                   // the target's full LM head
+      GemmBuffers bl = bufs();
+      bl.arg_keys = at<unsigned long long>(ws, s.arg_keys);
+      bl.ids = ids;
+      bl.maxv = maxv;
+      rc = cuda_status(launch_gemm_any(plan_gemm(B, m->vocab, dm, kGemmArgmax), kGemmArgmax, hn, m->w_lm, bl, st));
+    }
     if (rc) return rc;
     rc = cuda_status(launch_draft_collect(ids, maxv, B, k, step, drafts, draft_max, st));
     if (rc) return rc;
@@ -785,6 +855,25 @@ int spec_draft(const spec_model* m, const spec_drafter* d, const int32_t* block_
   if (k == 0) return SPEC_OK;
   return run_draft(m, d, block_table, max_pages, seq_lens, prev_hidden, prev_token, B, k, drafts,
                    draft_maxlogit, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+size_t spec_cluster_unembed_workspace_bytes(int M, int d, const spec_clusters* t) {
+  if (M < 1 || check_clusters(t, d)) return 0;
+  ClusterLayout c = cluster_layout(M, d, t, kWsHeaderBytes);
+  if (c.tickets > kMaxTickets) return 0;
+  return kWsHeaderBytes + c.bytes;
+}
+
+int spec_cluster_unembed(const void* h, int M, int d, const spec_clusters* t, int32_t* ids,
+                         float* maxlogit, void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_clusters(t, d);
+  if (rc) return rc;
+  if (!h || !ids || !ws || M < 1 || (reinterpret_cast<uintptr_t>(h) & 15)) return SPEC_EINVAL;
+  ClusterLayout c = cluster_layout(M, d, t, kWsHeaderBytes);
+  if (c.tickets > kMaxTickets) return SPEC_EUNSUPPORTED;
+  if (ws_bytes < kWsHeaderBytes + c.bytes) return SPEC_EINVAL;
+  return cuda_status(run_clusters(t, static_cast<const uint16_t*>(h), M, d, ids, maxlogit, ws, c,
+                                  static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

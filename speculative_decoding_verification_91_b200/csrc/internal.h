@@ -97,6 +97,17 @@ cudaError_t launch_draft_input(const uint16_t* prev_bf16, const float* prev_f32,
                                cudaStream_t st);
 cudaError_t launch_draft_collect(const int32_t* ids, const float* maxv, int B, int k, int s,
                                  int32_t* drafts, float* draft_max, cudaStream_t st);
+// Cheap unembedding over token clusters (cluster.cu).
+struct ClusterArgs {
+  int n_clusters, cluster_size, n_select;
+  const void* centroids;          // bf16 [C][d]
+  const int32_t* cluster_tokens;  // [C][S], -1 pads
+  const void* w_clustered;        // bf16 [C*S][d]
+};
+size_t cluster_logit_floats(int M, int C);
+cudaError_t launch_cluster_unembed(const ClusterArgs& t, const uint16_t* h, int M, int d,
+                                   int32_t* ids, float* maxv, float* cl_logits, int32_t* sel,
+                                   unsigned long long* keys, const GemmBuffers& gb, cudaStream_t st);
 cudaError_t launch_to_bf16(const float* x, size_t n, uint16_t* out, cudaStream_t st);
 cudaError_t launch_rmsnorm(const float* x, int M, int d, double eps, uint16_t* out,
                            cudaStream_t st);

@@ -196,6 +196,48 @@ def drafter_inputs(wl: Workload, b: int, attempt: int):
             int(gen.randint(wl.seed, key + "/tok", 0, 1, 0, wl.vocab)[0]))
 
 
+CLUSTER_SIZE = 128      # tokens per cluster of the cheap unembedding
+CANDIDATES = 4096       # candidate tokens per row it aims for (~4096)
+
+
+def _permutation(wl: Workload, name: str, n: int) -> np.ndarray:
+    u = gen.uniform(wl.seed, f"{wl.name}/{name}", 0, n)
+    perm = np.arange(n, dtype=np.int64)
+    for i in range(n - 1, 0, -1):           # Fisher-Yates, driven by the counter stream
+        j = int(u[i] * (i + 1))
+        perm[i], perm[j] = perm[j], perm[i]
+    return perm
+
+
+def _bf16_bits(x: np.ndarray) -> np.ndarray:
+    """float -> bf16 bit patterns, round to nearest even (storage format only)."""
+    u = np.ascontiguousarray(np.asarray(x, dtype=np.float32)).view(np.uint32).astype(np.uint64)
+    return (((u + 0x7FFF + ((u >> 16) & 1)) >> 16) & 0xFFFF).astype(np.uint16)
+
+
+def cluster_tables(wl: Workload, w_lm_bits=None):
+    """Synthetic token clusters for the cheap unembedding: a seeded random
+    partition of the vocabulary into clusters of CLUSTER_SIZE tokens (the
+    last one padded with -1), each cluster's centroid the mean of its
+    members' LM-head rows (bf16), and the LM-head rows copied in cluster
+    order (zero rows for the padding).  Returns (cluster_tokens [C][S]
+    int32, centroid bits [C][d], clustered LM-head bits [C*S][d],
+    n_select)."""
+    S, V, d = CLUSTER_SIZE, wl.vocab, wl.d_model
+    C = -(-V // S)
+    perm = _permutation(wl, "clusters", V)
+    toks = np.full(C * S, -1, dtype=np.int32)
+    toks[:V] = perm
+    w = lm_head_weight(wl) if w_lm_bits is None else w_lm_bits
+    wc = np.zeros((C * S, d), dtype=np.uint16)
+    wc[:V] = w[perm]
+    vals = (wc.astype(np.uint32) << 16).view(np.float32).reshape(C, S, d)
+    counts = (toks.reshape(C, S) >= 0).sum(axis=1)
+    cent = _bf16_bits(vals.astype(np.float64).sum(axis=1) / counts[:, None])
+    n_select = min(CANDIDATES // S, max(1, C // 8))
+    return toks.reshape(C, S), cent, wc, n_select
+
+
 def layer_weights(wl: Workload, l: int):
     """(W_qkv [Nqkv][d], W_o [d][Hq*D]) bf16 bits, rows = output features.
 

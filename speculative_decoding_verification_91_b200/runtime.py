@@ -108,7 +108,7 @@ class DeviceDrafter:
     descriptor.  blocks: (w_q bits, w_o bits, target layer) per block."""
 
     def __init__(self, *, d_draft, n_q_heads, w_emb_bits, w_down_bits, w_up_bits, blocks,
-                 device="cuda"):
+                 device="cuda", clusters=None):
         self.device = torch.device(device)
         self.d_draft, self.n_q_heads = d_draft, n_q_heads
         self.w_emb = to_device_bf16(w_emb_bits, self.device)
@@ -121,6 +121,22 @@ class DeviceDrafter:
         for i in range(len(blocks)):
             self._blocks_c[i] = B.SpecDraftBlock(self.w_q[i].data_ptr(), self.w_o[i].data_ptr(),
                                                  self.target_layers[i])
+        self.clusters = clusters
         self.desc = B.SpecDrafter(d_draft, n_q_heads, len(blocks), self.w_emb.data_ptr(),
                                   self.w_down.data_ptr(), self.w_up.data_ptr(),
-                                  ctypes.cast(self._blocks_c, ctypes.POINTER(B.SpecDraftBlock)))
+                                  ctypes.cast(self._blocks_c, ctypes.POINTER(B.SpecDraftBlock)),
+                                  ctypes.pointer(clusters.desc) if clusters is not None else None)
+
+
+class DeviceClusters:
+    """Token-cluster tables of the cheap unembedding on one GPU and their
+    spec_clusters descriptor."""
+
+    def __init__(self, *, cluster_tokens, centroid_bits, clustered_bits, n_select, device="cuda"):
+        self.device = torch.device(device)
+        C, S = cluster_tokens.shape
+        self.tokens = torch.from_numpy(np.ascontiguousarray(cluster_tokens, dtype=np.int32)).to(self.device)
+        self.centroids = to_device_bf16(centroid_bits, self.device)
+        self.w_clustered = to_device_bf16(clustered_bits, self.device)
+        self.desc = B.SpecClusters(int(C), int(S), int(n_select), self.centroids.data_ptr(),
+                                   self.tokens.data_ptr(), self.w_clustered.data_ptr())

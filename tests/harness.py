@@ -104,14 +104,14 @@ def oracle_drafter(wl: W.Workload):
                        for q, o, t in blocks])
 
 
-def guarded_draft_inputs(wl, model, drafter, caches, b, L, k, max_attempts=40):
+def guarded_draft_inputs(wl, model, drafter, caches, b, L, k, max_attempts=40, tables=None):
     """Redraw sequence b's drafter inputs (target activation, token) until every
     one of the k oracle draft steps has a safe top-2 margin.  Returns
     (attempt, activation bits, token, oracle steps)."""
     from oracle import draft as OD
     for t in range(max_attempts):
         h_bits, tok = W.drafter_inputs(wl, b, t)
-        steps = OD.draft(model, drafter, caches, L, oracle.bf16_from_bits(h_bits), tok, k)
+        steps = OD.draft(model, drafter, caches, L, oracle.bf16_from_bits(h_bits), tok, k, tables)
         if all(margin_ok(st.top1, st.top2) for st in steps):
             return t, h_bits, tok, steps
     raise RuntimeError(f"no margin-safe drafter inputs for sequence {b}")

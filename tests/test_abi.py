@@ -138,3 +138,18 @@ def test_drafter_workspace_and_validation(lib):
                           None) == B.SPEC_EINVAL
     assert lib.spec_draft(pm, ctypes.byref(_drafter(n_q_heads=12)), FAKE, 10, FAKE, FAKE, FAKE, 1, 4,
                           FAKE, None, FAKE, 1 << 30, None) == B.SPEC_EINVAL
+
+
+def test_cluster_unembed_validation(lib):
+    t = B.SpecClusters(2048, 128, 32, FAKE, FAKE, FAKE)
+    assert B.spec_cluster_unembed_workspace_bytes(4, 2560, t) > 4096
+    assert B.spec_cluster_unembed_workspace_bytes(4, 2561, t) == 0          # d not a multiple of 8
+    assert B.spec_cluster_unembed_workspace_bytes(4, 2560, B.SpecClusters(16, 8, 17, FAKE, FAKE, FAKE)) == 0
+    assert B.spec_cluster_unembed_workspace_bytes(4, 2560, B.SpecClusters(9000, 8, 4, FAKE, FAKE, FAKE)) == 0
+    assert lib.spec_cluster_unembed(FAKE, 4, 2560, ctypes.byref(t), FAKE, None, FAKE, 100,
+                                    None) == B.SPEC_EINVAL                   # workspace too small
+    assert lib.spec_cluster_unembed(FAKE + 2, 4, 2560, ctypes.byref(t), FAKE, None, FAKE, 1 << 30,
+                                    None) == B.SPEC_EINVAL                   # misaligned h
+    big = B.SpecClusters(9000, 8, 4, FAKE, FAKE, FAKE)
+    assert lib.spec_cluster_unembed(FAKE, 4, 2560, ctypes.byref(big), FAKE, None, FAKE, 1 << 30,
+                                    None) == B.SPEC_EUNSUPPORTED

@@ -35,11 +35,11 @@ def _bits(t):
     return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
 
 
-def device_drafter(wl):
+def device_drafter(wl, clusters=None):
     dd, hq, _ = W.drafter_spec(wl)
     emb, down, upw, blocks = W.drafter_weights(wl)
     return DeviceDrafter(d_draft=dd, n_q_heads=hq, w_emb_bits=emb, w_down_bits=down,
-                         w_up_bits=upw, blocks=blocks)
+                         w_up_bits=upw, blocks=blocks, clusters=clusters)
 
 
 @pytest.mark.parametrize("name,k", [("tiny", 3), ("small_b1", 4), ("small_ragged", 3),
