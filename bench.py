@@ -437,6 +437,35 @@ def run_lmhead_only(args):
                       "frac_tensor": (flops / us / 1e6 / tf) if tf else None}), flush=True)
 
 
+def lm_roofline(wl, r, lm_bytes, lm_s, peak_gbs, peak_kind):
+    """Roofline of the step's dominant kernel, the LM head + argmax.  Its
+    bound is the larger of bytes / measured copy bandwidth and FLOPs /
+    measured sustained bf16 GEMM throughput (it runs inside a long step):
+    HBM for few verify rows, the tensor cores at 256 rows."""
+    M = r["M"]
+    flops = 2.0 * M * wl.d_model * wl.vocab
+    tf = None
+    mp = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(mp):
+        tf = json.load(open(mp)).get("bf16_tflops_sustained")
+    kernel = ("tc_gemm_kernel<argmax> (tcgen05 LM head + argmax)" if 32 < M <= 256
+              else "stream_gemm_kernel<argmax> (LM head + argmax + acceptance)")
+    t_hbm = lm_bytes / (peak_gbs * 1e9)
+    t_tc = flops / (tf * 1e12) if tf else 0.0
+    out = {"kernel": kernel, "bytes_per_launch": lm_bytes, "flops_per_launch": flops,
+           "us_per_launch": lm_s * 1e6,
+           "traffic": measured_traffic(f"lm_head_argmax/{wl.name}")}
+    if t_tc > t_hbm:
+        ach = flops / lm_s / 1e12
+        out.update({"bound": "tensor", "achieved": ach, "peak": tf, "unit": "TFLOP/s",
+                    "frac": ach / tf, "peak_kind": "measured sustained bf16 GEMM"})
+    else:
+        ach = lm_bytes / lm_s / 1e9
+        out.update({"bound": "hbm", "achieved": ach, "peak": peak_gbs, "unit": "GB/s",
+                    "frac": ach / peak_gbs, "peak_kind": peak_kind})
+    return out
+
+
 def attention_roofline(wl, r, peak):
     """Per layer: visible KV bytes / (split + combine interval) of the
     per-launch breakdown (launches serialised by events there, so slightly
@@ -672,7 +701,6 @@ def main():
         lm_s = r["mean_lm"] / 1e3
         value = r["tokens_all"] / step_s
         lm_bytes = r["lm_b"] + r["M"] * wl.d_model * 2
-        achieved = lm_bytes / lm_s / 1e9
         step_bytes = r["kv_b"] + r["lm_b"]
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -689,11 +717,7 @@ def main():
                          "gbs": step_bytes / step_s / 1e9,
                          "frac_of_8tbs": step_bytes / step_s / 1e9 / NOMINAL_HBM_GBS,
                          "frac_of_measured": step_bytes / step_s / 1e9 / peak},
-            "roofline": {"kernel": "stream_gemm_kernel<argmax> (LM head + argmax)", "bound": "hbm",
-                         "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "peak_kind": peak_kind,
-                         "traffic": measured_traffic(f"lm_head_argmax/{wl.name}"),
-                         "bytes_per_launch": lm_bytes, "us_per_launch": r["mean_lm"] * 1e3},
+            "roofline": lm_roofline(wl, r, lm_bytes, lm_s, peak, peak_kind),
             "e2e": {"value": r["tokens_all"] / (r["mean_e2e"] / 1e3), "unit": "tokens/s",
                     "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
             "gpu_launches": r["launches"],
