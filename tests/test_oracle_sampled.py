@@ -1,0 +1,71 @@
+"""Pins of the sampled-verification oracle (CPU only).
+
+The pages state the property this must keep: the emitted tokens are
+distributed as if the target alone had sampled them.  It is checked by
+Monte Carlo on a tiny vocabulary (drafts drawn from the draft distribution,
+fresh uniforms per trial), together with the Gumbel-max draw's frequencies
+and the special cases p = q (every draft accepted) and p(d) = 0 (rejected).
+"""
+import numpy as np
+import pytest
+
+from oracle import sampled as OS
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def test_gumbel_draw_frequencies_follow_the_weights():
+    r = _rng(0)
+    w = np.array([0.5, 0.0, 0.2, 0.3])
+    n = 40000
+    counts = np.zeros(4)
+    for _ in range(n):
+        t, _, _ = OS.gumbel_draw(w, r.random(4))
+        counts[t] += 1
+    assert counts[1] == 0
+    np.testing.assert_allclose(counts / n, w, atol=0.012)
+
+
+@pytest.mark.parametrize("T", [1.0, 0.7])
+def test_emitted_tokens_follow_the_target_distribution(T):
+    r = _rng(1)
+    V, k, n = 5, 2, 30000
+    p_logits = r.standard_normal((k + 1, V)).astype(np.float32) * 1.5
+    q_logits = r.standard_normal((k, V)).astype(np.float32) * 1.5
+    p = OS.softmax(p_logits, T)
+    q = OS.softmax(q_logits, T)
+    first = np.zeros(V)
+    second = np.zeros(V)
+    n_second = 0
+    accepted = 0
+    for _ in range(n):
+        drafts = [r.choice(V, p=q[0]), r.choice(V, p=q[1])]
+        res = OS.speculative_sample(p_logits, q_logits, drafts, r.random(k), r.random(V), T)
+        first[res.emitted[0]] += 1
+        accepted += res.accept_len
+        if res.accept_len >= 1:          # token 1 followed the accepted draft 0
+            second[res.emitted[1]] += 1
+            n_second += 1
+    np.testing.assert_allclose(first / n, p[0], atol=0.012)
+    np.testing.assert_allclose(second / n_second, p[1], atol=0.02)
+    assert 0 < accepted < n * k
+
+
+def test_equal_distributions_accept_everything():
+    r = _rng(2)
+    V, k = 7, 3
+    logits = r.standard_normal((k + 1, V)).astype(np.float32)
+    drafts = [1, 4, 2]
+    res = OS.speculative_sample(logits, logits[:k], drafts, r.random(k) * 0.999, r.random(V))
+    assert res.accept_len == k and res.emitted[:k] == drafts
+
+
+def test_impossible_draft_is_rejected_and_redrawn_elsewhere():
+    V = 6
+    p_logits = np.zeros((2, V), np.float32)
+    p_logits[0, 3] = -1e4                 # the target never emits token 3 first
+    q_logits = np.zeros((1, V), np.float32)
+    res = OS.speculative_sample(p_logits, q_logits, [3], np.array([0.0]), _rng(3).random(V))
+    assert res.accept_len == 0 and res.emitted[0] != 3 and res.emitted[1] == -1
