@@ -231,6 +231,32 @@ int spec_prefill(const spec_model* m, const int32_t* block_table, int max_pages,
                  float* next_maxlogit, void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Sampled (distribution-preserving) verification.  The pages state the
+ * property ("Gemma 4 发布时未包含 MTP 数据——为什么这很重要" §MTP 能快多少: the output is
+ * what decoding the target alone would produce); for sampling this is
+ * speculative sampling (Leviathan, Kalman, Matias, ICML 2023, Algorithm 1):
+ * with p_i = softmax(target logits of verify row i / T) and q_i =
+ * softmax(draft_logits[b][i] / T), draft i is accepted iff
+ * u_accept[b][i] * q_i(d_i) < p_i(d_i); at the first rejection a token is
+ * drawn from max(0, p_i - q_i), and after k acceptances from p_k.  A draw
+ * from weights w is argmax_v log w_v - log(-log u_draw[b][v]) (w_v = 0
+ * never drawn; equal scores: lowest id).  Emits the accepted drafts and the
+ * drawn token, commits a+1 positions like spec_verify_step.
+ *   draft_logits [B][k][V] binary32, u_accept [B][k] in [0, 1), u_draw
+ *   [B][V] in (0, 1): device inputs; temperature > 0;
+ *   target_logits [B][k+1][V] (out, device) or NULL.
+ * ws: spec_verify_sampled_workspace_bytes (it holds the B*(k+1) x V target
+ * logits), set up once with spec_workspace_init.
+ * ------------------------------------------------------------------------- */
+size_t spec_verify_sampled_workspace_bytes(const spec_model* m, int B, int k, int max_pages);
+int spec_verify_step_sampled(const spec_model* m, const int32_t* block_table, int max_pages,
+                             const int32_t* last_token, const int32_t* drafts,
+                             const float* draft_logits, int B, int k, float temperature,
+                             const float* u_accept, const float* u_draw, int32_t* seq_lens,
+                             int32_t* accept_len, int32_t* emitted, int32_t* new_last_token,
+                             float* target_logits, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * MTP drafter on the target's shared KV cache ("Gemma 4 拆解 | 多模态怎么塞进端侧，
  * MTP drafter 又是怎么自带投机采样的" §4.2: the drafter's input is the target's
  * last-layer activation plus the embedding of the previous token, projected

@@ -36,7 +36,19 @@ from dataclasses import dataclass
 
 import numpy as np
 
-__all__ = ["softmax", "gumbel_draw", "SampledResult", "speculative_sample"]
+from .verify import bf16_from_bits, f32
+
+__all__ = ["softmax", "gumbel_draw", "SampledResult", "speculative_sample", "full_logits"]
+
+
+def full_logits(h, w_bits, chunk: int = 16384) -> np.ndarray:
+    """Logits h . W_v of every token (float64 products rounded to binary32),
+    the LM head's definition: h [M][d] bf16 values, w_bits [V][d] bf16 bits."""
+    h = np.asarray(h, dtype=np.float64)
+    out = np.empty((h.shape[0], w_bits.shape[0]), dtype=np.float32)
+    for v0 in range(0, w_bits.shape[0], chunk):
+        out[:, v0:v0 + chunk] = f32(h @ bf16_from_bits(w_bits[v0:v0 + chunk]).astype(np.float64).T)
+    return out
 
 
 def softmax(logits, T: float = 1.0) -> np.ndarray:
@@ -50,14 +62,16 @@ def softmax(logits, T: float = 1.0) -> np.ndarray:
 def gumbel_draw(w, g):
     """Token drawn from weights w >= 0 with uniforms g: argmax_v log w_v -
     log(-log g_v) (w_v = 0 excluded; ties: lowest id).  Returns (token, best
-    score, second score)."""
+    score, second score, second token)."""
     w = np.asarray(w, dtype=np.float64)
     g = np.asarray(g, dtype=np.float64)
     with np.errstate(divide="ignore"):
         score = np.where(w > 0, np.log(w) - np.log(-np.log(g)), -np.inf)
     j = int(np.argmax(score))
-    rest = np.delete(score, j)
-    return j, float(score[j]), float(rest.max()) if rest.size else -np.inf
+    rest = score.copy()
+    rest[j] = -np.inf
+    j2 = int(np.argmax(rest))
+    return j, float(score[j]), float(rest[j2]), j2
 
 
 @dataclass
@@ -65,8 +79,9 @@ class SampledResult:
     accept_len: int
     emitted: list                # accepted drafts, then the drawn token; -1 padding to k+1
     next_last_token: int
-    accept_margin: float         # min over tested drafts of |u q - p| (decision distance)
+    accept_margin: float         # min over tested drafts of |u q - p| / max(u q, p)
     draw_margin: float           # best minus second Gumbel score of the draw
+    draw_weights: tuple          # ((p, q) of the drawn token, (p, q) of the runner-up); q = 0 for p_k
 
 
 def speculative_sample(p_logits, q_logits, drafts, u, g, T: float = 1.0) -> SampledResult:
@@ -83,12 +98,14 @@ def speculative_sample(p_logits, q_logits, drafts, u, g, T: float = 1.0) -> Samp
     a = 0
     while a < k:
         pd, qd = p[a, drafts[a]], q[a, drafts[a]]
-        margin = min(margin, abs(u[a] * qd - pd))
+        margin = min(margin, abs(u[a] * qd - pd) / max(u[a] * qd, pd, 1e-300))
         if u[a] * qd < pd:
             a += 1
         else:
             break
-    w = np.maximum(p[a] - q[a], 0.0) if a < k else p[k]
-    tok, s1, s2 = gumbel_draw(w, g)
+    qa = q[a] if a < k else np.zeros_like(p[k])
+    w = np.maximum(p[a] - qa, 0.0)
+    tok, s1, s2, tok2 = gumbel_draw(w, g)
     emitted = drafts[:a] + [tok] + [-1] * (k - a)
-    return SampledResult(a, emitted, tok, float(margin), s1 - s2)
+    return SampledResult(a, emitted, tok, float(margin), s1 - s2,
+                         ((p[a, tok], qa[tok]), (p[a, tok2], qa[tok2])))

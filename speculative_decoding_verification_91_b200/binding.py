@@ -36,6 +36,7 @@ EXPORTED = [
     "spec_profile_launches", "spec_profile_launches_collect", "spec_launch_count",
     "spec_draft_workspace_bytes", "spec_draft",
     "spec_cluster_unembed_workspace_bytes", "spec_cluster_unembed",
+    "spec_verify_sampled_workspace_bytes", "spec_verify_step_sampled",
 ]
 SPEC_MAX_PREFILL = 256
 SPEC_NOALLOC_MAX_ROWS = 64
@@ -142,8 +143,13 @@ def lib():
         L.spec_cluster_unembed_workspace_bytes.argtypes = [c_int, c_int, pc]
         L.spec_cluster_unembed.argtypes = [c_void_p, c_int, c_int, pc, c_void_p, c_void_p, c_void_p,
                                            c_size_t, c_void_p]
+        L.spec_verify_sampled_workspace_bytes.argtypes = [pm, c_int, c_int, c_int]
+        L.spec_verify_step_sampled.argtypes = [pm, c_void_p, c_int, c_void_p, c_void_p, c_void_p,
+                                               c_int, c_int, c_float, c_void_p, c_void_p, c_void_p,
+                                               c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                               c_size_t, c_void_p]
         sizes = ("spec_prefill_workspace_bytes", "spec_draft_workspace_bytes",
-                 "spec_cluster_unembed_workspace_bytes")
+                 "spec_cluster_unembed_workspace_bytes", "spec_verify_sampled_workspace_bytes")
         for name in EXPORTED[4:]:
             if name not in sizes:
                 getattr(L, name).restype = c_int
@@ -316,3 +322,17 @@ def spec_cluster_unembed(h, M, d, clusters, ids, maxlogit, ws, ws_bytes, stream=
     return _check(lib().spec_cluster_unembed(_p(h), M, d, ctypes.byref(clusters), _p(ids),
                                              _p(maxlogit), _p(ws), ws_bytes, _s(stream)),
                   "spec_cluster_unembed")
+
+
+def spec_verify_sampled_workspace_bytes(model, B: int, k: int, max_pages: int) -> int:
+    return int(lib().spec_verify_sampled_workspace_bytes(ctypes.byref(model), B, k, max_pages))
+
+
+def spec_verify_step_sampled(model, block_table, max_pages, last_token, drafts, draft_logits, B, k,
+                             temperature, u_accept, u_draw, seq_lens, accept_len, emitted,
+                             new_last_token, target_logits, ws, ws_bytes, stream=None) -> int:
+    return _check(lib().spec_verify_step_sampled(
+        ctypes.byref(model), _p(block_table), max_pages, _p(last_token), _p(drafts), _p(draft_logits),
+        B, k, float(temperature), _p(u_accept), _p(u_draw), _p(seq_lens), _p(accept_len),
+        _p(emitted), _p(new_last_token), _p(target_logits), _p(ws), ws_bytes, _s(stream)),
+        "spec_verify_step_sampled")

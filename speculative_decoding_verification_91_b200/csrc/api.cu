@@ -5,6 +5,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <cmath>
 #include <atomic>
 #include <mutex>
 #include <vector>
@@ -127,7 +128,7 @@ StepLayout step_layout(const spec_model* m, int B, int q, int max_pages) {
     GemmPlan pq = plan_gemm(M, qkv_out(m, L), d, kGemmQkvRope);
     GemmPlan po = plan_gemm(M, d, m->n_q_heads * D, kGemmResidual);
     gemm_floats = std::max({gemm_floats, gemm_partial_floats(pq), gemm_partial_floats(po)});
-    tickets = std::max({tickets, gemm_tickets(pq), gemm_tickets(po)});
+    tickets = std::max({tickets, gemm_tickets(pq, kGemmQkvRope), gemm_tickets(po, kGemmResidual)});
   }
   GemmPlan pl = plan_gemm(M, m->vocab, d, kGemmArgmax);
   tickets = std::max(tickets, pl.mblocks);
@@ -200,6 +201,8 @@ struct ForwardIo {
   const int32_t* tokens = nullptr;     // prefill: [B][q]
   int32_t* next_token = nullptr;       // prefill: [B]
   float* next_maxlogit = nullptr;
+  float* logits = nullptr;             // sampled verify: LM head writes [M][V] logits, no argmax
+  float* logits_part = nullptr;        //   and its split-K partials (tensor-memory path)
 };
 
 // embed -> per layer (RMSNorm, QKV + RoPE + cache append, split-KV attention,
@@ -307,6 +310,21 @@ int run_forward(const spec_model* m, const int32_t* block_table, int max_pages, 
     bl.acc.copy_max = io.target_maxlogit;
   }
   prof_mark(1, st);
+  if (io.logits) {     // sampled verification: binary32 logits of every row
+    GemmBuffers bs{};
+    bs.out = io.logits;
+    bs.partial = io.logits_part;
+    bs.tickets = hdr.tickets;
+    bs.status = hdr.status;
+    rc = cuda_status(launch_gemm_any(plan_gemm(M, m->vocab, d, kGemmStore), kGemmStore, hn, m->w_lm,
+                                     bs, st));
+    prof_mark(2, st);
+    prof_mark(3, st);
+    detail_mark(st);
+    g_detail.on = false;
+    prof_step_done();
+    return rc;
+  }
   rc = cuda_status(launch_gemm_any(pl, kGemmArgmax, lm_x, m->w_lm, bl, st));
   prof_mark(2, st);
   detail_mark(st);
@@ -325,6 +343,30 @@ int run_forward(const spec_model* m, const int32_t* block_table, int max_pages, 
   g_detail.on = false;
   prof_step_done();
   return rc;
+}
+
+// ---------------------------------------------------------- sampled verify
+
+struct SampledLayout {
+  StepLayout s;
+  size_t logits, part, st_t, st_d, a, keys, total;
+  int tickets;
+};
+SampledLayout sampled_layout(const spec_model* m, int B, int k, int max_pages) {
+  SampledLayout L{};
+  L.s = step_layout(m, B, k + 1, max_pages);
+  const int M = B * (k + 1), V = m->vocab;
+  GemmPlan pl = plan_gemm(M, V, m->d_model, kGemmStore);
+  size_t off = L.s.total;
+  L.logits = off; off = up(off + (size_t)M * V * 4);
+  L.part = off;   off = up(off + ((pl.splits > 1 || tc_supported(M)) ? gemm_partial_floats(pl) : 0) * 4);
+  L.st_t = off;   off = up(off + (size_t)M * 8);
+  L.st_d = off;   off = up(off + (size_t)B * std::max(k, 1) * 8);
+  L.a = off;      off = up(off + (size_t)B * 4);
+  L.keys = off;   off = up(off + (size_t)B * 8);
+  L.total = off;
+  L.tickets = std::max(L.s.tickets, gemm_tickets(pl, kGemmStore));
+  return L;
 }
 
 // ---------------------------------------------------------------- clusters
@@ -368,7 +410,7 @@ ClusterLayout cluster_layout(int M, int d, const spec_clusters* t, size_t base) 
   c.sel = off;    off = up(off + (size_t)M * t->n_select * 4);
   c.keys = off;   off = up(off + (size_t)M * 8);
   c.bytes = off - base;
-  c.tickets = gemm_tickets(p);
+  c.tickets = gemm_tickets(p, kGemmStore);
   return c;
 }
 
@@ -426,13 +468,14 @@ DraftLayout draft_layout(const spec_model* m, const spec_drafter* d, int B, int 
     attn = std::max(attn, attn_partial_floats(g));
     if (g.n_splits_grid > kMaxSplits) s.splits_ok = false;
   }
-  const GemmPlan ps[4] = {plan_gemm(B, dd, dm + dd, kGemmStore), plan_gemm(B, nq, dd, kGemmQkvRope),
-                          plan_gemm(B, dd, nq, kGemmResidual), plan_gemm(B, dm, dd, kGemmStore)};
+  const int modes[4] = {kGemmStore, kGemmQkvRope, kGemmResidual, kGemmStore};
+  const GemmPlan ps[4] = {plan_gemm(B, dd, dm + dd, modes[0]), plan_gemm(B, nq, dd, modes[1]),
+                          plan_gemm(B, dd, nq, modes[2]), plan_gemm(B, dm, dd, modes[3])};
   size_t gp = 0;
   int tickets = plan_gemm(B, m->vocab, dm, kGemmArgmax).mblocks;
-  for (const GemmPlan& p : ps) {
-    gp = std::max(gp, gemm_partial_floats(p));
-    tickets = std::max(tickets, gemm_tickets(p));
+  for (int i = 0; i < 4; ++i) {
+    gp = std::max(gp, gemm_partial_floats(ps[i]));
+    tickets = std::max(tickets, gemm_tickets(ps[i], modes[i]));
   }
   size_t off = kWsHeaderBytes;
   s.u = off;         off = up(off + (size_t)B * (dm + dd) * 2);
@@ -874,6 +917,50 @@ int spec_cluster_unembed(const void* h, int M, int d, const spec_clusters* t, in
   if (ws_bytes < kWsHeaderBytes + c.bytes) return SPEC_EINVAL;
   return cuda_status(run_clusters(t, static_cast<const uint16_t*>(h), M, d, ids, maxlogit, ws, c,
                                   static_cast<cudaStream_t>(stream)));
+}
+
+size_t spec_verify_sampled_workspace_bytes(const spec_model* m, int B, int k, int max_pages) {
+  if (check_model(m) || B < 1 || k < 0 || k > SPEC_MAX_K || max_pages < 1) return 0;
+  SampledLayout L = sampled_layout(m, B, k, max_pages);
+  if (L.tickets > kMaxTickets || !L.s.splits_ok) return 0;
+  return L.total;
+}
+
+int spec_verify_step_sampled(const spec_model* m, const int32_t* block_table, int max_pages,
+                             const int32_t* last_token, const int32_t* drafts,
+                             const float* draft_logits, int B, int k, float temperature,
+                             const float* u_accept, const float* u_draw, int32_t* seq_lens,
+                             int32_t* accept_len, int32_t* emitted, int32_t* new_last_token,
+                             float* target_logits, void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_model(m);
+  if (rc) return rc;
+  if (!block_table || !last_token || !seq_lens || !accept_len || !emitted || !new_last_token ||
+      !u_draw || !ws)
+    return SPEC_EINVAL;
+  if (B < 1 || k < 0 || k > SPEC_MAX_K || max_pages < 1) return SPEC_EINVAL;
+  if (k > 0 && (!drafts || !draft_logits || !u_accept)) return SPEC_EINVAL;
+  if (!(temperature > 0.f) || !isfinite(temperature)) return SPEC_EINVAL;
+  SampledLayout L = sampled_layout(m, B, k, max_pages);
+  if (L.tickets > kMaxTickets || !L.s.splits_ok) return SPEC_EUNSUPPORTED;
+  if (ws_bytes < L.total) return SPEC_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ForwardIo io;
+  io.last_token = last_token;
+  io.drafts = drafts;
+  io.logits = at<float>(ws, L.logits);
+  io.logits_part = at<float>(ws, L.part);
+  rc = run_forward(m, block_table, max_pages, B, k + 1, seq_lens, io, ws, ws_bytes, st);
+  if (rc) return rc;
+  const int M = B * (k + 1), V = m->vocab;
+  if (target_logits &&
+      cudaMemcpyAsync(target_logits, io.logits, (size_t)M * V * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return SPEC_ECUDA;
+  WsHeader hdr = ws_header(ws);
+  return cuda_status(launch_sampled_tail(B, k, V, temperature, io.logits, draft_logits,
+                                         at<float2>(ws, L.st_t), at<float2>(ws, L.st_d), drafts,
+                                         u_accept, u_draw, at<int32_t>(ws, L.a),
+                                         at<unsigned long long>(ws, L.keys), seq_lens, accept_len,
+                                         emitted, new_last_token, hdr.status, st));
 }
 
 }  // extern "C"

@@ -420,10 +420,13 @@ size_t gemm_partial_floats(const GemmPlan& p) {
 }
 size_t gemm_argmax_entries(const GemmPlan& p) { return (size_t)p.M; }
 // Completion counters the fused last-CTA epilogue needs: one per (M-block,
-// tile) when it runs (few rows), none when the grid-wide reduce does the
-// epilogue (more rows).
-int gemm_tickets(const GemmPlan& p) {
-  return p.M > kFusedTailMaxRows ? 0 : p.mblocks * p.n_tiles;
+// tile) when it runs (few rows, more than one K split or the RoPE
+// epilogue), none when the tile is stored directly or the grid-wide reduce
+// does the epilogue (more rows).
+int gemm_tickets(const GemmPlan& p, int mode) {
+  if (p.M > kFusedTailMaxRows) return 0;
+  if (p.splits == 1 && mode != kGemmQkvRope) return 0;   // stored directly, no last-CTA tail
+  return p.mblocks * p.n_tiles;
 }
 
 cudaError_t launch_gemm(const GemmPlan& p, int mode, const void* x, const void* w,
@@ -461,7 +464,8 @@ cudaError_t launch_gemm(const GemmPlan& p, int mode, const void* x, const void* 
     case kGemmResidual: e = launch_mode<kGemmResidual>(p, tw, tx, a, st); break;
     case kGemmQkvRope: e = launch_mode<kGemmQkvRope>(p, tw, tx, a, st); break;
   }
-  if (e != cudaSuccess || !a.grid_reduce) return e;
+  // a single K split stores / adds its tile directly (no partials to reduce)
+  if (e != cudaSuccess || !a.grid_reduce || (p.splits == 1 && mode != kGemmQkvRope)) return e;
   return launch_splitk_reduce(a, mode, st);
 }
 

@@ -32,7 +32,7 @@ struct GemmPlan {
 GemmPlan plan_gemm(int M, int N, int K, int mode);
 size_t gemm_partial_floats(const GemmPlan& p);   // split-K partial sums
 size_t gemm_argmax_entries(const GemmPlan& p);   // argmax keys (one per row)
-int gemm_tickets(const GemmPlan& p);
+int gemm_tickets(const GemmPlan& p, int mode);
 
 // Acceptance fused into the LM-head argmax (B = 0: not fused).
 struct AcceptFuse {
@@ -108,6 +108,13 @@ size_t cluster_logit_floats(int M, int C);
 cudaError_t launch_cluster_unembed(const ClusterArgs& t, const uint16_t* h, int M, int d,
                                    int32_t* ids, float* maxv, float* cl_logits, int32_t* sel,
                                    unsigned long long* keys, const GemmBuffers& gb, cudaStream_t st);
+// Sampled verification tail (sampled.cu): softmax statistics, acceptance,
+// Gumbel-max draw, commit.
+cudaError_t launch_sampled_tail(int B, int k, int V, float T, const float* lt, const float* ld,
+                                float2* st_t, float2* st_d, const int32_t* drafts, const float* u,
+                                const float* g, int32_t* a_arr, unsigned long long* keys,
+                                int32_t* seq_lens, int32_t* accept_len, int32_t* emitted,
+                                int32_t* new_last, unsigned* status, cudaStream_t st);
 cudaError_t launch_to_bf16(const float* x, size_t n, uint16_t* out, cudaStream_t st);
 cudaError_t launch_rmsnorm(const float* x, int M, int d, double eps, uint16_t* out,
                            cudaStream_t st);

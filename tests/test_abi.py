@@ -153,3 +153,16 @@ def test_cluster_unembed_validation(lib):
     big = B.SpecClusters(9000, 8, 4, FAKE, FAKE, FAKE)
     assert lib.spec_cluster_unembed(FAKE, 4, 2560, ctypes.byref(big), FAKE, None, FAKE, 1 << 30,
                                     None) == B.SPEC_EUNSUPPORTED
+
+
+def test_sampled_verify_validation(lib):
+    m = _model()
+    pm = ctypes.byref(m)
+    assert B.spec_verify_sampled_workspace_bytes(m, 8, 4, 520) > B.spec_workspace_bytes(m, 8, 4, 520)
+    assert B.spec_verify_sampled_workspace_bytes(m, 8, 17, 520) == 0
+    args = lambda T, ws_bytes, dl=FAKE: (pm, FAKE, 10, FAKE, FAKE, dl, 1, 4, ctypes.c_float(T), FAKE,
+                                         FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, ws_bytes, None)
+    assert lib.spec_verify_step_sampled(*args(0.0, 1 << 40)) == B.SPEC_EINVAL       # temperature
+    assert lib.spec_verify_step_sampled(*args(float("nan"), 1 << 40)) == B.SPEC_EINVAL
+    assert lib.spec_verify_step_sampled(*args(1.0, 1 << 40, dl=None)) == B.SPEC_EINVAL   # draft logits
+    assert lib.spec_verify_step_sampled(*args(1.0, 100)) == B.SPEC_EINVAL            # workspace

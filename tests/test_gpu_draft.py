@@ -43,7 +43,7 @@ def device_drafter(wl, clusters=None):
 
 
 @pytest.mark.parametrize("name,k", [("tiny", 3), ("small_b1", 4), ("small_ragged", 3),
-                                    ("small_b16", 2), ("small_loop", 5)])
+                                    ("small_b16", 2), ("small_b32", 2), ("small_loop", 5)])
 def test_draft_matches_oracle(name, k):
     wl = W.get_workload(name)
     model = harness.oracle_model(wl)

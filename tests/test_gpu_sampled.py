@@ -1,0 +1,108 @@
+"""Parity of sampled verification (spec_verify_step_sampled) with the oracle.
+
+Draft logits are seeded synthetic inputs; the drafts are drawn from their
+softmax with seeded uniforms, and the acceptance and draw uniforms are
+seeded too.  A sequence's draws are redrawn (oracle only) until every
+acceptance decision is at least 5% away from its threshold and the Gumbel
+draw's winner leads by more than the logits' tolerance and is not a
+near-cancellation of p - q; then accept lengths, emitted tokens, next token
+and lengths must be identical, and the target logits within 2e-2 + 1e-2
+relative."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import sampled as OS
+from speculative_decoding_verification_91_b200 import binding as B
+from speculative_decoding_verification_91_b200.inputs import gen
+from speculative_decoding_verification_91_b200.inputs import workloads as W
+from speculative_decoding_verification_91_b200.runtime import Workspace
+from speculative_decoding_verification_91_b200.session import WorkloadSession
+
+from . import harness
+
+pytestmark = pytest.mark.gpu
+
+ATOL, RTOL = 2e-2, 1e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.fail("CUDA device required for -m gpu tests")
+    B.lib()
+    yield
+    torch.cuda.synchronize()
+
+
+def _safe(res):
+    if res.accept_margin < 5e-2 or res.draw_margin < 5e-2:
+        return False
+    for p, q in res.draw_weights:
+        if q > 0 and abs(p - q) < 0.2 * max(p, q):
+            return False
+    return True
+
+
+def _case(wl, model, caches, L, last, b, k, T, name):
+    V = wl.vocab
+    for t in range(60):
+        key = f"test/sampled/{name}/b{b}/a{t}"
+        dl = gen.normal_f32(7, key + "/dl", 0, k * V, 2.0).reshape(k, V)
+        q = OS.softmax(dl, T)
+        ud = gen.uniform(7, key + "/ud", 0, max(k, 1))
+        drafts = [int(min(np.searchsorted(np.cumsum(q[i]), ud[i]), V - 1)) for i in range(k)]
+        fw = oracle.verify_forward(model, caches, L, [last] + drafts, lm_rows=[])
+        pl = OS.full_logits(fw.h, model.w_lm_bits)
+        ua = gen.uniform(7, key + "/ua", 0, max(k, 1))[:k]
+        g = np.clip(gen.uniform(7, key + "/g", 0, V), 1e-7, 1 - 1e-7)
+        res = OS.speculative_sample(pl, dl, drafts, ua, g, T)
+        if _safe(res):
+            return drafts, dl, ua, g, pl, res
+    raise RuntimeError("no safe sampled case")
+
+
+@pytest.mark.parametrize("name,T,k", [("small_b1", 1.0, 4), ("small_ragged", 0.8, 4),
+                                      ("small_ragged", 1.0, 0), ("small_b32", 1.0, 3)])
+def test_sampled_verify_matches_oracle(name, T, k):
+    wl = W.get_workload(name)
+    model = harness.oracle_model(wl)
+    sess = WorkloadSession(wl)
+    Bn, V, q = wl.batch, wl.vocab, k + 1
+    drafts = np.zeros((Bn, max(k, 1)), np.int32)
+    dls = np.zeros((Bn, max(k, 1), V), np.float32)
+    uas = np.zeros((Bn, max(k, 1)), np.float32)
+    gs = np.zeros((Bn, V), np.float32)
+    lasts = np.zeros(Bn, np.int32)
+    want, logits = [], []
+    for b in range(Bn):
+        L = int(sess.lens[b])
+        caches = harness.context_caches(wl, model, b, 0, L)
+        last = W.last_token(wl, b, 0)
+        d, dl, ua, g, pl, res = _case(wl, model, caches, L, last, b, k, T, name)
+        lasts[b] = last
+        drafts[b, :k], dls[b, :k], uas[b, :k], gs[b] = d, dl, ua, g
+        want.append(res)
+        logits.append(pl)
+    ws = Workspace(B.spec_verify_sampled_workspace_bytes(sess.dm.desc, Bn, k, sess.max_pages))
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    acc = torch.zeros(Bn, dtype=torch.int32, device="cuda")
+    emitted = torch.zeros(Bn * q, dtype=torch.int32, device="cuda")
+    new_last = torch.zeros(Bn, dtype=torch.int32, device="cuda")
+    tl = torch.zeros(Bn * q * V, dtype=torch.float32, device="cuda")
+    B.spec_verify_step_sampled(sess.dm.desc, sess.block_table, sess.max_pages, dev(lasts),
+                               dev(drafts[:, :k].reshape(-1)) if k else None,
+                               dev(dls[:, :k].reshape(-1)) if k else None, Bn, k, T,
+                               dev(uas[:, :k].reshape(-1)) if k else None, dev(gs.reshape(-1)),
+                               sess.seq_lens, acc, emitted, new_last, tl, ws.buf, ws.nbytes)
+    torch.cuda.synchronize()
+    assert ws.device_status() == 0
+    acc, emitted, new_last = acc.cpu().numpy(), emitted.cpu().numpy().reshape(Bn, q), new_last.cpu().numpy()
+    tl = tl.cpu().numpy().reshape(Bn, q, V)
+    for b in range(Bn):
+        np.testing.assert_allclose(tl[b], logits[b], atol=ATOL, rtol=RTOL)
+        assert acc[b] == want[b].accept_len, (b, acc[b], want[b].accept_len)
+        assert list(emitted[b]) == want[b].emitted
+        assert new_last[b] == want[b].next_last_token
+    assert np.array_equal(sess.seq_lens.cpu().numpy(), sess.lens + acc + 1)

@@ -22,7 +22,7 @@ def test_gumbel_draw_frequencies_follow_the_weights():
     n = 40000
     counts = np.zeros(4)
     for _ in range(n):
-        t, _, _ = OS.gumbel_draw(w, r.random(4))
+        t, _, _, _ = OS.gumbel_draw(w, r.random(4))
         counts[t] += 1
     assert counts[1] == 0
     np.testing.assert_allclose(counts / n, w, atol=0.012)
