@@ -46,14 +46,21 @@ def _safe(res):
 
 
 def _case(wl, model, caches, L, last, b, k, T, name):
+    """Draft i is drawn from q_i = softmax((the oracle target's logits of row i
+    + seeded N(0, 0.3) noise) / T), row i seeing the drafts before it, so
+    that drafts are often accepted; then the acceptance and draw uniforms."""
     V = wl.vocab
     for t in range(60):
         key = f"test/sampled/{name}/b{b}/a{t}"
-        dl = gen.normal_f32(7, key + "/dl", 0, k * V, 2.0).reshape(k, V)
-        q = OS.softmax(dl, T)
         ud = gen.uniform(7, key + "/ud", 0, max(k, 1))
-        drafts = [int(min(np.searchsorted(np.cumsum(q[i]), ud[i]), V - 1)) for i in range(k)]
-        fw = oracle.verify_forward(model, caches, L, [last] + drafts, lm_rows=[])
+        drafts, dl = [], np.zeros((k, V), np.float32)
+        for i in range(k):
+            fw_i = oracle.verify_forward(model, caches, L, [last] + drafts, lm_rows=[i])
+            noise = gen.normal_f32(7, key + f"/dl{i}", 0, V, 0.3)
+            dl[i] = OS.full_logits(fw_i.h, model.w_lm_bits)[0] + noise
+            q = OS.softmax(dl[i], T)
+            drafts.append(int(min(np.searchsorted(np.cumsum(q), ud[i]), V - 1)))
+        fw = oracle.verify_forward(model, caches, L, [last] + drafts)
         pl = OS.full_logits(fw.h, model.w_lm_bits)
         ua = gen.uniform(7, key + "/ua", 0, max(k, 1))[:k]
         g = np.clip(gen.uniform(7, key + "/g", 0, V), 1e-7, 1 - 1e-7)
