@@ -81,8 +81,9 @@ def _case(wl, model, caches, L, last, b, k, T, name):
             drafts.append(int(min(np.searchsorted(np.cumsum(q), ud[i]), V - 1)))
         fw = oracle.verify_forward(model, caches, L, [last] + drafts)
         pl = OS.full_logits(fw.h, model.w_lm_bits)
-        ua = gen.uniform(7, key + "/ua", 0, max(k, 1))[:k]
-        g = np.clip(gen.uniform(7, key + "/g", 0, V), 1e-7, 1 - 1e-7)
+        # the device reads binary32 uniforms: the oracle gets the same values
+        ua = gen.uniform(7, key + "/ua", 0, max(k, 1))[:k].astype(np.float32)
+        g = np.clip(gen.uniform(7, key + "/g", 0, V), 1e-7, 1 - 1e-7).astype(np.float32)
         res = OS.speculative_sample(pl, dl, drafts, ua, g, T)
         if _safe(res, pl, dl, g, T, k):
             return drafts, dl, ua, g, pl, res
