@@ -533,7 +533,7 @@ constexpr int kCombineWarps = 4;
 constexpr int kMaxCombineSplits = kMaxSplits;
 __global__ void __launch_bounds__(kCombineWarps * 32) attn_combine_kernel(AttnArgs a, int D, int n_items,
                                                                           int warp_per_row,
-                                                                          uint16_t* __restrict__ out) {
+                                                                          uint16_t* out) {
   __shared__ float msh[kCombineWarps][kMaxCombineSplits];
   __shared__ float lsh[kCombineWarps][kMaxCombineSplits];
   __shared__ float part[kCombineWarps][256];

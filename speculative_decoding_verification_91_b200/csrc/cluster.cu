@@ -33,9 +33,9 @@ constexpr int kCandWarps = 8;
 constexpr int kRowsPerWarp = 2;
 constexpr int kRowsPerCta = kCandWarps * kRowsPerWarp;   // 16 tokens of a cluster per CTA
 
-__global__ void __launch_bounds__(kSelThreads) cluster_select_kernel(const float* __restrict__ logits,
+__global__ void __launch_bounds__(kSelThreads) cluster_select_kernel(const float* logits,
                                                                      int C, int P, int n_sel,
-                                                                     int32_t* __restrict__ sel) {
+                                                                     int32_t* sel) {
   extern __shared__ unsigned long long keys[];   // P = power of two >= C
   pdl_trigger();
   pdl_wait();
@@ -86,9 +86,9 @@ __device__ __forceinline__ float dot8(uint4 w, uint4 x, float acc) {
 
 // grid (n_sel * ceil(S / 16), M)
 __global__ void __launch_bounds__(kCandWarps * 32) cluster_cand_kernel(
-    const uint16_t* __restrict__ h, int d, const int32_t* __restrict__ sel, int n_sel,
-    const int32_t* __restrict__ tokens, int S, const uint16_t* __restrict__ wc,
-    unsigned long long* __restrict__ keys) {
+    const uint16_t* h, int d, const int32_t* sel, int n_sel,
+    const int32_t* tokens, int S, const uint16_t* wc,
+    unsigned long long* keys) {
   extern __shared__ uint4 hs[];   // the row's h, d / 8 chunks of 16 bytes
   __shared__ unsigned long long best_w[kCandWarps];
   pdl_trigger();
@@ -135,8 +135,8 @@ __global__ void __launch_bounds__(kCandWarps * 32) cluster_cand_kernel(
   }
 }
 
-__global__ void cluster_finish_kernel(unsigned long long* __restrict__ keys, int M,
-                                      int32_t* __restrict__ ids, float* __restrict__ maxv) {
+__global__ void cluster_finish_kernel(unsigned long long* keys, int M,
+                                      int32_t* ids, float* maxv) {
   pdl_trigger();
   pdl_wait();
   const int m = blockIdx.x * blockDim.x + threadIdx.x;

@@ -183,6 +183,10 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
 // data that grid (or an earlier one) may write; only constant weights are read
 // before the wait.  Both are no-ops for a launch without the PDL attribute.
 // ---------------------------------------------------------------------------
+// Data a kernel's predecessors wrote is read only after pdl_wait(), through
+// pointers without __restrict__: a `const __restrict__` pointer lets the
+// compiler treat its target as never written and move (non-coherent) loads
+// of it above the wait, reading values from before the predecessor finished.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 

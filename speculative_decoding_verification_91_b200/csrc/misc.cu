@@ -16,8 +16,8 @@ namespace {
 // normalised GEMM input differs from an exact evaluation only when the
 // float64 result sits within a few ulps of a binary32 rounding boundary.
 constexpr int kNormThreads = 256;
-__device__ __forceinline__ void norm_row(const float* __restrict__ row, int d, double eps,
-                                         uint16_t* __restrict__ o, double* red) {
+__device__ __forceinline__ void norm_row(const float* row, int d, double eps,
+                                         uint16_t* o, double* red) {
   double ss = 0.0;
   for (int e = threadIdx.x; e < d; e += kNormThreads) {
     const double v = row[e];
@@ -35,9 +35,9 @@ __device__ __forceinline__ void norm_row(const float* __restrict__ row, int d, d
     o[e] = f32_to_bf16((float)((double)row[e] / rms));
 }
 
-__global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(const float* __restrict__ x, int d,
+__global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(const float* x, int d,
                                                                double eps,
-                                                               uint16_t* __restrict__ out) {
+                                                               uint16_t* out) {
   __shared__ double red[kNormThreads / 32];
   pdl_trigger();
   pdl_wait();
@@ -48,11 +48,11 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(const float* __re
 // Embedding gather fused with the first layer's RMSNorm and with the
 // (cos, sin) table of the row's position for every rotary pair.
 __global__ void __launch_bounds__(kNormThreads) embed_norm_kernel(
-    const uint16_t* __restrict__ w_emb, int vocab, int d, const int32_t* __restrict__ last_token,
-    const int32_t* __restrict__ drafts, const int32_t* __restrict__ tokens_flat, int q, double eps,
-    float* __restrict__ x, uint16_t* __restrict__ out, unsigned* status,
-    const int32_t* __restrict__ seq_lens, InvFreq inv_freq, int half,
-    float2* __restrict__ rope_tab) {
+    const uint16_t* w_emb, int vocab, int d, const int32_t* last_token,
+    const int32_t* drafts, const int32_t* tokens_flat, int q, double eps,
+    float* x, uint16_t* out, unsigned* status,
+    const int32_t* seq_lens, InvFreq inv_freq, int half,
+    float2* rope_tab) {
   __shared__ double red[kNormThreads / 32];
   pdl_trigger();
   pdl_wait();
@@ -83,7 +83,7 @@ __global__ void __launch_bounds__(kNormThreads) embed_norm_kernel(
 // One warp per sequence: a = number of leading drafts equal to the target's
 // argmax (ballot of matches, first zero bit), emit them and target[a], commit
 // a+1 positions.
-__global__ void accept_kernel(const int32_t* __restrict__ drafts, const int32_t* __restrict__ target,
+__global__ void accept_kernel(const int32_t* drafts, const int32_t* target,
                               int B, int k, int32_t* seq_lens, int32_t* accept_len,
                               int32_t* emitted, int32_t* last_token, int32_t* copy_ids,
                               float* copy_max, const float* maxv) {
@@ -120,10 +120,10 @@ __global__ void accept_kernel(const int32_t* __restrict__ drafts, const int32_t*
 // Blocks past the B rows fill the (cos, sin) table of position
 // seq_lens[b] + pos_off for every rotary pair, as embed_norm_kernel does.
 __global__ void __launch_bounds__(kNormThreads) draft_input_kernel(
-    const uint16_t* __restrict__ prev_bf16, const float* __restrict__ prev_f32, int d_model,
-    const int32_t* __restrict__ token, const uint16_t* __restrict__ w_emb, int vocab, int d_draft,
-    uint16_t* __restrict__ u, unsigned* status, const int32_t* __restrict__ seq_lens, int pos_off,
-    InvFreq inv_freq, int half, float2* __restrict__ rope_tab, int B) {
+    const uint16_t* prev_bf16, const float* prev_f32, int d_model,
+    const int32_t* token, const uint16_t* w_emb, int vocab, int d_draft,
+    uint16_t* u, unsigned* status, const int32_t* seq_lens, int pos_off,
+    InvFreq inv_freq, int half, float2* rope_tab, int B) {
   pdl_trigger();
   pdl_wait();
   if ((int)blockIdx.x >= B) {
@@ -147,9 +147,9 @@ __global__ void __launch_bounds__(kNormThreads) draft_input_kernel(
 }
 
 // drafts[b][s] = argmax of step s, draft_max[b][s] its logit
-__global__ void draft_collect_kernel(const int32_t* __restrict__ ids, const float* __restrict__ maxv,
-                                     int B, int k, int s, int32_t* __restrict__ drafts,
-                                     float* __restrict__ draft_max) {
+__global__ void draft_collect_kernel(const int32_t* ids, const float* maxv,
+                                     int B, int k, int s, int32_t* drafts,
+                                     float* draft_max) {
   pdl_trigger();
   pdl_wait();
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
@@ -159,7 +159,7 @@ __global__ void draft_collect_kernel(const int32_t* __restrict__ ids, const floa
 }
 
 // out[i] = bf16(x[i]): a binary32 activation entering a projection
-__global__ void to_bf16_kernel(const float* __restrict__ x, size_t n, uint16_t* __restrict__ out) {
+__global__ void to_bf16_kernel(const float* x, size_t n, uint16_t* out) {
   pdl_trigger();
   pdl_wait();
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
@@ -184,7 +184,7 @@ cudaError_t launch_embed_norm(const void* w_emb, int vocab, int d, const int32_t
                   eps, x, out, status, seq_lens, f, half, rope_tab);
 }
 
-__global__ void prefill_commit_kernel(const int32_t* __restrict__ ids, const float* __restrict__ maxv,
+__global__ void prefill_commit_kernel(const int32_t* ids, const float* maxv,
                                       int B, int n, int32_t* seq_lens, int32_t* next_token,
                                       float* next_max) {
   pdl_trigger();

@@ -30,9 +30,9 @@ constexpr int kStatThreads = 1024;
 constexpr int kDrawThreads = 256;
 constexpr int kDrawChunk = 2048;
 
-__global__ void __launch_bounds__(kStatThreads) softmax_stats_kernel(const float* __restrict__ logits,
+__global__ void __launch_bounds__(kStatThreads) softmax_stats_kernel(const float* logits,
                                                                      int V, float T,
-                                                                     float2* __restrict__ stats) {
+                                                                     float2* stats) {
   __shared__ float red[kStatThreads / 32];
   pdl_trigger();
   pdl_wait();
@@ -64,10 +64,10 @@ __device__ __forceinline__ float prob(const float* row, float2 st, int v, float 
   return __fdiv_rn(expf(__fsub_rn(__fdiv_rn(row[v], T), st.x)), st.y);
 }
 
-__global__ void sampled_accept_kernel(int B, int k, int V, float T, const float* __restrict__ lt,
-                                      const float2* __restrict__ st_t, const float* __restrict__ ld,
-                                      const float2* __restrict__ st_d, const int32_t* __restrict__ drafts,
-                                      const float* __restrict__ u, int32_t* __restrict__ a_out,
+__global__ void sampled_accept_kernel(int B, int k, int V, float T, const float* lt,
+                                      const float2* st_t, const float* ld,
+                                      const float2* st_d, const int32_t* drafts,
+                                      const float* u, int32_t* a_out,
                                       unsigned* status) {
   pdl_trigger();
   pdl_wait();
@@ -91,9 +91,9 @@ __global__ void sampled_accept_kernel(int B, int k, int V, float T, const float*
 }
 
 __global__ void __launch_bounds__(kDrawThreads) sampled_draw_kernel(
-    int k, int V, float T, const float* __restrict__ lt, const float2* __restrict__ st_t,
-    const float* __restrict__ ld, const float2* __restrict__ st_d, const int32_t* __restrict__ a_arr,
-    const float* __restrict__ g, unsigned long long* __restrict__ keys) {
+    int k, int V, float T, const float* lt, const float2* st_t,
+    const float* ld, const float2* st_d, const int32_t* a_arr,
+    const float* g, unsigned long long* keys) {
   __shared__ unsigned long long best_w[kDrawThreads / 32];
   pdl_trigger();
   pdl_wait();
@@ -127,9 +127,9 @@ __global__ void __launch_bounds__(kDrawThreads) sampled_draw_kernel(
   }
 }
 
-__global__ void sampled_finish_kernel(int B, int k, const int32_t* __restrict__ drafts,
-                                      const int32_t* __restrict__ a_arr,
-                                      unsigned long long* __restrict__ keys, int32_t* seq_lens,
+__global__ void sampled_finish_kernel(int B, int k, const int32_t* drafts,
+                                      const int32_t* a_arr,
+                                      unsigned long long* keys, int32_t* seq_lens,
                                       int32_t* accept_len, int32_t* emitted, int32_t* new_last) {
   pdl_trigger();
   pdl_wait();
