@@ -20,6 +20,7 @@
 #include <math.h>
 
 #include <algorithm>
+#include <cstdlib>
 
 #include "common.cuh"
 #include "internal.h"
@@ -679,6 +680,22 @@ cudaError_t launch_rope_append(const RopeAppend& a, int B, cudaStream_t st) {
                   dim3(kRopeThreads), 0, st, a);
 }
 
+// 16-row MMA tiles per CTA of the mma.sync kernel.  One tile (16 query rows)
+// per CTA by default: the row blocks of a KV head re-read its keys, mostly
+// from L2, but the lighter CTAs (fewer registers and accumulators) let
+// several share an SM and hide the mma.sync latency chains.  With 40 rows per
+// KV head (batch 8, 32/4 heads, k 4) the split kernel takes 264 us with one
+// tile, 289 with two and 305 with three (everything in one CTA).
+// SPECVERIFY_ATTN_MT_MAX (1..4) sets the cap.
+int attn_mt(int rows) {
+  static const int cap = [] {
+    const char* v = getenv("SPECVERIFY_ATTN_MT_MAX");
+    const int c = v ? atoi(v) : 1;
+    return c < 1 ? 1 : (c > 4 ? 4 : c);
+  }();
+  return std::min(cap, (rows + 15) / 16);
+}
+
 AttnGeom plan_attn(int B, int q, int Hq, int Hkv, int D, int page, int num_pages, int max_pages,
                    int window, int kv_equal, int sb_width, int split_tokens) {
   AttnGeom g{};
@@ -697,7 +714,7 @@ AttnGeom plan_attn(int B, int q, int Hq, int Hkv, int D, int page, int num_pages
   g.rows = (Hq / Hkv) * q;
   g.qpos_off = 0;
   g.kend_off = q - 1;
-  const int mt = std::min(4, (g.rows + 15) / 16);
+  const int mt = attn_mt(g.rows);
   g.row_blocks = (g.rows + mt * 16 - 1) / (mt * 16);
   if (window > 0) {
     // keys of the rows span at most window + q - 1 positions: that many
@@ -748,7 +765,7 @@ cudaError_t launch_attention(const AttnGeom& g, const uint16_t* qrot, const void
   a.part_ml = part + slots * g.head_dim;
   a.status = status;
   a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)g.head_dim));
-  const int mt = std::min(4, (g.rows + 15) / 16);
+  const int mt = attn_mt(g.rows);
   cudaError_t e;
   if (attn_tc_supported(g)) {
     e = launch_attn_tc(g, tk, tv, qrot, block_table, seq_lens, a.part_o, a.part_ml, status,
