@@ -54,6 +54,9 @@ def parse():
                     help="with --draft: the cheap clustered unembedding picks each draft token")
     ap.add_argument("--sweep", action="store_true",
                     help="verify-step time over batch x k on the b1_ctx8k model; one JSON line")
+    ap.add_argument("--split-tokens", type=str, default=None,
+                    help="tuning: split size of every sliding-window / global layer, 'LOCAL,GLOBAL' "
+                         "(recorded in config)")
     ap.add_argument("--profile-case", action="store_true",
                     help="shrink the vocabulary to 4096 (attention and projection shapes kept) "
                          "so that a profiler capture of the layer kernels holds little device "
@@ -249,6 +252,11 @@ def run_cuda(args, rank, world, local_rank):
     wl = W.get_workload(args.workload)
     if args.profile_case:
         wl = wl.with_(vocab=4096)
+    if args.split_tokens:
+        import dataclasses
+        loc, glo = (int(x) for x in args.split_tokens.split(","))
+        wl = wl.with_(layers=tuple(dataclasses.replace(s, split_tokens=(loc if s.window else glo))
+                                   for s in wl.layers))
     B.lib()
     fixture = os.path.join(ROOT, "tests", "golden", f"verify_{wl.name}.json")
     if args.profile_case:
@@ -708,6 +716,7 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
             "config": {"workload": wl.name, "batch": wl.batch, "k": wl.k,
+                       "split_tokens": [s.split_tokens or wl.split_tokens for s in wl.layers],
                        "context": [int(x) for x in r["lens"]], "layers": len(wl.layers),
                        "d_model": wl.d_model, "vocab": wl.vocab,
                        "l2": f"flushed ({L2_FLUSH_BYTES >> 20} MiB write) before every timed step",

@@ -87,7 +87,7 @@ WORKLOADS = {
     # Batch 8 ragged 4k-32k, global key-equals-value layer only.
     "b8_ragged": Workload("b8_ragged", batch=8, k=4, d_model=5376, n_q_heads=32, n_kv_heads=4,
                           head_dim=256, vocab=262144, layers=(GLOBAL_KV,), ctx_lo=4096,
-                          ctx_hi=32768, accept=("geometric", 0.8), split_tokens=512),
+                          ctx_hi=32768, accept=("geometric", 0.8), split_tokens=1024),
     # Batch 64, k=3, 5 sliding-window layers + 1 key-equals-value global layer.
     # (64 sequences x 8 KV heads already fill the GPU: long splits keep the
     #  split-combine traffic small)
