@@ -152,6 +152,7 @@ struct AttnArgs {
   int q, Hq, Hkv, G, max_pages, num_pages, window, split, n_splits_grid, rows, n_rot;
   int qpos_off;   // row i of a sequence sits at position L + qpos_off + i
   int kend_off;   // its last cached key is at position L + kend_off
+  int row_blocks; // row blocks of a KV head (blockIdx.x = split * row_blocks + block)
   const uint16_t* qrot;
   const int32_t* block_table;
   const int32_t* seq_lens;
@@ -193,7 +194,10 @@ __global__ void __launch_bounds__(kThreads) attn_split_kernel(
   pdl_trigger();
   pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int b = blockIdx.z, kvh = blockIdx.y % a.Hkv, rb = blockIdx.y / a.Hkv;
+  // the row blocks of one split are neighbours in the grid, so the CTAs that
+  // read the same keys run together and share them through L2
+  const int b = blockIdx.z, kvh = blockIdx.y;
+  const int sidx = blockIdx.x / a.row_blocks, rb = blockIdx.x % a.row_blocks;
   const int L = a.seq_lens[b];
   if (L < 0 || L + a.q > a.max_pages * kPage) {
     if (threadIdx.x == 0 && blockIdx.x == 0 && kvh == 0 && rb == 0)
@@ -202,7 +206,7 @@ __global__ void __launch_bounds__(kThreads) attn_split_kernel(
   }
   int klo, khi;
   seq_key_range(L, a, klo, khi);
-  const int s_abs = klo / a.split + blockIdx.x;
+  const int s_abs = klo / a.split + sidx;
   if (s_abs * a.split > khi) return;  // beyond this sequence's last split
   const int lo = max(s_abs * a.split, klo);
   const int hi = min(s_abs * a.split + a.split - 1, khi);
@@ -227,7 +231,8 @@ __global__ void __launch_bounds__(kThreads) attn_split_kernel(
     if (lane == 0) {
       prefetch_tmap(&tk);
       prefetch_tmap(&tv);
-      const uint64_t pol = policy_evict_first();
+      // streamed once: evict first; shared by the split's row blocks: normal
+      const uint64_t pol = a.row_blocks > 1 ? policy_evict_normal() : policy_evict_first();
       int issued = 0;
       for (int it = 0; it < np; ++it) {
         const int s = it % C::kStages;
@@ -499,7 +504,7 @@ __global__ void __launch_bounds__(kThreads) attn_split_kernel(
   if (*fail) return;
 
   // ---- publish the partial (o unnormalised, m and l in the log2 domain)
-  const long slot = ((long)(b * a.Hkv + kvh) * a.n_splits_grid + blockIdx.x) * a.rows;
+  const long slot = ((long)(b * a.Hkv + kvh) * a.n_splits_grid + sidx) * a.rows;
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
@@ -653,7 +658,7 @@ cudaError_t launch_split(const AttnGeom& g, const CUtensorMap& tk, const CUtenso
   const int smem = ACfg<D, MT, KVEQ>::kSmem;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  return launch_k(kern, dim3(g.n_splits_grid, g.n_kv_heads * g.row_blocks, g.B), dim3(kThreads),
+  return launch_k(kern, dim3(g.n_splits_grid * g.row_blocks, g.n_kv_heads, g.B), dim3(kThreads),
                   smem, st, tk, tv, a);
 }
 
@@ -754,6 +759,7 @@ cudaError_t launch_attention(const AttnGeom& g, const uint16_t* qrot, const void
   a.split = g.split_tokens;
   a.qpos_off = g.qpos_off;
   a.kend_off = g.kend_off;
+  a.row_blocks = g.row_blocks;
   a.n_splits_grid = g.n_splits_grid;
   a.rows = g.rows;
   a.n_rot = g.sb_width / 2;
