@@ -122,6 +122,11 @@ WORKLOADS.update({
                                                 vocab=4100, ctx_lo=60, ctx_hi=700,
                                                 layers=(LayerSpec(window=200, split_tokens=64),
                                                         GLOBAL_KV)),
+    # the largest draft count the library takes: 17 verify rows
+    "small_b1_k16": WORKLOADS["b1_ctx8k"].with_(name="small_b1_k16", k=16, vocab=9000, ctx_lo=1500,
+                                                  ctx_hi=1500,
+                                                  layers=(LayerSpec(window=300, split_tokens=128),
+                                                          GLOBAL_KV)),
     "small_loop": WORKLOADS["loop_131k"].with_(name="small_loop", vocab=6000, d_model=512,
                                                 ctx_lo=700, ctx_hi=700, prompt_tokens=700,
                                                 layers=(LayerSpec(window=128),) * 3 + (GLOBAL_KV,),

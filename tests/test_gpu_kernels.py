@@ -194,7 +194,8 @@ def _run_step(wl, cases):
     return s, s.outputs()
 
 
-@pytest.mark.parametrize("name", ["tiny", "small_b1", "small_ragged", "small_b16", "small_b32"])
+@pytest.mark.parametrize("name", ["tiny", "small_b1", "small_ragged", "small_b16", "small_b32",
+                                  "small_b1_k16"])
 def test_verify_step_matches_oracle(name):
     wl = W.get_workload(name)
     model = harness.oracle_model(wl)
