@@ -405,15 +405,11 @@ GemmPlan plan_gemm(int M, int N, int K, int mode) {
       const int t = v ? atoi(v) : 0;
       return t > 0 ? t : 148;   // one CTA per SM of a B200
     }();
-    // the tensor-memory path (more rows) has its own target: its split
-    // partials are M x N floats per split
-    static const int tc_target = [] {
-      const char* v = getenv("SPECVERIFY_TC_SPLIT_TARGET");
-      const int t = v ? atoi(v) : 0;
-      return t > 0 ? t : 100;   // measured at 256 rows: 2 splits of the QKV GEMM beat 3
-    }();
-    const int tgt = tc_supported(M) ? tc_target : target;
-    int s = (tgt + p.n_tiles - 1) / p.n_tiles;
+    // One target for both GEMM paths: the K partition must not depend on M,
+    // so a row's sums (and the bits of its cache entries and logits) are the
+    // same whatever k is (a separate target for the many-row path was 2%
+    // faster at 256 rows but broke that).
+    int s = (target + p.n_tiles - 1) / p.n_tiles;
     s = std::min(s, std::max(1, p.kchunks / 4));
     p.splits = std::max(1, s);
   }
