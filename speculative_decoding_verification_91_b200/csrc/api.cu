@@ -156,17 +156,6 @@ T* at(void* ws, size_t off) {
 
 inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? SPEC_OK : SPEC_ECUDA; }
 
-// LM-head bytes the first kernel of a forward asks L2 to prefetch
-// (SPECVERIFY_LM_PREFETCH_MB, 0 = none).
-size_t lm_prefetch_bytes() {
-  static const size_t b = [] {
-    const char* v = getenv("SPECVERIFY_LM_PREFETCH_MB");
-    const long mb = v ? atol(v) : 0;
-    return (size_t)(mb > 0 ? mb : 0) << 20;
-  }();
-  return b;
-}
-
 // Profiling events: per recorded step {step start, LM-head start, LM-head
 // stop, step stop}.
 struct Prof {
@@ -242,8 +231,7 @@ int run_forward(const spec_model* m, const int32_t* block_table, int max_pages, 
   float2* rope_tab = at<float2>(ws, s.rope_tab);
   rc = cuda_status(launch_embed_norm(m->w_embed, m->vocab, d, io.last_token, io.drafts, io.tokens,
                                      B, q, m->rms_eps, x, hn, hdr.status, seq_lens, inv_freq, D / 2,
-                                     rope_tab, st, m->w_lm,
-                                     std::min(lm_prefetch_bytes(), (size_t)m->vocab * d * 2)));
+                                     rope_tab, st));
   if (rc) return rc;
   detail_mark(st);
   for (int l = 0; l < m->n_layers; ++l) {

@@ -127,8 +127,7 @@ cudaError_t launch_embed_norm(const void* w_emb, int vocab, int d, const int32_t
                               const int32_t* drafts, const int32_t* tokens_flat, int B, int q,
                               double eps, float* x, uint16_t* out, unsigned* status,
                               const int32_t* seq_lens, const double* inv_freq, int half,
-                              float2* rope_tab, cudaStream_t st,
-                              const void* prefetch = nullptr, size_t prefetch_bytes = 0);
+                              float2* rope_tab, cudaStream_t st);
 // Prefill commit: seq_lens[b] += n; next_token[b] = ids[b]; next_max[b] = maxv[b] (if set).
 cudaError_t launch_prefill_commit(const int32_t* ids, const float* maxv, int B, int n,
                                   int32_t* seq_lens, int32_t* next_token, float* next_max,

@@ -52,24 +52,9 @@ __global__ void __launch_bounds__(kNormThreads) embed_norm_kernel(
     const int32_t* drafts, const int32_t* tokens_flat, int q, double eps,
     float* x, uint16_t* out, unsigned* status,
     const int32_t* seq_lens, InvFreq inv_freq, int half,
-    float2* rope_tab, int n_rows, int tab_blocks, const uint8_t* pf, size_t pf_bytes) {
+    float2* rope_tab, int n_rows) {
   __shared__ double red[kNormThreads / 32];
   pdl_trigger();
-  if ((int)blockIdx.x >= n_rows + tab_blocks) {
-    // blocks past the rows and the table: ask L2 to fetch the first pf_bytes
-    // of the LM-head weights (never written, so no wait) with high retention,
-    // while the latency-bound layer kernels leave HBM mostly idle; the LM
-    // head later finds those tiles in L2
-    const size_t chunk = 64u << 10;
-    const size_t c = ((size_t)(blockIdx.x - n_rows - tab_blocks) * kNormThreads + threadIdx.x) * chunk;
-    if (c < pf_bytes) {
-      const uint32_t n = (uint32_t)min(chunk, pf_bytes - c);
-      asm volatile("cp.async.bulk.prefetch.L2.global.L2::cache_hint [%0], %1, %2;" ::"l"(pf + c),
-                   "r"(n), "l"(policy_evict_last())
-                   : "memory");
-    }
-    return;
-  }
   pdl_wait();
   if ((int)blockIdx.x >= n_rows) {
     // blocks past the rows: the (cos, sin) table, one (row, pair) per thread,
@@ -186,22 +171,16 @@ cudaError_t launch_embed_norm(const void* w_emb, int vocab, int d, const int32_t
                               const int32_t* drafts, const int32_t* tokens_flat, int B, int q,
                               double eps, float* x, uint16_t* out, unsigned* status,
                               const int32_t* seq_lens, const double* inv_freq, int half,
-                              float2* rope_tab, cudaStream_t st, const void* prefetch,
-                              size_t prefetch_bytes) {
+                              float2* rope_tab, cudaStream_t st) {
   InvFreq f{};
   for (int j = 0; j < half && j < 128; ++j) f.v[j] = inv_freq[j];
   // rows, then as many blocks again for the RoPE table (table blocks <= rows
-  // since half <= kNormThreads), then the L2-prefetch blocks (64 KB per thread)
+  // since half <= kNormThreads)
   const int rows = B * q;
   const int tab_blocks = rope_tab ? rows : 0;
-  prefetch_bytes &= ~(size_t)15;   // bulk prefetches move multiples of 16 bytes
-  if (!prefetch || (reinterpret_cast<uintptr_t>(prefetch) & 15)) prefetch_bytes = 0;
-  const size_t per_block = (size_t)kNormThreads * (64u << 10);
-  const int pf_blocks = (int)((prefetch_bytes + per_block - 1) / per_block);
-  return launch_k(embed_norm_kernel, dim3(rows + tab_blocks + pf_blocks), dim3(kNormThreads), 0, st,
+  return launch_k(embed_norm_kernel, dim3(rows + tab_blocks), dim3(kNormThreads), 0, st,
                   static_cast<const uint16_t*>(w_emb), vocab, d, last_token, drafts, tokens_flat, q,
-                  eps, x, out, status, seq_lens, f, half, rope_tab, rows, tab_blocks,
-                  static_cast<const uint8_t*>(prefetch), prefetch_bytes);
+                  eps, x, out, status, seq_lens, f, half, rope_tab, rows);
 }
 
 __global__ void prefill_commit_kernel(const int32_t* ids, const float* maxv,
