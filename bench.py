@@ -258,21 +258,17 @@ def run_cuda(args, rank, world, local_rank):
         wl = wl.with_(layers=tuple(dataclasses.replace(s, split_tokens=(loc if s.window else glo))
                                    for s in wl.layers))
     B.lib()
-    fixture = os.path.join(ROOT, "tests", "golden", f"verify_{wl.name}.json")
     if args.profile_case:
         sess = WorkloadSession(wl, device=dev, poison=False)
         last = np.array([W.last_token(wl, b, 0) for b in range(wl.batch)], dtype=np.int32)
         drafts = np.stack([gen.randint(wl.seed, f"{wl.name}/profile_drafts", b * wl.k, wl.k, 0, wl.vocab)
                            for b in range(wl.batch)]).astype(np.int32)
         inputs = "profile case: vocabulary 4096, random drafts"
-    elif os.path.exists(fixture):
+    elif fixture_inputs(wl) is not None:
         # margin-guarded inputs shared with the parity tests
-        with open(fixture) as f:
-            seqs = json.load(f)["sequences"]
-        sess = WorkloadSession(wl, attempts=[q["attempt"] for q in seqs], device=dev, poison=False)
-        last = np.array([q["last_token"] for q in seqs], dtype=np.int32)
-        drafts = np.array([q["drafts"] for q in seqs], dtype=np.int32)
-        inputs = "margin-guarded fixture " + os.path.relpath(fixture, ROOT)
+        fx = fixture_inputs(wl)
+        sess = WorkloadSession(wl, attempts=fx["attempts"], device=dev, poison=False)
+        last, drafts, inputs = fx["last"], fx["drafts"], fx["inputs"]
     else:
         sess = WorkloadSession(wl, device=dev, poison=False)
         last, drafts = gpu_greedy_drafts(sess, wl, W)
@@ -366,13 +362,43 @@ def run_cuda(args, rank, world, local_rank):
 # CPU oracle leg (baseline only; bounded sample)
 # --------------------------------------------------------------------------
 
+def fixture_inputs(wl):
+    """The margin-guarded step inputs stored for the workload (written by the
+    oracle-only script beside them), or None: per-sequence draw attempts, last
+    tokens, drafts, the emitted-token count of the step and a description."""
+    fixture = os.path.join(ROOT, "tests", "golden", f"verify_{wl.name}.json")
+    if not os.path.exists(fixture):
+        return None
+    with open(fixture) as f:
+        seqs = json.load(f)["sequences"]
+    return dict(attempts=[q["attempt"] for q in seqs],
+                last=np.array([q["last_token"] for q in seqs], dtype=np.int32),
+                drafts=np.array([q["drafts"] for q in seqs], dtype=np.int32),
+                tokens_per_step=int(sum(q["accept_len"] + 1 for q in seqs)),
+                inputs="margin-guarded fixture " + os.path.relpath(fixture, ROOT))
+
+
+def workload_config(wl, lens, tokens_per_step, inputs):
+    """The JSON line's `config`, the same object for both arms."""
+    return {"workload": wl.name, "batch": wl.batch, "k": wl.k,
+            "split_tokens": [s.split_tokens or wl.split_tokens for s in wl.layers],
+            "context": [int(x) for x in lens], "layers": len(wl.layers),
+            "d_model": wl.d_model, "vocab": wl.vocab,
+            "l2": f"flushed ({L2_FLUSH_BYTES >> 20} MiB write) before every timed step",
+            "tokens_per_step": tokens_per_step, "inputs": inputs}
+
+
 def oracle_setup(wl_name: str):
-    """The oracle's model, caches and inputs for sequence 0 of the workload."""
+    """The oracle's model, caches and inputs for sequence 0 of the workload
+    (the stored margin-guarded inputs when the workload has them, as in the
+    CUDA arm)."""
     import oracle
     from speculative_decoding_verification_91_b200.inputs import workloads as W
     from speculative_decoding_verification_91_b200.inputs import gen
     wl = W.get_workload(wl_name)
     L = int(W.context_lengths(wl)[0])
+    fx = fixture_inputs(wl)
+    attempt = fx["attempts"][0] if fx else 0
     layers = []
     for l, spec in enumerate(wl.layers):
         wqkv, wo = W.layer_weights(wl, l)
@@ -383,11 +409,14 @@ def oracle_setup(wl_name: str):
                          W.embedding_weight(wl))
     caches = []
     for l in range(len(wl.layers)):
-        lo, k, v = W.context_kv(wl, 0, 0, l, L)
+        lo, k, v = W.context_kv(wl, 0, attempt, l, L)
         caches.append(oracle.cache_from_raw(model, l, lo, oracle.bf16_from_bits(k),
                                             None if v is None else oracle.bf16_from_bits(v)))
-    last = W.last_token(wl, 0, 0)
-    drafts = gen.randint(wl.seed, f"{wl.name}/bench_drafts", 0, wl.k, 0, wl.vocab)
+    if fx:
+        last, drafts = int(fx["last"][0]), fx["drafts"][0]
+    else:
+        last = W.last_token(wl, 0, 0)
+        drafts = gen.randint(wl.seed, f"{wl.name}/bench_drafts", 0, wl.k, 0, wl.vocab)
     return wl, model, caches, L, last, drafts
 
 
@@ -427,7 +456,13 @@ def run_reference(args):
     desc = (f"oracle on sequence 0 of {wl.name} ({len(wl.layers)} layers, k={wl.k}, ctx {L}, vocab {V}); "
             f"layer stack timed once ({t_layers:.2f} s), each step times the LM head on {n_slice} "
             f"of {V} tokens and scales it to the vocabulary; numpy float64, BLAS threads={threads}")
-    return tps, sec, threads, desc
+    if wl.batch > 1:
+        desc += f"; the metric is sequence 0's emitted tokens over its step time (batch {wl.batch})"
+    from speculative_decoding_verification_91_b200.inputs import workloads as W
+    fx = fixture_inputs(wl)
+    config = workload_config(wl, W.context_lengths(wl), fx["tokens_per_step"] if fx else tokens_per_step,
+                             fx["inputs"] if fx else "attempt-0 draws; random drafts")
+    return tps, sec, threads, desc, config
 
 
 def oracle_sample(wl_name: str, budget_s: float = 25.0):
@@ -435,25 +470,7 @@ def oracle_sample(wl_name: str, budget_s: float = 25.0):
     step (all layers, all k+1 rows, full-vocabulary LM head).  Returns
     (tokens/s, seconds, threads, description)."""
     import oracle
-    from speculative_decoding_verification_91_b200.inputs import workloads as W
-    from speculative_decoding_verification_91_b200.inputs import gen
-    wl = W.get_workload(wl_name)
-    L = int(W.context_lengths(wl)[0])
-    layers = []
-    for l, spec in enumerate(wl.layers):
-        wqkv, wo = W.layer_weights(wl, l)
-        layers.append(oracle.LayerDef(spec.window, spec.kv_equal, spec.rope_fraction,
-                                      oracle.bf16_from_bits(wqkv), oracle.bf16_from_bits(wo)))
-    model = oracle.Model(wl.d_model, wl.n_q_heads, wl.n_kv_heads, wl.head_dim,
-                         W.lm_head_weight(wl), layers, wl.rope_theta, wl.rms_eps,
-                         W.embedding_weight(wl))
-    caches = []
-    for l in range(len(wl.layers)):
-        lo, k, v = W.context_kv(wl, 0, 0, l, L)
-        caches.append(oracle.cache_from_raw(model, l, lo, oracle.bf16_from_bits(k),
-                                            None if v is None else oracle.bf16_from_bits(v)))
-    last = W.last_token(wl, 0, 0)
-    drafts = gen.randint(wl.seed, f"{wl.name}/bench_drafts", 0, wl.k, 0, wl.vocab)
+    wl, model, caches, L, last, drafts = oracle_setup(wl_name)
     t0 = time.perf_counter()
     n = 0
     tokens = 0
@@ -738,12 +755,12 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        tps, sec, threads, desc = run_reference(args)
+        tps, sec, threads, desc, config = run_reference(args)
         line = {"metric": METRIC, "value": tps, "unit": "tokens/s", "n_gpus": args.gpus,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
                 "data": "synthetic", "impl": "reference",
-                "config": {"workload": args.workload},
+                "config": config,
                 "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": threads,
                                  "kind": "oracle", "sample": desc},
                 "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -773,12 +790,7 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["mean_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": wl.name, "batch": wl.batch, "k": wl.k,
-                       "split_tokens": [s.split_tokens or wl.split_tokens for s in wl.layers],
-                       "context": [int(x) for x in r["lens"]], "layers": len(wl.layers),
-                       "d_model": wl.d_model, "vocab": wl.vocab,
-                       "l2": f"flushed ({L2_FLUSH_BYTES >> 20} MiB write) before every timed step",
-                       "tokens_per_step": r["tokens_per_step"], "inputs": r["inputs"]},
+            "config": workload_config(wl, r["lens"], r["tokens_per_step"], r["inputs"]),
             "us_per_step": r["mean_step"] * 1e3,
             "step_hbm": {"bytes": step_bytes, "bytes_with_projections": step_bytes + r["proj_b"],
                          "gbs": step_bytes / step_s / 1e9,
