@@ -49,6 +49,10 @@
  * are asynchronous on the given stream (cudaStream_t passed as void*; NULL =
  * legacy default stream).  bf16 tensors are raw 16-bit bfloat16 patterns.
  *
+ * Empty work: a batch of zero sequences (B < 1) or zero rows (M < 1) is an
+ * invalid argument (SPEC_EINVAL, nothing launched), not a no-op; k = 0 (no
+ * drafts) is valid and is one plain greedy decode step.
+ *
  * Errors: arguments are validated on the host before any launch; on error
  * the call returns a negative spec_status and launches nothing (the cache is
  * untouched).  A launch failure returns SPEC_ECUDA.  Conditions only the

@@ -98,6 +98,22 @@ def test_invalid_arguments_are_rejected_before_any_launch(lib):
     assert L.spec_cache_write(pm, 0, FAKE, 2, 100, 60, FAKE, None, None) == B.SPEC_EINVAL
 
 
+def test_empty_batches_are_invalid_arguments(lib):
+    m = _model()
+    pm = ctypes.byref(m)
+    assert lib.spec_verify_step(pm, FAKE, 10, FAKE, FAKE, 0, 4, FAKE, FAKE, FAKE, FAKE, None, None,
+                                FAKE, 1 << 30, None) == B.SPEC_EINVAL
+    assert lib.spec_lmhead_argmax(FAKE, FAKE, 0, 512, 1000, FAKE, None, FAKE, 1 << 20,
+                                  None) == B.SPEC_EINVAL
+    assert lib.spec_lmhead_argmax(FAKE, FAKE, 4, 512, 0, FAKE, None, FAKE, 1 << 20,
+                                  None) == B.SPEC_EINVAL
+    assert lib.spec_accept_commit(FAKE, FAKE, 0, 4, FAKE, FAKE, FAKE, FAKE, None) == B.SPEC_EINVAL
+    assert lib.spec_verify_attn(pm, 0, FAKE, FAKE, FAKE, FAKE, 10, FAKE, 0, 4, FAKE, FAKE, 1 << 30,
+                                None) == B.SPEC_EINVAL
+    assert lib.spec_workspace_bytes(pm, 0, 4, 10) == 0
+    assert lib.spec_lmhead_workspace_bytes(0, 1000) == 0
+
+
 def test_unsupported_shapes_are_reported(lib):
     m = _model(D=192)
     assert lib.spec_verify_step(ctypes.byref(m), FAKE, 10, FAKE, FAKE, 1, 4, FAKE, FAKE, FAKE, FAKE,
