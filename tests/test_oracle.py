@@ -326,7 +326,11 @@ def test_forward_degenerate_zero_output_projection():
     E = torch.from_numpy(oracle.bf16_from_bits(m.w_lm_bits).astype(np.float64))
     hn = torch.nn.functional.rms_norm(E[toks], (m.d_model,), eps=1e-6)
     hn = torch.from_numpy(oracle.bf16(hn.numpy()).astype(np.float64))
-    assert np.array_equal(fw.g, (hn @ E.T).argmax(dim=1).numpy())
+    lg = hn @ E.T
+    assert np.array_equal(fw.g, lg.argmax(dim=1).numpy())
+    # the logit values too (an argmax alone cannot see a missing final norm,
+    # which only rescales each row); binary32 rounding of each logit
+    np.testing.assert_allclose(fw.top1, lg.max(dim=1).values.numpy(), rtol=1e-6)
 
 
 def _loop_model(seed):

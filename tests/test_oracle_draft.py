@@ -204,6 +204,24 @@ def test_cheap_unembed_keeps_the_best_clusters(n_select):
         assert ids[m] == cand[j] and t1[m] == float(lg[j])
 
 
+def test_cheap_unembed_tie_at_the_kept_boundary_keeps_the_lower_cluster_id():
+    # clusters 5 and 9 share the same centroid, aligned with h, so they tie
+    # for first place far above every other cluster; keeping one cluster
+    # must keep cluster 5, and the argmax then lies among its tokens
+    r = _rng(31)
+    V, S, d = 203, 8, 12
+    w = _bits(r.standard_normal((V, d)))
+    t = _tables(V, S, d, n_select=1)
+    h = OV.bf16(r.standard_normal((2, d)))
+    for m in range(2):
+        t.centroids_bits[5] = t.centroids_bits[9] = _bits(h[m] * 8.0)
+        cent = OV.bf16_from_bits(t.centroids_bits).astype(np.float64)
+        cl = cent @ h[m].astype(np.float64)
+        assert cl[5] == cl[9] and np.sum(cl >= cl[5]) == 2       # the tie is for first place
+        ids, _, _ = OD.cheap_unembed(h[m:m + 1], w, t)
+        assert ids[0] in set(int(x) for x in t.cluster_tokens[5] if x >= 0)
+
+
 def test_draft_step_with_clusters_uses_them():
     model, L = _model(0, False, 1.0), 9
     cache, dr = _cache(model, L), _drafter()

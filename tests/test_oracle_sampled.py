@@ -6,6 +6,8 @@ Monte Carlo on a tiny vocabulary (drafts drawn from the draft distribution,
 fresh uniforms per trial), together with the Gumbel-max draw's frequencies
 and the special cases p = q (every draft accepted) and p(d) = 0 (rejected).
 """
+import math
+
 import numpy as np
 import pytest
 
@@ -14,6 +16,18 @@ from oracle import sampled as OS
 
 def _rng(seed):
     return np.random.default_rng(seed)
+
+
+def test_softmax_temperature_closed_forms():
+    # logits (0, ln 2): weights 1 : 2 at T = 1, 1 : 4 at T = 1/2, 1 : sqrt 2 at T = 2
+    lg = np.array([[0.0, math.log(2.0)]])
+    np.testing.assert_allclose(OS.softmax(lg, 1.0), [[1 / 3, 2 / 3]], rtol=1e-15)
+    np.testing.assert_allclose(OS.softmax(lg, 0.5), [[1 / 5, 4 / 5]], rtol=1e-15)
+    r2 = math.sqrt(2.0)
+    np.testing.assert_allclose(OS.softmax(lg, 2.0), [[1 / (1 + r2), r2 / (1 + r2)]], rtol=1e-15)
+    # a common shift leaves it unchanged (up to the rounding of 1000 + ln 2);
+    # large logits do not overflow
+    np.testing.assert_allclose(OS.softmax(lg + 1000.0, 0.5), [[1 / 5, 4 / 5]], rtol=1e-12)
 
 
 def test_gumbel_draw_frequencies_follow_the_weights():
