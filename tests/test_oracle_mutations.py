@@ -142,6 +142,9 @@ CASES = [
      [_pin(TS.test_emitted_tokens_follow_the_target_distribution, 1.0)]),
     ("gumbel_sign", OS, "gumbel_draw", "np.log(w) - np.log(-np.log(g))", "np.log(w) + np.log(-np.log(g))",
      [_pin(TS.test_gumbel_draw_frequencies_follow_the_weights)]),
+    ("logits_chunk_misaligned", OS, "full_logits", "out[:, v0:v0 + chunk] = f32(h @ bf16_from_bits(w_bits[v0:v0 + chunk])",
+     "out[:, v0:v0 + chunk] = f32(h @ bf16_from_bits(w_bits[v0 + 1:v0 + chunk + 1])",
+     [_pin(TS.test_full_logits_match_torch_and_the_argmax_head)]),
     ("temperature_ignored", OS, "softmax", "z = np.asarray(logits, dtype=np.float64) / T",
      "z = np.asarray(logits, dtype=np.float64)", [_pin(TS.test_softmax_temperature_closed_forms)]),
 ]

@@ -30,6 +30,20 @@ def test_softmax_temperature_closed_forms():
     np.testing.assert_allclose(OS.softmax(lg + 1000.0, 0.5), [[1 / 5, 4 / 5]], rtol=1e-12)
 
 
+def test_full_logits_match_torch_and_the_argmax_head():
+    from oracle import verify as OV
+    import torch
+    r = _rng(5)
+    h = OV.bf16(r.standard_normal((3, 40)))
+    wb = OV.bits_from_bf16(r.standard_normal((2100, 40)) * 0.05)
+    lg = OS.full_logits(h, wb, chunk=512)
+    ref = (torch.from_numpy(h.astype(np.float64)) @
+           torch.from_numpy(OV.bf16_from_bits(wb).astype(np.float64)).T).float().numpy()
+    assert lg.dtype == np.float32 and np.array_equal(lg, ref)       # each logit rounded once
+    ids, top1, _ = OV.lm_head_top2(h, wb, chunk=700)
+    assert np.array_equal(np.argmax(lg, axis=1), ids) and np.array_equal(lg.max(axis=1), top1)
+
+
 def test_gumbel_draw_frequencies_follow_the_weights():
     r = _rng(0)
     w = np.array([0.5, 0.0, 0.2, 0.3])
