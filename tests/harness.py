@@ -43,6 +43,45 @@ def context_caches(wl: W.Workload, model: oracle.Model, b: int, attempt: int, L:
     return caches
 
 
+def snapshot_caches(model: oracle.Model, pools, table_row, L: int, page: int = 64) -> list:
+    """Oracle caches of one sequence rebuilt from the library's paged pools.
+
+    pools[l] = (k_pool, v_pool or None, ksb_pool or None), each [P][Hkv][page][*]
+    bf16 tensors (any device); table_row = the sequence's block-table row; L =
+    its committed length.  Positions [lo, L) are gathered page by page, with
+    lo = L - (window - 1) on sliding-window layers (0 on global ones).  On
+    key-equals-value layers the values (the pre-RoPE keys) are the post-RoPE
+    keys with their rotated dimensions taken from the side-band."""
+    import torch
+    out = []
+    D = model.head_dim
+    half = D // 2
+    table_row = np.asarray(table_row)
+    for l, spec in enumerate(model.layers):
+        k_pool, v_pool, sb_pool = pools[l]
+        lo = max(0, L - (spec.window - 1)) if spec.window > 0 else 0
+        p0, p1 = lo // page, (L + page - 1) // page
+        idx = torch.as_tensor(table_row[p0:p1].astype(np.int64), device=k_pool.device)
+
+        def rows(pool):
+            g = pool.index_select(0, idx)                          # [n_pages][Hkv][page][w]
+            g = g.permute(0, 2, 1, 3).reshape(-1, pool.shape[1], pool.shape[3])
+            bits = g[lo - p0 * page:L - p0 * page].contiguous().view(torch.int16).cpu().numpy()
+            return oracle.bf16_from_bits(bits.view(np.uint16))
+
+        k = rows(k_pool)
+        if spec.kv_equal:
+            n = sb_pool.shape[3] // 2
+            sb = rows(sb_pool)
+            kpre = k.copy()
+            kpre[..., :n] = sb[..., :n]
+            kpre[..., half:half + n] = sb[..., n:]
+            out.append(oracle.LayerCache(lo, k, None, kpre))
+        else:
+            out.append(oracle.LayerCache(lo, k, rows(v_pool), None))
+    return out
+
+
 def greedy_continuation(model, caches, L, last, n):
     """First n greedy tokens after `last` (one oracle forward per token)."""
     toks = [int(last)]
