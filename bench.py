@@ -224,19 +224,20 @@ def attention_bytes(wl, lens, layer):
     return int(kv)
 
 
-def reduce_over_ranks(times, tokens, world, device):
+def reduce_over_ranks(times, tokens, world, device, launches=0):
     """Whole-job figures of a multi-rank run: every time is the maximum over
-    the ranks (the job is as slow as its slowest rank) and the emitted tokens
-    are summed over the ranks.  One all-reduce each; every rank calls it."""
+    the ranks (the job is as slow as its slowest rank); the emitted tokens and
+    the kernel launches of the timed region are summed over the ranks.  One
+    all-reduce each; every rank calls it.  Returns (times, tokens, launches)."""
     if world == 1:
-        return [float(t) for t in times], int(tokens)
+        return [float(t) for t in times], int(tokens), int(launches)
     import torch
     import torch.distributed as dist
     t = torch.tensor([float(x) for x in times], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    n = torch.tensor([float(tokens)], dtype=torch.float64, device=device)
+    n = torch.tensor([float(tokens), float(launches)], dtype=torch.float64, device=device)
     dist.all_reduce(n, op=dist.ReduceOp.SUM)
-    return [float(v) for v in t.tolist()], int(round(n.item()))
+    return [float(v) for v in t.tolist()], int(round(n[0].item())), int(round(n[1].item()))
 
 
 def run_cuda(args, rank, world, local_rank):
@@ -347,8 +348,8 @@ def run_cuda(args, rank, world, local_rank):
     mean_step = float(np.mean(step_ms))
     mean_lm = float(np.mean(lm_ms))
     mean_e2e = float(np.mean(e2e_ms))
-    (mean_step, mean_e2e, mean_lm), tokens_all = reduce_over_ranks(
-        [mean_step, mean_e2e, mean_lm], tokens_per_step, world, dev)
+    (mean_step, mean_e2e, mean_lm), tokens_all, n_launches = reduce_over_ranks(
+        [mean_step, mean_e2e, mean_lm], tokens_per_step, world, dev, n_launches)
     kv_b, lm_b, proj_b = algorithmic_bytes(wl, sess.lens)
     return dict(wl=wl, lens=sess.lens, tokens_per_step=tokens_per_step, tokens_all=tokens_all,
                 mean_step=mean_step, inputs=inputs,

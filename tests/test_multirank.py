@@ -1,7 +1,7 @@
 """Multi-rank host logic of bench.py on CPU: two gloo ranks reduce their
-step times (maximum over ranks) and emitted tokens (sum over ranks) the way
-the N-GPU benchmark does; the aggregate throughput is whole-job tokens over
-the slowest rank's time."""
+step times (maximum over ranks), emitted tokens and kernel launches (sums
+over ranks) the way the N-GPU benchmark does; the aggregate throughput is
+whole-job tokens over the slowest rank's time."""
 import os
 import socket
 import sys
@@ -27,9 +27,10 @@ def _rank(rank, world, port):
     try:
         times = [1.0 + rank, 10.0 - rank, 0.5 * (rank + 1)]   # step, e2e, lm (ms)
         tokens = 3 + 2 * rank
-        got, total = bench.reduce_over_ranks(times, tokens, world, "cpu")
+        got, total, launches = bench.reduce_over_ranks(times, tokens, world, "cpu", 12 * (rank + 1))
         assert got == [float(world), 10.0, 0.5 * world], got
         assert total == sum(3 + 2 * r for r in range(world)), total
+        assert launches == sum(12 * (r + 1) for r in range(world)), launches
         # every rank sees the same whole-job figures
         value = total / (got[0] / 1e3)
         assert abs(value - 8 / 2e-3) < 1e-6 if world == 2 else True
@@ -44,5 +45,5 @@ def test_two_gloo_ranks_reduce_like_the_benchmark():
 def test_single_rank_is_identity():
     sys.path.insert(0, ROOT)
     import bench
-    got, total = bench.reduce_over_ranks([1.5, 2.5], 7, 1, "cpu")
-    assert got == [1.5, 2.5] and total == 7
+    got, total, launches = bench.reduce_over_ranks([1.5, 2.5], 7, 1, "cpu", 24000)
+    assert got == [1.5, 2.5] and total == 7 and launches == 24000
