@@ -259,6 +259,7 @@ def run_cuda(args, rank, world, local_rank):
         wl = wl.with_(layers=tuple(dataclasses.replace(s, split_tokens=(loc if s.window else glo))
                                    for s in wl.layers))
     B.lib()
+    draws = 0
     if args.profile_case:
         sess = WorkloadSession(wl, device=dev, poison=False)
         last = np.array([W.last_token(wl, b, 0) for b in range(wl.batch)], dtype=np.int32)
@@ -266,10 +267,14 @@ def run_cuda(args, rank, world, local_rank):
                            for b in range(wl.batch)]).astype(np.int32)
         inputs = "profile case: vocabulary 4096, random drafts"
     elif fixture_inputs(wl) is not None:
-        # margin-guarded inputs shared with the parity tests
+        # margin-guarded inputs shared with the parity tests; in draws mode
+        # every draw has its own context resident and each timed step runs
+        # one draw (batch 1), cycling through them
         fx = fixture_inputs(wl)
-        sess = WorkloadSession(wl, attempts=fx["attempts"], device=dev, poison=False)
+        sess_wl = wl.with_(batch=len(fx["attempts"])) if fx["draws"] else wl
+        sess = WorkloadSession(sess_wl, attempts=fx["attempts"], device=dev, poison=False)
         last, drafts, inputs = fx["last"], fx["drafts"], fx["inputs"]
+        draws = len(fx["attempts"]) if fx["draws"] else 0
     else:
         sess = WorkloadSession(wl, device=dev, poison=False)
         last, drafts = gpu_greedy_drafts(sess, wl, W)
@@ -280,15 +285,31 @@ def run_cuda(args, rank, world, local_rank):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     ev = lambda: torch.cuda.Event(enable_timing=True)
 
-    # ---- warm-up (untimed), also fixes the emitted-token count of the step
-    for _ in range(args.warmup):
+    def one_step(i, with_targets=False):
+        if draws:
+            sess.step_one(i % draws, stream=stream, with_targets=with_targets)
+        else:
+            sess.step(stream=stream, with_targets=with_targets)
+
+    # ---- warm-up (untimed), then one untimed pass that fixes the emitted-token
+    #      count of every step (of every draw)
+    for i in range(args.warmup):
         sess.reset_lengths()
-        sess.step(stream=stream)
+        one_step(i)
+    sess.reset_lengths()
+    for i in range(max(1, draws)):
+        one_step(i, with_targets=True)
     torch.cuda.synchronize(dev)
     out = sess.outputs()
     if sess.ws.device_status(stream) != 0:
         raise RuntimeError("device status flagged during warm-up")
-    tokens_per_step = int(np.sum(out["accept_len"] + 1))
+    if draws:
+        step_tokens = [int(a) + 1 for a in out["accept_len"]]       # per draw
+        if step_tokens != [int(t) for t in fx["draw_tokens"]]:
+            raise RuntimeError("emitted tokens differ from the stored oracle outcome")
+    else:
+        step_tokens = [int(np.sum(out["accept_len"] + 1))]
+    tokens_timed = sum(step_tokens[i % len(step_tokens)] for i in range(args.steps))
 
     # ---- timed: device-resident inputs, L2 flushed before every step; the
     #      library records its own CUDA events around each step and its
@@ -302,7 +323,7 @@ def run_cuda(args, rank, world, local_rank):
         for i in range(args.steps):
             flush.zero_()
             sess.reset_lengths()
-            sess.step(stream=stream, with_targets=False)
+            one_step(i)
         torch.cuda.synchronize(dev)
     n_launches = B.spec_launch_count() - n_launch0
     step_ms, lm_ms = B.spec_profile_collect(args.steps)
@@ -311,51 +332,63 @@ def run_cuda(args, rank, world, local_rank):
     if sess.ws.device_status(stream) != 0:
         raise RuntimeError("device status flagged during the timed steps")
 
-    # ---- e2e: the public C-ABI call fed from pinned host buffers
+    # ---- e2e: the public C-ABI call fed from pinned host buffers (the step's
+    #      draw's last token, drafts and length in; its acceptance outputs back)
     Bn, k = wl.batch, wl.k
-    h_in = torch.empty(Bn * (2 + k), dtype=torch.int32).pin_memory()
-    h_in[:Bn] = torch.from_numpy(last)
-    h_in[Bn:Bn + Bn * k] = torch.from_numpy(drafts.reshape(-1).astype(np.int32))
-    h_in[Bn + Bn * k:] = torch.from_numpy(sess.lens.astype(np.int32))
-    h_out = torch.empty(Bn * (k + 1) + 3 * Bn, dtype=torch.int32).pin_memory()
+    n_in = max(1, draws)
+    lens_all = sess.lens.astype(np.int32)
+    h_in = torch.empty(n_in, Bn * (2 + k), dtype=torch.int32).pin_memory()
+    for j in range(n_in):
+        sl = slice(j, j + 1) if draws else slice(0, Bn)
+        h_in[j, :Bn] = torch.from_numpy(np.ascontiguousarray(last[sl]))
+        h_in[j, Bn:Bn + Bn * k] = torch.from_numpy(np.ascontiguousarray(drafts[sl]).reshape(-1).astype(np.int32))
+        h_in[j, Bn + Bn * k:] = torch.from_numpy(np.ascontiguousarray(lens_all[sl]))
+    h_out = torch.empty(n_in, Bn * (k + 1) + 3 * Bn, dtype=torch.int32).pin_memory()
     e0 = [ev() for _ in range(args.steps)]
     e1 = [ev() for _ in range(args.steps)]
     torch.cuda.synchronize(dev)
+    q = k + 1
     for i in range(args.steps):
+        j = i % n_in
+        o = j if draws else 0                         # the draw's slot in the session buffers
         flush.zero_()
         e0[i].record(stream)
-        sess.last_token.copy_(h_in[:Bn], non_blocking=True)
-        sess.drafts[:Bn * k].copy_(h_in[Bn:Bn + Bn * k], non_blocking=True)
-        sess.seq_lens.copy_(h_in[Bn + Bn * k:], non_blocking=True)
-        sess.step(stream=stream, with_targets=False)
-        h_out[:Bn * (k + 1)].copy_(sess.emitted, non_blocking=True)
-        h_out[Bn * (k + 1):Bn * (k + 2)].copy_(sess.accept_len, non_blocking=True)
-        h_out[Bn * (k + 2):Bn * (k + 3)].copy_(sess.new_last, non_blocking=True)
-        h_out[Bn * (k + 3):].copy_(sess.seq_lens, non_blocking=True)
+        sess.last_token[o:o + Bn].copy_(h_in[j, :Bn], non_blocking=True)
+        sess.drafts[o * k:(o + Bn) * k].copy_(h_in[j, Bn:Bn + Bn * k], non_blocking=True)
+        sess.seq_lens[o:o + Bn].copy_(h_in[j, Bn + Bn * k:], non_blocking=True)
+        one_step(i)
+        h_out[j, :Bn * q].copy_(sess.emitted[o * q:(o + Bn) * q], non_blocking=True)
+        h_out[j, Bn * q:Bn * (q + 1)].copy_(sess.accept_len[o:o + Bn], non_blocking=True)
+        h_out[j, Bn * (q + 1):Bn * (q + 2)].copy_(sess.new_last[o:o + Bn], non_blocking=True)
+        h_out[j, Bn * (q + 2):].copy_(sess.seq_lens[o:o + Bn], non_blocking=True)
         e1[i].record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = [s.elapsed_time(e) for s, e in zip(e0, e1)]
-    got_acc = h_out[Bn * (k + 1):Bn * (k + 2)].numpy()
-    assert np.array_equal(got_acc, out["accept_len"]), "e2e step disagrees with the device-timed step"
+    for j in range(min(n_in, args.steps)):
+        got_acc = h_out[j, Bn * q:Bn * (q + 1)].numpy()
+        want = out["accept_len"][j:j + 1] if draws else out["accept_len"]
+        assert np.array_equal(got_acc, want), "e2e step disagrees with the device-timed step"
 
     # per-launch breakdown of one extra step (events serialise the launches)
     flush.zero_()
     sess.reset_lengths()
     B.spec_profile_launches(256)
-    sess.step(stream=stream, with_targets=False)
+    one_step(0)
     launch_ms = B.spec_profile_launches_collect(256)
 
     mean_step = float(np.mean(step_ms))
     mean_lm = float(np.mean(lm_ms))
     mean_e2e = float(np.mean(e2e_ms))
     (mean_step, mean_e2e, mean_lm), tokens_all, n_launches = reduce_over_ranks(
-        [mean_step, mean_e2e, mean_lm], tokens_per_step, world, dev, n_launches)
-    kv_b, lm_b, proj_b = algorithmic_bytes(wl, sess.lens)
-    return dict(wl=wl, lens=sess.lens, tokens_per_step=tokens_per_step, tokens_all=tokens_all,
-                mean_step=mean_step, inputs=inputs,
+        [mean_step, mean_e2e, mean_lm], tokens_timed, world, dev, n_launches)
+    lens = sess.lens[:1] if draws else sess.lens
+    kv_b, lm_b, proj_b = algorithmic_bytes(wl, lens)
+    tps = fx["tokens_per_step"] if draws else tokens_timed / args.steps
+    return dict(wl=wl, lens=lens, tokens_per_step=tps, tokens_all=tokens_all,
+                mean_step=mean_step, inputs=inputs, draws=draws,
                 mean_lm=mean_lm, mean_e2e=mean_e2e, kv_b=kv_b, lm_b=lm_b, proj_b=proj_b,
                 launches=n_launches, clocks=clocks.summary(),
-                h2d=int(h_in.numel() * 4), d2h=int(h_out.numel() * 4), step_ms=step_ms,
+                h2d=int(h_in[0].numel() * 4), d2h=int(h_out[0].numel() * 4), step_ms=step_ms,
                 M=wl.batch * wl.q_rows, launch_us=[round(x * 1e3, 1) for x in launch_ms])
 
 
@@ -372,11 +405,20 @@ def fixture_inputs(wl):
         return None
     with open(fixture) as f:
         seqs = json.load(f)["sequences"]
+    with open(fixture) as f:
+        draws = json.load(f).get("mode") == "draws"
+    toks = [q["accept_len"] + 1 for q in seqs]
+    inputs = "margin-guarded fixture " + os.path.relpath(fixture, ROOT)
+    if draws:
+        inputs += (f"; {len(seqs)} draws cycled one per step (batch 1 each), mean emitted tokens "
+                   f"per step {np.mean(toks):.4f}")
     return dict(attempts=[q["attempt"] for q in seqs],
                 last=np.array([q["last_token"] for q in seqs], dtype=np.int32),
                 drafts=np.array([q["drafts"] for q in seqs], dtype=np.int32),
-                tokens_per_step=int(sum(q["accept_len"] + 1 for q in seqs)),
-                inputs="margin-guarded fixture " + os.path.relpath(fixture, ROOT))
+                draws=draws, draw_tokens=toks,
+                # draws: mean emitted tokens of one batch-1 step; else of the batched step
+                tokens_per_step=round(float(np.mean(toks)), 4) if draws else int(sum(toks)),
+                inputs=inputs)
 
 
 def workload_config(wl, lens, tokens_per_step, inputs):
@@ -441,7 +483,9 @@ def run_reference(args):
     g, _, _ = oracle.lm_head_top2(h, model.w_lm_bits)
     t_lm = time.perf_counter() - t0
     a, _, _ = oracle.accept_longest_prefix([int(t) for t in drafts], g)
-    tokens_per_step = a + 1
+    fx = fixture_inputs(wl)
+    # draws mode: the stored draws' mean emitted tokens (each draw's step costs the same)
+    tokens_per_step = fx["tokens_per_step"] if fx and fx["draws"] else a + 1
     V = model.vocab
     budget = max(0.005, 120.0 / max(1, args.steps + args.warmup))
     n_slice = int(min(V, max(1024, V * budget / max(t_lm, 1e-9))))
@@ -738,8 +782,146 @@ def run_draft_bench(args):
                       "l2": "flushed before every timed call", "clocks": clocks.summary()}), flush=True)
 
 
+def loop_drafter(wl, greedy_stream):
+    """The loop workload's corrupted-greedy drafter: draft i of a step is the
+    true greedy token (from the precomputed greedy stream, at the sequence's
+    emitted position) with probability p, else a random id (seeded flips)."""
+    def drafter(step, n_emitted):
+        flips, ids = W_mod().loop_draft_flips(wl, step)
+        out = []
+        for i in range(wl.k):
+            e = n_emitted + i
+            truth = greedy_stream[e] if e < len(greedy_stream) else 0
+            out.append(truth if flips[i] < wl.accept[1] else int(ids[i]))
+        return np.asarray(out, dtype=np.int32)
+    return drafter
+
+
+def W_mod():
+    from speculative_decoding_verification_91_b200.inputs import workloads as W
+    return W
+
+
+def run_loop(args):
+    """--workload loop_131k: the speculative loop after a 131,072-token prompt.
+
+    Untimed: the prompt is prefilled on the GPU (spec_prefill, 256-token
+    chunks) and the greedy stream the drafter corrupts is produced by k = 0
+    steps; then the lengths are rolled back to the prompt.  Timed: the loop's
+    verify steps (min(--steps, 512)), each with drafts built on the host from
+    the tokens emitted so far; L2 flushed before every step.  Per step the
+    library's CUDA events give the device time of spec_verify_step; the e2e
+    figure adds the host->device copy of the step's inputs (last token,
+    drafts) and the device->host copy of its outputs, which the loop needs
+    anyway to build the next drafts.  --warmup steps run first and are rolled
+    back (rollback = resetting the length)."""
+    import torch
+    from speculative_decoding_verification_91_b200 import binding as B
+    from speculative_decoding_verification_91_b200.session import WorkloadSession
+    W = W_mod()
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    wl = W.get_workload(args.workload)
+    steps = max(1, min(args.steps, wl.steps))
+    s = WorkloadSession(wl, fill_context=False, lens=np.zeros(wl.batch, np.int64), device=dev,
+                        poison=False, extra_tokens=wl.prompt_tokens + (steps + args.warmup + 2) * (wl.k + 1))
+    t0 = time.time()
+    nxt, _ = s.prefill(W.prompt_tokens(wl)[None, :])
+    t_prefill = time.time() - t0
+    L0 = int(s.seq_lens[0].item())
+    n_greedy = steps * (wl.k + 1) + 1
+    greedy, _ = s.greedy(nxt, n_greedy)
+    stream_tokens = [int(t) for t in greedy[0]]
+    drafter = loop_drafter(wl, stream_tokens)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    k, q = wl.k, wl.k + 1
+    h_in = torch.empty(1 + k, dtype=torch.int32).pin_memory()
+    h_out = torch.empty(q + 3, dtype=torch.int32).pin_memory()
+
+    def run(n, timed):
+        s.seq_lens.fill_(L0)
+        cur, emitted, accepts = int(nxt[0]), 0, []
+        e0 = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        e1 = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        if timed:
+            B.spec_profile_start(n)
+        for st in range(n):
+            h_in[0] = cur
+            h_in[1:] = torch.from_numpy(drafter(st, emitted))
+            flush.zero_()
+            e0[st].record(stream)
+            s.last_token.copy_(h_in[:1], non_blocking=True)
+            s.drafts[:k].copy_(h_in[1:], non_blocking=True)
+            s.step(stream=stream, with_targets=False)
+            h_out[:q].copy_(s.emitted[:q], non_blocking=True)
+            h_out[q:q + 1].copy_(s.accept_len[:1], non_blocking=True)
+            h_out[q + 1:q + 2].copy_(s.new_last[:1], non_blocking=True)
+            h_out[q + 2:].copy_(s.seq_lens[:1], non_blocking=True)
+            e1[st].record(stream)
+            stream.synchronize()               # the drafter needs this step's tokens
+            a = int(h_out[q])
+            got = [int(x) for x in h_out[:a + 1]]
+            if got != stream_tokens[emitted:emitted + a + 1]:
+                raise RuntimeError(f"loop step {st} emitted tokens that differ from greedy decoding")
+            accepts.append(a)
+            emitted += a + 1
+            cur = int(h_out[q + 1])
+        torch.cuda.synchronize(dev)
+        e2e = [x.elapsed_time(y) for x, y in zip(e0, e1)]
+        dev_ms = B.spec_profile_collect(n)[0] if timed else None
+        return accepts, dev_ms, e2e
+
+    if args.warmup:
+        run(args.warmup, False)
+    n0 = B.spec_launch_count()
+    with ClockSampler(0) as clocks:
+        accepts, dev_ms, e2e = run(steps, True)
+    launches = B.spec_launch_count() - n0
+    if s.ws.device_status(stream) != 0:
+        raise RuntimeError("device status flagged during the loop")
+    tokens = int(sum(a + 1 for a in accepts))
+    total_s = float(np.sum(dev_ms)) / 1e3
+    e2e_s = float(np.sum(e2e)) / 1e3
+    # bytes of each step at its own committed length
+    lens, L = [], L0
+    for a in accepts:
+        lens.append(L)
+        L += a + 1
+    kv = [algorithmic_bytes(wl, [x])[0] for x in lens]
+    _, lm_b, proj_b = algorithmic_bytes(wl, [L0])
+    step_bytes = float(np.mean(kv)) + lm_b
+    mean_step = total_s / steps
+    peak, peak_kind = measured_peaks()
+    value = tokens / total_s
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": 1, "steps": steps,
+            "warmup": args.warmup, "ms_per_step": mean_step * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name, "batch": wl.batch, "k": wl.k,
+                       "prompt": wl.prompt_tokens, "loop_steps": steps,
+                       "context": [L0, L], "layers": len(wl.layers), "d_model": wl.d_model,
+                       "vocab": wl.vocab, "l2": f"flushed ({L2_FLUSH_BYTES >> 20} MiB write) before every step",
+                       "tokens_per_step": tokens / steps,
+                       "inputs": "131,072 random prompt tokens prefilled on the GPU (untimed); "
+                                 "corrupted-greedy drafts (p = 0.8) built on the host each step; "
+                                 "every step's emitted tokens checked against greedy decoding"},
+            "us_per_step": mean_step * 1e6,
+            "step_hbm": {"bytes": step_bytes, "bytes_with_projections": step_bytes + proj_b,
+                         "gbs": step_bytes / mean_step / 1e9,
+                         "frac_of_8tbs": step_bytes / mean_step / 1e9 / NOMINAL_HBM_GBS,
+                         "frac_of_measured": step_bytes / mean_step / 1e9 / peak},
+            "accept_len_mean": float(np.mean(accepts)),
+            "e2e": {"value": tokens / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": int(h_in.numel() * 4),
+                    "d2h_bytes_per_step": int(h_out.numel() * 4)},
+            "gpu_launches": launches, "prefill_s": round(t_prefill, 2), "clocks": clocks.summary()}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
+    if args.workload == "loop_131k" and args.impl == "cuda":
+        run_loop(args)
+        return
     if args.draft:
         run_draft_bench(args)
         return
@@ -783,7 +965,8 @@ def main():
         peak, peak_kind = measured_peaks()
         step_s = r["mean_step"] / 1e3
         lm_s = r["mean_lm"] / 1e3
-        value = r["tokens_all"] / step_s
+        # whole job: tokens emitted over the timed steps (all ranks) / their time
+        value = r["tokens_all"] / (args.steps * step_s)
         lm_bytes = r["lm_b"] + r["M"] * wl.d_model * 2
         step_bytes = r["kv_b"] + r["lm_b"]
         line = {
@@ -798,7 +981,7 @@ def main():
                          "frac_of_8tbs": step_bytes / step_s / 1e9 / NOMINAL_HBM_GBS,
                          "frac_of_measured": step_bytes / step_s / 1e9 / peak},
             "roofline": lm_roofline(wl, r, lm_bytes, lm_s, peak, peak_kind),
-            "e2e": {"value": r["tokens_all"] / (r["mean_e2e"] / 1e3), "unit": "tokens/s",
+            "e2e": {"value": r["tokens_all"] / (args.steps * r["mean_e2e"] / 1e3), "unit": "tokens/s",
                     "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
             "gpu_launches": r["launches"],
             "launch_breakdown_us": dict(zip(launch_labels(wl), r["launch_us"]))

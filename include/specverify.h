@@ -4,7 +4,7 @@
  * The operation: a target model checks k drafted tokens in ONE forward.  The
  * last accepted token and the k drafts run as k+1 causal query rows through
  * grouped-query attention against the KV cache the drafter and the target
- * share; the rows' final hidden states go through the tied LM head and an
+ * share; the rows' final hidden states go through the LM head and an
  * argmax over the vocabulary; the longest prefix of drafts that agrees with
  * the target is accepted, the target's own token at the first disagreement
  * (or after the last draft) is added, and the cache keeps exactly the
@@ -354,26 +354,37 @@ int spec_draft(const spec_model* m, const spec_drafter* d, const int32_t* block_
  * gives only its input and output tensors, a latency-critical loop that
  * cannot take cudaMalloc's implicit device synchronisation.
  *
- * Same operation, arguments and errors as spec_lmhead_argmax, minus the
- * workspace.  Its scratch (one argmax key per row, a completion counter, a
- * status word) is a file-scope __device__ array inside the library, of about
- * 4.5 KiB, that every GPU which loads the library holds until the process
- * exits.
- * Limits: M <= SPEC_NOALLOC_MAX_ROWS and ceil(V / 128) * M <=
- * SPEC_NOALLOC_MAX_TILE_ROWS (so V = 262,144 allows M <= 64); larger
- * problems return SPEC_EUNSUPPORTED and launch nothing.
+ * Same operation and arguments as spec_lmhead_argmax, minus the workspace,
+ * and the same kernels (the tensor-memory GEMM above 32 rows, the streaming
+ * one below).  Its scratch (a status word, the completion counters and one
+ * argmax key per row) is a file-scope __device__ array inside the library,
+ * of 4 KiB + 8 bytes per row, that every GPU which loads the library holds
+ * until the process exits.
+ * Limit: M <= SPEC_NOALLOC_MAX_ROWS (the keys the array holds); larger M
+ * returns SPEC_EUNSUPPORTED and launches nothing.
  *
  * The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture.  Each call clears the counter and status word
- * and keys (an async memset on `stream`) and allocates nothing.  All calls share the
- * one array, which keeps the last call's contents: calls that overlap on the
- * GPU (different streams, or concurrent host threads on one device) race and
- * must be serialised by the caller. */
+ * before any stream capture.  Each call clears the counters and the keys (an
+ * async memset on `stream`) and allocates nothing.  Device-detected errors
+ * (a bounded wait that ran out) set bits in the array's status word, which
+ * calls do not clear: they accumulate until spec_noalloc_read_status reads
+ * and clears them.  All calls share the one array, which keeps the last
+ * call's contents: calls that overlap on the GPU (different streams, or
+ * concurrent host threads on one device) race and must be serialised by the
+ * caller. */
 #define SPEC_NOALLOC_MAX_ROWS 64
-#define SPEC_NOALLOC_MAX_TILE_ROWS 131072
 int spec_lmhead_argmax_noalloc(const void* h, const void* w, int M, int d, int V, int32_t* ids,
                                float* maxlogit, void* stream);
+/* Reads and clears the status word of spec_lmhead_argmax_noalloc's scratch on
+ * the current device (synchronises the stream).  *status receives SPEC_DEV_*
+ * bits; returns SPEC_ETIMEOUT if SPEC_DEV_TIMEOUT was set, SPEC_EDEVICE for
+ * any other bit, else SPEC_OK. */
+int spec_noalloc_read_status(void* stream, unsigned* status);
+/* Fault injection on the host side: ORs `bits` into that status word (one
+ * one-thread kernel on `stream`), so that callers can test their handling of
+ * device-detected errors without making the device fail. */
+int spec_noalloc_inject_status(unsigned bits, void* stream);
 
 /* Timing hook (no counterpart in the pages; measurement only).
  * spec_profile_start(n): the next n spec_verify_step calls record CUDA events

@@ -37,10 +37,10 @@ EXPORTED = [
     "spec_draft_workspace_bytes", "spec_draft",
     "spec_cluster_unembed_workspace_bytes", "spec_cluster_unembed",
     "spec_verify_sampled_workspace_bytes", "spec_verify_step_sampled",
+    "spec_noalloc_read_status", "spec_noalloc_inject_status",
 ]
 SPEC_MAX_PREFILL = 256
 SPEC_NOALLOC_MAX_ROWS = 64
-SPEC_NOALLOC_MAX_TILE_ROWS = 131072
 
 
 class SpecError(RuntimeError):
@@ -127,6 +127,8 @@ def lib():
                                        c_void_p, c_size_t, c_void_p]
         L.spec_lmhead_argmax_noalloc.argtypes = [c_void_p, c_void_p, c_int, c_int, c_int, c_void_p,
                                                  c_void_p, c_void_p]
+        L.spec_noalloc_read_status.argtypes = [c_void_p, POINTER(c_uint)]
+        L.spec_noalloc_inject_status.argtypes = [c_uint, c_void_p]
         L.spec_prefill_workspace_bytes.restype = c_size_t
         L.spec_prefill_workspace_bytes.argtypes = [pm, c_int, c_int, c_int]
         L.spec_prefill.argtypes = [pm, c_void_p, c_int, c_void_p, c_int, c_int, c_void_p, c_void_p,
@@ -264,13 +266,26 @@ def spec_profile_collect(n_steps: int):
 def spec_lmhead_argmax_noalloc(h, w, M, d, V, ids, maxlogit, stream=None) -> int:
     """spec_lmhead_argmax without a workspace: the scratch is a fixed device
     array inside the library, for callers that cannot allocate device memory.
-    Raises SpecError(SPEC_EUNSUPPORTED) when M > 64 or ceil(V/128)*M > 131072."""
+    Raises SpecError(SPEC_EUNSUPPORTED) when M > SPEC_NOALLOC_MAX_ROWS."""
     rc = lib().spec_lmhead_argmax_noalloc(_p(h), _p(w), M, d, V, _p(ids), _p(maxlogit), _s(stream))
     if rc == SPEC_EUNSUPPORTED:
-        raise SpecError(rc, f"spec_lmhead_argmax_noalloc: M={M}, V={V} exceeds the fixed scratch "
-                            f"(M <= {SPEC_NOALLOC_MAX_ROWS}, ceil(V/128)*M <= "
-                            f"{SPEC_NOALLOC_MAX_TILE_ROWS})")
+        raise SpecError(rc, f"spec_lmhead_argmax_noalloc: M={M} exceeds the fixed scratch "
+                            f"(M <= {SPEC_NOALLOC_MAX_ROWS})")
     return _check(rc, "spec_lmhead_argmax_noalloc")
+
+
+def spec_noalloc_read_status(stream=None) -> int:
+    """SPEC_DEV_* bits of spec_lmhead_argmax_noalloc's scratch (read and
+    cleared; synchronises the stream); never raises on bits."""
+    v = c_uint(0)
+    rc = lib().spec_noalloc_read_status(_s(stream), ctypes.byref(v))
+    if rc not in (SPEC_OK, SPEC_EDEVICE, SPEC_ETIMEOUT):
+        raise SpecError(rc, "spec_noalloc_read_status")
+    return int(v.value)
+
+
+def spec_noalloc_inject_status(bits: int, stream=None) -> int:
+    return _check(lib().spec_noalloc_inject_status(bits, _s(stream)), "spec_noalloc_inject_status")
 
 
 def spec_prefill_workspace_bytes(model: SpecModel, max_batch: int, max_n: int, max_pages: int) -> int:

@@ -1,8 +1,8 @@
 // LM head + argmax for callers that cannot allocate device memory.
 //
-// spec_lmhead_argmax needs a caller-provided workspace for its per-tile
-// argmax partials and its completion counter.  Some callers have no way to
-// provide one: code that runs where device allocation is not permitted or
+// spec_lmhead_argmax needs a caller-provided workspace for its per-row argmax
+// keys, its completion counter and its status word.  Some callers have no way
+// to provide one: code that runs where device allocation is not permitted or
 // not wanted (an inference runtime whose memory plan is fixed before the
 // first token and forbids allocations on the decode path, a plugin handed
 // only its input and output tensors by a host framework that owns every
@@ -10,6 +10,9 @@
 // implicit device synchronisation).  spec_lmhead_argmax_noalloc serves them:
 // its scratch is a file-scope __device__ array below, loaded with the
 // library, so the call itself allocates nothing.
+//
+// Layout of the array: the 4 KiB header of every workspace (status word,
+// then the completion counters), then one 64-bit argmax key per row.
 #include <mutex>
 
 #include "../../include/specverify.h"
@@ -22,6 +25,8 @@ namespace {
 constexpr size_t kNoAllocHeader = kWsHeaderBytes;                       // status + counters
 constexpr size_t kNoAllocEntries = (size_t)SPEC_NOALLOC_MAX_ROWS;       // argmax keys (one per row)
 constexpr size_t kNoAllocBytes = kNoAllocHeader + kNoAllocEntries * 8;
+// the status word is the header's first 4 bytes; counters start at word kTicketBase
+constexpr size_t kNoAllocClearFrom = (size_t)kTicketBase * 4;
 
 // One copy per GPU that loads the library; it stays allocated until exit.
 __device__ __align__(256) uint8_t g_lmhead_scratch[kNoAllocBytes];
@@ -47,6 +52,13 @@ int scratch_for_current_device(void** out) {
   return SPEC_OK;
 }
 
+// Host-side fault injection: OR bits into the status word (one thread).
+__global__ void noalloc_inject_kernel(unsigned* status, unsigned bits) {
+  pdl_trigger();
+  pdl_wait();
+  atomicOr(status, bits);
+}
+
 }  // namespace
 }  // namespace sv
 
@@ -56,17 +68,20 @@ extern "C" int spec_lmhead_argmax_noalloc(const void* h, const void* w, int M, i
                                           int32_t* ids, float* maxlogit, void* stream) {
   if (!h || !w || !ids || M < 1 || V < 1 || d < 8 || d % 8) return SPEC_EINVAL;
   if ((reinterpret_cast<uintptr_t>(h) & 15) || (reinterpret_cast<uintptr_t>(w) & 15)) return SPEC_EINVAL;
+  // the fixed scratch holds one argmax key per row
+  if (M > SPEC_NOALLOC_MAX_ROWS) return SPEC_EUNSUPPORTED;
   GemmPlan p = plan_gemm(M, V, d, kGemmArgmax);
-  // The fixed scratch holds one key per row; the tile count is bounded as documented.
-  if (M > SPEC_NOALLOC_MAX_ROWS || (size_t)p.n_tiles * M > (size_t)SPEC_NOALLOC_MAX_TILE_ROWS)
-    return SPEC_EUNSUPPORTED;
   void* scratch = nullptr;
   int rc = scratch_for_current_device(&scratch);
   if (rc) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // The array keeps the previous call's contents: the status word, the
-  // completion counter and the argmax keys must start at zero.
-  if (cudaMemsetAsync(scratch, 0, kNoAllocBytes, st) != cudaSuccess) return SPEC_ECUDA;
+  // The array keeps the previous call's contents: the completion counters and
+  // the argmax keys must start at zero (a call cut short by a timed-out wait
+  // may have left them set).  The status word is kept: its bits accumulate
+  // until spec_noalloc_read_status reads and clears them.
+  if (cudaMemsetAsync(static_cast<uint8_t*>(scratch) + kNoAllocClearFrom, 0,
+                      kNoAllocBytes - kNoAllocClearFrom, st) != cudaSuccess)
+    return SPEC_ECUDA;
   WsHeader hdr = ws_header(scratch);
   GemmBuffers b{};
   b.arg_keys = reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(scratch) + kNoAllocHeader);
@@ -74,5 +89,31 @@ extern "C" int spec_lmhead_argmax_noalloc(const void* h, const void* w, int M, i
   b.maxv = maxlogit;
   b.tickets = hdr.tickets;
   b.status = hdr.status;
-  return launch_gemm(p, kGemmArgmax, h, w, b, st) == cudaSuccess ? SPEC_OK : SPEC_ECUDA;
+  // the same kernel choice as spec_lmhead_argmax (tcgen05 above 32 rows)
+  return launch_gemm_any(p, kGemmArgmax, h, w, b, st) == cudaSuccess ? SPEC_OK : SPEC_ECUDA;
+}
+
+extern "C" int spec_noalloc_read_status(void* stream, unsigned* status) {
+  if (!status) return SPEC_EINVAL;
+  void* scratch = nullptr;
+  int rc = scratch_for_current_device(&scratch);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned v = 0;
+  if (cudaMemcpyAsync(&v, scratch, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess) return SPEC_ECUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return SPEC_ECUDA;
+  if (v && cudaMemsetAsync(scratch, 0, 4, st) != cudaSuccess) return SPEC_ECUDA;
+  *status = v;
+  if (v & SPEC_DEV_TIMEOUT) return SPEC_ETIMEOUT;
+  return v ? SPEC_EDEVICE : SPEC_OK;
+}
+
+extern "C" int spec_noalloc_inject_status(unsigned bits, void* stream) {
+  void* scratch = nullptr;
+  int rc = scratch_for_current_device(&scratch);
+  if (rc) return rc;
+  return launch_k(noalloc_inject_kernel, dim3(1), dim3(1), 0, static_cast<cudaStream_t>(stream),
+                  ws_header(scratch).status, bits) == cudaSuccess
+             ? SPEC_OK
+             : SPEC_ECUDA;
 }

@@ -127,6 +127,13 @@ WORKLOADS.update({
                                                   ctx_hi=1500,
                                                   layers=(LayerSpec(window=300, split_tokens=128),
                                                           GLOBAL_KV)),
+    # 40 sequences x 9 rows = 360 verify rows: more rows than one tensor-memory
+    # accumulator holds (256), so every GEMM takes the multi-block path
+    "small_b40_k8": WORKLOADS["b64_6layer"].with_(name="small_b40_k8", batch=40, k=8, d_model=768,
+                                                   vocab=5000, ctx_lo=60, ctx_hi=500,
+                                                   accept=("geometric", 0.8),
+                                                   layers=(LayerSpec(window=200, split_tokens=64),
+                                                           GLOBAL_KV)),
     "small_loop": WORKLOADS["loop_131k"].with_(name="small_loop", vocab=6000, d_model=512,
                                                 ctx_lo=700, ctx_hi=700, prompt_tokens=700,
                                                 layers=(LayerSpec(window=128),) * 3 + (GLOBAL_KV,),
@@ -332,13 +339,17 @@ def rejection_point(wl: Workload, b: int, attempt: int) -> int:
     return r
 
 
-def make_drafts(wl: Workload, b: int, attempt: int, greedy: np.ndarray) -> tuple[np.ndarray, int]:
+def make_drafts(wl: Workload, b: int, attempt: int, greedy: np.ndarray,
+                r: int | None = None) -> tuple[np.ndarray, int]:
     """Drafts from the greedy continuation `greedy` (at least r+1 tokens).
 
     drafts[i] = greedy[i] for i < r; drafts[r] = a random id != greedy[r];
     later drafts are random ids.  one_wrong keeps greedy tokens after the
-    replaced position.  Returns (drafts[k] int32, r)."""
-    r = rejection_point(wl, b, attempt)
+    replaced position.  r defaults to rejection_point(wl, b, attempt); a
+    caller that keeps a sequence's rejection point fixed across redraws of
+    its context passes it.  Returns (drafts[k] int32, r)."""
+    if r is None:
+        r = rejection_point(wl, b, attempt)
     stream = f"{wl.name}/b{b}/t{attempt}/draft_rand"
     ids = gen.randint(wl.seed, stream, 0, 4 * wl.k + 64, 0, wl.vocab)
     drafts = np.empty(wl.k, dtype=np.int32)

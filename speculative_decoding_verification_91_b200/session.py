@@ -85,6 +85,19 @@ class WorkloadSession:
                            self.target_max if with_targets else None,
                            self.ws.buf, self.ws.nbytes, stream)
 
+    def step_one(self, b: int, stream=None, with_targets=True):
+        """One batch-1 spec_verify_step on sequence slot b alone (its block-table
+        row, length, inputs and outputs; the workspace is shared)."""
+        wl = self.wl
+        k, q = wl.k, wl.q_rows
+        B.spec_verify_step(self.dm.desc, self.block_table[b], self.max_pages, self.last_token[b:b + 1],
+                           self.drafts[b * k:(b + 1) * k] if k > 0 else None, 1, k,
+                           self.seq_lens[b:b + 1], self.accept_len[b:b + 1],
+                           self.emitted[b * q:(b + 1) * q], self.new_last[b:b + 1],
+                           self.target_ids[b * q:(b + 1) * q] if with_targets else None,
+                           self.target_max[b * q:(b + 1) * q] if with_targets else None,
+                           self.ws.buf, self.ws.nbytes, stream)
+
     # ---------------------------------------------------------------- prefill
 
     def prefill(self, tokens: np.ndarray, chunk: int = 256):

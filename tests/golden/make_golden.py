@@ -10,7 +10,15 @@ implementation within that tolerance takes the same decisions.
 LM-head passes are batched over all sequences of a round so that the
 262,144-row vocabulary is streamed once per round, not once per row.
 
-  python tests/golden/make_golden.py b1_ctx8k [b8_ragged ...]
+Draws mode (`name:draws=N`): N independent single-sequence steps of the
+workload, draw b seeded as sequence b of its seed space.  Each draw's
+rejection point is taken once from the recipe (attempt 0's coin flips) and
+kept while its context and last token are redrawn for the margin guard, so
+the stored draws follow the recipe's acceptance distribution (a guard that
+also redrew the rejection point would favour short accepted runs, which
+have fewer rows to guard).
+
+  python tests/golden/make_golden.py b1_ctx8k:draws=24 [b8_ragged ...]
 """
 from __future__ import annotations
 
@@ -35,7 +43,7 @@ def _forward_rows(model, caches, L, tokens):
     return fw
 
 
-def solve(wl: W.Workload, max_rounds: int = 60, log=print):
+def solve(wl: W.Workload, max_rounds: int = 60, log=print, fixed_r: bool = False):
     model = harness.oracle_model(wl)
     lens = W.context_lengths(wl)
     attempt = [0] * wl.batch
@@ -50,7 +58,7 @@ def solve(wl: W.Workload, max_rounds: int = 60, log=print):
             L = int(lens[b])
             caches = harness.context_caches(wl, model, b, attempt[b], L)
             last = W.last_token(wl, b, attempt[b])
-            r = W.rejection_point(wl, b, attempt[b])
+            r = W.rejection_point(wl, b, 0 if fixed_r else attempt[b])
             need = wl.k if (r == wl.k or wl.accept[0] == "one_wrong") else r + 1
             state[b] = dict(L=L, caches=caches, last=last, r=r, need=need, greedy=[])
         # greedy continuation, one batched LM pass per position
@@ -71,7 +79,8 @@ def solve(wl: W.Workload, max_rounds: int = 60, log=print):
         rows, spans = [], []
         for b in todo:
             st = state[b]
-            drafts, r2 = W.make_drafts(wl, b, attempt[b], np.array(st["greedy"] + [0], np.int64))
+            drafts, r2 = W.make_drafts(wl, b, attempt[b], np.array(st["greedy"] + [0], np.int64),
+                                       r=st["r"])
             st["drafts"] = drafts
             fw = _forward_rows(model, st["caches"], st["L"], [st["last"]] + [int(x) for x in drafts])
             h = oracle.bf16(oracle.rmsnorm(fw.x_out, model.rms_eps))
@@ -100,9 +109,14 @@ def solve(wl: W.Workload, max_rounds: int = 60, log=print):
 
 
 def main(names):
-    for name in names:
+    for arg in names:
+        name, _, opt = arg.partition(":")
         wl = W.get_workload(name)
-        seqs = solve(wl)
+        draws = int(opt.split("=")[1]) if opt.startswith("draws=") else 0
+        if draws:
+            seqs = solve(wl.with_(batch=draws), fixed_r=True)
+        else:
+            seqs = solve(wl)
         out = {
             "_about": ("Margin-guarded inputs and the oracle's outcome of one verify step; "
                        "written by tests/golden/make_golden.py (oracle + seeded inputs only)."),
@@ -110,6 +124,11 @@ def main(names):
             "margin": {"abs": harness.MARGIN_ABS, "rel": harness.MARGIN_REL},
             "sequences": seqs,
         }
+        if draws:
+            out["mode"] = "draws"
+            out["_about"] += (f" Draws mode: {draws} independent batch-1 steps (draw b = sequence b "
+                              "of the seed space); rejection points fixed per draw from the "
+                              "recipe, contexts redrawn for the margin guard.")
         path = os.path.join(HERE, f"verify_{name}.json")
         with open(path, "w") as f:
             json.dump(out, f, indent=1)

@@ -23,16 +23,26 @@ ATOL, RTOL = 2e-2, 1e-2
 
 @pytest.mark.parametrize("name", FIXTURES)
 def test_full_size_step_matches_oracle(name):
+    """Fixtures in draws mode hold independent batch-1 steps (draw b seeded as
+    sequence b); each runs alone, as the benchmark times it.  Other fixtures
+    run as one batched step."""
     with open(os.path.join(GOLDEN, f"verify_{name}.json")) as f:
         fx = json.load(f)
-    wl = W.get_workload(fx["workload"])
     seqs = fx["sequences"]
+    draws = fx.get("mode") == "draws"
+    wl = W.get_workload(fx["workload"])
+    if draws:
+        wl = wl.with_(batch=len(seqs))
     s = WorkloadSession(wl, attempts=[q["attempt"] for q in seqs])
     s.set_inputs([q["last_token"] for q in seqs],
                  np.array([q["drafts"] for q in seqs], dtype=np.int32) if wl.k else [])
     for rep in range(2):        # a second identical step: counters and status were left clean
         s.reset_lengths()
-        s.step()
+        if draws:
+            for b in range(len(seqs)):
+                s.step_one(b)
+        else:
+            s.step()
         out = s.outputs()
         assert s.ws.device_status() == 0
         for b, q in enumerate(seqs):
@@ -46,3 +56,5 @@ def test_full_size_step_matches_oracle(name):
                 assert abs(out["target_max"][b][i] - t1) <= ATOL + RTOL * abs(t1), (b, i)
                 if q["margin_ok"][i]:
                     assert out["target_ids"][b][i] == q["target_ids"][i], (b, i)
+    if draws:                   # the draws exercise acceptance at full size
+        assert max(q["accept_len"] for q in seqs) >= 1

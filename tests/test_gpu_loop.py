@@ -74,6 +74,33 @@ def test_prefill_matches_oracle():
             assert np.all(np.isclose(oracle.bf16_from_bits(v), c.v, atol=ATOL, rtol=RTOL))
 
 
+def test_prefill_of_two_sequences_matches_oracle():
+    """A prefill chunk of 2 sequences x 256 tokens (512 rows: the projections
+    take the many-row GEMM path) fills each sequence's cache as the oracle's
+    prefill of that sequence alone does."""
+    wl = W.get_workload("small_loop").with_(name="small_loop_b2", batch=2, prompt_tokens=600)
+    s = _session(wl, 0)
+    prompt = np.stack([W.prompt_tokens(wl, b) for b in range(2)])
+    nxt, nmax = s.prefill(prompt, chunk=256)
+    assert s.ws.device_status() == 0 and s.pws.device_status() == 0
+    model = harness.oracle_model(wl)
+    n = wl.prompt_tokens
+    for b in range(2):
+        caches, g, t1, t2 = oracle.prefill(model, prompt[b], chunk=256)
+        assert int(s.seq_lens[b].item()) == n
+        if harness.margin_ok(t1, t2):
+            assert int(nxt[b]) == g, b
+        assert abs(float(nmax[b]) - t1) <= ATOL + RTOL * abs(t1)
+        for l, spec in enumerate(wl.layers):
+            k, v, sb = s.read_cache(l, b, 0, n)
+            c = caches[l]
+            assert np.all(np.isclose(oracle.bf16_from_bits(k), c.k, atol=ATOL, rtol=RTOL)), (b, l)
+            if l == 0:
+                assert np.mean(k == oracle.bits_from_bf16(c.k)) >= 0.99
+            if not spec.kv_equal:
+                assert np.all(np.isclose(oracle.bf16_from_bits(v), c.v, atol=ATOL, rtol=RTOL)), (b, l)
+
+
 def test_greedy_stream_matches_oracle():
     wl = W.get_workload("small_loop")
     n_tok = 24
