@@ -57,6 +57,24 @@ bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64
   return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                       uint64_t stride1, uint64_t stride2, uint32_t b0, uint32_t b1, uint32_t b2) {
+  std::call_once(g_encode_once, resolve_encode);
+  if (!g_encode || !base) return false;
+  if ((reinterpret_cast<uintptr_t>(base) & 15) || (stride1 * 2) % 16 || (stride2 * 2) % 16 ||
+      b0 * 2 != 128 || b1 < 1 || b1 > 256 || b2 < 1 || b2 > 256)
+    return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {stride1 * 2, stride2 * 2};
+  cuuint32_t box[3] = {b0, b1, b2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 namespace {
 
 constexpr size_t kAlign = 256;
@@ -326,6 +344,8 @@ int run_forward(const spec_model* m, const int32_t* block_table, int max_pages, 
     prof_step_done();
     return rc;
   }
+  int fused = 0;
+  bl.accept_fused = &fused;
   rc = cuda_status(launch_gemm_any(pl, kGemmArgmax, lm_x, m->w_lm, bl, st));
   prof_mark(2, st);
   detail_mark(st);
@@ -333,8 +353,8 @@ int run_forward(const spec_model* m, const int32_t* block_table, int max_pages, 
   if (prefill) {
     rc = cuda_status(launch_prefill_commit(at<int32_t>(ws, s.ids), at<float>(ws, s.maxv), B, q,
                                            seq_lens, io.next_token, io.next_maxlogit, st));
-  } else if (pl.mblocks > 1 && !tc_supported(pl.M)) {
-    // acceptance is fused into the LM head when all rows share one block
+  } else if (!fused) {
+    // the LM head runs the acceptance itself when all rows share one block
     rc = cuda_status(launch_accept(io.drafts, at<int32_t>(ws, s.ids), B, k, seq_lens, io.accept_len,
                                    io.emitted, io.new_last_token, io.target_ids,
                                    io.target_maxlogit, at<float>(ws, s.maxv), st));

@@ -524,13 +524,19 @@ __global__ void __launch_bounds__(kThreads) attn_split_kernel(
 }
 
 // out[b][i][h] = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s.
-// The split maxima and weighted denominators are butterfly reductions over a
-// warp's lanes.  The numerator is summed in four parts: part v takes the
-// splits s with (s / 4) % 4 == v in ascending order (lane: 8 output dims),
-// and the parts are added in order.  The grouping is by absolute split
-// index, so splits past a row's own keys (more of them for larger k) only
-// append exact zeros: a row's result does not depend on k.  Both thread
-// mappings compute exactly this:
+// Every reduction tree here is keyed by the ABSOLUTE split index a (split a
+// covers keys [a*split, a*split + split)), never by a split's position in the
+// sequence's list, whose first entry depends on where the layer's window
+// starts for the first query row (on sliding-window layers it moves with k):
+//   - the denominator: lane a % 32 sums its splits in ascending order, then a
+//     butterfly over the lanes;
+//   - the numerator: four parts, part v taking the chunks of four splits
+//     c = a / 4 with c % 4 == v in ascending order (lane: 8 output dims), the
+//     parts added in order.
+// Splits that hold none of a row's keys (m at or below the no-key reference,
+// l = 0, o = 0) only add exact zeros at their fixed places, so a row's result
+// is the same whichever other rows, and so whichever k, the step had.  Both
+// thread mappings compute exactly this:
 //   warp_per_row = 1: one warp per query row (4 rows per CTA) walks the four
 //                     parts itself (few splits, many rows);
 //   warp_per_row = 0: one CTA of four warps per query row, warp v sums part
@@ -560,7 +566,8 @@ __global__ void __launch_bounds__(kCombineWarps * 32) attn_combine_kernel(AttnAr
   }
   int klo, khi;
   seq_key_range(L, a, klo, khi);
-  const int ns = khi < klo ? 0 : min(khi / a.split - klo / a.split + 1, kMaxCombineSplits);
+  const int sf = klo / a.split;   // absolute index of the sequence's first split (partial slot 0)
+  const int ns = khi < klo ? 0 : min(khi / a.split - sf + 1, kMaxCombineSplits);
   const long slot0 = ((long)(b * a.Hkv + kvh) * a.n_splits_grid) * a.rows + r;
   float* m_s = msh[warp_per_row ? warp : 0];
   float* l_s = lsh[warp_per_row ? warp : 0];
@@ -577,8 +584,10 @@ __global__ void __launch_bounds__(kCombineWarps * 32) attn_combine_kernel(AttnAr
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, off));
   const float M = mloc;
+  // lane (sf + s) % 32 owns split s: the first split of this lane is s0
+  const int s0_lane = ((lane - sf) % 32 + 32) % 32;
   float den = 0.f;
-  for (int s = lane; s < ns; s += 32) {
+  for (int s = s0_lane; s < ns; s += 32) {
     const float m = m_s[s];
     den = __fadd_rn(den, __fmul_rn((m == -INFINITY) ? 0.f : exp2f(__fsub_rn(m, M)), l_s[s]));
   }
@@ -593,26 +602,29 @@ __global__ void __launch_bounds__(kCombineWarps * 32) attn_combine_kernel(AttnAr
   const int per_lane = D / 32;   // 8 (D = 256) or 4 (D = 128)
   const float* po = a.part_o + slot0 * D + lane * per_lane;
   const long sstride = (long)a.rows * D;
-  // part v: chunks of four splits c = v, v + 4, v + 8, ..., ascending, the
-  // chunk's four loads in flight together
+  // part v: chunks c = a / 4 of absolute splits with c % 4 == v, ascending,
+  // each chunk's (up to) four loads in flight together
+  const int c_first = sf >> 2, c_last = (sf + ns - 1) >> 2;
   auto part_sum = [&](int v, float (&acc)[8]) {
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.f;
     constexpr int U = 4;
-    for (int s0 = v * U; s0 < ns; s0 += 4 * U) {
+    for (int c = c_first + ((v - c_first) % 4 + 4) % 4; c <= c_last; c += 4) {
       float4 x[U][2];
 #pragma unroll
       for (int u = 0; u < U; ++u) {
-        const bool in = s0 + u < ns;
-        const float* pp = po + (s0 + u) * sstride;
+        const int s = 4 * c + u - sf;          // position of absolute split 4c + u in the list
+        const bool in = s >= 0 && s < ns;
+        const float* pp = po + (long)s * sstride;
         x[u][0] = in ? __ldcg(reinterpret_cast<const float4*>(pp)) : make_float4(0, 0, 0, 0);
         x[u][1] = (in && per_lane == 8) ? __ldcg(reinterpret_cast<const float4*>(pp + 4))
                                         : make_float4(0, 0, 0, 0);
       }
 #pragma unroll
       for (int u = 0; u < U; ++u) {
-        if (s0 + u >= ns) break;
-        const float m = m_s[s0 + u];
+        const int s = 4 * c + u - sf;
+        if (s < 0 || s >= ns) continue;
+        const float m = m_s[s];
         const float ws = (m == -INFINITY) ? 0.f : exp2f(__fsub_rn(m, M));
         const float xs[8] = {x[u][0].x, x[u][0].y, x[u][0].z, x[u][0].w,
                              x[u][1].x, x[u][1].y, x[u][1].z, x[u][1].w};

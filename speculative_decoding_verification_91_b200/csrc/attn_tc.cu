@@ -1,31 +1,44 @@
-// Split-KV verify attention on the 5th-generation tensor cores (sm_100a).
+// Split-KV verify attention on the 5th-generation tensor cores (sm_100a),
+// head_dim 256, persistent.
 //
-// One CTA per (sequence, KV head, absolute split of `split_tokens` keys, row
-// block of up to NP query rows); 6 warps:
+// Work item = (sequence b, KV head, row block, absolute split of split_tokens
+// keys).  Items are ordered (b, kv head, row block, split) and every CTA (one
+// per SM) takes a contiguous range of them, so consecutive items mostly share
+// their queries; its producer streams their keys without a break between
+// items.  10 warps:
 //   warp 0    TMA producer.  Keys arrive in blocks of 128 (two 64-token pages)
 //             as four 128 x 64 swizzled atoms; on key-equals-value layers the
-//             side-band atom (pre-RoPE rotated dims) rides with the keys, on
-//             separate-K/V layers the values have their own buffer.
+//             side-band atom (pre-RoPE rotated dims) rides with the keys (two
+//             stages), on separate-K/V layers keys have two stages and values
+//             one buffer.  Queries come by a 3D TMA box {64 dims, G heads, PB
+//             positions} straight from the rotated-query buffer, once per
+//             (b, kv head, row block).
 //   warp 1    allocates TMEM and issues the MMAs (one thread):
 //               S^T[128 keys][NP rows] = K . Q^T          (A = K, K-major)
-//               O^T[dims][NP rows]   += V^T . P_hi^T + V^T . P_lo^T
-//                                                          (A = V^T, MN-major)
-//             with the accumulators in TMEM (lane = key or value dim,
-//             column = query row).
-//   warps 2-5 softmax: thread t owns key t of the block (TMEM lane t): it
-//             reads its NP scores, the row maxima and sums are reduced over
-//             the 128 keys (warp transpose-reduce, then 4 warps in order),
-//             it writes its probabilities as bf16 head + bf16 tail into the
-//             P tiles, and it rescales its lanes of O when a row maximum
-//             moved.  At the end it writes the partial (o, m, l) of its
-//             rows, the same layout the mma.sync kernel writes.
+//               O^T[dims][NP rows]    += V^T . P^T        (A = V^T, MN-major)
+//             accumulators in TMEM (lane = key or value dim, column = query
+//             row); the scores of the next block are computed while the
+//             softmax works on the current one (two score buffers).
+//   warps 2-9 softmax: thread t of a lane quadrant owns key t of the block;
+//             the warps of one half of the columns (query rows) form a group
+//             of 128 threads.  Per block: the scores of the thread's key for
+//             its NP/2 rows; p = 2^(s - m) against a per-row reference maximum
+//             m that moves only when a block maximum exceeds it by more than
+//             2^8 (one OR-vote per block decides; the exact block maxima are
+//             reduced only then, and the running output is rescaled in TMEM
+//             only for rows that moved); p is written once as bf16 for P . V
+//             and summed unrounded into per-thread row sums, reduced over the
+//             keys at the end of the item.  The partial (o, m, l) of every row
+//             goes out in the layout the split combine reads.
 //
-// Value rows of keys outside the split's valid range (or on pages that were
-// not loaded) are zeroed in shared memory before the PV product, so stale or
-// poisoned slots never reach it.  Keys are visited in blocks at absolute
-// 128-key boundaries and every reduction tree depends only on absolute key
-// positions, so a row's partial does not depend on k, the batch or its row
-// slot.  Every wait is bounded; the CTA always frees its TMEM.
+// Value rows of keys outside the item's range (or on pages that were not
+// loaded) are zeroed in shared memory before P . V, so stale or poisoned
+// slots never reach it.  Keys are visited in blocks at absolute 128-key
+// boundaries; a row's reference maximum, its probabilities and the reduction
+// trees depend only on its own scores and absolute key positions, so a row's
+// partial does not depend on k, the batch, its row slot or the CTA that
+// computed it.  Every wait is bounded; after a timeout the CTA stops issuing
+// work, drains what it issued, writes nothing and frees its TMEM.
 #include <math.h>
 
 #include <algorithm>
@@ -39,49 +52,66 @@ namespace sv {
 
 namespace {
 
-constexpr int kTaThreads = 192;
 constexpr int kBlk = 128;                    // keys per MMA block
 constexpr int kPg = 64;                      // tokens per page
 constexpr int kDim = 256;                    // head_dim of this kernel
 constexpr uint32_t kAtom = kBlk * 128;       // 128 keys x 64 dims of bf16: 16 KB
 constexpr uint32_t kHalfAtom = kPg * 128;    // one page's rows of an atom: 8 KB
+constexpr int kSoftWarps = 8;
+constexpr int kFaThreads = (2 + kSoftWarps) * 32;
+constexpr uint32_t kSmemMax = 227u * 1024u;
+constexpr uint32_t kTailBytes = 4096;
+// p <= 2^kLazy: a row's reference maximum moves only when a block maximum
+// exceeds it by more than this (log2 domain)
+constexpr float kLazy = 8.f;
+constexpr int kMaxItemPages = 128;           // pages one item (split) may span
+// Reference maximum of a row that has seen no key yet: finite, so that
+// 2^(s - m) is exactly 0 for a masked score (s = -inf) and any visible score
+// exceeds it by more than the lazy margin.  A partial whose rows saw no key
+// carries m = kNoKey, l = 0, o = 0, which the split combine weighs by
+// 2^(kNoKey - M) = 0.
+constexpr float kNoKey = -1e30f;
+
+// 2^x (the hardware approximation, relative error ~2^-22; 2^-inf = +0)
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 template <bool KVEQ, int NP>
-struct TaCfg {
-  static constexpr uint32_t kKsBytes = 4 * kAtom + (KVEQ ? kAtom : 0);   // K atoms (+ side-band)
-  static constexpr uint32_t kVBytes = KVEQ ? 0 : 4 * kAtom;
+struct FaCfg {
+  static constexpr uint32_t kStage = 4 * kAtom + (KVEQ ? kAtom : 0);   // keys (+ side-band)
+  static constexpr uint32_t kVBytes = KVEQ ? 0 : 4 * kAtom;           // separate values
   static constexpr uint32_t kQBytes = 4u * NP * 128u;
-  static constexpr uint32_t kPBytes = 2u * NP * 128u;                   // one of P_hi / P_lo
-  static constexpr uint32_t kTailBytes = 4096;
-  // P_hi/P_lo are double-buffered when shared memory allows (the softmax of
-  // block j+1 then writes its P while the PV product of block j reads its own)
-  static constexpr int kPBufs =
-      (1024 + 2 * kKsBytes + kVBytes + kQBytes + 4 * kPBytes + kTailBytes <= 227 * 1024) ? 2 : 1;
-  static constexpr uint32_t kOffV = 2 * kKsBytes;
-  static constexpr uint32_t kOffQ = kOffV + kVBytes;
-  static constexpr uint32_t kOffP = kOffQ + kQBytes;                    // [buf][hi, lo]
-  static constexpr uint32_t kOffTail = kOffP + 2 * kPBufs * kPBytes;
+  static constexpr uint32_t kPBytes = 2u * NP * 128u;                 // [NP rows][128 keys]
+  static constexpr uint32_t bytes(int pb, int qb) {
+    return 1024u + 2u * kStage + kVBytes + pb * kPBytes + qb * kQBytes + kTailBytes;
+  }
+  static constexpr int kPBufs = bytes(2, 1) <= kSmemMax ? 2 : 1;
+  static constexpr int kQBufs = bytes(kPBufs, 2) <= kSmemMax ? 2 : 1;
+  static constexpr uint32_t kOffV = 2 * kStage;
+  static constexpr uint32_t kOffP = kOffV + kVBytes;
+  static constexpr uint32_t kOffQ = kOffP + kPBufs * kPBytes;
+  static constexpr uint32_t kOffTail = kOffQ + kQBufs * kQBytes;
   static constexpr uint32_t kSmem = 1024 + kOffTail + kTailBytes;
   static constexpr int kOTiles = KVEQ ? 3 : 2;
-  // TMEM columns: O tiles, then two score buffers
-  static constexpr uint32_t kColS = kOTiles * NP;
-  static constexpr uint32_t kColsUsed = (kOTiles + 2) * NP;
-  static constexpr uint32_t kTmemCols = kColsUsed <= 32 ? 32 : kColsUsed <= 64 ? 64
-                                      : kColsUsed <= 128 ? 128 : 256;
+  static constexpr uint32_t kColS = kOTiles * NP;       // two score buffers after the O tiles
+  static constexpr uint32_t kCols = (kOTiles + 2) * NP;
+  static constexpr uint32_t kTmemCols =
+      kCols <= 32 ? 32 : kCols <= 64 ? 64 : kCols <= 128 ? 128 : kCols <= 256 ? 256 : 512;
   static_assert(NP % 16 == 0 && NP >= 16 && NP <= 64, "rows per block");
-  static_assert(kColsUsed <= 256, "TMEM columns");
-  static_assert(kSmem <= 227 * 1024, "shared memory");
+  static_assert(kSmem <= kSmemMax, "shared memory");
+  // the side-band MMA pairs each side-band atom with the next 16 KB of shared
+  // memory (lanes never read); for the second stage that is what follows it
+  static_assert(!KVEQ || kOffTail + kTailBytes >= 2 * kStage + kAtom, "side-band pairing");
 };
 
-// A row's exponentials are taken against a reference maximum that moves only
-// when the block maximum exceeds it by more than 2^kLazy (in the log2 domain),
-// so the running output is rescaled in TMEM only then; p <= 2^kLazy.
-constexpr float kLazy = 8.f;
-constexpr int kMaxSplitPages = 256;          // page ids of one split kept in shared memory
-
-struct TaArgs {
-  int q, Hq, Hkv, G, max_pages, num_pages, window, split, n_splits_grid, rows;
-  const uint16_t* qrot;
+struct FaArgs {
+  int B, q, Hq, Hkv, G, max_pages, num_pages, window, split, n_splits_grid, rows;
+  int qpos_off, kend_off;
+  int PB, RB;                 // query positions per row block, row blocks per KV head
+  int lgG;                    // log2 G (G is a power of two)
   const int32_t* block_table;
   const int32_t* seq_lens;
   float* part_o;
@@ -90,9 +120,75 @@ struct TaArgs {
   float scale_log2;
 };
 
+// Keys any row of sequence b may see and the number of absolute splits they
+// touch (0 for an invalid length: the combine then writes zeros).
+__device__ __forceinline__ int seq_splits(const FaArgs& a, int L, int& klo, int& khi) {
+  klo = a.window > 0 ? max(0, L + a.qpos_off - a.window + 1) : 0;
+  khi = L + a.kend_off;
+  if (L < 0 || L + a.q > a.max_pages * kPg || khi < klo) return 0;
+  return khi / a.split - klo / a.split + 1;
+}
+
+// Walks this CTA's items in order.  Every role keeps its own walker; all
+// walkers see the same sequence.
+struct Walker {
+  const FaArgs* a;
+  int b, kvh, rb, sidx, ns, L, lo, hi, blk0, nb;
+  bool new_q;           // this item's queries differ from the previous item's
+  __device__ void load_seq() {
+    L = a->seq_lens[b];
+    int klo, khi;
+    ns = seq_splits(*a, L, klo, khi);
+  }
+  __device__ void derive() {
+    int klo, khi;
+    seq_splits(*a, L, klo, khi);
+    const int s_abs = klo / a->split + sidx;
+    lo = max(s_abs * a->split, klo);
+    hi = min(s_abs * a->split + a->split - 1, khi);
+    blk0 = lo / kBlk;
+    nb = hi / kBlk - blk0 + 1;
+  }
+  __device__ void start(const FaArgs* args, int b0, int kvh0, int rb0, int s0) {
+    a = args;
+    b = b0;
+    kvh = kvh0;
+    rb = rb0;
+    sidx = s0;
+    load_seq();
+    derive();
+    new_q = true;
+  }
+  __device__ void next() {
+    new_q = false;
+    if (++sidx < ns) {
+      derive();
+      return;
+    }
+    sidx = 0;
+    new_q = true;
+    if (++rb < a->RB) {
+      derive();
+      return;
+    }
+    rb = 0;
+    if (++kvh < a->Hkv) {
+      derive();
+      return;
+    }
+    kvh = 0;
+    do {
+      ++b;
+      if (b >= a->B) return;   // past the last item; callers stop by count
+      load_seq();
+    } while (ns == 0);
+    derive();
+  }
+};
+
 // v[0..31] per lane in, lane l out: the max (or sum) over the warp's 32 lanes
-// of column l.  Each round halves the columns a lane keeps; the pairing is
-// by lane bit 4, 3, 2, 1, 0 for every column, so every column gets the same
+// of column l.  Each round halves the columns a lane keeps; the pairing is by
+// lane bit 4, 3, 2, 1, 0 for every column, so every column gets the same
 // reduction tree.
 template <bool MAX>
 __device__ __forceinline__ float transpose_reduce32(float (&v)[32], int lane) {
@@ -122,435 +218,631 @@ __device__ __forceinline__ int o_dim0(int t, int quad) {
   return quad == 0 ? 0 : (quad == 1 ? 128 : -1);
 }
 
+// Bounded wait that gives up at once after an earlier timeout in the CTA.
+__device__ __forceinline__ bool fwait(uint64_t* bar, uint32_t parity, unsigned* status,
+                                      volatile int* fail) {
+  if (*fail) return false;
+  if (mbar_wait(bar, parity, status)) return true;
+  *fail = 1;
+  return false;
+}
+
 template <bool KVEQ, int NP>
-__global__ void __launch_bounds__(kTaThreads, 1) attn_tc_kernel(
-    const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv, TaArgs a) {
-  using C = TaCfg<KVEQ, NP>;
+__global__ void __launch_bounds__(kFaThreads, 1) attn_fa_kernel(
+    const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
+    const __grid_constant__ CUtensorMap tq, const __grid_constant__ FaArgs a) {
+  using C = FaCfg<KVEQ, NP>;
+  constexpr int NH = NP / 2;                 // columns (query rows) per softmax half
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* ks = smem;                      // [2][K atoms (+ side-band)]
-  uint8_t* vb = smem + C::kOffV;           // separate-K/V values
-  uint8_t* qs = smem + C::kOffQ;
-  uint8_t* pbase = smem + C::kOffP;        // P_hi of buffer u at u * 2 * kPBytes, P_lo after it
+  uint8_t* stage = smem;                     // [2][K atoms (+ side-band)]
+  uint8_t* vbuf = smem + C::kOffV;           // separate-K/V values
+  uint8_t* pbuf = smem + C::kOffP;           // [kPBufs][P]
+  uint8_t* qbuf = smem + C::kOffQ;           // [kQBufs][Q]
   uint8_t* tail = smem + C::kOffTail;
-  uint64_t* ks_full = reinterpret_cast<uint64_t*>(tail);   // [2]
-  uint64_t* ks_empty = ks_full + 2;                         // [2]
-  uint64_t* v_full = ks_empty + 2;
+  uint64_t* k_full = reinterpret_cast<uint64_t*>(tail);    // [2]
+  uint64_t* k_empty = k_full + 2;                           // [2]
+  uint64_t* v_full = k_empty + 2;
   uint64_t* v_empty = v_full + 1;
-  uint64_t* s_full = v_empty + 1;                           // [2] per score buffer
-  uint64_t* p_full = s_full + 2;
-  uint64_t* pv_done = p_full + 1;
-  uint64_t* o_full = pv_done + 1;
-  uint64_t* q_full = o_full + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_full + 1);
+  uint64_t* q_full = v_empty + 1;                           // [2]
+  uint64_t* q_empty = q_full + 2;                           // [2]
+  uint64_t* s_full = q_empty + 2;                           // [2]
+  uint64_t* p_full = s_full + 2;                            // [2] by block parity
+  uint64_t* pv_done = p_full + 2;                           // [2] by block parity
+  uint64_t* o_free = pv_done + 2;
+  uint64_t* mma_done = o_free + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* fail = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* red = reinterpret_cast<float*>(tail + 256);       // [4][64]
-  float* m_sh = red + 4 * 64;                               // [64] reference max of each row
-  float* al_sh = m_sh + 64;                                 // [64] rescale factor of the block
-  int* rpos = reinterpret_cast<int*>(al_sh + 64);           // [64] position of each row
-  int* pid_sh = rpos + 64;                                  // [kMaxSplitPages] page ids
+  int* start = reinterpret_cast<int*>(tmem_slot + 4);      // b, kvh, rb, sidx, count
+  float* red = reinterpret_cast<float*>(tail + 256);       // [2 halves][2 bufs][4 quads][32]
+  int* pvalid_all = reinterpret_cast<int*>(red + 512);      // [2][kMaxItemPages] page validity of an item
 
-  pdl_trigger();
-  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int b = blockIdx.z, kvh = blockIdx.y % a.Hkv, rb = blockIdx.y / a.Hkv;
-  const int L = a.seq_lens[b];
-  if (L < 0 || L + a.q > a.max_pages * kPg) {
-    if (threadIdx.x == 0 && blockIdx.x == 0 && kvh == 0 && rb == 0)
-      flag_status(a.status, SPEC_DEV_BAD_LENGTH);
-    return;
-  }
-  const int klo = a.window > 0 ? max(0, L - a.window + 1) : 0;
-  const int khi = L + a.q - 1;
-  const int s_abs = klo / a.split + blockIdx.x;
-  if (s_abs * a.split > khi) return;   // beyond this sequence's last split
-  const int lo = max(s_abs * a.split, klo);
-  const int hi = min(s_abs * a.split + a.split - 1, khi);
-  const int blk0 = lo / kBlk, nb = hi / kBlk - blk0 + 1;
-  const int r0 = rb * NP;
-  const int nrows = min(NP, a.rows - r0);
-  const int32_t* bt = a.block_table + (long)b * a.max_pages;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&ks_full[i], 1);
-      mbar_init(&ks_empty[i], 1);
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&pv_done[i], 1);
+      mbar_init(&p_full[i], kSoftWarps);
     }
     mbar_init(v_full, 1);
     mbar_init(v_empty, 1);
-    mbar_init(&s_full[0], 1);
-    mbar_init(&s_full[1], 1);
-    mbar_init(p_full, 1);
-    mbar_init(pv_done, 1);
-    mbar_init(o_full, 1);
-    mbar_init(q_full, 1);
+    mbar_init(o_free, kSoftWarps);
+    mbar_init(mma_done, 1);
     *fail = 0;
     fence_barrier_init();
   }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tk);
+    prefetch_tmap(&tv);
+    prefetch_tmap(&tq);
+  }
   if (warp == 1) tmem_alloc(tmem_slot, C::kTmemCols);
+  pdl_trigger();
+  pdl_wait();
+
+  // ---- this CTA's items: [i0, i1) of the (b, kvh, rb, split) list
+  if (warp == 2) {
+    const int per_b = a.Hkv * a.RB;
+    long total = 0;
+    for (int b0 = 0; b0 < a.B; b0 += 32) {
+      int klo, khi, n = 0;
+      if (b0 + lane < a.B) n = seq_splits(a, a.seq_lens[b0 + lane], klo, khi);
+      if (n == 0 && b0 + lane < a.B && blockIdx.x == 0) {
+        const int L = a.seq_lens[b0 + lane];
+        if (L < 0 || L + a.q > a.max_pages * kPg) flag_status(a.status, SPEC_DEV_BAD_LENGTH);
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) n += __shfl_xor_sync(0xffffffffu, n, off);
+      total += (long)n * per_b;
+    }
+    const long i0 = (long)blockIdx.x * total / gridDim.x;
+    const long i1 = (long)(blockIdx.x + 1) * total / gridDim.x;
+    // locate item i0
+    long pre = 0;
+    int found_b = -1;
+    long found_pre = 0;
+    for (int b0 = 0; b0 < a.B && found_b < 0 && i1 > i0; b0 += 32) {
+      int klo, khi, n = 0;
+      if (b0 + lane < a.B) n = seq_splits(a, a.seq_lens[b0 + lane], klo, khi);
+      long c = (long)n * per_b, incl = c;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const long o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+      }
+      const long excl = pre + incl - c;
+      const bool mine = c > 0 && i0 >= excl && i0 < excl + c;
+      const unsigned bal = __ballot_sync(0xffffffffu, mine);
+      if (bal) {
+        const int src = __ffs(bal) - 1;
+        found_b = b0 + src;
+        found_pre = __shfl_sync(0xffffffffu, excl, src);
+      }
+      pre += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) {
+      if (found_b >= 0) {
+        int klo, khi;
+        const int ns = seq_splits(a, a.seq_lens[found_b], klo, khi);
+        const long rem = i0 - found_pre;
+        start[0] = found_b;
+        start[1] = (int)(rem / ((long)a.RB * ns));
+        start[2] = (int)((rem / ns) % a.RB);
+        start[3] = (int)(rem % ns);
+        start[4] = (int)(i1 - i0);
+      } else {
+        start[4] = 0;
+      }
+    }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
-  // cache page of absolute page index pg if it holds keys of [lo, hi]: its id,
-  // -1 when it is not needed, -2 when the block table entry is invalid
-  auto page_of = [&](int pg) -> int {
-    if (pg * kPg > hi || pg * kPg + kPg - 1 < lo) return -1;
-    const int id = bt[pg];
-    return (id >= 0 && id < a.num_pages) ? id : -2;
-  };
+  const int count = start[4];
+  const int32_t* bt_all = a.block_table;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      prefetch_tmap(&tk);
-      prefetch_tmap(&tv);
+    if (lane == 0 && count > 0) {
       const uint64_t pol = policy_evict_first();
-      auto load_ks = [&](int j) {
-        const int slot = j & 1;
-        uint8_t* dst = ks + slot * C::kKsBytes;
+      const uint64_t pol_q = policy_evict_normal();
+      Walker w;
+      w.start(&a, start[0], start[1], start[2], start[3]);
+      int gk = 0, gv = 0, nq = 0;
+      auto page_id = [&](const Walker& it, int pg) -> int {   // -1 not needed, -2 invalid
+        if (pg * kPg > it.hi || pg * kPg + kPg - 1 < it.lo) return -1;
+        const int id = bt_all[(long)it.b * a.max_pages + pg];
+        return (id >= 0 && id < a.num_pages) ? id : -2;
+      };
+      auto load_k = [&](const Walker& it, int j) -> bool {
+        const int s = gk & 1;
+        if (gk >= 2 && !fwait(&k_empty[s], ((gk >> 1) - 1) & 1, a.status, fail)) return false;
+        uint8_t* dst = stage + s * C::kStage;
         int id[2];
         uint32_t bytes = 0;
         for (int h = 0; h < 2; ++h) {
-          id[h] = page_of((blk0 + j) * 2 + h);
+          id[h] = page_id(it, (it.blk0 + j) * 2 + h);
           if (id[h] == -2) flag_status(a.status, SPEC_DEV_BAD_PAGE);
           if (id[h] >= 0) bytes += (KVEQ ? 5u : 4u) * kHalfAtom;
         }
-        mbar_arrive_expect_tx(&ks_full[slot], bytes);
+        mbar_arrive_expect_tx(&k_full[s], bytes);
         for (int h = 0; h < 2; ++h) {
           if (id[h] < 0) continue;
-          const int y = (id[h] * a.Hkv + kvh) * kPg;
+          const int y = (id[h] * a.Hkv + it.kvh) * kPg;
+#pragma unroll
           for (int at = 0; at < 4; ++at)
-            tma_load_2d(dst + at * kAtom + h * kHalfAtom, &tk, &ks_full[slot], at * 64, y, pol);
-          if (KVEQ) tma_load_2d(dst + 4 * kAtom + h * kHalfAtom, &tv, &ks_full[slot], 0, y, pol);
+            tma_load_2d(dst + at * kAtom + h * kHalfAtom, &tk, &k_full[s], at * 64, y, pol);
+          if (KVEQ) tma_load_2d(dst + 4 * kAtom + h * kHalfAtom, &tv, &k_full[s], 0, y, pol);
         }
+        ++gk;
+        return true;
       };
-      auto load_v = [&](int j) {
+      auto load_v = [&](const Walker& it, int j) -> bool {
+        if (gv >= 1 && !fwait(v_empty, (gv - 1) & 1, a.status, fail)) return false;
         int id[2];
         uint32_t bytes = 0;
         for (int h = 0; h < 2; ++h) {
-          id[h] = page_of((blk0 + j) * 2 + h);
+          id[h] = page_id(it, (it.blk0 + j) * 2 + h);
           if (id[h] >= 0) bytes += 4u * kHalfAtom;
         }
         mbar_arrive_expect_tx(v_full, bytes);
         for (int h = 0; h < 2; ++h) {
           if (id[h] < 0) continue;
-          const int y = (id[h] * a.Hkv + kvh) * kPg;
+          const int y = (id[h] * a.Hkv + it.kvh) * kPg;
+#pragma unroll
           for (int at = 0; at < 4; ++at)
-            tma_load_2d(vb + at * kAtom + h * kHalfAtom, &tv, v_full, at * 64, y, pol);
+            tma_load_2d(vbuf + at * kAtom + h * kHalfAtom, &tv, v_full, at * 64, y, pol);
         }
+        ++gv;
+        return true;
       };
-      int ks_issued = 0, v_issued = 0;
+      auto load_q = [&](const Walker& it) -> bool {
+        const int qb = nq % C::kQBufs;
+        if (nq >= C::kQBufs && !fwait(&q_empty[qb], ((nq / C::kQBufs) - 1) & 1, a.status, fail))
+          return false;
+        uint8_t* dst = qbuf + qb * C::kQBytes;
+        mbar_arrive_expect_tx(&q_full[qb], C::kQBytes);
+        const int z = it.b * a.q + it.rb * a.PB;
+#pragma unroll
+        for (int sub = 0; sub < 4; ++sub)
+          tma_load_3d(dst + sub * (NP * 128), &tq, &q_full[qb], sub * 64, it.kvh * a.G, z, pol_q);
+        ++nq;
+        return true;
+      };
+      bool ok = true;
       if (KVEQ) {
-        for (int j = 0; j < nb; ++j) {
-          if (j >= 2 && (*fail || !mbar_wait(&ks_empty[j & 1], ((j >> 1) - 1) & 1, a.status))) {
-            *fail = 1;
-            break;
-          }
-          load_ks(j);
-          ks_issued = j + 1;
+        for (int i = 0; ok && i < count; ++i, w.next()) {
+          if (w.new_q) ok = load_q(w);
+          for (int j = 0; ok && j < w.nb; ++j) ok = load_k(w, j);
         }
       } else {
-        // keys run two blocks ahead of values: K slot j+2 frees when QK_j is
-        // done, the value buffer when PV_j is done
-        load_ks(0);
-        ks_issued = 1;
-        if (nb > 1) {
-          load_ks(1);
-          ks_issued = 2;
-        }
-        for (int j = 0; j < nb; ++j) {
-          if (j >= 1 && (*fail || !mbar_wait(v_empty, (j - 1) & 1, a.status))) {
-            *fail = 1;
-            break;
-          }
-          load_v(j);
-          v_issued = j + 1;
-          if (j + 2 < nb) {
-            if (*fail || !mbar_wait(&ks_empty[j & 1], (j >> 1) & 1, a.status)) {
-              *fail = 1;
-              break;
+        // keys run up to two blocks ahead of the values (a key stage frees
+        // when its scores are done, the value buffer when P . V is done)
+        Walker wk = w;
+        int ik = 0, jk = 0;          // next key block to load: item ik, block jk of wk
+        auto key_ahead = [&](int limit) -> bool {   // load keys while gk < limit
+          while (ik < count && gk < limit) {
+            if (jk == 0 && wk.new_q && !load_q(wk)) return false;
+            if (!load_k(wk, jk)) return false;
+            if (++jk >= wk.nb) {
+              jk = 0;
+              ++ik;
+              if (ik < count) wk.next();
             }
-            load_ks(j + 2);
-            ks_issued = j + 3;
+          }
+          return true;
+        };
+        int gblk = 0;
+        for (int i = 0; ok && i < count; ++i, w.next()) {
+          for (int j = 0; ok && j < w.nb; ++j, ++gblk) {
+            ok = key_ahead(gblk + 2) && load_v(w, j);
           }
         }
       }
-      // every issued copy has landed before the CTA may exit
-      for (int j = (ks_issued > 2 ? ks_issued - 2 : 0); j < ks_issued; ++j)
-        mbar_wait(&ks_full[j & 1], (j >> 1) & 1, a.status);
-      if (v_issued > 0) mbar_wait(v_full, (v_issued - 1) & 1, a.status);
+      // every issued copy must land before the CTA may exit
+      for (int i = (gk > 2 ? gk - 2 : 0); i < gk; ++i) mbar_wait(&k_full[i & 1], (i >> 1) & 1, a.status);
+      if (gv > 0) mbar_wait(v_full, (gv - 1) & 1, a.status);
+      for (int i = (nq > C::kQBufs ? nq - C::kQBufs : 0); i < nq; ++i)
+        mbar_wait(&q_full[i % C::kQBufs], (i / C::kQBufs) & 1, a.status);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
-    // order: QK_0, then per block j: QK_{j+1} (other score buffer, as soon as
-    // its keys landed), wait for P_j, PV_j.  The tensor core thus computes the
-    // next scores while the softmax works on the current ones.
-    if (lane == 0) {
+    if (lane == 0 && count > 0) {
       const uint32_t id_qk = idesc_bf16(NP);
       const uint32_t id_pv = idesc_bf16(NP, true);
-      const uint32_t q_addr = smem_u32(qs);
-      const uint32_t p_addr = smem_u32(pbase);
-      auto issue_qk = [&](int j) -> bool {
-        if (*fail || !mbar_wait(&ks_full[j & 1], (j >> 1) & 1, a.status)) return false;
-        tc_fence_after();
-        const uint32_t k_addr = smem_u32(ks + (j & 1) * C::kKsBytes);
-        const uint32_t t_s = tmem + C::kColS + (j & 1) * NP;
+      // The scores of block g (QK) and the product P . V of block g - 1 are
+      // independent: each is issued as soon as its inputs are ready, so P . V
+      // never waits for the next block's keys (which, on key-equals-value
+      // layers, could not be requested before that P . V frees its stage).
+      //   QK(g):  keys of g landed; score buffer g % 2 read by the softmax
+      //           (g <= npv + 1); new queries landed at a query-group start.
+      //   PV(g):  P(g) written; values landed (separate-K/V); the previous
+      //           item's output read out (first block of an item).
+      Walker ws, wp;
+      ws.start(&a, start[0], start[1], start[2], start[3]);
+      wp = ws;
+      int is = 0, js = 0, ip = 0, jp = 0;   // QK / PV positions: item, block in item
+      int nqk = 0, npv = 0, nq_used = -1;
+      uint64_t t_last = globaltimer_ns();
+      uint32_t polls = 0;
+      while (ip < count) {
+        bool progressed = false;
+        if (is < count && nqk <= npv + 1) {
+          const bool newq = js == 0 && ws.new_q;
+          const int qb = (nq_used + 1) % C::kQBufs;
+          bool ready = !newq || mbar_try_wait(&q_full[qb], ((nq_used + 1) / C::kQBufs) & 1);
+          ready = ready && mbar_try_wait(&k_full[nqk & 1], (nqk >> 1) & 1);
+          if (ready) {
+            if (newq) ++nq_used;
+            tc_fence_after();
+            const int s = nqk & 1;
+            const uint32_t k_addr = smem_u32(stage + s * C::kStage);
+            const uint32_t q_addr = smem_u32(qbuf + (nq_used % C::kQBufs) * C::kQBytes);
+            const uint32_t t_s = tmem + C::kColS + s * NP;
 #pragma unroll
-        for (int kk = 0; kk < kDim / 16; ++kk)   // K = 16 dims per MMA
-          umma_bf16(t_s, sw128_desc(k_addr + (kk >> 2) * kAtom + (kk & 3) * 32),
-                    sw128_desc(q_addr + (kk >> 2) * (NP * 128) + (kk & 3) * 32), id_qk, kk > 0);
-        umma_commit(&s_full[j & 1]);
-        if (!KVEQ) umma_commit(&ks_empty[j & 1]);   // keys no longer needed
-        return true;
-      };
-      bool ok = mbar_wait(q_full, 0, a.status) && (nb < 1 || issue_qk(0));
-      for (int j = 0; ok && j < nb; ++j) {
-        if (j + 1 < nb && !issue_qk(j + 1)) {
-          ok = false;
-          break;
-        }
-        if (!mbar_wait(p_full, j & 1, a.status) ||
-            (!KVEQ && !mbar_wait(v_full, j & 1, a.status))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t v_addr = KVEQ ? smem_u32(ks + (j & 1) * C::kKsBytes) : smem_u32(vb);
-        const uint32_t ph_addr = p_addr + (j % C::kPBufs) * 2 * C::kPBytes;
-        const uint32_t pl_addr = ph_addr + C::kPBytes;
-#pragma unroll
-        for (int t = 0; t < C::kOTiles; ++t) {
-          // [atom 2t ; atom 2t+1] (the side-band tile pairs its atom with the
-          // next 16 KB of shared memory, whose lanes are never read)
-          const uint32_t a0 = v_addr + 2 * t * kAtom;
-#pragma unroll
-          for (int kk = 0; kk < kBlk / 16; ++kk) {   // K = 16 keys per MMA
-            const uint64_t ad = sw128_desc_mn(a0 + kk * 2048, kAtom);
-            const uint32_t po = (kk >> 2) * (NP * 128) + (kk & 3) * 32;
-            umma_bf16(tmem + t * NP, ad, sw128_desc(ph_addr + po), id_pv, (j > 0 || kk > 0));
-            umma_bf16(tmem + t * NP, ad, sw128_desc(pl_addr + po), id_pv, 1u);
+            for (int kk = 0; kk < kDim / 16; ++kk)   // K = 16 dims per MMA
+              umma_bf16(t_s, sw128_desc(k_addr + (kk >> 2) * kAtom + (kk & 3) * 32),
+                        sw128_desc(q_addr + (kk >> 2) * (NP * 128) + (kk & 3) * 32), id_qk, kk > 0);
+            umma_commit(&s_full[s]);
+            if (!KVEQ) umma_commit(&k_empty[s]);     // keys no longer needed
+            // last block of the last item of this query group: release the queries
+            bool last_of_group = false;
+            if (js + 1 >= ws.nb) {
+              if (is + 1 >= count) {
+                last_of_group = true;
+              } else {
+                Walker peek = ws;
+                peek.next();
+                last_of_group = peek.new_q;
+              }
+            }
+            if (last_of_group) umma_commit(&q_empty[nq_used % C::kQBufs]);
+            ++nqk;
+            if (++js >= ws.nb) {
+              js = 0;
+              ++is;
+              if (is < count) ws.next();
+            }
+            progressed = true;
           }
         }
-        umma_commit(pv_done);
-        umma_commit(KVEQ ? &ks_empty[j & 1] : v_empty);
+        if (npv < nqk) {
+          bool ready = mbar_try_wait(&p_full[npv & 1], (npv >> 1) & 1);
+          if (!KVEQ) ready = ready && mbar_try_wait(v_full, npv & 1);
+          if (jp == 0 && ip > 0) ready = ready && mbar_try_wait(o_free, (ip - 1) & 1);
+          if (ready) {
+            tc_fence_after();
+            const uint32_t v_addr = KVEQ ? smem_u32(stage + (npv & 1) * C::kStage) : smem_u32(vbuf);
+            const uint32_t p_addr = smem_u32(pbuf + (npv % C::kPBufs) * C::kPBytes);
+#pragma unroll
+            for (int t = 0; t < C::kOTiles; ++t) {
+              // [atom 2t ; atom 2t+1] (the side-band tile pairs its atom with the
+              // next 16 KB of shared memory, whose lanes are never read)
+              const uint32_t a0 = v_addr + 2 * t * kAtom;
+#pragma unroll
+              for (int kk = 0; kk < kBlk / 16; ++kk) {   // K = 16 keys per MMA
+                const uint64_t ad = sw128_desc_mn(a0 + kk * 2048, kAtom);
+                const uint32_t po = (kk >> 2) * (NP * 128) + (kk & 3) * 32;
+                umma_bf16(tmem + t * NP, ad, sw128_desc(p_addr + po), id_pv, (jp > 0 || kk > 0) ? 1u : 0u);
+              }
+            }
+            umma_commit(&pv_done[npv & 1]);
+            umma_commit(KVEQ ? &k_empty[npv & 1] : v_empty);
+            ++npv;
+            if (++jp >= wp.nb) {
+              jp = 0;
+              ++ip;
+              if (ip < count) wp.next();
+            }
+            progressed = true;
+          }
+        }
+        if (progressed) {
+          polls = 0;
+        } else if ((++polls & 255u) == 0) {
+          const uint64_t now = globaltimer_ns();
+          if (polls == 256) t_last = now;       // first idle check of this stretch
+          else if (now - t_last > kWaitNs || *fail) {
+            flag_status(a.status, SPEC_DEV_TIMEOUT);
+            *fail = 1;
+            break;
+          }
+        }
       }
-      if (!ok) *fail = 1;
-      umma_commit(o_full);
-      // nothing may be in flight when TMEM is freed
-      mbar_wait(o_full, 0, a.status);
+    }
+    // nothing may be in flight when TMEM is freed
+    if (lane == 0) {
+      umma_commit(mma_done);
+      mbar_wait(mma_done, 0, a.status);
     }
   } else {
     // ------------------------------------------------------------ softmax
-    const int ctid = threadIdx.x - 64;       // 0..127
-    const int quad = warp & 3;               // TMEM lanes 32*quad ..
+    const int sw = warp - 2;                 // 0..7
+    const int quad = warp & 3;               // TMEM lanes 32*quad .. (fixed by the warp id)
+    const int half = sw >> 2;                // columns [half*NH, half*NH + NH)
+    const int c0 = half * NH;
     const int t = quad * 32 + lane;          // key of the block / O lane
-    const uint32_t tq = tmem + ((uint32_t)(quad * 32) << 16);
-
-    // Q rows of this block -> K-major swizzled tile (zero padding rows)
-    for (int idx = ctid; idx < NP * (kDim / 8); idx += 128) {
-      const int r = idx / (kDim / 8), c = idx % (kDim / 8);
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (r < nrows) {
-        const int rg = r0 + r, gh = rg / a.q, i = rg % a.q;
-        const int h = kvh * a.G + gh;
-        v = *reinterpret_cast<const uint4*>(a.qrot + (((long)b * a.q + i) * a.Hq + h) * kDim + c * 8);
+    const uint32_t tq_lane = tmem + ((uint32_t)(quad * 32) << 16);
+    const int bar_id = 1 + half;
+    float* red_h = red + half * (2 * 128);
+    // P tile address of (row c0 + r, key t): a per-thread base plus the
+    // 128-byte swizzle term (chunk ^ (row & 7)) << 4, where row & 7 = r & 7
+    // because c0 is a multiple of 8
+    const uint32_t chs = (uint32_t)((t & 63) >> 3) << 4;
+    const uint32_t p_off = (t >> 6) * (NP * 128) + c0 * 128 + ((t & 7) << 1);
+    Walker w;
+    if (count > 0) w.start(&a, start[0], start[1], start[2], start[3]);
+    int g = 0;                                // global block counter
+    int nslow = 0;                            // slow-path rounds (double-buffered reductions)
+    for (int i = 0; i < count; ++i, w.next()) {
+      // rows of this half: column c = i_pos * G + gh holds query position
+      // i_pos of the row block (position L + qpos_off + rb*PB + i_pos), or
+      // nothing past the sequence's q positions
+      const int npos = min(a.PB, a.q - w.rb * a.PB);            // positions in this row block
+      const int pos0 = w.L + a.qpos_off + w.rb * a.PB;
+      auto row_pos = [&](int r) -> int {                         // -1: padding column
+        const int ip = (c0 + r) >> a.lgG;
+        return ip < npos ? pos0 + ip : -1;
+      };
+      // a half whose columns are all padding only keeps the barriers going
+      const bool active = row_pos(0) >= 0;
+      const int pmin = pos0, pmax = pos0 + npos - 1;
+      // page ids of the item's blocks -> validity bits in shared memory (one
+      // load per page, before the first block; two buffers by item parity, so
+      // that the next item's writes never meet this item's reads)
+      int* pvalid = pvalid_all + (i & 1) * kMaxItemPages;
+      {
+        const int np_item = 2 * w.nb;
+        const int st_ = sw * 32 + lane;
+        if (st_ < np_item) {
+          const int pg = 2 * w.blk0 + st_;
+          int ok = 0;
+          if (pg < a.max_pages) {
+            const int id = bt_all[(long)w.b * a.max_pages + pg];
+            ok = id >= 0 && id < a.num_pages;
+          }
+          pvalid[st_] = ok;
+        }
+        named_bar(3, kSoftWarps * 32);
       }
-      *reinterpret_cast<uint4*>(qs + (c >> 3) * (NP * 128) + swz128(r, c & 7)) = v;
-    }
-    if (ctid < NP) rpos[ctid] = ctid < nrows ? L + (r0 + ctid) % a.q : -1;
-    // cache page ids of the split's pages (-1 / -2: not loaded)
-    for (int i = ctid; i < 2 * nb; i += 128) pid_sh[i] = page_of(2 * blk0 + i);
-    float m_ref = -INFINITY, l_run = 0.f;    // row ctid (ctid < NP)
-    fence_proxy_async_smem();
-    named_bar(1, 128);
-    if (ctid == 0) mbar_arrive(q_full);
-
-    for (int j = 0; j < nb; ++j) {
-      bool ok = !*fail && mbar_wait(&s_full[j & 1], (j >> 1) & 1, a.status);
-      ok = __all_sync(0xffffffffu, ok);   // TMEM loads are warp-collective
-      if (!ok) *fail = 1;
-      tc_fence_after();
-      const int key = (blk0 + j) * kBlk + t;
-      const bool in_range = key >= lo && key <= hi && pid_sh[2 * j + (t >> 6)] >= 0;
-      float s[NP];
-      if (ok) {
+      // running state per row: the reference maximum (log2 domain; kNoKey
+      // until the row has seen a key, so that 2^(s - m) of a masked score is
+      // exactly 0 and every visible score moves it) and the row sum
+      float mref[NH], lt[NH];
 #pragma unroll
-        for (int c0 = 0; c0 < NP; c0 += 16) {
-          uint32_t r[16];
-          tmem_ld16_nowait(tq + C::kColS + (j & 1) * NP + c0, r);
+      for (int r = 0; r < NH; ++r) {
+        mref[r] = kNoKey;
+        lt[r] = 0.f;
+      }
+      for (int j = 0; j < w.nb; ++j, ++g) {
+        const int s = g & 1;
+        const int kb = (w.blk0 + j) * kBlk;
+        const bool pv0 = pvalid[2 * j] != 0, pv1 = pvalid[2 * j + 1] != 0;
+        const bool interior = kb >= w.lo && kb + kBlk - 1 <= w.hi && pv0 && pv1 &&
+                              kb + kBlk - 1 <= pmin && (a.window == 0 || kb > pmax - a.window);
+        const int key = kb + t;
+        const bool in_range = key >= w.lo && key <= w.hi && ((t < kPg) ? pv0 : pv1);
+        fwait(&s_full[s], (g >> 1) & 1, a.status, fail);
+        tc_fence_after();
+        float sc[NH];
+        bool need = false;
+        if (active) {
+          uint32_t r8[NH / 8][8];
+#pragma unroll
+          for (int c = 0; c < NH / 8; ++c) tmem_ld8_nowait(tq_lane + C::kColS + s * NP + c0 + 8 * c, r8[c]);
           tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 16; ++i) s[c0 + i] = __uint_as_float(r[i]);
+          for (int c = 0; c < NH / 8; ++c)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) sc[8 * c + e] = __fmul_rn(__uint_as_float(r8[c][e]), a.scale_log2);
+          if (!interior) {
+#pragma unroll
+            for (int r = 0; r < NH; ++r) {
+              const int p = row_pos(r);
+              const bool vis = in_range && key <= p && (a.window == 0 || key > p - a.window);
+              if (!vis) sc[r] = -INFINITY;
+            }
+          }
+#pragma unroll
+          for (int r = 0; r < NH; ++r) need |= sc[r] > __fadd_rn(mref[r], kLazy);
         }
-      }
+        // ---- the reference maxima move only when some row needs it
+        if (bar_red_or(bar_id, 128, need)) {
+          float* rb_ = red_h + (nslow & 1) * 128;
+          ++nslow;
+          float v[32];
 #pragma unroll
-      for (int r = 0; r < NP; ++r) {
-        const int p = rpos[r];
-        const bool vis = ok && in_range && key <= p && (a.window == 0 || key > p - a.window);
-        s[r] = vis ? __fmul_rn(s[r], a.scale_log2) : -INFINITY;
-      }
-      // ---- row maxima of the block -> reference maxima
+          for (int e = 0; e < 32; ++e) v[e] = e < NH ? sc[e] : -INFINITY;
+          const float mx = transpose_reduce32<true>(v, lane);
+          rb_[quad * 32 + lane] = mx;
+          named_bar(bar_id, 128);
+          float alpha[NH];
+          bool moved = false;
 #pragma unroll
-      for (int c0 = 0; c0 < NP; c0 += 32) {
-        float v[32];
+          for (int r = 0; r < NH; ++r) {
+            const float bm = fmaxf(fmaxf(rb_[r], rb_[32 + r]), fmaxf(rb_[64 + r], rb_[96 + r]));
+            alpha[r] = 1.f;
+            if (bm > __fadd_rn(mref[r], kLazy)) {
+              alpha[r] = ex2_approx(__fsub_rn(mref[r], bm));   // 0 while the row had no key
+              mref[r] = bm;
+              lt[r] = __fmul_rn(lt[r], alpha[r]);
+              moved = true;
+            }
+          }
+          if (moved && j > 0) {
+            // rescale this half's columns of the running output (all P . V of
+            // the earlier blocks must have completed)
+            fwait(&pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1, a.status, fail);
+            tc_fence_after();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = (c0 + i < NP) ? s[c0 + i] : -INFINITY;
-        const float mx = transpose_reduce32<true>(v, lane);
-        if (c0 + lane < NP) red[quad * 64 + c0 + lane] = mx;
-      }
-      named_bar(1, 128);
-      if (ctid < NP) {
-        const float mb = fmaxf(fmaxf(red[ctid], red[64 + ctid]), fmaxf(red[128 + ctid], red[192 + ctid]));
-        float al = 1.f;
-        if (m_ref == -INFINITY) {
-          m_ref = mb;                          // nothing accumulated yet: no rescale
-        } else if (mb > __fadd_rn(m_ref, kLazy)) {
-          al = exp2f(__fsub_rn(m_ref, mb));
-          m_ref = mb;
-        }
-        m_sh[ctid] = m_ref;
-        al_sh[ctid] = al;
-      }
-      named_bar(1, 128);
-      // ---- probabilities and the block's row sums
-      float p[NP];
+            for (int tt = 0; tt < C::kOTiles; ++tt) {
 #pragma unroll
-      for (int r = 0; r < NP; ++r)
-        p[r] = (s[r] == -INFINITY) ? 0.f : exp2f(__fsub_rn(s[r], m_sh[r]));
+              for (int c = 0; c < NH; c += 8) {
+                uint32_t r8[8];
+                tmem_ld8_nowait(tq_lane + tt * NP + c0 + c, r8);
+                tmem_ld_wait();
 #pragma unroll
-      for (int c0 = 0; c0 < NP; c0 += 32) {
-        float v[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = (c0 + i < NP) ? p[c0 + i] : 0.f;
-        const float sm = transpose_reduce32<false>(v, lane);
-        if (c0 + lane < NP) red[quad * 64 + c0 + lane] = sm;
-      }
-      bool moved = false;
-#pragma unroll
-      for (int r = 0; r < NP; ++r) moved |= al_sh[r] != 1.f;
-      // PV of the previous block must be done before its P buffer is
-      // rewritten (single buffer) or its output is rescaled
-      if (ok && j > 0 && (C::kPBufs == 1 || moved)) ok = mbar_wait(pv_done, (j - 1) & 1, a.status);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) *fail = 1;
-      // ---- P = P_hi + P_lo as bf16 (K-major tiles: row r, key t)
-      {
-        uint8_t* ph = pbase + (j % C::kPBufs) * 2 * C::kPBytes;
-        uint8_t* pl = ph + C::kPBytes;
-        const uint32_t off = (t >> 6) * (NP * 128) + ((t & 7) << 1);
-        const uint32_t ch = (t & 63) >> 3;
-#pragma unroll
-        for (int r = 0; r < NP; ++r) {
-          const uint16_t hb = f32_to_bf16(p[r]);
-          const uint16_t lb = f32_to_bf16(__fsub_rn(p[r], bf16_to_f32(hb)));
-          const uint32_t o = off + swz128(r, ch);
-          *reinterpret_cast<uint16_t*>(ph + o) = hb;
-          *reinterpret_cast<uint16_t*>(pl + o) = lb;
-        }
-      }
-      // ---- value rows of keys outside the valid range: zero them
-      if (ok && !in_range && (KVEQ || mbar_wait(v_full, j & 1, a.status))) {
-        // (separate values: their copy must have landed first)
-        uint8_t* base = KVEQ ? ks + (j & 1) * C::kKsBytes : vb;
-        const int n_at = KVEQ ? 5 : 4;
-        for (int at = 0; at < n_at; ++at)
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint4*>(base + at * kAtom + t * 128 + c * 16) = make_uint4(0, 0, 0, 0);
-      }
-      // ---- rescale the running output of rows whose reference max moved
-      if (ok && j > 0 && moved) {
-#pragma unroll
-        for (int tt = 0; tt < C::kOTiles; ++tt) {
-          if (o_dim0<KVEQ>(tt, quad) < 0) continue;
-#pragma unroll
-          for (int c0 = 0; c0 < NP; c0 += 16) {
-            uint32_t r[16];
-            tmem_ld16_nowait(tq + tt * NP + c0, r);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__fmul_rn(__uint_as_float(r[i]), al_sh[c0 + i]));
-            tmem_st16(tq + tt * NP + c0, r);
+                for (int e = 0; e < 8; ++e)
+                  r8[e] = __float_as_uint(__fmul_rn(__uint_as_float(r8[e]), alpha[c + e]));
+                tmem_st8(tq_lane + tt * NP + c0 + c, r8);
+              }
+            }
+            tmem_st_wait();
           }
         }
-        tmem_st_wait();
+        // the P buffer of this block was last read by P . V of block g - kPBufs
+        if (g >= C::kPBufs)
+          fwait(&pv_done[(g - C::kPBufs) & 1], ((g - C::kPBufs) >> 1) & 1, a.status, fail);
+        if (active) {
+          // ---- probabilities: unrounded into the row sums, bf16 into P
+          // (2^-inf = 0: masked keys and rows without a key so far give 0)
+          uint8_t* pp = pbuf + (g % C::kPBufs) * C::kPBytes + p_off;
+#pragma unroll
+          for (int r = 0; r < NH; ++r) {
+            const float p = ex2_approx(__fsub_rn(sc[r], mref[r]));
+            lt[r] = __fadd_rn(lt[r], p);
+            *reinterpret_cast<uint16_t*>(pp + r * 128 + (chs ^ ((uint32_t)(r & 7) << 4))) = f32_to_bf16(p);
+          }
+        }
+        // ---- value rows of keys no row of the item may use: zero them
+        if (!interior && !in_range && half == 0) {
+          if (KVEQ) {
+            uint8_t* base = stage + s * C::kStage;
+#pragma unroll
+            for (int at = 0; at < 5; ++at)
+#pragma unroll
+              for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<uint4*>(base + at * kAtom + t * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+          } else if ((g == 0 || fwait(&pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1, a.status, fail)) &&
+                     fwait(v_full, g & 1, a.status, fail)) {
+            // the single value buffer takes block g's values only after P . V
+            // of block g - 1; from then on its current phase is block g's
+#pragma unroll
+            for (int at = 0; at < 4; ++at)
+#pragma unroll
+              for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<uint4*>(vbuf + at * kAtom + t * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+          }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[g & 1]);
       }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      named_bar(1, 128);
-      if (ctid < NP) {
-        const float rs = __fadd_rn(__fadd_rn(red[ctid], red[64 + ctid]), __fadd_rn(red[128 + ctid], red[192 + ctid]));
-        l_run = __fadd_rn(__fmul_rn(l_run, al_sh[ctid]), rs);
-      }
-      if (ctid == 0) mbar_arrive(p_full);
-      named_bar(1, 128);   // red / m_sh / al_sh are rewritten by the next block
-    }
 
-    // ---- partial (o unnormalised, m and l in the log2 domain) of each row
-    const bool ok = __all_sync(0xffffffffu, !*fail && mbar_wait(o_full, 0, a.status));
-    tc_fence_after();
-    if (ok) {
-      const long slot = ((long)(b * a.Hkv + kvh) * a.n_splits_grid + blockIdx.x) * a.rows + r0;
+      // ---- the item's partial: o unnormalised, m and l in the log2 domain
+      float v[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) v[e] = e < NH ? lt[e] : 0.f;
+      const float lq = transpose_reduce32<false>(v, lane);
+      float* rl = red_h + (nslow & 1) * 128;
+      ++nslow;
+      rl[quad * 32 + lane] = lq;
+      named_bar(bar_id, 128);
+      fwait(&pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1, a.status, fail);
+      tc_fence_after();
+      const long slot = ((long)(w.b * a.Hkv + w.kvh) * a.n_splits_grid + w.sidx) * a.rows;
+      const bool out_ok = !*fail && active;
 #pragma unroll
       for (int tt = 0; tt < C::kOTiles; ++tt) {
         const int d0 = o_dim0<KVEQ>(tt, quad);
-        if (d0 < 0) continue;
-        const int dim = d0 + lane;
+        if (d0 < 0 || !out_ok) continue;
+        float ov[NH];
+        {
+          uint32_t r8[NH / 8][8];
 #pragma unroll
-        for (int c0 = 0; c0 < NP; c0 += 16) {
-          uint32_t r[16];
-          tmem_ld16_nowait(tq + tt * NP + c0, r);
+          for (int c = 0; c < NH / 8; ++c) tmem_ld8_nowait(tq_lane + tt * NP + c0 + 8 * c, r8[c]);
           tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            if (c0 + i < nrows) __stcg(a.part_o + (slot + c0 + i) * kDim + dim, __uint_as_float(r[i]));
+          for (int c = 0; c < NH / 8; ++c)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) ov[8 * c + e] = __uint_as_float(r8[c][e]);
+        }
+#pragma unroll
+        for (int r = 0; r < NH; ++r) {
+          if (row_pos(r) < 0) continue;
+          const int c = c0 + r;
+          const int prow = (c & (a.G - 1)) * a.q + w.rb * a.PB + (c >> a.lgG);
+          __stcg(a.part_o + (slot + prow) * kDim + d0 + lane, ov[r]);
         }
       }
-      if (ctid < nrows)
-        __stcg(reinterpret_cast<float2*>(a.part_ml + (slot + ctid) * 2), make_float2(m_ref, l_run));
+      if (quad == 0 && lane < NH && out_ok) {
+        const int c = c0 + lane;
+        const int ip = w.rb * a.PB + (c >> a.lgG);
+        if (ip < a.q) {
+          float mv = kNoKey;
+#pragma unroll
+          for (int r = 0; r < NH; ++r)
+            if (r == lane) mv = mref[r];
+          const float l = __fadd_rn(__fadd_rn(rl[lane], rl[32 + lane]), __fadd_rn(rl[64 + lane], rl[96 + lane]));
+          const int prow = (c & (a.G - 1)) * a.q + ip;
+          __stcg(reinterpret_cast<float2*>(a.part_ml + (slot + prow) * 2), make_float2(mv, l));
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(o_free);
     }
-    tc_fence_before();
   }
+  tc_fence_before();
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, C::kTmemCols);
 }
 
+int g_num_sms = 0;
+
 template <bool KVEQ, int NP>
-cudaError_t launch_ta(const AttnGeom& g, int row_blocks, const CUtensorMap& tk, const CUtensorMap& tv,
-                      const TaArgs& a, cudaStream_t st) {
-  using C = TaCfg<KVEQ, NP>;
-  auto kern = attn_tc_kernel<KVEQ, NP>;
+cudaError_t launch_fa(int grid, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
+                      const FaArgs& a, cudaStream_t st) {
+  using C = FaCfg<KVEQ, NP>;
+  auto kern = attn_fa_kernel<KVEQ, NP>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
-  return launch_k(kern, dim3(g.n_splits_grid, g.n_kv_heads * row_blocks, g.B), dim3(kTaThreads),
-                  C::kSmem, st, tk, tv, a);
+  return launch_k(kern, dim3(grid), dim3(kFaThreads), C::kSmem, st, tk, tv, tq, a);
 }
 
-int ta_np(const AttnGeom& g) {
-  if (!g.kv_equal) return 16;
-  const int r = std::min(g.rows, 48);
-  return (r + 15) / 16 * 16;
+// Rows per CTA tile: the KV head's G*q rows rounded up to 16 when they fit
+// (64 on key-equals-value layers, 32 with separate values, whose larger
+// stages leave less shared memory), else row blocks of whole query positions.
+int fa_np(const AttnGeom& g, int G) {
+  const int cap = g.kv_equal ? 64 : 32;
+  const int rows = G * g.q;
+  if (rows <= cap) return (rows + 15) / 16 * 16;
+  return cap;
 }
 
 }  // namespace
 
-// Opt-in (SPECVERIFY_TC_ATTN=1): at the verify shapes measured so far (8 to
-// 40 query rows per KV head) the mma.sync kernel is faster, because the
-// skinny tcgen05 MMAs and the per-block softmax chain leave the tensor core
-// and the load pipe idle most of the time.
+// Which layers take the tensor-memory attention: head_dim 256 with 64-token
+// pages, and at least SPECVERIFY_TC_ATTN_MIN_G query heads per KV head
+// (default 4).  The choice depends on the model only, never on k or the
+// batch, so a row is computed by the same kernel whatever k is.  With G = 2
+// (8 to 10 rows per KV head at the benchmark's k) the mma.sync kernel's lighter
+// per-block work is faster (batch 64 global layer 479 vs 660 us, batch 1
+// sliding-window layer 12 vs 19 us); from G = 4 on the tensor cores win
+// (batch 8, G = 8: 168 vs 255 us).  SPECVERIFY_NO_TC_ATTN=1 or SPECVERIFY_NO_TC=1
+// turns the path off.
 bool attn_tc_supported(const AttnGeom& g) {
-  static const bool on = [] {
-    const char* v = getenv("SPECVERIFY_TC_ATTN");
+  static const int min_g = [] {
+    const char* v = getenv("SPECVERIFY_NO_TC_ATTN");
     const char* off = getenv("SPECVERIFY_NO_TC");
-    return v && v[0] == '1' && !(off && off[0] == '1');
+    if ((v && v[0] == '1') || (off && off[0] == '1')) return 1 << 30;
+    const char* m = getenv("SPECVERIFY_TC_ATTN_MIN_G");
+    const int r = m ? atoi(m) : 4;
+    return r < 1 ? 1 : r;
   }();
-  return on && g.qpos_off == 0 && g.kend_off == g.q - 1 &&   // verify rows only
-         g.head_dim == kDim && g.page_size == kPg && g.split_tokens % kBlk == 0 &&
-         g.split_tokens <= kPg * kMaxSplitPages && (!g.kv_equal || g.sb_width == 64);
+  const int G = g.n_q_heads / g.n_kv_heads;
+  return G >= min_g && g.head_dim == kDim && g.page_size == kPg && (!g.kv_equal || g.sb_width == 64) &&
+         G <= 16 && 16 % G == 0 && g.split_tokens % kPg == 0 &&
+         g.split_tokens / kPg + 2 <= kMaxItemPages;
 }
 
 cudaError_t launch_attn_tc(const AttnGeom& g, const CUtensorMap& tk, const CUtensorMap& tv,
@@ -558,31 +850,57 @@ cudaError_t launch_attn_tc(const AttnGeom& g, const CUtensorMap& tk, const CUten
                            float* part_o, float* part_ml, unsigned* status, float scale_log2,
                            cudaStream_t st) {
   if (!attn_tc_supported(g)) return cudaErrorInvalidValue;
-  TaArgs a{};
+  const int G = g.n_q_heads / g.n_kv_heads;
+  const int np = fa_np(g, G);
+  FaArgs a{};
+  a.B = g.B;
   a.q = g.q;
   a.Hq = g.n_q_heads;
   a.Hkv = g.n_kv_heads;
-  a.G = g.n_q_heads / g.n_kv_heads;
+  a.G = G;
   a.max_pages = g.max_pages;
   a.num_pages = g.num_pages;
   a.window = g.window;
   a.split = g.split_tokens;
   a.n_splits_grid = g.n_splits_grid;
   a.rows = g.rows;
-  a.qrot = qrot;
+  a.qpos_off = g.qpos_off;
+  a.kend_off = g.kend_off;
+  a.PB = np / G;
+  a.lgG = __builtin_ctz((unsigned)G);
+  a.RB = (g.q + a.PB - 1) / a.PB;
   a.block_table = block_table;
   a.seq_lens = seq_lens;
   a.part_o = part_o;
   a.part_ml = part_ml;
   a.status = status;
   a.scale_log2 = scale_log2;
-  const int np = ta_np(g);
-  const int row_blocks = (g.rows + np - 1) / np;
-  if (!g.kv_equal) return launch_ta<false, 16>(g, row_blocks, tk, tv, a, st);
+  // queries: [B*q positions][Hq heads][D], box {64 dims, G heads, PB positions}
+  CUtensorMap tq;
+  if (!make_tmap_bf16_3d(&tq, qrot, kDim, g.n_q_heads, (uint64_t)g.B * g.q, kDim,
+                         (uint64_t)g.n_q_heads * kDim, 64, G, a.PB))
+    return cudaErrorInvalidValue;
+  if (g_num_sms == 0) {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+      return cudaErrorInvalidValue;
+    g_num_sms = n;
+  }
+  const long items = (long)g.B * g.n_kv_heads * a.RB * g.n_splits_grid;   // upper bound
+  const int grid = (int)std::max(1L, std::min<long>(items, g_num_sms));
+  if (!g.kv_equal) {
+    switch (np) {
+      case 16: return launch_fa<false, 16>(grid, tk, tv, tq, a, st);
+      case 32: return launch_fa<false, 32>(grid, tk, tv, tq, a, st);
+    }
+    return cudaErrorInvalidValue;
+  }
   switch (np) {
-    case 16: return launch_ta<true, 16>(g, row_blocks, tk, tv, a, st);
-    case 32: return launch_ta<true, 32>(g, row_blocks, tk, tv, a, st);
-    case 48: return launch_ta<true, 48>(g, row_blocks, tk, tv, a, st);
+    case 16: return launch_fa<true, 16>(grid, tk, tv, tq, a, st);
+    case 32: return launch_fa<true, 32>(grid, tk, tv, tq, a, st);
+    case 48: return launch_fa<true, 48>(grid, tk, tv, tq, a, st);
+    case 64: return launch_fa<true, 64>(grid, tk, tv, tq, a, st);
   }
   return cudaErrorInvalidValue;
 }

@@ -419,7 +419,7 @@ GemmPlan plan_gemm(int M, int N, int K, int mode) {
 // Split-K partial floats of either path: the tensor-memory kernel writes
 // rows padded to 16 (tc_np), the mma.sync kernel to its M-block width.
 size_t gemm_partial_floats(const GemmPlan& p) {
-  const size_t ldp = tc_supported(p.M) ? std::max<size_t>(mma_ldp(p), (size_t)tc_np(p.M)) : mma_ldp(p);
+  const size_t ldp = tc_supported(p.M) ? std::max<size_t>(mma_ldp(p), (size_t)tc_ldp(p.M)) : mma_ldp(p);
   return (size_t)p.splits * p.n_tiles * kTileN * ldp;
 }
 size_t gemm_argmax_entries(const GemmPlan& p) { return (size_t)p.M; }
@@ -458,7 +458,8 @@ cudaError_t launch_gemm(const GemmPlan& p, int mode, const void* x, const void* 
   a.ldp = mma_ldp(p);
   // more than a few rows: reduce the split partials with the whole grid
   a.grid_reduce = (mode != kGemmArgmax && p.M > kFusedTailMaxRows) ? 1 : 0;
-  if (mode != kGemmArgmax || p.mblocks != 1) a.acc.B = 0;
+  if (mode != kGemmArgmax || p.mblocks != 1) a.acc.B = 0;   // acceptance needs every row
+  if (b.accept_fused) *b.accept_fused = a.acc.B > 0 ? 1 : 0;
   switch (mode) {
     case kGemmArgmax: return launch_mode<kGemmArgmax>(p, tw, tx, a, st);
   }

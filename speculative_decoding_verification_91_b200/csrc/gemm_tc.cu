@@ -32,6 +32,7 @@ namespace sv {
 namespace {
 
 constexpr int kTcThreads = 192;
+constexpr int kTcMaxRows = 256;              // verify rows per TMEM accumulator (MMA N)
 constexpr int kTcEpiWarp0 = 2;
 constexpr uint32_t kABytes = kTileN * 128;   // 16 KB weight tile per stage
 
@@ -76,7 +77,8 @@ __global__ void __launch_bounds__(kTcThreads, 2) tc_gemm_kernel(
 
   pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_tile = blockIdx.x, split = blockIdx.y;
+  const int n_tile = blockIdx.x, split = blockIdx.y, mblk = blockIdx.z;
+  const int m0 = mblk * kTcMaxRows;          // first verify row of this block
   const int kc0 = (int)((long)split * a.kchunks / a.splits);
   const int kc1 = (int)((long)(split + 1) * a.kchunks / a.splits);
   const int nk = kc1 - kc0;
@@ -112,7 +114,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) tc_gemm_kernel(
       }
       pdl_wait();
       for (int it = 0; it < pre; ++it)
-        tma_load_2d(smem + it * L.stage_bytes + kABytes, &tx, &full[it], (kc0 + it) * kTileK, 0, pol_x);
+        tma_load_2d(smem + it * L.stage_bytes + kABytes, &tx, &full[it], (kc0 + it) * kTileK, m0, pol_x);
       int issued = pre;
       for (int it = pre; it < nk; ++it) {
         const int s = it % L.stages;
@@ -124,7 +126,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) tc_gemm_kernel(
         mbar_arrive_expect_tx(&full[s], L.stage_bytes);
         const int kx = (kc0 + it) * kTileK;
         tma_load_2d(st, &tw, &full[s], kx, n_tile * kTileN, pol_w);
-        tma_load_2d(st + kABytes, &tx, &full[s], kx, 0, pol_x);
+        tma_load_2d(st + kABytes, &tx, &full[s], kx, m0, pol_x);
         issued = it + 1;
       }
       for (int it = (issued > L.stages ? issued - L.stages : 0); it < issued; ++it)
@@ -203,7 +205,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) tc_gemm_kernel(
           }
         }
         named_bar(1, kEpiThreads);
-        for (int c = ctid; c < np && c < a.M; c += kEpiThreads) {
+        for (int c = ctid; c < np && m0 + c < a.M; c += kEpiThreads) {
           float bv = red_v[c];
           int bi = red_i[c];
           for (int q2 = 1; q2 < 4; ++q2)
@@ -211,11 +213,11 @@ __global__ void __launch_bounds__(kTcThreads, 2) tc_gemm_kernel(
               bv = red_v[q2 * 256 + c];
               bi = red_i[q2 * 256 + c];
             }
-          atomicMax(&a.arg_keys[c], pack_arg(bv, bi));
+          atomicMax(&a.arg_keys[m0 + c], pack_arg(bv, bi));
         }
       } else {
         // split-K partial tile [128 rows][np], then the shared epilogues
-        float* mine = a.partial + ((size_t)split * a.n_tiles + n_tile) * kTileN * a.ldp;
+        float* mine = a.partial + ((size_t)split * a.n_tiles + n_tile) * kTileN * a.ldp + m0;
         for (int c0 = 0; c0 < np; c0 += 32) {
           float v[32];
           tmem_ld32(tq + c0, v);
@@ -239,7 +241,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) tc_gemm_kernel(
   //      the whole grid instead of one CTA per tile
   if (MODE == kGemmArgmax) {
     const int ctid = threadIdx.x - kTcEpiWarp0 * 32;
-    argmax_finish(a, a.n_tiles, 0, 0, np, ctid, flag, red_i);
+    argmax_finish(a, a.n_tiles, mblk, m0, np, ctid, flag, red_i);
   }
 }
 
@@ -250,7 +252,7 @@ cudaError_t launch_tc_mode(const GemmPlan& p, const CUtensorMap& tw, const CUten
   const TcLayout L = tc_layout(a.np);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.smem);
   if (e != cudaSuccess) return e;
-  e = launch_k(kern, dim3(p.n_tiles, p.splits, 1), dim3(kTcThreads), L.smem, st, tw, tx, a);
+  e = launch_k(kern, dim3(p.n_tiles, p.splits, tc_mblocks(p.M)), dim3(kTcThreads), L.smem, st, tw, tx, a);
   if (e != cudaSuccess || MODE == kGemmArgmax) return e;
   return launch_splitk_reduce(a, MODE, st);
 }
@@ -259,8 +261,10 @@ cudaError_t launch_tc_mode(const GemmPlan& p, const CUtensorMap& tw, const CUten
 
 // Row counts for the tensor-memory GEMM: above 32 (up to there the mma.sync
 // kernel streams the weights at the same HBM speed; at 40 and 64 rows it
-// becomes compute-bound: LM head at d 2560, 64 rows 442 us vs 230 us here)
-// and up to 256 (one TMEM accumulator of N = 256 columns).
+// becomes compute-bound: LM head at d 2560, 64 rows 442 us vs 230 us here).
+// Up to 256 rows sit in one TMEM accumulator (N = 256 columns); more rows run
+// as blocks of 256 (grid z), each streaming the weights once -- against the
+// mma.sync kernel's blocks of 64 rows, a quarter of the weight traffic.
 // SPECVERIFY_TC_MIN_ROWS overrides the lower bound (>= 16),
 // SPECVERIFY_NO_TC=1 turns the path off.
 bool tc_supported(int M) {
@@ -271,10 +275,12 @@ bool tc_supported(int M) {
     const int r = m ? atoi(m) : 32;
     return r < 16 ? 16 : r;
   }();
-  return M > min_rows && M <= 256;
+  return M > min_rows && M <= kTcMaxRows * kMaxTickets;
 }
 
-int tc_np(int M) { return (M + 15) / 16 * 16; }
+int tc_np(int M) { return M <= kTcMaxRows ? (M + 15) / 16 * 16 : kTcMaxRows; }
+int tc_mblocks(int M) { return (M + kTcMaxRows - 1) / kTcMaxRows; }
+int tc_ldp(int M) { return M <= kTcMaxRows ? tc_np(M) : tc_mblocks(M) * kTcMaxRows; }
 
 cudaError_t launch_gemm_tc(const GemmPlan& p, int mode, const void* x, const void* w,
                            const GemmBuffers& b, cudaStream_t st) {
@@ -291,7 +297,7 @@ cudaError_t launch_gemm_tc(const GemmPlan& p, int mode, const void* x, const voi
   a.splits = p.splits;
   a.n_tiles = p.n_tiles;
   a.np = np;
-  a.ldp = np;
+  a.ldp = tc_ldp(p.M);
   a.grid_reduce = 1;
   a.out = b.out;
   a.partial = b.partial;
@@ -302,7 +308,8 @@ cudaError_t launch_gemm_tc(const GemmPlan& p, int mode, const void* x, const voi
   a.status = b.status;
   a.acc = b.acc;
   a.rope = b.rope;
-  if (mode != kGemmArgmax) a.acc.B = 0;
+  if (mode != kGemmArgmax || tc_mblocks(p.M) > 1) a.acc.B = 0;   // acceptance needs every row
+  if (b.accept_fused) *b.accept_fused = a.acc.B > 0 ? 1 : 0;
   switch (mode) {
     case kGemmStore: return launch_tc_mode<kGemmStore>(p, tw, tx, a, st);
     case kGemmResidual: return launch_tc_mode<kGemmResidual>(p, tw, tx, a, st);

@@ -14,6 +14,10 @@ namespace sv {
 // fails (the caller reports SPEC_ECUDA) or the layout is not encodable.
 bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                        uint32_t box_rows, uint32_t box_cols, uint64_t row_stride = 0);
+// 3D row-major bf16 tensor [d2][d1][d0] (strides in elements), box {b0, b1, b2},
+// 128-byte swizzle (b0 * 2 must be 128), zero fill outside the tensor.
+bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                       uint64_t stride1, uint64_t stride2, uint32_t b0, uint32_t b1, uint32_t b2);
 
 // --------------------------------------------------------- streaming GEMM
 // Y = X . W^T with X [M][K] bf16 (row-major), W [N][K] bf16 (row-major),
@@ -71,6 +75,7 @@ struct GemmBuffers {
   unsigned* status;
   AcceptFuse acc;      // kGemmArgmax with a single M-block only
   RopeFuse rope;       // kGemmQkvRope
+  int* accept_fused;   // set by the launcher: 1 if the argmax kernel runs the acceptance
 };
 cudaError_t launch_gemm(const GemmPlan& p, int mode, const void* x, const void* w,
                         const GemmBuffers& buf, cudaStream_t st);
@@ -79,7 +84,9 @@ cudaError_t launch_gemm(const GemmPlan& p, int mode, const void* x, const void* 
 // outside that range (SPECVERIFY_TC_MIN_ROWS moves the lower bound) or when
 // SPECVERIFY_NO_TC=1.
 bool tc_supported(int M);
-int tc_np(int M);   // rows of the tensor-memory GEMM (M rounded up to 16)
+int tc_np(int M);        // rows per tensor-memory block (M rounded up to 16, at most 256)
+int tc_mblocks(int M);   // blocks of 256 rows
+int tc_ldp(int M);       // row stride of its split-K partials
 cudaError_t launch_gemm_tc(const GemmPlan& p, int mode, const void* x, const void* w,
                            const GemmBuffers& buf, cudaStream_t st);
 // tcgen05 path when it applies, else the mma.sync path

@@ -122,6 +122,13 @@ WORKLOADS.update({
                                                 vocab=4100, ctx_lo=60, ctx_hi=700,
                                                 layers=(LayerSpec(window=200, split_tokens=64),
                                                         GLOBAL_KV)),
+    # the window of the first verify row starts on the last key of a split
+    # (1450 - 300 + 1 = 9 * 128 - 1), so each later row's window starts in the
+    # next split: the split combine must not depend on where the list begins
+    "small_b1_edge": WORKLOADS["b1_ctx8k"].with_(name="small_b1_edge", vocab=9000, ctx_lo=1450,
+                                                   ctx_hi=1450,
+                                                   layers=(LayerSpec(window=300, split_tokens=128),
+                                                           GLOBAL_KV)),
     # the largest draft count the library takes: 17 verify rows
     "small_b1_k16": WORKLOADS["b1_ctx8k"].with_(name="small_b1_k16", k=16, vocab=9000, ctx_lo=1500,
                                                   ctx_hi=1500,

@@ -1,6 +1,11 @@
-"""The tcgen05 split-KV attention kernel (opt-in through SPECVERIFY_TC_ATTN=1)
-against the oracle: the attention-level and whole-step parity tests run
-again in a child process with the tensor-memory path switched on."""
+"""The two split-KV attention kernels against the oracle on every shape.
+
+By default a layer takes the tcgen05 kernel when it has at least four query
+heads per KV head, else the mma.sync kernel.  Here the attention-level,
+whole-step and k-invariance parity tests run again in child processes with
+each kernel forced on for every layer (head_dim 256): the tcgen05 kernel
+(SPECVERIFY_TC_ATTN_MIN_G=1) and the mma.sync kernel
+(SPECVERIFY_NO_TC_ATTN=1)."""
 import os
 import subprocess
 import sys
@@ -11,10 +16,11 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 @pytest.mark.gpu
-def test_tc_attention_parity():
-    env = dict(os.environ, SPECVERIFY_TC_ATTN="1")
+@pytest.mark.parametrize("env", [{"SPECVERIFY_TC_ATTN_MIN_G": "1"}, {"SPECVERIFY_NO_TC_ATTN": "1"}])
+def test_attention_kernels_forced_parity(env):
     r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
                         os.path.join(ROOT, "tests", "test_gpu_kernels.py"),
                         "-k", "verify_attn or verify_step or invariant"],
-                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=900)
+                       cwd=ROOT, env=dict(os.environ, **env), capture_output=True, text=True,
+                       timeout=900)
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]

@@ -250,7 +250,7 @@ def test_verify_step_matches_oracle(name):
     assert flips[0] <= max(4, total[0] // 200), (flips[0], total[0])
 
 
-@pytest.mark.parametrize("name", ["small_b1", "small_ragged"])
+@pytest.mark.parametrize("name", ["small_b1", "small_ragged", "small_b1_edge"])
 def test_step_is_invariant_to_k(name):
     """Greedy decoding with k = 0, one token per step, and one verify step with
     k = 8 whose drafts are those greedy tokens give bit-identical rows: the
