@@ -319,12 +319,14 @@ def run_cuda(args, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     B.spec_profile_start(args.steps)
     n_launch0 = B.spec_launch_count()
+    torch.cuda.nvtx.range_push("timed")     # selects the timed launches in a profiler
     with ClockSampler(local_rank) as clocks:
         for i in range(args.steps):
             flush.zero_()
             sess.reset_lengths()
             one_step(i)
         torch.cuda.synchronize(dev)
+    torch.cuda.nvtx.range_pop()
     n_launches = B.spec_launch_count() - n_launch0
     step_ms, lm_ms = B.spec_profile_collect(args.steps)
     if world > 1:
@@ -846,6 +848,7 @@ def run_loop(args):
         e1 = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
         if timed:
             B.spec_profile_start(n)
+            torch.cuda.nvtx.range_push("timed")
         for st in range(n):
             h_in[0] = cur
             h_in[1:] = torch.from_numpy(drafter(st, emitted))
@@ -868,12 +871,26 @@ def run_loop(args):
             emitted += a + 1
             cur = int(h_out[q + 1])
         torch.cuda.synchronize(dev)
+        if timed:
+            torch.cuda.nvtx.range_pop()
         e2e = [x.elapsed_time(y) for x, y in zip(e0, e1)]
         dev_ms = B.spec_profile_collect(n)[0] if timed else None
         return accepts, dev_ms, e2e
 
     if args.warmup:
         run(args.warmup, False)
+    # per-launch breakdown of one verify step at the prompt's end (events
+    # serialise the launches; rolled back afterwards)
+    s.seq_lens.fill_(L0)
+    s.last_token.fill_(int(nxt[0]))
+    s.drafts[:k].copy_(torch.from_numpy(drafter(0, 0)))
+    flush.zero_()
+    B.spec_profile_launches(256)
+    s.step(stream=stream, with_targets=False)
+    launch_ms = B.spec_profile_launches_collect(256)
+    labels = launch_labels(wl)
+    breakdown = (dict(zip(labels, [round(x * 1e3, 1) for x in launch_ms])) if len(labels) == len(launch_ms)
+                 else [round(x * 1e3, 1) for x in launch_ms])
     n0 = B.spec_launch_count()
     with ClockSampler(0) as clocks:
         accepts, dev_ms, e2e = run(steps, True)
@@ -913,7 +930,8 @@ def run_loop(args):
             "accept_len_mean": float(np.mean(accepts)),
             "e2e": {"value": tokens / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": int(h_in.numel() * 4),
                     "d2h_bytes_per_step": int(h_out.numel() * 4)},
-            "gpu_launches": launches, "prefill_s": round(t_prefill, 2), "clocks": clocks.summary()}
+            "gpu_launches": launches, "launch_breakdown_us": breakdown,
+            "prefill_s": round(t_prefill, 2), "clocks": clocks.summary()}
     print(json.dumps(line), flush=True)
 
 

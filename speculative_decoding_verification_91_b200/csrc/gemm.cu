@@ -34,7 +34,7 @@ namespace {
 constexpr int kConsumerWarps = 4;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kMBlock = 64;
-constexpr int kFusedTailMaxRows = 16;   // up to this many rows the last CTA runs the epilogue
+constexpr int kFusedTailMaxRows = kEpiMaxRows;   // up to this many rows the last CTA runs the epilogue
 
 template <int NT>
 struct Cfg {
@@ -271,24 +271,46 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(Args a) {
   const int ld = a.ldp, tx = threadIdx.x, ty = threadIdx.y;   // 32 x 8
   const int m_base = blockIdx.y * 32;
   const size_t split_stride = (size_t)a.n_tiles * kTileN * ld;
+  // Each thread sums four (feature or pair, row) elements; the loads of four
+  // splits of all four are in flight together, then added in split order.
   if (MODE != kGemmQkvRope) {
     const int n_base = blockIdx.x * 32;
-    for (int r = ty; r < 32; r += 8) {             // r: feature within the tile
-      const int n = n_base + r, m = m_base + tx;
-      float s = 0.f;
-      if (n < a.N && m < a.M) {
+    float s[4] = {0.f, 0.f, 0.f, 0.f};
+    const int m = m_base + tx;
+    for (int sp0 = 0; sp0 < a.splits; sp0 += 4) {
+      float v[4][4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {                // u: feature ty + 8u of the tile
+        const int n = n_base + ty + 8 * u;
         const float* p = a.partial + (size_t)n * ld + m;
-        for (int sp = 0; sp < a.splits; ++sp) s = __fadd_rn(s, __ldcg(p + (size_t)sp * split_stride));
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+          v[u][w] = (n < a.N && m < a.M && sp0 + w < a.splits) ? __ldcg(p + (size_t)(sp0 + w) * split_stride)
+                                                               : 0.f;
       }
-      t0[r][tx] = s;
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+          if (sp0 + w < a.splits) s[u] = __fadd_rn(s[u], v[u][w]);
     }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) t0[ty + 8 * u][tx] = s[u];
     __syncthreads();
-    for (int r = ty; r < 32; r += 8) {             // r: row within the tile
-      const int n = n_base + tx, m = m_base + r;
-      if (n < a.N && m < a.M) {
-        float* dst = a.out + (size_t)m * a.N + n;
-        *dst = (MODE == kGemmResidual) ? __fadd_rn(*dst, t0[tx][r]) : t0[tx][r];
-      }
+    // the residuals are read before the first store (a store may alias a
+    // later load as far as the compiler knows)
+    const int n = n_base + tx;
+    float res[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {                  // u: row ty + 8u of the tile
+      const int m = m_base + ty + 8 * u;
+      res[u] = (MODE == kGemmResidual && n < a.N && m < a.M) ? a.out[(size_t)m * a.N + n] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int r = ty + 8 * u, m = m_base + r;
+      if (n < a.N && m < a.M)
+        a.out[(size_t)m * a.N + n] = (MODE == kGemmResidual) ? __fadd_rn(res[u], t0[tx][r]) : t0[tx][r];
     }
     return;
   }
@@ -296,51 +318,81 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(Args a) {
   const int D = f.head_dim, half = D / 2;
   const int pairs_per_head = half / 32;
   const int head = blockIdx.x / pairs_per_head, j0 = (blockIdx.x % pairs_per_head) * 32;
-  for (int r = ty; r < 32; r += 8) {               // r: pair within the tile
-    const int m = m_base + tx, j = j0 + r;
-    float x0 = 0.f, x1 = 0.f;
-    if (m < a.M) {
-      const float* p0 = a.partial + (size_t)(head * D + j) * ld + m;
-      const float* p1 = a.partial + (size_t)(head * D + j + half) * ld + m;
-      for (int sp = 0; sp < a.splits; ++sp) {
-        x0 = __fadd_rn(x0, __ldcg(p0 + (size_t)sp * split_stride));
-        x1 = __fadd_rn(x1, __ldcg(p1 + (size_t)sp * split_stride));
+  {
+    const int m = m_base + tx;
+    float x0[4] = {0.f, 0.f, 0.f, 0.f}, x1[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int sp0 = 0; sp0 < a.splits; sp0 += 2) {
+      float v0[4][2], v1[4][2];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {                // u: pair ty + 8u of the tile
+        const int j = j0 + ty + 8 * u;
+        const float* p0 = a.partial + (size_t)(head * D + j) * ld + m;
+        const float* p1 = a.partial + (size_t)(head * D + j + half) * ld + m;
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          const bool ok = m < a.M && sp0 + w < a.splits;
+          v0[u][w] = ok ? __ldcg(p0 + (size_t)(sp0 + w) * split_stride) : 0.f;
+          v1[u][w] = ok ? __ldcg(p1 + (size_t)(sp0 + w) * split_stride) : 0.f;
+        }
       }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int w = 0; w < 2; ++w)
+          if (sp0 + w < a.splits) {
+            x0[u] = __fadd_rn(x0[u], v0[u][w]);
+            x1[u] = __fadd_rn(x1[u], v1[u][w]);
+          }
     }
-    t0[r][tx] = x0;
-    t1[r][tx] = x1;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      t0[ty + 8 * u][tx] = x0[u];
+      t1[ty + 8 * u][tx] = x1[u];
+    }
   }
   __syncthreads();
-  for (int r = ty; r < 32; r += 8) {               // r: row within the tile
-    const int m = m_base + r, j = j0 + tx;
+  // every load (table entries, lengths, pages) before the first store
+  const int j = j0 + tx;
+  const bool rot = j < f.n_rot && head < f.n_q_heads + f.n_kv_heads;
+  const bool kv_head = head >= f.n_q_heads;
+  const int kvh = head < f.n_q_heads + f.n_kv_heads ? head - f.n_q_heads
+                                                    : head - f.n_q_heads - f.n_kv_heads;
+  float2 cs[4];
+  long long rowi[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {                    // u: row ty + 8u of the tile
+    const int m = m_base + ty + 8 * u;
+    cs[u] = (m < a.M && rot) ? f.rope_tab[(size_t)m * half + j] : make_float2(1.f, 0.f);
+    rowi[u] = -1;
+    if (m < a.M && kv_head) {
+      const int b = m / f.q, i = m % f.q;
+      const int pos = f.seq_lens[b] + i;
+      if (pos < 0 || pos / f.page_size >= f.max_pages) {
+        flag_status(a.status, SPEC_DEV_BAD_LENGTH);
+      } else {
+        const int page = f.block_table[(size_t)b * f.max_pages + pos / f.page_size];
+        if (page < 0 || page >= f.num_pages)
+          flag_status(a.status, SPEC_DEV_BAD_PAGE);
+        else
+          rowi[u] = ((long long)page * f.n_kv_heads + kvh) * f.page_size + pos % f.page_size;
+      }
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int r = ty + 8 * u, m = m_base + r;
     if (m >= a.M) continue;
     const float x0 = t0[tx][r], x1 = t1[tx][r];
-    const int b = m / f.q, i = m % f.q;
-    const bool rot = j < f.n_rot && head < f.n_q_heads + f.n_kv_heads;
     float y0 = x0, y1 = x1;
-    if (rot) {
-      const float2 cs = f.rope_tab[(size_t)m * half + j];
-      rope_pair(x0, x1, cs.x, cs.y, y0, y1);
-    }
+    if (rot) rope_pair(x0, x1, cs[u].x, cs[u].y, y0, y1);
     if (head < f.n_q_heads) {
       uint16_t* qo = f.q_out + ((size_t)m * f.n_q_heads + head) * D;
       qo[j] = f32_to_bf16(y0);
       qo[j + half] = f32_to_bf16(y1);
       continue;
     }
-    const int pos = f.seq_lens[b] + i;
-    if (pos < 0 || pos / f.page_size >= f.max_pages) {
-      flag_status(a.status, SPEC_DEV_BAD_LENGTH);
-      continue;
-    }
-    const int page = f.block_table[(size_t)b * f.max_pages + pos / f.page_size];
-    if (page < 0 || page >= f.num_pages) {
-      flag_status(a.status, SPEC_DEV_BAD_PAGE);
-      continue;
-    }
-    const int kvh = head < f.n_q_heads + f.n_kv_heads ? head - f.n_q_heads
-                                                      : head - f.n_q_heads - f.n_kv_heads;
-    const size_t row = ((size_t)page * f.n_kv_heads + kvh) * f.page_size + pos % f.page_size;
+    if (rowi[u] < 0) continue;
+    const size_t row = (size_t)rowi[u];
     if (head < f.n_q_heads + f.n_kv_heads) {
       f.k_pool[row * D + j] = f32_to_bf16(y0);
       f.k_pool[row * D + j + half] = f32_to_bf16(y1);

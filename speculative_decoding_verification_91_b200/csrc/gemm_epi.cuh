@@ -12,6 +12,7 @@ namespace sv {
 constexpr int kTileN = 128;     // weight rows (output features / vocab entries) per tile
 constexpr int kTileK = 64;      // bf16 elements per 128-byte K chunk
 constexpr int kEpiThreads = 128;
+constexpr int kEpiMaxRows = 16;   // rows the last-CTA epilogues handle (more: the grid-wide reduce)
 
 struct Args {
   int M, N, K, kchunks, splits, n_tiles;
@@ -101,11 +102,25 @@ __device__ __forceinline__ void argmax_finish(const Args& a, int n_parts, int mb
   }
 }
 
+// The split partials of one 128-feature tile are, per split, one contiguous
+// block of 128 x ldp floats (feature-major, rows contiguous, ldp a multiple of
+// 8).  The last-CTA epilogues below read them as float4 runs of four rows of
+// one feature, so that a warp's loads cover 512 contiguous bytes, and keep the
+// loads of several splits in flight before adding them in split order
+// (starting from 0, exactly as splitk_reduce_kernel does).
+__device__ __forceinline__ float4 add4_rn(float4 s, float4 v) {
+  return make_float4(__fadd_rn(s.x, v.x), __fadd_rn(s.y, v.y), __fadd_rn(s.z, v.z), __fadd_rn(s.w, v.w));
+}
+__device__ __forceinline__ float lane4(const float4& v, int e) {
+  return e == 0 ? v.x : e == 1 ? v.y : e == 2 ? v.z : v.w;
+}
+
 // QKV projection epilogue: after this CTA published its split partial, the
 // last CTA to finish a head (all splits of its D/128 column tiles) sums the
 // partials in split order, rotates each (j, j + D/2) pair of query and key
 // heads at its row's position and writes queries to the workspace and keys,
-// values and the key-equals-value side-band to the cache pools.
+// values and the key-equals-value side-band to the cache pools.  Work item =
+// (pair j, four consecutive rows).
 __device__ __forceinline__ void rope_epilogue(const Args& a, int MP, int n_tile, int mblk, int m0,
                                               int ctid, int* flag) {
   const RopeFuse& f = a.rope;
@@ -119,84 +134,116 @@ __device__ __forceinline__ void rope_epilogue(const Args& a, int MP, int n_tile,
   if (!*flag) return;
   __threadfence();
   const int mcount = min(MP, a.M - m0);
-  const size_t split_stride = (size_t)a.n_tiles * kTileN * a.ldp;
-  const int n_items = half * mcount;
-  for (int it0 = ctid; it0 < n_items; it0 += 2 * kEpiThreads) {
-   float xs0[2] = {0.f, 0.f}, xs1[2] = {0.f, 0.f};
-   for (int sp0 = 0; sp0 < a.splits; sp0 += 8) {
-    float u0[2][8], u1[2][8];
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int item = it0 + u * kEpiThreads;
-      const int mm = item / half, j = item % half;
-      const int f0 = head * D + j, f1 = f0 + half;
-      const float* p0 = a.partial + (size_t)f0 * a.ldp + m0 + mm;
-      const float* p1 = a.partial + (size_t)f1 * a.ldp + m0 + mm;
-#pragma unroll
-      for (int w = 0; w < 8; ++w) {
-        const bool ok = item < n_items && sp0 + w < a.splits;
-        u0[u][w] = ok ? __ldcg(p0 + (size_t)(sp0 + w) * split_stride) : 0.f;
-        u1[u][w] = ok ? __ldcg(p1 + (size_t)(sp0 + w) * split_stride) : 0.f;
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < 2; ++u)
-#pragma unroll
-      for (int w = 0; w < 8; ++w)
-        if (sp0 + w < a.splits) {
-          xs0[u] = __fadd_rn(xs0[u], u0[u][w]);
-          xs1[u] = __fadd_rn(xs1[u], u1[u][w]);
-        }
-   }
-   for (int u = 0; u < 2; ++u) {
-    const int item = it0 + u * kEpiThreads;
-    if (item >= n_items) break;
-    const int mm = item / half, j = item % half;
-    const float x0 = xs0[u], x1 = xs1[u];
-    const int m = m0 + mm, b = m / f.q, i = m % f.q;
-    const bool rot = j < f.n_rot && head < f.n_q_heads + f.n_kv_heads;
-    float y0 = x0, y1 = x1;
-    if (rot) {
-      const float2 cs = f.rope_tab[(size_t)m * half + j];
-      rope_pair(x0, x1, cs.x, cs.y, y0, y1);
-    }
-    if (head < f.n_q_heads) {
-      uint16_t* qo = f.q_out + ((size_t)m * f.n_q_heads + head) * D;
-      qo[j] = f32_to_bf16(y0);
-      qo[j + half] = f32_to_bf16(y1);
-      continue;
-    }
-    const int pos = f.seq_lens[b] + i;
-    if (pos < 0 || pos / f.page_size >= f.max_pages) {
-      flag_status(a.status, SPEC_DEV_BAD_LENGTH);
-      continue;
-    }
-    const int page = f.block_table[(size_t)b * f.max_pages + pos / f.page_size];
-    if (page < 0 || page >= f.num_pages) {
-      flag_status(a.status, SPEC_DEV_BAD_PAGE);
-      continue;
-    }
+  const int ld = a.ldp, q4 = ld / 4;
+  const size_t split_stride = (size_t)a.n_tiles * kTileN * ld;
+  const int n_items = half * q4;
+  // cache row of every verify row of a key or value head, once per row
+  // (-1: invalid length or page, flagged)
+  __shared__ long long row_s[kEpiMaxRows];
+  if (head >= f.n_q_heads && ctid < mcount) {
+    const int m = m0 + ctid, b = m / f.q, i = m % f.q;
     const int kvh = head < f.n_q_heads + f.n_kv_heads ? head - f.n_q_heads
                                                       : head - f.n_q_heads - f.n_kv_heads;
-    const size_t row = ((size_t)page * f.n_kv_heads + kvh) * f.page_size + pos % f.page_size;
-    if (head < f.n_q_heads + f.n_kv_heads) {
-      f.k_pool[row * D + j] = f32_to_bf16(y0);
-      f.k_pool[row * D + j + half] = f32_to_bf16(y1);
-      if (f.ksb_pool && j < f.n_rot) {
-        f.ksb_pool[row * 2 * f.n_rot + j] = f32_to_bf16(x0);
-        f.ksb_pool[row * 2 * f.n_rot + f.n_rot + j] = f32_to_bf16(x1);
-      }
+    const int pos = f.seq_lens[b] + i;
+    long long r = -1;
+    if (pos < 0 || pos / f.page_size >= f.max_pages) {
+      flag_status(a.status, SPEC_DEV_BAD_LENGTH);
     } else {
-      f.v_pool[row * D + j] = f32_to_bf16(x0);
-      f.v_pool[row * D + j + half] = f32_to_bf16(x1);
+      const int page = f.block_table[(size_t)b * f.max_pages + pos / f.page_size];
+      if (page < 0 || page >= f.num_pages)
+        flag_status(a.status, SPEC_DEV_BAD_PAGE);
+      else
+        r = ((long long)page * f.n_kv_heads + kvh) * f.page_size + pos % f.page_size;
     }
-   }
+    row_s[ctid] = r;
+  }
+  named_bar(1, kEpiThreads);
+  constexpr int kU = 4;                  // items per thread per pass
+  for (int it0 = ctid; it0 < n_items; it0 += kU * kEpiThreads) {
+    float4 s0[kU], s1[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) s0[u] = s1[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int sp0 = 0; sp0 < a.splits; sp0 += 2) {
+      float4 v0[kU][2], v1[kU][2];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int item = it0 + u * kEpiThreads;
+        const int j = item / q4, mq = (item % q4) * 4;
+        const float* p0 = a.partial + (size_t)(head * D + j) * ld + m0 + mq;
+        const float* p1 = p0 + (size_t)half * ld;
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          const bool ok = item < n_items && sp0 + w < a.splits;
+          const size_t o = (size_t)(sp0 + w) * split_stride;
+          v0[u][w] = ok ? __ldcg(reinterpret_cast<const float4*>(p0 + o)) : make_float4(0.f, 0.f, 0.f, 0.f);
+          v1[u][w] = ok ? __ldcg(reinterpret_cast<const float4*>(p1 + o)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u)
+#pragma unroll
+        for (int w = 0; w < 2; ++w)
+          if (sp0 + w < a.splits) {
+            s0[u] = add4_rn(s0[u], v0[u][w]);
+            s1[u] = add4_rn(s1[u], v1[u][w]);
+          }
+    }
+    // every load before the first store (a store may alias a later load as
+    // far as the compiler knows): the (cos, sin) entries of rotated pairs
+    const bool rot_head = head < f.n_q_heads + f.n_kv_heads;
+    float2 cs[kU][4];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int item = it0 + u * kEpiThreads;
+      const int j = item / q4, mq = (item % q4) * 4;
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        cs[u][e] = (item < n_items && mq + e < mcount && rot_head && j < f.n_rot)
+                       ? f.rope_tab[(size_t)(m0 + mq + e) * half + j]
+                       : make_float2(1.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int item = it0 + u * kEpiThreads;
+      if (item >= n_items) break;
+      const int j = item / q4, mq = (item % q4) * 4;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int mm = mq + e;
+        if (mm >= mcount) break;
+        const float x0 = lane4(s0[u], e), x1 = lane4(s1[u], e);
+        const int m = m0 + mm;
+        float y0 = x0, y1 = x1;
+        if (rot_head && j < f.n_rot) rope_pair(x0, x1, cs[u][e].x, cs[u][e].y, y0, y1);
+        if (head < f.n_q_heads) {
+          uint16_t* qo = f.q_out + ((size_t)m * f.n_q_heads + head) * D;
+          qo[j] = f32_to_bf16(y0);
+          qo[j + half] = f32_to_bf16(y1);
+          continue;
+        }
+        const long long rowi = row_s[mm];
+        if (rowi < 0) continue;
+        const size_t row = (size_t)rowi;
+        if (head < f.n_q_heads + f.n_kv_heads) {
+          f.k_pool[row * D + j] = f32_to_bf16(y0);
+          f.k_pool[row * D + j + half] = f32_to_bf16(y1);
+          if (f.ksb_pool && j < f.n_rot) {
+            f.ksb_pool[row * 2 * f.n_rot + j] = f32_to_bf16(x0);
+            f.ksb_pool[row * 2 * f.n_rot + f.n_rot + j] = f32_to_bf16(x1);
+          }
+        } else {
+          f.v_pool[row * D + j] = f32_to_bf16(x0);
+          f.v_pool[row * D + j + half] = f32_to_bf16(x1);
+        }
+      }
+    }
   }
   if (ctid == 0) a.tickets[mblk * n_heads + head] = 0u;
 }
 
 // After this CTA published its split partial: the last split of the tile
 // sums all partials in split order and applies the store / residual epilogue.
+// Work item = (output feature r, four consecutive rows).
 template <int MODE>
 __device__ __forceinline__ void splitk_finish(const Args& a, int MP, int n_tile, int mblk, int m0,
                                               int ctid, int* flag) {
@@ -208,46 +255,61 @@ __device__ __forceinline__ void splitk_finish(const Args& a, int MP, int n_tile,
   named_bar(1, kEpiThreads);
   if (!*flag) return;
   __threadfence();
-  // last split of this tile: sum partials in split order, then the epilogue.
-  // Work item = (output feature r, row mm); the split loads of an item are
-  // issued together (independent) and then added in split order.
   const int mcount = min(MP, a.M - m0);
-  const size_t split_stride = (size_t)a.n_tiles * kTileN * a.ldp;
-  const float* base = a.partial + (size_t)n_tile * kTileN * a.ldp + m0;
-  const int n_items = kTileN * mcount;
-  // four items per thread at a time, their split loads issued together
-  for (int it0 = ctid; it0 < n_items; it0 += 4 * kEpiThreads) {
-    float s[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int sp0 = 0; sp0 < a.splits; sp0 += 8) {
-      float v[4][8];
+  const int ld = a.ldp, q4 = ld / 4;
+  const size_t split_stride = (size_t)a.n_tiles * kTileN * ld;
+  const float* base = a.partial + (size_t)n_tile * kTileN * ld + m0;
+  const int n_items = kTileN * q4;
+  constexpr int kU = 4;
+  for (int it0 = ctid; it0 < n_items; it0 += kU * kEpiThreads) {
+    float4 s[kU];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < kU; ++u) s[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int sp0 = 0; sp0 < a.splits; sp0 += 4) {
+      float4 v[kU][4];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
         const int item = it0 + u * kEpiThreads;
-        const int mm = item / kTileN, r = item % kTileN;
-        const float* p = base + (size_t)r * a.ldp + mm;
+        const float* p = base + (size_t)(item / q4) * ld + (item % q4) * 4;
 #pragma unroll
-        for (int w = 0; w < 8; ++w)
-          v[u][w] = (item < n_items && sp0 + w < a.splits) ? __ldcg(p + (size_t)(sp0 + w) * split_stride)
-                                                           : 0.f;
+        for (int w = 0; w < 4; ++w)
+          v[u][w] = (item < n_items && sp0 + w < a.splits)
+                        ? __ldcg(reinterpret_cast<const float4*>(p + (size_t)(sp0 + w) * split_stride))
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
+      for (int u = 0; u < kU; ++u)
 #pragma unroll
-        for (int w = 0; w < 8; ++w)
-          if (sp0 + w < a.splits) s[u] = __fadd_rn(s[u], v[u][w]);
+        for (int w = 0; w < 4; ++w)
+          if (sp0 + w < a.splits) s[u] = add4_rn(s[u], v[u][w]);
+    }
+    // the residuals are read before the first store (a store may alias a
+    // later load as far as the compiler knows)
+    float res[kU][4];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int item = it0 + u * kEpiThreads;
+      const int n = n_tile * kTileN + item / q4, mq = (item % q4) * 4;
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        res[u][e] = (MODE == kGemmResidual && item < n_items && n < a.N && mq + e < mcount)
+                        ? a.out[(size_t)(m0 + mq + e) * a.N + n]
+                        : 0.f;
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < kU; ++u) {
       const int item = it0 + u * kEpiThreads;
-      if (item >= n_items) continue;
-      const int mm = item / kTileN, r = item % kTileN;
+      if (item >= n_items) break;
+      const int r = item / q4, mq = (item % q4) * 4;
       const int n = n_tile * kTileN + r;
       if (n >= a.N) continue;
-      float* dst = a.out + (size_t)(m0 + mm) * a.N + n;
-      if (MODE == kGemmResidual)
-        *dst = __fadd_rn(*dst, s[u]);
-      else
-        *dst = s[u];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int mm = mq + e;
+        if (mm >= mcount) break;
+        float* dst = a.out + (size_t)(m0 + mm) * a.N + n;
+        *dst = (MODE == kGemmResidual) ? __fadd_rn(res[u][e], lane4(s[u], e)) : lane4(s[u], e);
+      }
     }
   }
   if (ctid == 0) a.tickets[mblk * a.n_tiles + n_tile] = 0u;
