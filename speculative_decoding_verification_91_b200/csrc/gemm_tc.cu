@@ -35,6 +35,8 @@ constexpr int kTcThreads = 192;
 constexpr int kTcMaxRows = 256;              // verify rows per TMEM accumulator (MMA N)
 constexpr int kTcEpiWarp0 = 2;
 constexpr uint32_t kABytes = kTileN * 128;   // 16 KB weight tile per stage
+// LM heads with more (padded) rows than this take two weight tiles per CTA
+constexpr int kPairMinRows = 128;
 
 // barriers, TMEM slot, flags, then red_v / red_i [4][256] for the argmax
 constexpr uint32_t kTailBytes = 256u + 2u * 4u * 256u * 4u;
@@ -45,11 +47,12 @@ struct TcLayout {
   uint32_t smem;          // dynamic shared memory bytes
 };
 
-__host__ __device__ inline TcLayout tc_layout(int np) {
+// nw weight tiles per CTA: 1 (two CTAs per SM when the ring fits 2 stages in
+// ~110 KB), or 2 (one CTA per SM, the whole shared memory)
+__host__ __device__ inline TcLayout tc_layout(int np, int nw) {
   TcLayout t{};
-  t.stage_bytes = kABytes + (uint32_t)np * 128u;
-  // two CTAs per SM when the ring fits 2 stages in ~110 KB, else one
-  const uint32_t budget = 110u * 1024u;
+  t.stage_bytes = (uint32_t)nw * kABytes + (uint32_t)np * 128u;
+  const uint32_t budget = nw == 1 ? 110u * 1024u : 227u * 1024u;
   int s = (int)((budget - 1024u - kTailBytes) / t.stage_bytes);
   s = s < 2 ? 2 : (s > 6 ? 6 : s);
   t.stages = s;
@@ -57,11 +60,12 @@ __host__ __device__ inline TcLayout tc_layout(int np) {
   return t;
 }
 
-template <int MODE>
-__global__ void __launch_bounds__(kTcThreads, 2) tc_gemm_kernel(
+template <int MODE, int NW>
+__global__ void __launch_bounds__(kTcThreads, NW == 1 ? 2 : 1) tc_gemm_kernel(
     const __grid_constant__ CUtensorMap tw, const __grid_constant__ CUtensorMap tx, Args a) {
+  static_assert(NW == 1 || (NW == 2 && MODE == kGemmArgmax), "weight tiles per CTA");
   const int np = a.np;
-  const TcLayout L = tc_layout(np);
+  const TcLayout L = tc_layout(np, NW);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -77,7 +81,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) tc_gemm_kernel(
 
   pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_tile = blockIdx.x, split = blockIdx.y, mblk = blockIdx.z;
+  const int n_tile = blockIdx.x * NW, split = blockIdx.y, mblk = blockIdx.z;   // first weight tile
   const int m0 = mblk * kTcMaxRows;          // first verify row of this block
   const int kc0 = (int)((long)split * a.kchunks / a.splits);
   const int kc1 = (int)((long)(split + 1) * a.kchunks / a.splits);
@@ -93,7 +97,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) tc_gemm_kernel(
     *fail = 0;
     fence_barrier_init();
   }
-  if (warp == 1) tmem_alloc(tmem_slot, ncols);
+  if (warp == 1) tmem_alloc(tmem_slot, ncols * NW);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -107,14 +111,18 @@ __global__ void __launch_bounds__(kTcThreads, 2) tc_gemm_kernel(
       const uint64_t pol_w = policy_evict_first();
       const uint64_t pol_x = policy_evict_last();
       const int pre = min(nk, L.stages);
+      // (a weight tile past N reads zeros; its rows are masked in the epilogue)
       for (int it = 0; it < pre; ++it) {
         mbar_arrive_expect_tx(&full[it], L.stage_bytes);
-        tma_load_2d(smem + it * L.stage_bytes, &tw, &full[it], (kc0 + it) * kTileK, n_tile * kTileN,
-                    pol_w);
+#pragma unroll
+        for (int w = 0; w < NW; ++w)
+          tma_load_2d(smem + it * L.stage_bytes + w * kABytes, &tw, &full[it], (kc0 + it) * kTileK,
+                      (n_tile + w) * kTileN, pol_w);
       }
       pdl_wait();
       for (int it = 0; it < pre; ++it)
-        tma_load_2d(smem + it * L.stage_bytes + kABytes, &tx, &full[it], (kc0 + it) * kTileK, m0, pol_x);
+        tma_load_2d(smem + it * L.stage_bytes + NW * kABytes, &tx, &full[it], (kc0 + it) * kTileK, m0,
+                    pol_x);
       int issued = pre;
       for (int it = pre; it < nk; ++it) {
         const int s = it % L.stages;
@@ -125,8 +133,9 @@ __global__ void __launch_bounds__(kTcThreads, 2) tc_gemm_kernel(
         uint8_t* st = smem + s * L.stage_bytes;
         mbar_arrive_expect_tx(&full[s], L.stage_bytes);
         const int kx = (kc0 + it) * kTileK;
-        tma_load_2d(st, &tw, &full[s], kx, n_tile * kTileN, pol_w);
-        tma_load_2d(st + kABytes, &tx, &full[s], kx, m0, pol_x);
+#pragma unroll
+        for (int w = 0; w < NW; ++w) tma_load_2d(st + w * kABytes, &tw, &full[s], kx, (n_tile + w) * kTileN, pol_w);
+        tma_load_2d(st + NW * kABytes, &tx, &full[s], kx, m0, pol_x);
         issued = it + 1;
       }
       for (int it = (issued > L.stages ? issued - L.stages : 0); it < issued; ++it)
@@ -145,11 +154,13 @@ __global__ void __launch_bounds__(kTcThreads, 2) tc_gemm_kernel(
         }
         tc_fence_after();
         const uint32_t a_addr = smem_u32(smem + s * L.stage_bytes);
-        const uint32_t b_addr = a_addr + kABytes;
+        const uint32_t b_addr = a_addr + NW * kABytes;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)   // K = 16 per MMA: +32 bytes inside the swizzled rows
-          umma_bf16(tmem, sw128_desc(a_addr + kk * 32), sw128_desc(b_addr + kk * 32), idesc,
-                    (it > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+          for (int w = 0; w < NW; ++w)   // accumulator w: weight tile n_tile + w
+            umma_bf16(tmem + w * ncols, sw128_desc(a_addr + w * kABytes + kk * 32), sw128_desc(b_addr + kk * 32),
+                      idesc, (it > 0 || kk > 0) ? 1u : 0u);
         umma_commit(&empty[s]);
         done = it + 1;
       }
@@ -170,7 +181,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) tc_gemm_kernel(
     if (!*fail) {
       const uint32_t tq = tmem + ((uint32_t)(quad * 32) << 16);
       if (MODE == kGemmArgmax) {
-        // per verify row (column): max over this tile's 128 weight rows
+        // per verify row (column): max over this CTA's NW x 128 weight rows
         const int n = n_tile * kTileN + row;
         for (int c0 = 0; c0 < np; c0 += 32) {
           float v[32];
@@ -180,6 +191,21 @@ __global__ void __launch_bounds__(kTcThreads, 2) tc_gemm_kernel(
           for (int j = 0; j < 32; ++j) {
             id[j] = n;
             if (n >= a.N) v[j] = -INFINITY;
+          }
+          if (NW == 2) {
+            // the second tile's row of this thread (ids n + 128 > n: on equal
+            // values the first tile's row wins, as the lower id must)
+            float v2[32];
+            tmem_ld32(tq + ncols + c0, v2);
+            const int n2 = n + kTileN;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float x = n2 < a.N ? v2[j] : -INFINITY;
+              if (better(x, n2, v[j], id[j])) {
+                v[j] = x;
+                id[j] = n2;
+              }
+            }
           }
           // transpose-reduce: after the 5 rounds lane l holds column c0 + l
 #pragma unroll
@@ -233,7 +259,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) tc_gemm_kernel(
   }
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, ncols);
+  if (warp == 1) tmem_dealloc(tmem, ncols * NW);
   if (warp < kTcEpiWarp0 || *fail) return;
 
   // ---- cross-CTA completion of the argmax (epilogue warps only); the other
@@ -241,18 +267,19 @@ __global__ void __launch_bounds__(kTcThreads, 2) tc_gemm_kernel(
   //      the whole grid instead of one CTA per tile
   if (MODE == kGemmArgmax) {
     const int ctid = threadIdx.x - kTcEpiWarp0 * 32;
-    argmax_finish(a, a.n_tiles, mblk, m0, np, ctid, flag, red_i);
+    argmax_finish(a, gridDim.x, mblk, m0, np, ctid, flag, red_i);
   }
 }
 
-template <int MODE>
+template <int MODE, int NW>
 cudaError_t launch_tc_mode(const GemmPlan& p, const CUtensorMap& tw, const CUtensorMap& tx,
                            const Args& a, cudaStream_t st) {
-  auto kern = tc_gemm_kernel<MODE>;
-  const TcLayout L = tc_layout(a.np);
+  auto kern = tc_gemm_kernel<MODE, NW>;
+  const TcLayout L = tc_layout(a.np, NW);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.smem);
   if (e != cudaSuccess) return e;
-  e = launch_k(kern, dim3(p.n_tiles, p.splits, tc_mblocks(p.M)), dim3(kTcThreads), L.smem, st, tw, tx, a);
+  e = launch_k(kern, dim3((p.n_tiles + NW - 1) / NW, p.splits, tc_mblocks(p.M)), dim3(kTcThreads), L.smem,
+               st, tw, tx, a);
   if (e != cudaSuccess || MODE == kGemmArgmax) return e;
   return launch_splitk_reduce(a, MODE, st);
 }
@@ -311,10 +338,14 @@ cudaError_t launch_gemm_tc(const GemmPlan& p, int mode, const void* x, const voi
   if (mode != kGemmArgmax || tc_mblocks(p.M) > 1) a.acc.B = 0;   // acceptance needs every row
   if (b.accept_fused) *b.accept_fused = a.acc.B > 0 ? 1 : 0;
   switch (mode) {
-    case kGemmStore: return launch_tc_mode<kGemmStore>(p, tw, tx, a, st);
-    case kGemmResidual: return launch_tc_mode<kGemmResidual>(p, tw, tx, a, st);
-    case kGemmArgmax: return launch_tc_mode<kGemmArgmax>(p, tw, tx, a, st);
-    case kGemmQkvRope: return launch_tc_mode<kGemmQkvRope>(p, tw, tx, a, st);
+    case kGemmStore: return launch_tc_mode<kGemmStore, 1>(p, tw, tx, a, st);
+    case kGemmResidual: return launch_tc_mode<kGemmResidual, 1>(p, tw, tx, a, st);
+    case kGemmArgmax:
+      // many rows: the MMAs bound the LM head, and two weight tiles per CTA
+      // halve the re-reads of the row tile from L2
+      return np > kPairMinRows ? launch_tc_mode<kGemmArgmax, 2>(p, tw, tx, a, st)
+                               : launch_tc_mode<kGemmArgmax, 1>(p, tw, tx, a, st);
+    case kGemmQkvRope: return launch_tc_mode<kGemmQkvRope, 1>(p, tw, tx, a, st);
   }
   return cudaErrorInvalidValue;
 }

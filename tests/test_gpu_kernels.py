@@ -70,7 +70,7 @@ def test_accept_commit_matches_oracle(k):
 @pytest.mark.parametrize("M,d,V", [(1, 512, 4096), (5, 2560, 9000), (9, 256, 1000),
                                    (40, 1024, 5000), (100, 512, 3000), (64, 2048, 131),
                                    (256, 1024, 5000), (72, 3840, 1000), (300, 1024, 5000),
-                                   (520, 512, 3000)])
+                                   (520, 512, 3000), (144, 768, 4400), (256, 512, 129)])
 def test_lmhead_argmax_matches_oracle(M, d, V):
     h = gen.normal_bf16(1, f"test/lm/h/{M}/{d}", 0, M * d, 1.0).reshape(M, d)
     w = gen.normal_bf16(1, f"test/lm/w/{d}/{V}", 0, V * d, 0.02).reshape(V, d)
