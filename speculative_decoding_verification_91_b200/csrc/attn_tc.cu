@@ -466,6 +466,37 @@ __global__ void __launch_bounds__(kFaThreads, 1) attn_fa_kernel(
       uint32_t polls = 0;
       while (ip < count) {
         bool progressed = false;
+        // P . V first: it frees a stage for the next copy
+        if (npv < nqk) {
+          bool ready = mbar_test_wait(&p_full[npv % NPB], (npv / NPB) & 1);
+          if (jp == 0 && ip >= NOB) ready = ready && mbar_test_wait(&o_free[ip % NOB], ((ip / NOB) - 1) & 1);
+          if (ready) {
+            tc_fence_after();
+            const uint32_t v_addr = smem_u32(stage + (npv % NS) * C::kStage) + (KVEQ ? 0u : 4u * kAtom);
+            const uint32_t p_addr = smem_u32(pbuf + (npv % NPB) * C::kPBytes);
+            const uint32_t t_o = tmem + (ip % NOB) * (C::kOTiles * NP);
+#pragma unroll
+            for (int t = 0; t < C::kOTiles; ++t) {
+              // [atom 2t ; atom 2t+1] (the side-band tile pairs its atom with the
+              // next 8 KB of shared memory, whose lanes are never read)
+              const uint32_t a0 = v_addr + 2 * t * kAtom;
+#pragma unroll
+              for (int kk = 0; kk < kPg / 16; ++kk) {    // K = 16 keys per MMA
+                const uint64_t ad = sw128_desc_mn(a0 + kk * 2048, kAtom);
+                umma_bf16(t_o + t * NP, ad, sw128_desc(p_addr + kk * 32), id_pv, (jp > 0 || kk > 0) ? 1u : 0u);
+              }
+            }
+            umma_commit(&pv_done[npv % NPB]);
+            umma_commit(&k_empty[npv % NS]);
+            ++npv;
+            if (++jp >= wp.np) {
+              jp = 0;
+              ++ip;
+              if (ip < count) wp.next();
+            }
+            progressed = true;
+          }
+        }
         if (is < count && nqk - npv < NSB) {
           const bool newq = js == 0 && ws.new_q;
           const int qb = (nq_used + 1) % C::kQBufs;
@@ -499,36 +530,6 @@ __global__ void __launch_bounds__(kFaThreads, 1) attn_fa_kernel(
               js = 0;
               ++is;
               if (is < count) ws.next();
-            }
-            progressed = true;
-          }
-        }
-        if (npv < nqk) {
-          bool ready = mbar_test_wait(&p_full[npv % NPB], (npv / NPB) & 1);
-          if (jp == 0 && ip >= NOB) ready = ready && mbar_test_wait(&o_free[ip % NOB], ((ip / NOB) - 1) & 1);
-          if (ready) {
-            tc_fence_after();
-            const uint32_t v_addr = smem_u32(stage + (npv % NS) * C::kStage) + (KVEQ ? 0u : 4u * kAtom);
-            const uint32_t p_addr = smem_u32(pbuf + (npv % NPB) * C::kPBytes);
-            const uint32_t t_o = tmem + (ip % NOB) * (C::kOTiles * NP);
-#pragma unroll
-            for (int t = 0; t < C::kOTiles; ++t) {
-              // [atom 2t ; atom 2t+1] (the side-band tile pairs its atom with the
-              // next 8 KB of shared memory, whose lanes are never read)
-              const uint32_t a0 = v_addr + 2 * t * kAtom;
-#pragma unroll
-              for (int kk = 0; kk < kPg / 16; ++kk) {    // K = 16 keys per MMA
-                const uint64_t ad = sw128_desc_mn(a0 + kk * 2048, kAtom);
-                umma_bf16(t_o + t * NP, ad, sw128_desc(p_addr + kk * 32), id_pv, (jp > 0 || kk > 0) ? 1u : 0u);
-              }
-            }
-            umma_commit(&pv_done[npv % NPB]);
-            umma_commit(&k_empty[npv % NS]);
-            ++npv;
-            if (++jp >= wp.np) {
-              jp = 0;
-              ++ip;
-              if (ip < count) wp.next();
             }
             progressed = true;
           }
