@@ -5,46 +5,43 @@
 // keys).  Items are ordered (b, kv head, row block, split) and every CTA (one
 // per SM) takes a contiguous range of them, so consecutive items mostly share
 // their queries; its producer streams their keys without a break between
-// items.  Keys are visited one 64-token page at a time, so that several pages
-// are in flight per SM (a page is held from its copy until P . V of it has
-// completed).  10 warps:
-//   warp 0    TMA producer.  A page arrives as four 64 x 64 swizzled key atoms
-//             plus, on key-equals-value layers, the side-band atom (pre-RoPE
-//             rotated dims; 40 KB, four stages), or plus four value atoms on
-//             separate-K/V layers (64 KB, three stages).  Queries come by a 3D
-//             TMA box {64 dims, G heads, PB positions} straight from the
-//             rotated-query buffer, once per (b, kv head, row block).
+// items.  10 warps:
+//   warp 0    TMA producer.  Keys arrive in blocks of 128 (two 64-token pages)
+//             as four 128 x 64 swizzled atoms; on key-equals-value layers the
+//             side-band atom (pre-RoPE rotated dims) rides with the keys (two
+//             stages), on separate-K/V layers keys have two stages and values
+//             one buffer.  Queries come by a 3D TMA box {64 dims, G heads, PB
+//             positions} straight from the rotated-query buffer, once per
+//             (b, kv head, row block).
 //   warp 1    allocates TMEM and issues the MMAs (one thread):
-//               S^T[64 keys][NP rows]  = K . Q^T          (M = 64, A = K)
-//               O^T[dims][NP rows]    += V^T . P^T        (M = 128, A = V^T,
-//                                                          MN-major)
+//               S^T[128 keys][NP rows] = K . Q^T          (A = K, K-major)
+//               O^T[dims][NP rows]    += V^T . P^T        (A = V^T, MN-major)
 //             accumulators in TMEM (lane = key or value dim, column = query
-//             row).  Scores run up to kSBufs pages ahead of the softmax; the
-//             output has two buffers, so P . V of an item's first page does
-//             not wait for the previous item's output to be read out.
-//   warps 2-9 softmax: in the M = 64 score layout key 16q + l of the page sits
-//             on TMEM lane 32q + l, so lanes 0-15 of the warp of lane
-//             quadrant q own one key each; the warps of one half of the
-//             columns (query rows) form a group of 128 threads.  Per page:
-//             the scores of the thread's key for its NP/2 rows; p = 2^(s - m)
-//             against a per-row reference maximum m that moves only when a
-//             page maximum exceeds it by more than 2^8 (one OR-vote per page
-//             decides; the exact page maxima are reduced only then, and the
-//             running output is rescaled in TMEM only for rows that moved);
-//             p is written once as bf16 for P . V and summed unrounded into
-//             per-thread row sums, reduced over the keys at the end of the
-//             item, when (m, l) go out.  The output o of an item is read out
-//             of TMEM one page later, after the next item's first page, when
-//             its last P . V has long completed.  Partials go out in the
-//             layout the split combine reads.
+//             row); the scores of the next block are computed while the
+//             softmax works on the current one (two score buffers), and the
+//             output has two buffers by item parity, so P . V of an item's
+//             first block never waits for the previous item's read-out.
+//   warps 2-9 softmax: thread t of a lane quadrant owns key t of the block;
+//             the warps of one half of the columns (query rows) form a group
+//             of 128 threads.  Per block: the scores of the thread's key for
+//             its NP/2 rows; p = 2^(s - m) against a per-row reference maximum
+//             m that moves only when a block maximum exceeds it by more than
+//             2^8 (one OR-vote per block decides; the exact block maxima are
+//             reduced only then, and the running output is rescaled in TMEM
+//             only for rows that moved); p is written once as bf16 for P . V
+//             and summed unrounded into per-thread row sums, reduced over the
+//             keys at the end of the item, when (m, l) go out; the item's o is
+//             read out of TMEM one block later, after the next item's first
+//             block.  The partials go out in the layout the split combine reads.
 //
 // Value rows of keys outside the item's range (or on pages that were not
 // loaded) are zeroed in shared memory before P . V, so stale or poisoned
-// slots never reach it.  A row's reference maximum, its probabilities and the
-// reduction trees depend only on its own scores and absolute key positions,
-// so a row's partial does not depend on k, the batch, its row slot or the
-// CTA that computed it.  Every wait is bounded; after a timeout the CTA stops
-// issuing work, drains what it issued, writes nothing and frees its TMEM.
+// slots never reach it.  Keys are visited in blocks at absolute 128-key
+// boundaries; a row's reference maximum, its probabilities and the reduction
+// trees depend only on its own scores and absolute key positions, so a row's
+// partial does not depend on k, the batch, its row slot or the CTA that
+// computed it.  Every wait is bounded; after a timeout the CTA stops issuing
+// work, drains what it issued, writes nothing and frees its TMEM.
 #include <math.h>
 
 #include <algorithm>
@@ -58,14 +55,16 @@ namespace sv {
 
 namespace {
 
-constexpr int kPg = 64;                      // tokens per page = keys per block
+constexpr int kBlk = 128;                    // keys per MMA block
+constexpr int kPg = 64;                      // tokens per page
 constexpr int kDim = 256;                    // head_dim of this kernel
-constexpr uint32_t kAtom = kPg * 128;        // 64 keys x 64 dims of bf16: 8 KB
+constexpr uint32_t kAtom = kBlk * 128;       // 128 keys x 64 dims of bf16: 16 KB
+constexpr uint32_t kHalfAtom = kPg * 128;    // one page's rows of an atom: 8 KB
 constexpr int kSoftWarps = 8;
 constexpr int kFaThreads = (2 + kSoftWarps) * 32;
 constexpr uint32_t kSmemMax = 227u * 1024u;
 constexpr uint32_t kTailBytes = 4096;
-// p <= 2^kLazy: a row's reference maximum moves only when a page maximum
+// p <= 2^kLazy: a row's reference maximum moves only when a block maximum
 // exceeds it by more than this (log2 domain)
 constexpr float kLazy = 8.f;
 constexpr int kMaxItemPages = 128;           // pages one item (split) may span
@@ -83,40 +82,34 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// Instruction descriptor, kind::f16 with M = 64: D fp32, A and B bf16, both
-// K-major, N = n.
-__device__ __forceinline__ uint32_t idesc_bf16_m64(int n) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(64 >> 4) << 24);
-}
-
 template <bool KVEQ, int NP>
 struct FaCfg {
-  static constexpr int kStages = KVEQ ? 4 : 3;
-  static constexpr uint32_t kStage = (KVEQ ? 5u : 8u) * kAtom;   // keys + side-band, or keys + values
+  static constexpr uint32_t kStage = 4 * kAtom + (KVEQ ? kAtom : 0);   // keys (+ side-band)
+  static constexpr uint32_t kVBytes = KVEQ ? 0 : 4 * kAtom;           // separate values
   static constexpr uint32_t kQBytes = 4u * NP * 128u;
-  static constexpr uint32_t kPBytes = NP * 128u;                 // [NP rows][64 keys]
+  static constexpr uint32_t kPBytes = 2u * NP * 128u;                 // [NP rows][128 keys]
   static constexpr uint32_t bytes(int pb, int qb) {
-    return 1024u + kStages * kStage + pb * kPBytes + qb * kQBytes + kTailBytes;
+    return 1024u + 2u * kStage + kVBytes + pb * kPBytes + qb * kQBytes + kTailBytes;
   }
-  static constexpr int kPBufs = bytes(4, 1) <= kSmemMax ? 4 : bytes(3, 1) <= kSmemMax ? 3 : 2;
+  static constexpr int kPBufs = bytes(2, 1) <= kSmemMax ? 2 : 1;
   static constexpr int kQBufs = bytes(kPBufs, 2) <= kSmemMax ? 2 : 1;
-  static constexpr uint32_t kOffP = kStages * kStage;
+  static constexpr uint32_t kOffV = 2 * kStage;
+  static constexpr uint32_t kOffP = kOffV + kVBytes;
   static constexpr uint32_t kOffQ = kOffP + kPBufs * kPBytes;
   static constexpr uint32_t kOffTail = kOffQ + kQBufs * kQBytes;
   static constexpr uint32_t kSmem = 1024 + kOffTail + kTailBytes;
   static constexpr int kOTiles = KVEQ ? 3 : 2;
-  static constexpr int kOBufs = 2;
-  static constexpr uint32_t kColS = kOBufs * kOTiles * NP;        // score buffers after the outputs
-  static constexpr int kSBufs = (512 - (int)kColS) / NP >= 4 ? 4 : (512 - (int)kColS) / NP;
-  static constexpr uint32_t kCols = kColS + kSBufs * NP;
+  static constexpr int kOBufs = 2;                       // output accumulators (by item parity)
+  static constexpr uint32_t kColS = kOBufs * kOTiles * NP;   // two score buffers after the outputs
+  static constexpr uint32_t kCols = kColS + 2 * NP;
   static constexpr uint32_t kTmemCols =
       kCols <= 32 ? 32 : kCols <= 64 ? 64 : kCols <= 128 ? 128 : kCols <= 256 ? 256 : 512;
   static_assert(NP % 16 == 0 && NP >= 16 && NP <= 64, "rows per block");
-  static_assert(kSBufs >= 2 && kCols <= 512, "tensor memory");
-  static_assert(bytes(2, 1) <= kSmemMax && kSmem <= kSmemMax, "shared memory");
-  // the side-band MMA pairs each side-band atom with the next 8 KB of shared
-  // memory (lanes never read); for the last stage that is what follows it
-  static_assert(!KVEQ || kOffTail + kTailBytes >= kStages * kStage + kAtom, "side-band pairing");
+  static_assert(kCols <= 512, "tensor memory");
+  static_assert(kSmem <= kSmemMax, "shared memory");
+  // the side-band MMA pairs each side-band atom with the next 16 KB of shared
+  // memory (lanes never read); for the second stage that is what follows it
+  static_assert(!KVEQ || kOffTail + kTailBytes >= 2 * kStage + kAtom, "side-band pairing");
 };
 
 struct FaArgs {
@@ -145,7 +138,7 @@ __device__ __forceinline__ int seq_splits(const FaArgs& a, int L, int& klo, int&
 // walkers see the same sequence.
 struct Walker {
   const FaArgs* a;
-  int b, kvh, rb, sidx, ns, L, lo, hi, pg0, np;
+  int b, kvh, rb, sidx, ns, L, lo, hi, blk0, nb;
   bool new_q;           // this item's queries differ from the previous item's
   __device__ void load_seq() {
     L = a->seq_lens[b];
@@ -158,8 +151,8 @@ struct Walker {
     const int s_abs = klo / a->split + sidx;
     lo = max(s_abs * a->split, klo);
     hi = min(s_abs * a->split + a->split - 1, khi);
-    pg0 = lo / kPg;
-    np = hi / kPg - pg0 + 1;
+    blk0 = lo / kBlk;
+    nb = hi / kBlk - blk0 + 1;
   }
   __device__ void start(const FaArgs* args, int b0, int kvh0, int rb0, int s0) {
     a = args;
@@ -219,26 +212,6 @@ __device__ __forceinline__ float transpose_reduce32(float (&v)[32], int lane) {
   return v[0];
 }
 
-// v[0..15] per lane in, lane l out: the max (or sum) over the 16 lanes of
-// l's half-warp of column l & 15.  Pairing by lane bit 3, 2, 1, 0 for every
-// column, so every column gets the same reduction tree.
-template <bool MAX>
-__device__ __forceinline__ float transpose_reduce16(float (&v)[16], int lane) {
-#pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    const int off = 8 >> r;
-    const bool up = (lane & off) != 0;
-#pragma unroll
-    for (int j = 0; j < off; ++j) {
-      const float send = up ? v[j] : v[j + off];
-      const float keep = up ? v[j + off] : v[j];
-      const float got = __shfl_xor_sync(0xffffffffu, send, off);
-      v[j] = MAX ? fmaxf(keep, got) : __fadd_rn(keep, got);
-    }
-  }
-  return v[0];
-}
-
 // Value dims held by TMEM lane quadrant `quad` of O tile `t`: first dim, or -1.
 // Key-equals-value tiles: [K0;K1] dims 0..127, [K2;K3] dims 128..255 (the
 // rotated dims 0..31 and 128..159 there hold post-RoPE keys and are not
@@ -264,53 +237,48 @@ __global__ void __launch_bounds__(kFaThreads, 1) attn_fa_kernel(
     const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
     const __grid_constant__ CUtensorMap tq, const __grid_constant__ FaArgs a) {
   using C = FaCfg<KVEQ, NP>;
-  constexpr int NS = C::kStages;
-  constexpr int NPB = C::kPBufs;
-  constexpr int NSB = C::kSBufs;
-  constexpr int NOB = C::kOBufs;
   constexpr int NH = NP / 2;                 // columns (query rows) per softmax half
-  constexpr int NQ = NH / 2;                 // columns per thread (a half-warp's share)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* stage = smem;                     // [NS][key atoms + side-band or value atoms]
-  uint8_t* pbuf = smem + C::kOffP;           // [NPB][P]
+  uint8_t* stage = smem;                     // [2][K atoms (+ side-band)]
+  uint8_t* vbuf = smem + C::kOffV;           // separate-K/V values
+  uint8_t* pbuf = smem + C::kOffP;           // [kPBufs][P]
   uint8_t* qbuf = smem + C::kOffQ;           // [kQBufs][Q]
   uint8_t* tail = smem + C::kOffTail;
-  uint64_t* k_full = reinterpret_cast<uint64_t*>(tail);    // [NS]
-  uint64_t* k_empty = k_full + NS;                          // [NS]
-  uint64_t* q_full = k_empty + NS;                          // [2]
+  uint64_t* k_full = reinterpret_cast<uint64_t*>(tail);    // [2]
+  uint64_t* k_empty = k_full + 2;                           // [2]
+  uint64_t* v_full = k_empty + 2;
+  uint64_t* v_empty = v_full + 1;
+  uint64_t* q_full = v_empty + 1;                           // [2]
   uint64_t* q_empty = q_full + 2;                           // [2]
-  uint64_t* s_full = q_empty + 2;                           // [NSB]
-  uint64_t* p_full = s_full + NSB;                          // [NPB]
-  uint64_t* pv_done = p_full + NPB;                         // [NPB]
-  uint64_t* o_free = pv_done + NPB;                         // [NOB]
-  uint64_t* mma_done = o_free + NOB;
+  uint64_t* s_full = q_empty + 2;                           // [2]
+  uint64_t* p_full = s_full + 2;                            // [2] by block parity
+  uint64_t* pv_done = p_full + 2;                           // [2] by block parity
+  uint64_t* o_free = pv_done + 2;                           // [2] by item parity
+  uint64_t* mma_done = o_free + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* fail = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* start = reinterpret_cast<int*>(tmem_slot + 4);      // b, kvh, rb, sidx, count
-  float* red = reinterpret_cast<float*>(tail + 512);       // [2 halves][2 bufs][4 quads][32]
+  float* red = reinterpret_cast<float*>(tail + 256);       // [2 halves][2 bufs][4 quads][32]
   int* pvalid_all = reinterpret_cast<int*>(red + 512);      // [2][kMaxItemPages] page validity of an item
-  static_assert(512 + 512 * 4 + 2 * kMaxItemPages * 4 <= (int)kTailBytes, "tail layout");
-  static_assert((2 * NS + 4 + NSB + 2 * NPB + NOB + 1) * 8 + 32 <= 512, "barriers");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NS; ++i) {
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&k_empty[i], 1);
-    }
-    for (int i = 0; i < 2; ++i) {
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
-    }
-    for (int i = 0; i < NSB; ++i) mbar_init(&s_full[i], 1);
-    for (int i = 0; i < NPB; ++i) {
-      mbar_init(&p_full[i], kSoftWarps);
+      mbar_init(&s_full[i], 1);
       mbar_init(&pv_done[i], 1);
+      mbar_init(&p_full[i], kSoftWarps);
     }
-    for (int i = 0; i < NOB; ++i) mbar_init(&o_free[i], kSoftWarps);
+    mbar_init(v_full, 1);
+    mbar_init(v_empty, 1);
+    mbar_init(&o_free[0], kSoftWarps);
+    mbar_init(&o_free[1], kSoftWarps);
     mbar_init(mma_done, 1);
     *fail = 0;
     fence_barrier_init();
@@ -393,31 +361,52 @@ __global__ void __launch_bounds__(kFaThreads, 1) attn_fa_kernel(
       const uint64_t pol_q = policy_evict_normal();
       Walker w;
       w.start(&a, start[0], start[1], start[2], start[3]);
-      int gk = 0, nq = 0;
-      auto load_page = [&](const Walker& it, int j) -> bool {
-        const int s = gk % NS;
-        if (gk >= NS && !fwait(&k_empty[s], ((gk / NS) - 1) & 1, a.status, fail)) return false;
+      int gk = 0, gv = 0, nq = 0;
+      auto page_id = [&](const Walker& it, int pg) -> int {   // -1 not needed, -2 invalid
+        if (pg * kPg > it.hi || pg * kPg + kPg - 1 < it.lo) return -1;
+        const int id = bt_all[(long)it.b * a.max_pages + pg];
+        return (id >= 0 && id < a.num_pages) ? id : -2;
+      };
+      auto load_k = [&](const Walker& it, int j) -> bool {
+        const int s = gk & 1;
+        if (gk >= 2 && !fwait(&k_empty[s], ((gk >> 1) - 1) & 1, a.status, fail)) return false;
         uint8_t* dst = stage + s * C::kStage;
-        const int pg = it.pg0 + j;
-        int id = bt_all[(long)it.b * a.max_pages + pg];
-        if (id < 0 || id >= a.num_pages) {
-          flag_status(a.status, SPEC_DEV_BAD_PAGE);
-          id = -1;
+        int id[2];
+        uint32_t bytes = 0;
+        for (int h = 0; h < 2; ++h) {
+          id[h] = page_id(it, (it.blk0 + j) * 2 + h);
+          if (id[h] == -2) flag_status(a.status, SPEC_DEV_BAD_PAGE);
+          if (id[h] >= 0) bytes += (KVEQ ? 5u : 4u) * kHalfAtom;
         }
-        mbar_arrive_expect_tx(&k_full[s], id >= 0 ? C::kStage : 0u);
-        if (id >= 0) {
-          const int y = (id * a.Hkv + it.kvh) * kPg;
+        mbar_arrive_expect_tx(&k_full[s], bytes);
+        for (int h = 0; h < 2; ++h) {
+          if (id[h] < 0) continue;
+          const int y = (id[h] * a.Hkv + it.kvh) * kPg;
 #pragma unroll
-          for (int at = 0; at < 4; ++at) tma_load_2d(dst + at * kAtom, &tk, &k_full[s], at * 64, y, pol);
-          if (KVEQ) {
-            tma_load_2d(dst + 4 * kAtom, &tv, &k_full[s], 0, y, pol);
-          } else {
-#pragma unroll
-            for (int at = 0; at < 4; ++at)
-              tma_load_2d(dst + (4 + at) * kAtom, &tv, &k_full[s], at * 64, y, pol);
-          }
+          for (int at = 0; at < 4; ++at)
+            tma_load_2d(dst + at * kAtom + h * kHalfAtom, &tk, &k_full[s], at * 64, y, pol);
+          if (KVEQ) tma_load_2d(dst + 4 * kAtom + h * kHalfAtom, &tv, &k_full[s], 0, y, pol);
         }
         ++gk;
+        return true;
+      };
+      auto load_v = [&](const Walker& it, int j) -> bool {
+        if (gv >= 1 && !fwait(v_empty, (gv - 1) & 1, a.status, fail)) return false;
+        int id[2];
+        uint32_t bytes = 0;
+        for (int h = 0; h < 2; ++h) {
+          id[h] = page_id(it, (it.blk0 + j) * 2 + h);
+          if (id[h] >= 0) bytes += 4u * kHalfAtom;
+        }
+        mbar_arrive_expect_tx(v_full, bytes);
+        for (int h = 0; h < 2; ++h) {
+          if (id[h] < 0) continue;
+          const int y = (id[h] * a.Hkv + it.kvh) * kPg;
+#pragma unroll
+          for (int at = 0; at < 4; ++at)
+            tma_load_2d(vbuf + at * kAtom + h * kHalfAtom, &tv, v_full, at * 64, y, pol);
+        }
+        ++gv;
         return true;
       };
       auto load_q = [&](const Walker& it) -> bool {
@@ -434,33 +423,59 @@ __global__ void __launch_bounds__(kFaThreads, 1) attn_fa_kernel(
         return true;
       };
       bool ok = true;
-      for (int i = 0; ok && i < count; ++i, w.next()) {
-        if (w.new_q) ok = load_q(w);
-        for (int j = 0; ok && j < w.np; ++j) ok = load_page(w, j);
+      if (KVEQ) {
+        for (int i = 0; ok && i < count; ++i, w.next()) {
+          if (w.new_q) ok = load_q(w);
+          for (int j = 0; ok && j < w.nb; ++j) ok = load_k(w, j);
+        }
+      } else {
+        // keys run up to two blocks ahead of the values (a key stage frees
+        // when its scores are done, the value buffer when P . V is done)
+        Walker wk = w;
+        int ik = 0, jk = 0;          // next key block to load: item ik, block jk of wk
+        auto key_ahead = [&](int limit) -> bool {   // load keys while gk < limit
+          while (ik < count && gk < limit) {
+            if (jk == 0 && wk.new_q && !load_q(wk)) return false;
+            if (!load_k(wk, jk)) return false;
+            if (++jk >= wk.nb) {
+              jk = 0;
+              ++ik;
+              if (ik < count) wk.next();
+            }
+          }
+          return true;
+        };
+        int gblk = 0;
+        for (int i = 0; ok && i < count; ++i, w.next()) {
+          for (int j = 0; ok && j < w.nb; ++j, ++gblk) {
+            ok = key_ahead(gblk + 2) && load_v(w, j);
+          }
+        }
       }
       // every issued copy must land before the CTA may exit
-      for (int i = (gk > NS ? gk - NS : 0); i < gk; ++i) mbar_wait(&k_full[i % NS], (i / NS) & 1, a.status);
+      for (int i = (gk > 2 ? gk - 2 : 0); i < gk; ++i) mbar_wait(&k_full[i & 1], (i >> 1) & 1, a.status);
+      if (gv > 0) mbar_wait(v_full, (gv - 1) & 1, a.status);
       for (int i = (nq > C::kQBufs ? nq - C::kQBufs : 0); i < nq; ++i)
         mbar_wait(&q_full[i % C::kQBufs], (i / C::kQBufs) & 1, a.status);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0 && count > 0) {
-      const uint32_t id_qk = idesc_bf16_m64(NP);
+      const uint32_t id_qk = idesc_bf16(NP);
       const uint32_t id_pv = idesc_bf16(NP, true);
-      // The scores of page g (QK) and the product P . V of an earlier page are
+      // The scores of block g (QK) and the product P . V of block g - 1 are
       // independent: each is issued as soon as its inputs are ready (polled
-      // with the non-blocking test, so that waiting for one never delays the
-      // other).
-      //   QK(g):  keys of g landed; score buffer g % NSB read by the softmax
-      //           (P . V of page g - NSB issued); new queries landed at a
-      //           query-group start.
-      //   PV(g):  P(g) written; at an item's first page, the output buffer
-      //           of two items back read out.
+      // with the non-blocking test, P . V first), so P . V never waits for
+      // the next block's keys (which, on key-equals-value layers, could not be
+      // requested before that P . V frees its stage).
+      //   QK(g):  keys of g landed; score buffer g % 2 read by the softmax
+      //           (g <= npv + 1); new queries landed at a query-group start.
+      //   PV(g):  P(g) written; values landed (separate-K/V); at an item's
+      //           first block, the output buffer of two items back read out.
       Walker ws, wp;
       ws.start(&a, start[0], start[1], start[2], start[3]);
       wp = ws;
-      int is = 0, js = 0, ip = 0, jp = 0;   // QK / PV positions: item, page in item
+      int is = 0, js = 0, ip = 0, jp = 0;   // QK / PV positions: item, block in item
       int nqk = 0, npv = 0, nq_used = -1;
       uint64_t t_last = globaltimer_ns();
       uint32_t polls = 0;
@@ -468,28 +483,30 @@ __global__ void __launch_bounds__(kFaThreads, 1) attn_fa_kernel(
         bool progressed = false;
         // P . V first: it frees a stage for the next copy
         if (npv < nqk) {
-          bool ready = mbar_test_wait(&p_full[npv % NPB], (npv / NPB) & 1);
-          if (jp == 0 && ip >= NOB) ready = ready && mbar_test_wait(&o_free[ip % NOB], ((ip / NOB) - 1) & 1);
+          bool ready = mbar_test_wait(&p_full[npv & 1], (npv >> 1) & 1);
+          if (!KVEQ) ready = ready && mbar_test_wait(v_full, npv & 1);
+          if (jp == 0 && ip >= 2) ready = ready && mbar_test_wait(&o_free[ip & 1], ((ip >> 1) - 1) & 1);
           if (ready) {
             tc_fence_after();
-            const uint32_t v_addr = smem_u32(stage + (npv % NS) * C::kStage) + (KVEQ ? 0u : 4u * kAtom);
-            const uint32_t p_addr = smem_u32(pbuf + (npv % NPB) * C::kPBytes);
-            const uint32_t t_o = tmem + (ip % NOB) * (C::kOTiles * NP);
+            const uint32_t v_addr = KVEQ ? smem_u32(stage + (npv & 1) * C::kStage) : smem_u32(vbuf);
+            const uint32_t p_addr = smem_u32(pbuf + (npv % C::kPBufs) * C::kPBytes);
+            const uint32_t t_o = tmem + (ip & 1) * (C::kOTiles * NP);
 #pragma unroll
             for (int t = 0; t < C::kOTiles; ++t) {
               // [atom 2t ; atom 2t+1] (the side-band tile pairs its atom with the
-              // next 8 KB of shared memory, whose lanes are never read)
+              // next 16 KB of shared memory, whose lanes are never read)
               const uint32_t a0 = v_addr + 2 * t * kAtom;
 #pragma unroll
-              for (int kk = 0; kk < kPg / 16; ++kk) {    // K = 16 keys per MMA
+              for (int kk = 0; kk < kBlk / 16; ++kk) {   // K = 16 keys per MMA
                 const uint64_t ad = sw128_desc_mn(a0 + kk * 2048, kAtom);
-                umma_bf16(t_o + t * NP, ad, sw128_desc(p_addr + kk * 32), id_pv, (jp > 0 || kk > 0) ? 1u : 0u);
+                const uint32_t po = (kk >> 2) * (NP * 128) + (kk & 3) * 32;
+                umma_bf16(t_o + t * NP, ad, sw128_desc(p_addr + po), id_pv, (jp > 0 || kk > 0) ? 1u : 0u);
               }
             }
-            umma_commit(&pv_done[npv % NPB]);
-            umma_commit(&k_empty[npv % NS]);
+            umma_commit(&pv_done[npv & 1]);
+            umma_commit(KVEQ ? &k_empty[npv & 1] : v_empty);
             ++npv;
-            if (++jp >= wp.np) {
+            if (++jp >= wp.nb) {
               jp = 0;
               ++ip;
               if (ip < count) wp.next();
@@ -497,25 +514,27 @@ __global__ void __launch_bounds__(kFaThreads, 1) attn_fa_kernel(
             progressed = true;
           }
         }
-        if (is < count && nqk - npv < NSB) {
+        if (is < count && nqk <= npv + 1) {
           const bool newq = js == 0 && ws.new_q;
           const int qb = (nq_used + 1) % C::kQBufs;
           bool ready = !newq || mbar_test_wait(&q_full[qb], ((nq_used + 1) / C::kQBufs) & 1);
-          ready = ready && mbar_test_wait(&k_full[nqk % NS], (nqk / NS) & 1);
+          ready = ready && mbar_test_wait(&k_full[nqk & 1], (nqk >> 1) & 1);
           if (ready) {
             if (newq) ++nq_used;
             tc_fence_after();
-            const uint32_t k_addr = smem_u32(stage + (nqk % NS) * C::kStage);
+            const int s = nqk & 1;
+            const uint32_t k_addr = smem_u32(stage + s * C::kStage);
             const uint32_t q_addr = smem_u32(qbuf + (nq_used % C::kQBufs) * C::kQBytes);
-            const uint32_t t_s = tmem + C::kColS + (nqk % NSB) * NP;
+            const uint32_t t_s = tmem + C::kColS + s * NP;
 #pragma unroll
             for (int kk = 0; kk < kDim / 16; ++kk)   // K = 16 dims per MMA
               umma_bf16(t_s, sw128_desc(k_addr + (kk >> 2) * kAtom + (kk & 3) * 32),
                         sw128_desc(q_addr + (kk >> 2) * (NP * 128) + (kk & 3) * 32), id_qk, kk > 0);
-            umma_commit(&s_full[nqk % NSB]);
-            // last page of the last item of this query group: release the queries
+            umma_commit(&s_full[s]);
+            if (!KVEQ) umma_commit(&k_empty[s]);     // keys no longer needed
+            // last block of the last item of this query group: release the queries
             bool last_of_group = false;
-            if (js + 1 >= ws.np) {
+            if (js + 1 >= ws.nb) {
               if (is + 1 >= count) {
                 last_of_group = true;
               } else {
@@ -526,7 +545,7 @@ __global__ void __launch_bounds__(kFaThreads, 1) attn_fa_kernel(
             }
             if (last_of_group) umma_commit(&q_empty[nq_used % C::kQBufs]);
             ++nqk;
-            if (++js >= ws.np) {
+            if (++js >= ws.nb) {
               js = 0;
               ++is;
               if (is < count) ws.next();
@@ -560,24 +579,18 @@ __global__ void __launch_bounds__(kFaThreads, 1) attn_fa_kernel(
     const int quad = warp & 3;               // TMEM lanes 32*quad .. (fixed by the warp id)
     const int half = sw >> 2;                // columns [half*NH, half*NH + NH)
     const int c0 = half * NH;
-    const int hs = lane >> 4;                // column group of this half-warp
-    const int t = quad * 16 + (lane & 15);   // key of the page
-    // The M = 64 scores of key t sit on TMEM lane 32*quad + (t & 15); a
-    // split-half load gives both half-warps those 16 lanes, each its own
-    // columns: half-warp hs owns columns c0 + 8i + 4hs + e (i < NH/8, e < 4),
-    // listed as j = 4i + e < NQ.
+    const int t = quad * 32 + lane;          // key of the block / O lane
     const uint32_t tq_lane = tmem + ((uint32_t)(quad * 32) << 16);
     const int bar_id = 1 + half;
     float* red_h = red + half * (2 * 128);
-    auto colj = [&](int j) -> int { return 8 * (j >> 2) + 4 * hs + (j & 3); };   // column in the half
-    // P tile address of (row c0 + colj(j), key t): a per-thread base plus the
-    // 128-byte swizzle term (chunk ^ (row & 7)) << 4, where row & 7 = 4hs + e
+    // P tile address of (row c0 + r, key t): a per-thread base plus the
+    // 128-byte swizzle term (chunk ^ (row & 7)) << 4, where row & 7 = r & 7
     // because c0 is a multiple of 8
-    const uint32_t chs = (uint32_t)(t >> 3) << 4;
-    const uint32_t p_off = c0 * 128 + ((t & 7) << 1);
+    const uint32_t chs = (uint32_t)((t & 63) >> 3) << 4;
+    const uint32_t p_off = (t >> 6) * (NP * 128) + c0 * 128 + ((t & 7) << 1);
     Walker w;
     if (count > 0) w.start(&a, start[0], start[1], start[2], start[3]);
-    int g = 0;                                // global page counter
+    int g = 0;                                // global block counter
     int nslow = 0;                            // slow-path rounds (double-buffered reductions)
     // the item whose output still waits in TMEM to be read out
     bool pend = false;
@@ -585,13 +598,13 @@ __global__ void __launch_bounds__(kFaThreads, 1) attn_fa_kernel(
     long pend_slot = 0;
     auto read_out = [&]() {
       // o of item pend_item: all its P . V done (the last one committed on
-      // pv_done of page pend_g - 1)
+      // pv_done of block pend_g - 1)
       const int gl = pend_g - 1;
-      fwait(&pv_done[gl % NPB], (gl / NPB) & 1, a.status, fail);
+      fwait(&pv_done[gl & 1], (gl >> 1) & 1, a.status, fail);
       tc_fence_after();
-      const uint32_t ob = (uint32_t)((pend_item % NOB) * (C::kOTiles * NP));
+      const uint32_t ob = (uint32_t)((pend_item & 1) * (C::kOTiles * NP));
       const bool out_ok = !*fail && (c0 >> a.lgG) < pend_npos;
-      // eight columns at a time (few registers: this runs inside the page loop)
+      // eight columns at a time (few registers: this runs inside the block loop)
 #pragma unroll 1
       for (int tt = 0; tt < C::kOTiles; ++tt) {
         const int d0 = o_dim0<KVEQ>(tt, quad);
@@ -612,7 +625,7 @@ __global__ void __launch_bounds__(kFaThreads, 1) attn_fa_kernel(
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&o_free[pend_item % NOB]);
+      if (lane == 0) mbar_arrive(&o_free[pend_item & 1]);
       pend = false;
     };
     for (int i = 0; i < count; ++i, w.next()) {
@@ -621,106 +634,100 @@ __global__ void __launch_bounds__(kFaThreads, 1) attn_fa_kernel(
       // nothing past the sequence's q positions
       const int npos = min(a.PB, a.q - w.rb * a.PB);            // positions in this row block
       const int pos0 = w.L + a.qpos_off + w.rb * a.PB;
-      auto row_pos = [&](int r) -> int {                         // r: column in the half; -1: padding
+      auto row_pos = [&](int r) -> int {                         // -1: padding column
         const int ip = (c0 + r) >> a.lgG;
         return ip < npos ? pos0 + ip : -1;
       };
       // a half whose columns are all padding only keeps the barriers going
       const bool active = row_pos(0) >= 0;
       const int pmin = pos0, pmax = pos0 + npos - 1;
-      const uint32_t t_ob = (uint32_t)((i % NOB) * (C::kOTiles * NP));
-      // page ids of the item -> validity bits in shared memory (one load per
-      // page, before the first page; two buffers by item parity, so that the
-      // next item's writes never meet this item's reads)
+      const uint32_t t_ob = (uint32_t)((i & 1) * (C::kOTiles * NP));   // this item's output buffer
+      // page ids of the item's blocks -> validity bits in shared memory (one
+      // load per page, before the first block; two buffers by item parity, so
+      // that the next item's writes never meet this item's reads)
       int* pvalid = pvalid_all + (i & 1) * kMaxItemPages;
       {
+        const int np_item = 2 * w.nb;
         const int st_ = sw * 32 + lane;
-        if (st_ < w.np) {
-          const int id = bt_all[(long)w.b * a.max_pages + w.pg0 + st_];
-          pvalid[st_] = id >= 0 && id < a.num_pages;
+        if (st_ < np_item) {
+          const int pg = 2 * w.blk0 + st_;
+          int ok = 0;
+          if (pg < a.max_pages) {
+            const int id = bt_all[(long)w.b * a.max_pages + pg];
+            ok = id >= 0 && id < a.num_pages;
+          }
+          pvalid[st_] = ok;
         }
         named_bar(3, kSoftWarps * 32);
       }
       // running state per row: the reference maximum (log2 domain; kNoKey
       // until the row has seen a key, so that 2^(s - m) of a masked score is
-      // exactly 0 and every visible score moves it), kept for every column of
-      // the half (the output rescale needs all of them), and the row sum over
-      // this thread's key, for its own NQ columns
-      // (mq: mref of the thread's own columns; every array index below is a
-      // compile-time constant, the half-warp picks by predicate)
-      float mref[NH], mq[NQ], lt[NQ];
+      // exactly 0 and every visible score moves it) and the row sum
+      float mref[NH], lt[NH];
 #pragma unroll
-      for (int r = 0; r < NH; ++r) mref[r] = kNoKey;
-#pragma unroll
-      for (int j = 0; j < NQ; ++j) {
-        mq[j] = kNoKey;
-        lt[j] = 0.f;
+      for (int r = 0; r < NH; ++r) {
+        mref[r] = kNoKey;
+        lt[r] = 0.f;
       }
-      for (int jp = 0; jp < w.np; ++jp, ++g) {
-        const int kb = (w.pg0 + jp) * kPg;
-        const bool pv = pvalid[jp] != 0;
-        const bool interior = kb >= w.lo && kb + kPg - 1 <= w.hi && pv && kb + kPg - 1 <= pmin &&
-                              (a.window == 0 || kb > pmax - a.window);
+      for (int j = 0; j < w.nb; ++j, ++g) {
+        const int s = g & 1;
+        const int kb = (w.blk0 + j) * kBlk;
+        const bool pv0 = pvalid[2 * j] != 0, pv1 = pvalid[2 * j + 1] != 0;
+        const bool interior = kb >= w.lo && kb + kBlk - 1 <= w.hi && pv0 && pv1 &&
+                              kb + kBlk - 1 <= pmin && (a.window == 0 || kb > pmax - a.window);
         const int key = kb + t;
-        const bool in_range = pv && key >= w.lo && key <= w.hi;
-        fwait(&s_full[g % NSB], (g / NSB) & 1, a.status, fail);
+        const bool in_range = key >= w.lo && key <= w.hi && ((t < kPg) ? pv0 : pv1);
+        fwait(&s_full[s], (g >> 1) & 1, a.status, fail);
         tc_fence_after();
-        float sc[NQ];
+        float sc[NH];
         bool need = false;
         if (active) {
-          uint32_t r4[NH / 8][4];
+          uint32_t r8[NH / 8][8];
 #pragma unroll
-          for (int c = 0; c < NH / 8; ++c)
-            tmem_ld16x2_4_nowait(tq_lane + C::kColS + (g % NSB) * NP + c0 + 8 * c, r4[c]);
+          for (int c = 0; c < NH / 8; ++c) tmem_ld8_nowait(tq_lane + C::kColS + s * NP + c0 + 8 * c, r8[c]);
           tmem_ld_wait();
 #pragma unroll
           for (int c = 0; c < NH / 8; ++c)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) sc[4 * c + e] = __fmul_rn(__uint_as_float(r4[c][e]), a.scale_log2);
+            for (int e = 0; e < 8; ++e) sc[8 * c + e] = __fmul_rn(__uint_as_float(r8[c][e]), a.scale_log2);
           if (!interior) {
 #pragma unroll
-            for (int j = 0; j < NQ; ++j) {
-              const int p = row_pos(colj(j));
+            for (int r = 0; r < NH; ++r) {
+              const int p = row_pos(r);
               const bool vis = in_range && key <= p && (a.window == 0 || key > p - a.window);
-              if (!vis) sc[j] = -INFINITY;
+              if (!vis) sc[r] = -INFINITY;
             }
           }
 #pragma unroll
-          for (int j = 0; j < NQ; ++j) need |= sc[j] > __fadd_rn(mq[j], kLazy);
+          for (int r = 0; r < NH; ++r) need |= sc[r] > __fadd_rn(mref[r], kLazy);
         }
         // ---- the reference maxima move only when some row needs it
         if (bar_red_or(bar_id, 128, need)) {
           float* rb_ = red_h + (nslow & 1) * 128;
           ++nslow;
-          float v[16];
+          float v[32];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) v[e] = e < NQ ? sc[e] : -INFINITY;
-          const float mx = transpose_reduce16<true>(v, lane);
-          rb_[quad * 32 + lane] = mx;     // column j = lane & 15 of half-warp hs
+          for (int e = 0; e < 32; ++e) v[e] = e < NH ? sc[e] : -INFINITY;
+          const float mx = transpose_reduce32<true>(v, lane);
+          rb_[quad * 32 + lane] = mx;
           named_bar(bar_id, 128);
           float alpha[NH];
           bool moved = false;
 #pragma unroll
           for (int r = 0; r < NH; ++r) {
-            const int ix = ((r >> 2) & 1) * 16 + 4 * (r >> 3) + (r & 3);   // (hs, j) of column r
-            const float bm = fmaxf(fmaxf(rb_[ix], rb_[32 + ix]), fmaxf(rb_[64 + ix], rb_[96 + ix]));
+            const float bm = fmaxf(fmaxf(rb_[r], rb_[32 + r]), fmaxf(rb_[64 + r], rb_[96 + r]));
             alpha[r] = 1.f;
             if (bm > __fadd_rn(mref[r], kLazy)) {
               alpha[r] = ex2_approx(__fsub_rn(mref[r], bm));   // 0 while the row had no key
               mref[r] = bm;
+              lt[r] = __fmul_rn(lt[r], alpha[r]);
               moved = true;
             }
           }
-#pragma unroll
-          for (int j = 0; j < NQ; ++j) {
-            const int lo_ = 8 * (j >> 2) + (j & 3);
-            mq[j] = hs ? mref[lo_ + 4] : mref[lo_];
-            lt[j] = __fmul_rn(lt[j], hs ? alpha[lo_ + 4] : alpha[lo_]);
-          }
-          if (moved && jp > 0) {
+          if (moved && j > 0) {
             // rescale this half's columns of the running output (all P . V of
-            // the item's earlier pages must have completed)
-            fwait(&pv_done[(g - 1) % NPB], ((g - 1) / NPB) & 1, a.status, fail);
+            // the earlier blocks must have completed)
+            fwait(&pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1, a.status, fail);
             tc_fence_after();
 #pragma unroll
             for (int tt = 0; tt < C::kOTiles; ++tt) {
@@ -738,43 +745,54 @@ __global__ void __launch_bounds__(kFaThreads, 1) attn_fa_kernel(
             tmem_st_wait();
           }
         }
-        // the P buffer of this page was last read by P . V of page g - NPB
-        if (g >= NPB) fwait(&pv_done[g % NPB], ((g / NPB) - 1) & 1, a.status, fail);
+        // the P buffer of this block was last read by P . V of block g - kPBufs
+        if (g >= C::kPBufs)
+          fwait(&pv_done[(g - C::kPBufs) & 1], ((g - C::kPBufs) >> 1) & 1, a.status, fail);
         if (active) {
           // ---- probabilities: unrounded into the row sums, bf16 into P
           // (2^-inf = 0: masked keys and rows without a key so far give 0)
-          uint8_t* pp = pbuf + (g % NPB) * C::kPBytes + p_off;
+          uint8_t* pp = pbuf + (g % C::kPBufs) * C::kPBytes + p_off;
 #pragma unroll
-          for (int j = 0; j < NQ; ++j) {
-            const int r = colj(j);
-            const float p = ex2_approx(__fsub_rn(sc[j], mq[j]));
-            lt[j] = __fadd_rn(lt[j], p);
-            *reinterpret_cast<uint16_t*>(pp + r * 128 + (chs ^ ((uint32_t)(4 * hs + (j & 3)) << 4))) =
-                f32_to_bf16(p);
+          for (int r = 0; r < NH; ++r) {
+            const float p = ex2_approx(__fsub_rn(sc[r], mref[r]));
+            lt[r] = __fadd_rn(lt[r], p);
+            *reinterpret_cast<uint16_t*>(pp + r * 128 + (chs ^ ((uint32_t)(r & 7) << 4))) = f32_to_bf16(p);
           }
         }
         // ---- value rows of keys no row of the item may use: zero them
         if (!interior && !in_range && half == 0) {
-          uint8_t* base = stage + (g % NS) * C::kStage + (KVEQ ? 0u : 4u * kAtom);
-          constexpr int kVAtoms = KVEQ ? 5 : 4;
-          for (int at = hs; at < kVAtoms; at += 2)
+          if (KVEQ) {
+            uint8_t* base = stage + s * C::kStage;
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-              *reinterpret_cast<uint4*>(base + at * kAtom + t * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+            for (int at = 0; at < 5; ++at)
+#pragma unroll
+              for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<uint4*>(base + at * kAtom + t * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+          } else if ((g == 0 || fwait(&pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1, a.status, fail)) &&
+                     fwait(v_full, g & 1, a.status, fail)) {
+            // the single value buffer takes block g's values only after P . V
+            // of block g - 1; from then on its current phase is block g's
+#pragma unroll
+            for (int at = 0; at < 4; ++at)
+#pragma unroll
+              for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<uint4*>(vbuf + at * kAtom + t * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+          }
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[g % NPB]);
-        // the previous item's output, one page after its last P . V
+        if (lane == 0) mbar_arrive(&p_full[g & 1]);
+        // the previous item's output, one block after its last P . V
         if (pend) read_out();
       }
 
-      // ---- the item's (m, l) now; its o after the next item's first page
-      float v[16];
+      // ---- the item's (m, l) now (log2 domain); its o, unnormalised, after
+      //      the next item's first block
+      float v[32];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) v[e] = e < NQ ? lt[e] : 0.f;
-      const float lq = transpose_reduce16<false>(v, lane);
+      for (int e = 0; e < 32; ++e) v[e] = e < NH ? lt[e] : 0.f;
+      const float lq = transpose_reduce32<false>(v, lane);
       float* rl = red_h + (nslow & 1) * 128;
       ++nslow;
       rl[quad * 32 + lane] = lq;
@@ -788,8 +806,7 @@ __global__ void __launch_bounds__(kFaThreads, 1) attn_fa_kernel(
 #pragma unroll
           for (int r = 0; r < NH; ++r)
             if (r == lane) mv = mref[r];
-          const int ix = ((lane >> 2) & 1) * 16 + 4 * (lane >> 3) + (lane & 3);
-          const float l = __fadd_rn(__fadd_rn(rl[ix], rl[32 + ix]), __fadd_rn(rl[64 + ix], rl[96 + ix]));
+          const float l = __fadd_rn(__fadd_rn(rl[lane], rl[32 + lane]), __fadd_rn(rl[64 + lane], rl[96 + lane]));
           const int prow = (c & (a.G - 1)) * a.q + ip;
           __stcg(reinterpret_cast<float2*>(a.part_ml + (slot + prow) * 2), make_float2(mv, l));
         }
