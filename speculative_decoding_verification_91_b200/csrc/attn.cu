@@ -135,7 +135,7 @@ struct ACfg {
   static constexpr int kVBytes = KVEQ ? kPage * kSbw * 2 : kPage * D * 2;
   static constexpr int kStageBytes = kKBytes + kVBytes;
   static constexpr int kQBytes = kRowsPad * D * 2;
-  static constexpr int kPBytes = 2 * kRowsPad * 128;   // P = P_hi + P_lo, both bf16
+  static constexpr int kPBytes = kRowsPad * 128;       // P as bf16
   static constexpr int kRedBytes = 2 * kCW * kRowsPad * 4;
   static constexpr int kFixed = 1024 + kQBytes + kPBytes + kRedBytes + 256;
   // Prefer a footprint that lets two CTAs share an SM (two pages in flight
@@ -422,16 +422,12 @@ __global__ void __launch_bounds__(kThreads) attn_split_kernel(
         }
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          // split p into a bf16 head and a bf16 tail: P V = P_hi V + P_lo V is
-          // then exact to ~2^-16 relative instead of 2^-9
+          // p rounded once to bf16 for P V (the row sums keep the unrounded
+          // values), as in the tensor-memory kernel
           const int r = mt * 16 + g + 8 * h;
           const uint32_t addr = p_base + swz128(r, 2 * warp + nt) + 4 * t;
-          const float a0 = pv[2 * h], a1 = pv[2 * h + 1];
-          const uint32_t hi = pack_bf16x2(a0, a1);
-          const float h0 = __uint_as_float(hi << 16), h1 = __uint_as_float(hi & 0xffff0000u);
-          const uint32_t lo = pack_bf16x2(__fsub_rn(a0, h0), __fsub_rn(a1, h1));
-          asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(hi));
-          asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr + RP * 128), "r"(lo));
+          const uint32_t pb = pack_bf16x2(pv[2 * h], pv[2 * h + 1]);
+          asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(pb));
         }
       }
 #pragma unroll
@@ -465,12 +461,11 @@ __global__ void __launch_bounds__(kThreads) attn_split_kernel(
     if (valid) {
 #pragma unroll
       for (int kk = 0; kk < kPage / 16; ++kk) {
-        uint32_t af[MT][4], al[MT][4];
+        uint32_t af[MT][4];
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
           const uint32_t pa = p_base + swz128(mt * 16 + (lane & 15), kk * 2 + (lane >> 4));
           ldsm_x4(pa, af[mt][0], af[mt][1], af[mt][2], af[mt][3]);
-          ldsm_x4(pa + RP * 128, al[mt][0], al[mt][1], al[mt][2], al[mt][3]);
         }
         const uint32_t vrow = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
@@ -491,8 +486,6 @@ __global__ void __launch_bounds__(kThreads) attn_split_kernel(
           for (int mt = 0; mt < MT; ++mt) {
             mma_bf16(o[mt][2 * np2], af[mt], b0, b1);
             mma_bf16(o[mt][2 * np2 + 1], af[mt], b2, b3);
-            mma_bf16(o[mt][2 * np2], al[mt], b0, b1);
-            mma_bf16(o[mt][2 * np2 + 1], al[mt], b2, b3);
           }
         }
       }
