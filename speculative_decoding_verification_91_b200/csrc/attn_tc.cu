@@ -851,18 +851,18 @@ int fa_np(const AttnGeom& g, int G) {
 }  // namespace
 
 // Which layers take the tensor-memory attention: head_dim 256 with 64-token
-// pages, and at least SPECVERIFY_TC_ATTN_MIN_G query heads per KV head
-// (default 4).  The choice depends on the model only, never on k or the
-// batch, so a row is computed by the same kernel whatever k is.  With G = 2
-// (8 to 10 rows per KV head at the benchmark's k) the mma.sync kernel's lighter
-// per-block work is faster (batch 64 global layer 479 vs 660 us, batch 1
-// sliding-window layer 12 vs 19 us); from G = 4 on the tensor cores win
-// (batch 8, G = 8: 168 vs 255 us).  Sliding-window layers stay on the mma.sync
-// kernel: a window of about a thousand keys leaves one or two 128-key blocks
-// per split, too little work to cover this kernel's set-up (one sequence,
-// 2 KV heads, G = 4, 9 query positions, window 1024: 16-21 vs 12 us);
-// SPECVERIFY_TC_ATTN_LOCAL=1 admits them.  SPECVERIFY_NO_TC_ATTN=1 or
-// SPECVERIFY_NO_TC=1 turns the path off.
+// pages, no sliding window, and at least SPECVERIFY_TC_ATTN_MIN_G query heads
+// per KV head (default 4).  The choice depends on the model only, never on k
+// or the batch, so a row is computed by the same kernel whatever k is.  With
+// G = 2 (8 to 10 rows per KV head at the benchmark's k) the mma.sync kernel's
+// lighter per-block work is faster (batch 64 global layer 475-500 vs about
+// 800 us, batch 1 layers 11 / 18 vs 15 / 27 us); from G = 4 on the tensor
+// cores win (batch 8, G = 8: 143 vs 255 us).  Sliding-window layers stay on
+// the mma.sync kernel: a window of about a thousand keys leaves one or two
+// 128-key blocks per split, too little work to cover this kernel's set-up
+// (one sequence, 2 KV heads, G = 4, 9 query positions, window 1024: 15-16 vs
+// 11-12 us); SPECVERIFY_TC_ATTN_LOCAL=1 admits them.  SPECVERIFY_NO_TC_ATTN=1
+// or SPECVERIFY_NO_TC=1 turns the path off.
 bool attn_tc_supported(const AttnGeom& g) {
   static const bool local_ok = [] {
     const char* v = getenv("SPECVERIFY_TC_ATTN_LOCAL");

@@ -1,21 +1,25 @@
 // Streaming GEMM on the 5th-generation tensor cores (tcgen05 + TMEM) for
-// verify steps with many rows (M = B*(k+1) up to 256, e.g. batch 64 x 4
-// rows): Y = X . W^T with W [N][K] streamed once from HBM and every verify
-// row in the MMA's N dimension, so the weights are read once whatever M is.
+// verify steps with many rows (M = B*(k+1) above 32, e.g. batch 64 x 4
+// rows): Y = X . W^T with W [N][K] streamed once from HBM and up to 256
+// verify rows in the MMA's N dimension, so the weights are read once per
+// 256 rows whatever M is (more rows: blocks of 256 on grid z).
 //
-// One CTA per (128-row weight tile, K split); 6 warps:
-//   warp 0   TMA producer: W box 128 x 64 and X box NP x 64 (128-byte
-//            swizzle) into a ring of stages (mbarrier full/empty); the first
+// One CTA per (NW 128-row weight tiles, K split, row block); 6 warps:
+//   warp 0   TMA producer: NW W boxes 128 x 64 and an X box NP x 64 (128-byte
+//            swizzle) per stage into a ring (mbarrier full/empty); the first
 //            ring of W tiles is requested before the programmatic-launch wait;
-//   warp 1   allocates the TMEM accumulator (128 lanes x NP fp32 columns) and
+//   warp 1   allocates NW TMEM accumulators (128 lanes x NP fp32 columns) and
 //            one elected thread issues tcgen05.mma kind::f16 (A = W tile,
 //            B = X tile, both K-major SW128 shared-memory descriptors), 4 MMAs
-//            of K = 16 per stage; tcgen05.commit releases each stage and, after
-//            the last, signals the accumulator;
-//   warps 2-5 read the accumulator with tcgen05.ld (warp w owns TMEM lanes
-//            32*(w%4)..: one weight row per thread) and run the epilogue:
-//            per-tile argmax over the 128 rows of every verify row, or the
-//            split-K partial tile for the store / residual / RoPE epilogues.
+//            of K = 16 per stage and accumulator; tcgen05.commit releases each
+//            stage and, after the last, signals the accumulators;
+//   warps 2-5 read the accumulators with tcgen05.ld (warp w owns TMEM lanes
+//            32*(w%4)..: one weight row per thread and tile) and run the
+//            epilogue: the argmax over the CTA's weight rows of every verify
+//            row, or the split-K partial tile for the store / residual / RoPE
+//            epilogues (NW = 1).  NW = 2 serves LM heads above 128 padded
+//            rows, where the tensor cores bound the kernel: the row tile is
+//            then read from L2 once per 256 weight rows.
 //
 // Every wait is bounded; the CTA always reaches its final barrier and frees
 // its TMEM, also after a timeout.
