@@ -1,11 +1,13 @@
 """Host-side measurement logic of bench.py, on CPU: algorithmic bytes by
 hand, the roofline's bound choice and arithmetic, the guard that drops a
-recorded ncu traffic figure once its kernel's sources change, and the
-parsing of sampled clocks and throttle reasons."""
+recorded ncu traffic figure once its kernel's sources change, the parsing of
+sampled clocks and throttle reasons, the expected-tokens law of the sweep and
+the loop bench's drafter."""
 import json
 import os
 import types
 
+import numpy as np
 import pytest
 
 import bench
@@ -91,3 +93,45 @@ def test_clock_summary_reports_median_and_active_reasons():
     assert s["reasons"] == ["sw_power_cap"]
     c.lines, c.skip = [], 0
     assert c.summary()["reasons"] == ["unsampled"]
+
+
+def test_expected_tokens_is_the_mean_of_the_accepted_run_plus_one():
+    """E[a + 1] for i.i.d. acceptance alpha, a = leading accepted drafts of k:
+    the closed form (1 - alpha^(k+1)) / (1 - alpha), and brute force over all
+    2^k accept/reject patterns."""
+    import itertools
+    for alpha in (0.5, 0.8, 0.9):
+        for k in (0, 1, 4, 8):
+            closed = (1 - alpha ** (k + 1)) / (1 - alpha)
+            brute = 0.0
+            for pat in itertools.product((0, 1), repeat=k):
+                prob = 1.0
+                for ok in pat:
+                    prob *= alpha if ok else 1 - alpha
+                a = next((i for i, ok in enumerate(pat) if not ok), k)
+                brute += prob * (a + 1)
+            assert bench.expected_tokens(alpha, k) == pytest.approx(closed, rel=1e-12)
+            assert brute == pytest.approx(closed, rel=1e-12)
+
+
+def test_loop_drafter_keeps_the_greedy_token_where_its_coin_says_so():
+    """The loop bench's corrupted-greedy drafter: draft i of step s is the
+    greedy stream's token at the sequence's emitted position + i when the
+    step's seeded flip i is below the acceptance probability, else the
+    step's seeded random id; the same step gives the same drafts."""
+    wl = W.get_workload("loop_131k")
+    p = wl.accept[1]
+    stream = [1000 + 3 * i for i in range(200)]
+    drafter = bench.loop_drafter(wl, stream)
+    kept = total = 0
+    for step, emitted in ((0, 0), (1, 5), (7, 40), (30, 150)):
+        flips, ids = W.loop_draft_flips(wl, step)
+        d = drafter(step, emitted)
+        assert d.dtype == np.int32 and d.shape == (wl.k,)
+        assert np.array_equal(d, drafter(step, emitted))
+        for i in range(wl.k):
+            want = stream[emitted + i] if flips[i] < p else int(ids[i])
+            assert int(d[i]) == want
+            kept += int(flips[i] < p)
+            total += 1
+    assert 0.5 < kept / total < 1.0           # p = 0.8 over 32 seeded flips
